@@ -1,0 +1,438 @@
+"""CPU oracle for the token-choice MoE expert layer, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  It shares no code with the CUDA library and never imports it.
+
+Everything is plain numpy in float64.  Each function restates one step of the
+method as the source pages define it; a library primitive (matmul, argsort,
+bincount) may serve as a step, with no blocking or fusion beyond that.
+
+Sources (cited by page title and section):
+  [Beam]     "From 501B to 23B: what is Beam doing" -- sec. 2.2 (router, top-k,
+             weighted sum of experts), sec. 5.3 (MoELayer: top-k, then softmax
+             of the k values, per-expert masked loop), sec. 5.4 (expert counts).
+  [Trinity]  "Trinity Large: open 400B sparse MoE" commentary -- example 1
+             (gate logits, torch.topk, softmax of the top-k), example 2
+             (bincount of expert ids), example 3 (dispatch tokens into
+             per-expert input lists, run experts, add outputs back per token).
+  [SonicMoE] techwalker summary of SonicMoE -- sec. 1 (router-score gradient
+             dS = <dA', A> instead of <dO, Y>; recompute instead of store),
+             sec. 3 (token rounding: snap each expert's token count to the
+             nearest multiple of the GEMM tile, e.g. 145 -> 128).
+  [Olmo]     Olmo-core 3 news piece -- "row-wise expert parallelism puts data
+             straight into expert input buffers", GPU-resident routing,
+             grouped GEMM.
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * top-k then softmax over the k selected logits (sec. 5.3 / example 1); ties
+    in the logits go to the lowest expert id.
+  * experts are SwiGLU: A = silu(x W1) * (x W3), Y = A W2.
+  * rows of one expert are stored in ascending token order, and each expert's
+    segment starts at a multiple of the tile (128 rows); padding rows are
+    empty (token -1, weight 0).
+  * bf16 "staging": in the bf16 path every tensor that is stored in bf16 or
+    fed to a bf16 GEMM (H, A, Y, g*A, dH, dX_perm) is rounded to bf16
+    (round-to-nearest-even) at the same point here; ``staged=False`` gives the
+    ideal fp64 value.
+  * token rounding: r_e = tile*round(c_e/tile) with halves rounding up, capped
+    at tile*floor(T/tile); ranking key s_te = exp(l_te - LSE over the token's
+    top-k logits); drops take the smallest keys (ties: larger token first),
+    additions take the largest keys among unassigned tokens (ties: smaller
+    token first); final weights are s_te without renormalisation.
+
+parity pins: tests/test_oracle_pins.py (brute force, dense masked evaluation,
+closed-form 2-expert example, central finite differences, the 145 -> 128
+rounding example, invariants).  No function here is unpinned.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TILE = 128
+
+
+# --------------------------------------------------------------------------
+# elementary pieces
+# --------------------------------------------------------------------------
+
+def bf16_round(a):
+    """Round float64 values to the nearest bfloat16 value (ties to even).
+
+    bfloat16 keeps 8 significant bits and the float32 exponent range, so the
+    spacing of representable values around |a| in [2^(e-1), 2^e) is 2^(e-8),
+    and never finer than the subnormal spacing 2^-133.
+    """
+    a = np.asarray(a, dtype=np.float64)
+    out = np.zeros_like(a)
+    nz = a != 0
+    if not np.any(nz):
+        return out
+    _, e = np.frexp(a[nz])                    # a = m * 2^e, 0.5 <= |m| < 1
+    e = np.maximum(e, -125)
+    ulp = np.ldexp(1.0, e - 8)
+    out[nz] = np.rint(a[nz] / ulp) * ulp      # np.rint rounds halves to even
+    return out
+
+
+def _stage(a, staged):
+    return bf16_round(a) if staged else a
+
+
+def sigmoid(z):
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * (1.0 + np.tanh(0.5 * z))
+
+
+def silu(z):
+    """silu(z) = z * sigmoid(z)."""
+    return np.asarray(z, dtype=np.float64) * sigmoid(z)
+
+
+def silu_grad(z):
+    """d silu / dz = sigmoid(z) * (1 + z * (1 - sigmoid(z)))."""
+    s = sigmoid(z)
+    return s * (1.0 + z * (1.0 - s))
+
+
+# --------------------------------------------------------------------------
+# router: logits, top-k, softmax over the top-k  ([Beam] 2.2, 5.3; [Trinity] ex. 1)
+# --------------------------------------------------------------------------
+
+def route(x, w_gate, k, logits_override=None, logit_bias=None):
+    """Router logits l = x W_gate (+ optional per-expert bias), the k largest
+    logits of each token (ties: lowest expert id first), and their softmax.
+
+    Returns (logits [T,E] f64, idx [T,k] int32, gate [T,k] f64).
+    """
+    if logits_override is not None:
+        logits = np.array(logits_override, dtype=np.float64)
+    else:
+        logits = np.asarray(x, np.float64) @ np.asarray(w_gate, np.float64)
+    if logit_bias is not None:
+        logits = logits + np.asarray(logit_bias, np.float64)[None, :]
+    # a stable sort of the negated logits keeps equal values in ascending id
+    idx = np.argsort(-logits, axis=1, kind="stable")[:, :k]
+    top = np.take_along_axis(logits, idx, axis=1)
+    ex = np.exp(top - top[:, :1])
+    gate = ex / ex.sum(axis=1, keepdims=True)
+    return logits, idx.astype(np.int32), gate
+
+
+# --------------------------------------------------------------------------
+# permutation into expert-contiguous rows  ([Trinity] ex. 2-3; [Olmo]; [Beam] 5.4)
+# --------------------------------------------------------------------------
+
+def _pad(n, tile):
+    return ((n + tile - 1) // tile) * tile
+
+
+def row_capacity(T, E, k, tile=TILE):
+    """Rows any plan may occupy: every slot plus a tile of slack per expert."""
+    return T * k + E * tile
+
+
+def exact_plan(idx, gate, E, tile=TILE):
+    """Dropless permutation.  counts[e] = number of tokens that chose e;
+    expert e owns rows [offsets[e], offsets[e] + counts[e]) in ascending token
+    order; offsets are the exclusive prefix sum of counts padded to the tile.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    cap = row_capacity(T, E, k, tile)
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.int64)
+    offsets = np.zeros(E + 1, np.int64)
+    offsets[1:] = np.cumsum(_pad(counts, tile))
+    row_token = np.full(cap, -1, np.int64)
+    row_slot = np.full(cap, -1, np.int64)
+    row_gate = np.zeros(cap, np.float64)
+    slot_row = np.full(T * k, -1, np.int64)
+    flat = idx.ravel()
+    # slots are numbered token-major (s = t*k + j); a stable sort by expert
+    # keeps ascending token order inside each expert
+    order = np.argsort(flat, kind="stable")
+    start = np.zeros(E + 1, np.int64)
+    start[1:] = np.cumsum(counts)
+    for e in range(E):
+        slots = order[start[e]:start[e + 1]]
+        rows = offsets[e] + np.arange(len(slots))
+        row_token[rows] = slots // k
+        row_slot[rows] = slots
+        row_gate[rows] = np.asarray(gate, np.float64).ravel()[slots]
+        slot_row[slots] = rows
+    return dict(mode="exact", T=T, E=E, k=k, tile=tile, cap=cap, counts=counts,
+                offsets=offsets, row_token=row_token, row_slot=row_slot,
+                row_gate=row_gate, slot_row=slot_row, extra_row=None,
+                R=int(offsets[-1]))
+
+
+def rounded_target(counts, T, tile=TILE):
+    """Token rounding target ([SonicMoE] sec. 3): the multiple of the tile
+    nearest to each count (an exact half rounds up), capped at the largest
+    multiple of the tile that does not exceed T."""
+    counts = np.asarray(counts, np.int64)
+    r = tile * ((counts + tile // 2) // tile)
+    return np.minimum(r, tile * (T // tile))
+
+
+def rounding_keys(logits, idx):
+    """Log-domain ranking key l_te - LSE_{j in top-k(t)} l_tj for every
+    (token, expert) pair; exp(key) is the routing weight of a selected pair."""
+    logits = np.asarray(logits, np.float64)
+    top = np.take_along_axis(logits, np.asarray(idx), axis=1)
+    m = top.max(axis=1)
+    lse = m + np.log(np.exp(top - m[:, None]).sum(axis=1))
+    return logits - lse[:, None]
+
+
+def rounded_plan(idx, logits, E, tile=TILE):
+    """Token-rounded permutation ([SonicMoE] sec. 3 with the readings in the
+    module docstring).  Adds ``extra_row[T,E]`` (row of an added pair, else -1)
+    and ``dropped``/``added`` masks for checking."""
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    cap = row_capacity(T, E, k, tile)
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.int64)
+    target = rounded_target(counts, T, tile)
+    key = rounding_keys(logits, idx)
+    assigned = np.zeros((T, E), bool)
+    assigned[np.arange(T)[:, None], idx] = True
+    final = assigned.copy()
+    toks = np.arange(T)
+    for e in range(E):
+        if target[e] < counts[e]:
+            cand = toks[assigned[:, e]]
+            # order by key descending, then token ascending; keep the first r_e
+            order = cand[np.lexsort((cand, -key[cand, e]))]
+            final[order[target[e]:], e] = False
+        elif target[e] > counts[e]:
+            cand = toks[~assigned[:, e]]
+            order = cand[np.lexsort((cand, -key[cand, e]))]
+            final[order[:target[e] - counts[e]], e] = True
+    offsets = np.zeros(E + 1, np.int64)
+    offsets[1:] = np.cumsum(target)
+    row_token = np.full(cap, -1, np.int64)
+    row_slot = np.full(cap, -1, np.int64)
+    row_gate = np.zeros(cap, np.float64)
+    slot_row = np.full(T * k, -1, np.int64)
+    extra_row = np.full((T, E), -1, np.int64)
+    slot_of = np.full((T, E), -1, np.int64)
+    slot_of[np.arange(T)[:, None], idx] = np.arange(T * k).reshape(T, k)
+    for e in range(E):
+        members = toks[final[:, e]]
+        rows = offsets[e] + np.arange(len(members))
+        row_token[rows] = members
+        row_gate[rows] = np.exp(key[members, e])
+        s = slot_of[members, e]
+        row_slot[rows] = s
+        kept = s >= 0
+        slot_row[s[kept]] = rows[kept]
+        extra_row[members[~kept], e] = rows[~kept]
+    return dict(mode="rounded", T=T, E=E, k=k, tile=tile, cap=cap, counts=counts,
+                target=target, offsets=offsets, row_token=row_token,
+                row_slot=row_slot, row_gate=row_gate, slot_row=slot_row,
+                extra_row=extra_row, dropped=assigned & ~final,
+                added=final & ~assigned, R=int(offsets[-1]), key=key)
+
+
+def token_rows(plan, t):
+    """All rows of token t: its kept slots in slot order, then the rows added
+    by token rounding in ascending expert order."""
+    k = plan["k"]
+    rows = [int(r) for r in plan["slot_row"][t * k:(t + 1) * k] if r >= 0]
+    if plan["extra_row"] is not None:
+        rows += [int(r) for r in plan["extra_row"][t] if r >= 0]
+    return rows
+
+
+def row_expert(plan, rows):
+    """Expert owning each row (the segment the row falls in)."""
+    return np.searchsorted(plan["offsets"], np.asarray(rows), side="right") - 1
+
+
+# --------------------------------------------------------------------------
+# expert SwiGLU FFN on the rows of one expert
+# --------------------------------------------------------------------------
+
+def expert_rows_forward(xr, w1e, w3e, w2e, staged):
+    """H = [x W1 | x W3] (bf16-staged if ``staged``), A = silu(h1) * h3,
+    Y = A W2, for the rows ``xr`` [n,d] routed to one expert."""
+    xr = np.asarray(xr, np.float64)
+    h1 = _stage(xr @ w1e, staged)
+    h3 = _stage(xr @ w3e, staged)
+    a = _stage(silu(h1) * h3, staged)
+    y = _stage(a @ w2e, staged)
+    return h1, h3, a, y
+
+
+def expert_rows_backward(dor, gr, h1, h3, w1e, w3e, w2e, staged):
+    """Backward of one expert's rows given dO rows ``dor`` and row weights ``gr``.
+
+    dA' = dO W2^T                       (gradient of A before gate scaling)
+    dS  = <dA', A>                      ([SonicMoE] sec. 1: no stored Y needed)
+    dA  = g dA';  da3 = dA silu(h1);  da1 = dA h3 silu'(h1)
+    g*A (operand of dW2), dX_perm = da1 W1^T + da3 W3^T.
+    """
+    dor = np.asarray(dor, np.float64)
+    a = _stage(silu(h1) * h3, staged)
+    dap = dor @ w2e.T
+    ds = np.sum(dap * a, axis=1)
+    da = gr[:, None] * dap
+    da3 = _stage(da * silu(h1), staged)
+    da1 = _stage(da * h3 * silu_grad(h1), staged)
+    ga = _stage(gr[:, None] * a, staged)
+    dxp = _stage(da1 @ w1e.T + da3 @ w3e.T, staged)
+    return ds, da1, da3, ga, dxp
+
+
+# --------------------------------------------------------------------------
+# full layer, and the same quantities on a subset of tokens / experts
+# --------------------------------------------------------------------------
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
+    """Forward (and, given dout, backward) quantities of the listed rows.
+
+    Rows are grouped by the expert that owns them; padding rows give zeros.
+    Returns a dict of arrays aligned with ``rows``: H [n,2f], A [n,f],
+    Y [n,d] and, with dout, dS [n], dH [n,2f], gA [n,f], dXp [n,d].
+    """
+    rows = np.asarray(rows, np.int64)
+    x, w1, w3, w2 = map(_f64, (x, w1, w3, w2))
+    n, d, f = len(rows), x.shape[1], w1.shape[2]
+    res = dict(H=np.zeros((n, 2 * f)), A=np.zeros((n, f)), Y=np.zeros((n, d)))
+    if dout is not None:
+        dout = _f64(dout)
+        res.update(dS=np.zeros(n), dH=np.zeros((n, 2 * f)), gA=np.zeros((n, f)),
+                   dXp=np.zeros((n, d)))
+    toks_all = plan["row_token"][rows]
+    es = row_expert(plan, rows)
+    for e in np.unique(es[toks_all >= 0]):
+        sel = np.nonzero((es == e) & (toks_all >= 0))[0]
+        toks = toks_all[sel]
+        h1, h3, a, y = expert_rows_forward(x[toks], w1[e], w3[e], w2[e], staged)
+        res["H"][sel, :f], res["H"][sel, f:], res["A"][sel], res["Y"][sel] = h1, h3, a, y
+        if dout is not None:
+            g = plan["row_gate"][rows[sel]]
+            ds, da1, da3, ga, dxp = expert_rows_backward(
+                dout[toks], g, h1, h3, w1[e], w3[e], w2[e], staged)
+            res["dS"][sel] = ds
+            res["dH"][sel, :f], res["dH"][sel, f:] = da1, da3
+            res["gA"][sel] = ga
+            res["dXp"][sel] = dxp
+    return res
+
+
+def token_router_grad(plan, idx, gate, t, rows, dS_rows):
+    """dlogits of token t from the router-score gradients of its rows.
+
+    With F_t the final rows of token t (weights s), K_t its top-k experts and
+    p = softmax over K_t:
+        dl_te = [e in F_t] s_te dS_te - [e in K_t] p_te * sum_{e' in F_t} s_te' dS_te'.
+    For the dropless plan F_t = K_t and s = p = g, giving g_e (dS_e - sum g dS).
+    """
+    E, k = plan["E"], plan["k"]
+    dl = np.zeros(E)
+    tot = 0.0
+    for r, ds, e in zip(rows, dS_rows, row_expert(plan, rows)):
+        v = plan["row_gate"][r] * ds
+        dl[e] += v
+        tot += v
+    for j in range(k):
+        dl[idx[t, j]] -= gate[t, j] * tot
+    return dl
+
+
+def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
+              logits_override=None, logit_bias=None, staged=True):
+    """Full forward: route, permute, expert FFN on every row, combine."""
+    logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias)
+    T, E = logits.shape
+    plan = exact_plan(idx, gate, E, tile) if round_mode == 0 else rounded_plan(idx, logits, E, tile)
+    rows = np.arange(plan["R"])
+    res = rows_compute(rows, plan, x, w1, w3, w2, None, staged)
+    out = np.zeros((T, np.shape(x)[1]))
+    for t in range(T):
+        for r in token_rows(plan, t):
+            out[t] += plan["row_gate"][r] * res["Y"][r]
+    return dict(logits=logits, idx=idx, gate=gate, plan=plan, H=res["H"],
+                A=res["A"], Y=res["Y"], out=out)
+
+
+def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True):
+    """Full backward from the saved set {x, logits, idx, gate, plan, H}.
+
+    dW2_e = sum_rows (g A)^T dO,  [dW1|dW3]_e = sum_rows x^T dH,
+    dx_t = sum over the rows of t of dX_perm + dlogits_t W_gate^T,
+    dW_gate = x^T dlogits.  Returns dx, dw_gate, dw1, dw3, dw2, dS [R], dlogits.
+    """
+    dout, x, w_gate, w1, w3, w2 = map(_f64, (dout, x, w_gate, w1, w3, w2))
+    plan = fwd["plan"]
+    T, d = x.shape
+    E, _, f = w1.shape
+    R = plan["R"]
+    rows = np.arange(R)
+    res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged)
+    dw1, dw3, dw2 = np.zeros_like(w1), np.zeros_like(w3), np.zeros_like(w2)
+    for e in range(E):
+        lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
+        toks = plan["row_token"][lo:hi]
+        live = toks >= 0
+        r = np.arange(lo, hi)[live]
+        dw2[e] = res["gA"][r].T @ dout[toks[live]]
+        dw1[e] = x[toks[live]].T @ res["dH"][r, :f]
+        dw3[e] = x[toks[live]].T @ res["dH"][r, f:]
+    dlogits = np.zeros((T, E))
+    dx = np.zeros((T, d))
+    for t in range(T):
+        tr = token_rows(plan, t)
+        dlogits[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][tr])
+        for r in tr:
+            dx[t] += res["dXp"][r]
+    dw_gate = np.zeros((d, E))
+    if router_grad_on:
+        dx += dlogits @ w_gate.T
+        dw_gate = x.T @ dlogits
+    return dict(dx=dx, dw_gate=dw_gate, dw1=dw1, dw3=dw3, dw2=dw2, dS=res["dS"],
+                dlogits=dlogits, dXp=res["dXp"], dH=res["dH"])
+
+
+def sampled_tokens(tokens, dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True):
+    """out, dx, dlogits and per-row dS for a subset of tokens only.  Each of
+    these depends on nothing but the token itself and its experts' weights,
+    so the values equal those of the full layer."""
+    plan = fwd["plan"]
+    dout, x, w_gate = map(_f64, (dout, x, w_gate))
+    out, dx, dl, dS = {}, {}, {}, {}
+    for t in tokens:
+        tr = token_rows(plan, t)
+        res = rows_compute(tr, plan, x, w1, w3, w2, dout, staged)
+        out[t] = (plan["row_gate"][tr][:, None] * res["Y"]).sum(axis=0)
+        dl[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"])
+        dx[t] = res["dXp"].sum(axis=0)
+        if router_grad_on:
+            dx[t] = dx[t] + dl[t] @ w_gate.T
+        for r, v in zip(tr, res["dS"]):
+            dS[r] = v
+    return dict(out=out, dx=dx, dlogits=dl, dS=dS)
+
+
+def sampled_expert_grads(experts, dout, x, w1, w3, w2, fwd, staged=True):
+    """dW1, dW3, dW2 of the listed experts (sums over that expert's rows)."""
+    plan = fwd["plan"]
+    dout, x = _f64(dout), _f64(x)
+    f = np.shape(w1)[2]
+    out = {}
+    for e in experts:
+        lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
+        toks = plan["row_token"][lo:hi]
+        live = toks >= 0
+        rows = np.arange(lo, hi)[live]
+        res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged)
+        tk = toks[live]
+        out[e] = dict(dw2=res["gA"].T @ dout[tk], dw1=x[tk].T @ res["dH"][:, :f],
+                      dw3=x[tk].T @ res["dH"][:, f:])
+    return out

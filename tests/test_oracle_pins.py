@@ -1,0 +1,379 @@
+"""Pins for the CPU oracle: each check compares the oracle with something other
+than itself (a library routine, brute force, a dense masked evaluation, a
+closed form, finite differences, or the pages' worked example), so that a
+dropped term, a wrong sign or index, or a transposed operand fails here."""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def _rand_layer(rng, T, d, f, E, scale=0.5):
+    x = rng.standard_normal((T, d))
+    wg = rng.standard_normal((d, E)) * scale
+    w1 = rng.standard_normal((E, d, f)) * scale
+    w3 = rng.standard_normal((E, d, f)) * scale
+    w2 = rng.standard_normal((E, f, d)) * scale
+    dout = rng.standard_normal((T, d))
+    return x, wg, w1, w3, w2, dout
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_bf16_round_matches_torch_conversion():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-30).astype(np.float32),
+        (rng.standard_normal(2000) * 1e30).astype(np.float32),
+        # exact halfway cases between bf16 neighbours (ties to even)
+        np.array([1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8)], np.float32),
+    ])
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.bf16_round(v.astype(np.float64)), ref)
+
+
+def test_silu_and_grad_closed_forms():
+    z = np.linspace(-8, 8, 101)
+    np.testing.assert_allclose(O.silu(z), z / (1 + np.exp(-z)), rtol=1e-14, atol=1e-15)
+    h = 1e-6
+    num = (O.silu(z + h) - O.silu(z - h)) / (2 * h)
+    np.testing.assert_allclose(O.silu_grad(z), num, rtol=1e-8, atol=1e-9)
+
+
+# ---------------------------------------------------------------- routing
+
+def test_route_matches_brute_force_sort_with_ties():
+    rng = np.random.default_rng(2)
+    T, E, k = 64, 8, 3
+    logits = rng.integers(0, 3, size=(T, E)).astype(np.float64)  # many exact ties
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    for t in range(T):
+        brute = sorted(range(E), key=lambda e: (-logits[t, e], e))[:k]
+        assert list(idx[t]) == brute
+        vals = [logits[t, e] for e in brute]
+        z = sum(math.exp(v) for v in vals)
+        assert np.allclose(gate[t], [math.exp(v) / z for v in vals], rtol=1e-14)
+    assert np.allclose(gate.sum(1), 1.0, rtol=1e-14)
+
+
+def test_route_matches_torch_topk_softmax_without_ties():
+    rng = np.random.default_rng(3)
+    x, wg = rng.standard_normal((40, 16)), rng.standard_normal((16, 6))
+    logits, idx, gate = O.route(x, wg, 2)
+    tl = torch.from_numpy(x) @ torch.from_numpy(wg)
+    v, i = torch.topk(tl, 2, dim=-1)
+    np.testing.assert_allclose(logits, tl.numpy(), rtol=1e-13)
+    np.testing.assert_array_equal(idx, i.numpy())
+    np.testing.assert_allclose(gate, torch.softmax(v, -1).numpy(), rtol=1e-13)
+
+
+def test_route_bias_shifts_logits():
+    rng = np.random.default_rng(4)
+    x, wg = rng.standard_normal((10, 8)), rng.standard_normal((8, 4))
+    b = np.array([0.0, -1.0, 2.0, 0.5])
+    logits, _, _ = O.route(x, wg, 2, logit_bias=b)
+    np.testing.assert_allclose(logits, x @ wg + b, rtol=1e-13)
+
+
+# ---------------------------------------------------------------- permutation
+
+def test_exact_plan_matches_brute_force_dispatch():
+    rng = np.random.default_rng(5)
+    T, E, k, tile = 37, 5, 2, 4
+    logits = rng.standard_normal((T, E))
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    plan = O.exact_plan(idx, gate, E, tile)
+    # brute force: per-expert lists in token order (the structure of a
+    # dispatch into per-expert input lists), then tile-aligned placement
+    lists = {e: [] for e in range(E)}
+    for t in range(T):
+        for j in range(k):
+            lists[int(idx[t, j])].append((t, j))
+    off = 0
+    for e in range(E):
+        assert plan["offsets"][e] == off
+        assert plan["counts"][e] == len(lists[e])
+        for i, (t, j) in enumerate(lists[e]):
+            r = off + i
+            assert plan["row_token"][r] == t
+            assert plan["row_slot"][r] == t * k + j
+            assert plan["slot_row"][t * k + j] == r
+            assert plan["row_gate"][r] == gate[t, j]
+        for r in range(off + len(lists[e]), off + -(-len(lists[e]) // tile) * tile):
+            assert plan["row_token"][r] == -1 and plan["row_gate"][r] == 0
+        off += -(-len(lists[e]) // tile) * tile
+    assert plan["R"] == off
+
+
+def test_exact_plan_invariants():
+    rng = np.random.default_rng(6)
+    T, E, k = 1000, 16, 4
+    _, idx, gate = O.route(None, None, k, logits_override=rng.standard_normal((T, E)))
+    plan = O.exact_plan(idx, gate, E)
+    assert plan["counts"].sum() == T * k
+    assert np.all(plan["offsets"] % O.TILE == 0)
+    # slot_row is a bijection between the T*k slots and the live rows
+    live = np.nonzero(plan["row_token"] >= 0)[0]
+    assert len(live) == T * k
+    assert sorted(plan["slot_row"]) == sorted(live)
+    np.testing.assert_array_equal(plan["row_slot"][plan["slot_row"]], np.arange(T * k))
+    for e in range(E):
+        seg = plan["row_token"][plan["offsets"][e]:plan["offsets"][e] + plan["counts"][e]]
+        assert np.all(np.diff(seg) > 0)
+
+
+# ---------------------------------------------------------------- token rounding
+
+def test_token_rounding_page_example():
+    for cnt, tile, want in _golden("token_rounding_example.txt"):
+        assert O.rounded_target([int(cnt)], T=10 ** 6, tile=int(tile))[0] == int(want)
+
+
+def test_token_rounding_targets():
+    c = np.array([0, 1, 63, 64, 65, 127, 128, 191, 192, 193, 300])
+    r = O.rounded_target(c, T=10 ** 6, tile=128)
+    np.testing.assert_array_equal(r, [0, 0, 0, 128, 128, 128, 128, 128, 256, 256, 256])
+    assert np.all(np.abs(r - c) <= 64)
+    # capped at the largest tile multiple not above T
+    assert O.rounded_target([250], T=250, tile=128)[0] == 128
+
+
+def test_rounded_plan_brute_force_subsets():
+    """On tiny inputs the kept set of each shrunk expert is the size-r_e
+    subset of its tokens with the largest total score, and the added set of
+    each grown expert the size-(r_e - c_e) subset of the others with the
+    largest total score; checked by enumerating every subset."""
+    rng = np.random.default_rng(7)
+    T, E, k, tile = 11, 3, 2, 4
+    for trial in range(20):
+        logits = rng.standard_normal((T, E))
+        _, idx, gate = O.route(None, None, k, logits_override=logits)
+        plan = O.rounded_plan(idx, logits, E, tile)
+        counts = np.bincount(idx.ravel(), minlength=E)
+        top = np.take_along_axis(logits, idx, 1)
+        score = np.exp(logits) / np.exp(top).sum(1, keepdims=True)
+        for e in range(E):
+            assigned = [t for t in range(T) if e in idx[t]]
+            others = [t for t in range(T) if e not in idx[t]]
+            r = plan["target"][e]
+            assert r % tile == 0 and abs(r - counts[e]) <= tile // 2
+            members = set(int(t) for t in plan["row_token"][plan["offsets"][e]:plan["offsets"][e + 1]])
+            assert len(members) == r
+            if r <= counts[e]:
+                best = max(itertools.combinations(assigned, r), key=lambda s: sum(score[t, e] for t in s))
+                assert members == set(best)
+            else:
+                best = max(itertools.combinations(others, r - counts[e]),
+                           key=lambda s: sum(score[t, e] for t in s))
+                assert members == set(assigned) | set(best)
+            seg = plan["row_gate"][plan["offsets"][e]:plan["offsets"][e + 1]]
+            toks = plan["row_token"][plan["offsets"][e]:plan["offsets"][e + 1]]
+            np.testing.assert_allclose(seg, score[toks, e], rtol=1e-13)
+            assert np.all(np.diff(toks) > 0)
+
+
+def test_rounded_plan_tie_rules():
+    # every token has the same logits, so all keys of one expert are equal;
+    # drops take the largest token ids, additions the smallest
+    T, E, k, tile = 10, 3, 1, 4
+    logits = np.tile(np.array([[1.0, 0.5, 0.0]]), (T, 1))
+    logits[:6, 1] = 2.0          # tokens 0..5 choose expert 1, 6..9 choose 0
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    plan = O.rounded_plan(idx, logits, E, tile)
+    seg = lambda e: list(plan["row_token"][plan["offsets"][e]:plan["offsets"][e + 1]])
+    assert seg(1) == [0, 1, 2, 3, 4, 5, 6, 7]   # 6 -> 8: adds the smallest ids
+    assert seg(0) == [6, 7, 8, 9]               # 4 stays 4
+    assert seg(2) == []                         # 0 stays 0
+    logits2 = logits.copy()
+    logits2[:, 2] = -1.0
+    logits2[:7, 1] = 2.0                        # 7 tokens on expert 1 -> round to 8
+    logits2[7:, 0] = 3.0                        # 3 on expert 0 -> round to 4
+    _, idx2, _ = O.route(None, None, k, logits_override=logits2)
+    p2 = O.rounded_plan(idx2, logits2, E, tile)
+    s0 = list(p2["row_token"][p2["offsets"][0]:p2["offsets"][1]])
+    assert s0 == [0, 7, 8, 9]
+
+
+# ---------------------------------------------------------------- forward
+
+def _dense_forward(x, wg, w1, w3, w2, k):
+    """Every expert on every token, masked to the top-k (no permutation)."""
+    logits = x @ wg
+    T, E = logits.shape
+    out = np.zeros_like(x)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-logits[t, e], e))[:k]
+        z = sum(math.exp(logits[t, e] - logits[t, order[0]]) for e in order)
+        for e in range(E):
+            mask = e in order
+            h1 = x[t] @ w1[e]
+            h3 = x[t] @ w3[e]
+            y = ((h1 / (1 + np.exp(-h1))) * h3) @ w2[e]
+            g = math.exp(logits[t, e] - logits[t, order[0]]) / z if mask else 0.0
+            out[t] += g * y
+    return out
+
+
+def test_forward_matches_dense_masked_evaluation():
+    rng = np.random.default_rng(8)
+    x, wg, w1, w3, w2, _ = _rand_layer(rng, 23, 6, 5, 4)
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4, staged=False)
+    np.testing.assert_allclose(fwd["out"], _dense_forward(x, wg, w1, w3, w2, 2), rtol=1e-12, atol=1e-12)
+
+
+def test_forward_matches_per_expert_masked_loop():
+    """The structure of the Beam article's MoELayer: loop over the k slots and
+    the experts with a boolean mask (here with SwiGLU experts)."""
+    rng = np.random.default_rng(9)
+    x, wg, w1, w3, w2, _ = _rand_layer(rng, 19, 4, 3, 5)
+    k = 3
+    scores = torch.from_numpy(x @ wg)
+    vals, ids = scores.topk(k, dim=-1)
+    vals = torch.softmax(vals, -1).numpy()
+    ids = ids.numpy()
+    out = np.zeros_like(x)
+    for j in range(k):
+        for e in range(5):
+            m = ids[:, j] == e
+            if m.any():
+                h1 = x[m] @ w1[e]
+                y = (h1 / (1 + np.exp(-h1)) * (x[m] @ w3[e])) @ w2[e]
+                out[m] += vals[m, j][:, None] * y
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=k, tile=4, staged=False)
+    np.testing.assert_allclose(fwd["out"], out, rtol=1e-12, atol=1e-12)
+
+
+def test_staged_forward_close_to_ideal():
+    rng = np.random.default_rng(10)
+    x, wg, w1, w3, w2, _ = _rand_layer(rng, 50, 32, 16, 4, scale=0.2)
+    a = O.layer_fwd(x, wg, w1, w3, w2, k=2, staged=False)["out"]
+    b = O.layer_fwd(x, wg, w1, w3, w2, k=2, staged=True)["out"]
+    err = np.abs(a - b).sum() / np.abs(a).sum()
+    assert 1e-5 < err < 2e-2
+
+
+# ---------------------------------------------------------------- backward
+
+def test_two_expert_hand_example():
+    want = {n: float(v) for n, v in _golden("two_expert_example.txt")}
+    x = np.array([[1.0]])
+    wg = np.array([[math.log(3.0), 0.0]])
+    w1 = np.array([[[0.0]], [[1.0]]])
+    w3 = np.array([[[1.0]], [[2.0]]])
+    w2 = np.array([[[1.0]], [[1.0]]])
+    dout = np.array([[1.0]])
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=1, staged=False)
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
+    assert abs(fwd["out"][0, 0] - want["out"]) < 1e-9
+    rows = fwd["plan"]["slot_row"]      # slot 0 -> expert 0, slot 1 -> expert 1
+    assert abs(bwd["dS"][rows[0]] - want["dS0"]) < 1e-9
+    assert abs(bwd["dS"][rows[1]] - want["dS1"]) < 1e-9
+    for n, arr in (("dw_gate", bwd["dw_gate"][0]), ("dw1_", bwd["dw1"][:, 0, 0]),
+                   ("dw3_", bwd["dw3"][:, 0, 0]), ("dw2_", bwd["dw2"][:, 0, 0])):
+        for e in range(2):
+            assert abs(arr[e] - want[f"{n}{e}"]) < 1e-9, (n, e)
+    assert abs(bwd["dx"][0, 0] - want["dx"]) < 1e-9
+
+
+def _loss(params, dout, k, tile, round_mode):
+    x, wg, w1, w3, w2 = params
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=k, tile=tile, round_mode=round_mode, staged=False)
+    return float(np.sum(fwd["out"] * dout)), fwd
+
+
+@pytest.mark.parametrize("round_mode", [0, 1])
+def test_backward_matches_central_differences(round_mode):
+    rng = np.random.default_rng(11 + round_mode)
+    T, d, f, E, k, tile = 9, 4, 3, 4, 2, 4
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, T, d, f, E)
+    params = [x, wg, w1, w3, w2]
+    _, fwd = _loss(params, dout, k, tile, round_mode)
+    if round_mode:
+        assert fwd["plan"]["dropped"].any() or fwd["plan"]["added"].any()
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
+    grads = [bwd["dx"], bwd["dw_gate"], bwd["dw1"], bwd["dw3"], bwd["dw2"]]
+    h = 1e-6
+    for p, g in zip(params, grads):
+        num = np.zeros_like(p)
+        for i in np.ndindex(p.shape):
+            old = p[i]
+            p[i] = old + h
+            lp, fp = _loss(params, dout, k, tile, round_mode)
+            p[i] = old - h
+            lm, fm = _loss(params, dout, k, tile, round_mode)
+            p[i] = old
+            # the discrete routing must not change under the probe
+            assert np.array_equal(fp["idx"], fwd["idx"]) and np.array_equal(fm["idx"], fwd["idx"])
+            num[i] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-7)
+
+
+def test_dS_identity_inner_products():
+    """<dA', A> computed by the oracle equals <dO, Y> (the quantity it replaces)."""
+    rng = np.random.default_rng(12)
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, 30, 8, 6, 4)
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4, staged=False)
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
+    rows = np.nonzero(fwd["plan"]["row_token"] >= 0)[0]
+    toks = fwd["plan"]["row_token"][rows]
+    np.testing.assert_allclose(bwd["dS"][rows], np.sum(dout[toks] * fwd["Y"][rows], 1), rtol=1e-11)
+
+
+def test_router_grad_rows_sum_to_zero_in_exact_mode():
+    """Softmax over the top-k is shift invariant, so each token's dlogits sums
+    to zero over its k experts and vanishes elsewhere."""
+    rng = np.random.default_rng(13)
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, 25, 6, 4, 5)
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4, staged=False)
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
+    np.testing.assert_allclose(bwd["dlogits"].sum(1), 0, atol=1e-12)
+    mask = np.ones_like(bwd["dlogits"], bool)
+    mask[np.arange(25)[:, None], fwd["idx"]] = False
+    assert np.all(bwd["dlogits"][mask] == 0)
+
+
+def test_sampled_views_equal_full_layer():
+    rng = np.random.default_rng(14)
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, 40, 8, 6, 4, scale=0.3)
+    for rm in (0, 1):
+        fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4, round_mode=rm)
+        bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd)
+        s = O.sampled_tokens([0, 7, 39], dout, x, wg, w1, w3, w2, fwd)
+        for t in (0, 7, 39):
+            np.testing.assert_allclose(s["out"][t], fwd["out"][t], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(s["dx"][t], bwd["dx"][t], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(s["dlogits"][t], bwd["dlogits"][t], rtol=1e-12, atol=1e-14)
+        ge = O.sampled_expert_grads([1, 3], dout, x, w1, w3, w2, fwd)
+        for e in (1, 3):
+            for n in ("dw1", "dw3", "dw2"):
+                np.testing.assert_allclose(ge[e][n], bwd[n][e], rtol=1e-12, atol=1e-14)
+
+
+def test_rounded_plan_drop_tie_takes_largest_token():
+    # 5 tokens on expert 0 with equal keys, tile 4 -> 4 rows: token 4 is dropped
+    T, E, k, tile = 8, 2, 1, 4
+    logits = np.zeros((T, E))
+    logits[:5, 0] = 1.0
+    logits[5:, 1] = 1.0
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    plan = O.rounded_plan(idx, logits, E, tile)
+    assert list(plan["row_token"][0:4]) == [0, 1, 2, 3]
+    assert plan["slot_row"][4] == -1 and plan["dropped"][4, 0]
