@@ -1,0 +1,189 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) token-choice mixture-of-experts layer.
+ *
+ * One layer, forward and backward, on one GPU:
+ *   route      logits = x W_gate (+bias); top-k per token; softmax over the k
+ *   permute    histogram of expert choices, prefix sum, stable scatter into
+ *              expert-contiguous rows (optionally token-rounded)
+ *   ffn_fwd    grouped GEMM [x W1 | x W3] with fused SwiGLU, grouped GEMM A W2
+ *   combine    O_t = sum over the rows of token t of weight * Y(row)
+ *   layer_bwd  dS = <dA', A>, SwiGLU backward, dX / dW grouped GEMMs, router
+ *              gradient
+ *
+ * Sources, cited by page title and section:
+ *   [Beam]     "From 501B to 23B: what is Beam doing", sec. 2.2 (MoE layer:
+ *              router W_gate [d_model, N], top-k, weighted sum of experts),
+ *              sec. 5.3 (MoELayer: topk, softmax of the k values, per-expert
+ *              loop that grouped GEMM replaces), sec. 5.4 (expert counts).
+ *   [Trinity]  "Trinity Large: open 400B sparse MoE" commentary, examples 1-3
+ *              (top-k + softmax gating, bincount, dispatch / combine).
+ *   [SonicMoE] techwalker summary of SonicMoE, sec. 1 (dS = <dA', A>, Y not
+ *              stored) and sec. 3 (token rounding to multiples of the tile).
+ *   [Olmo]     Olmo-core 3 news piece (rows placed straight into expert input
+ *              buffers; GPU-resident routing; grouped GEMM).
+ *
+ * Conventions for every call:
+ *   - Tensor arguments are DEVICE pointers on the current CUDA device,
+ *     allocated and owned by the caller, row-major and contiguous.  The
+ *     library allocates no device memory; scratch comes from a caller
+ *     workspace whose size the matching *_workspace_size() call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue kernels on it; none synchronises or copies routing metadata to
+ *     the host, so the row count R lives on the device only (offsets[E]).
+ *   - dtype MOE_BF16: bf16 activations/weights, fp32 accumulation,
+ *     tcgen05 tensor cores.  MOE_F32: fp32 everywhere, CUDA-core path.
+ *   - Return value: MOE_OK or a negative MOE_ERR_* code; moe_last_error()
+ *     gives a message.  Arguments are checked on the host before any launch;
+ *     a failed check launches nothing.  Device-side waits are bounded: if one
+ *     expires the kernel records MOE_ERR_DEVICE_TIMEOUT in a device flag,
+ *     returns, and moe_check_status() reports it.
+ *   - Shapes: 1 <= k <= 8, k <= E <= 256, T >= 0.  The bf16 path needs
+ *     d % 128 == 0 and f % 128 == 0; the f32 path d % 64 == 0 and f % 64 == 0.
+ *   - Row space: expert e owns rows [offsets[e], offsets[e+1]); each segment
+ *     starts at a multiple of `tile` (128) and padding rows are empty (token
+ *     -1, weight 0).  Row buffers hold cap = moe_row_capacity(T,E,k,tile)
+ *     rows; only rows < offsets[E] are touched.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)
+#define MOE_ERR_UNSUPPORTED (-2)
+#define MOE_ERR_CUDA (-3)
+#define MOE_ERR_DEVICE_TIMEOUT (-4)
+#define MOE_ERR_WORKSPACE (-5)
+
+#define MOE_F32 0
+#define MOE_BF16 1
+
+#define MOE_ROUND_NONE 0
+#define MOE_ROUND_NEAREST 1
+
+/* Library version (major*10000 + minor*100 + patch). */
+int moe_version(void);
+
+/* Message describing the last error returned on the calling host thread. */
+const char* moe_last_error(void);
+
+/* Number of rows a plan may occupy: T*k + E*tile. */
+size_t moe_row_capacity(int T, int E, int k, int tile);
+
+/*
+ * moe_route -- router logits, top-k and softmax over the top-k.
+ * [Beam] sec. 2.2 and 5.3; [Trinity] example 1.
+ *   x [T,d] (dtype), w_gate [d,E] (dtype).
+ *   logits_override [T,E] fp32 or NULL: when given, x and w_gate are not read
+ *     and these values replace x W_gate (random-routing workloads).
+ *   logit_bias [E] fp32 or NULL: added to every token's logits.
+ *   logits [T,E] fp32 out; idx [T,k] int32 out: the k largest logits in
+ *   descending order, ties to the lowest expert id; gate [T,k] fp32 out:
+ *   softmax of those k logits.
+ */
+int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
+              const float* logits_override, const float* logit_bias,
+              float* logits, int32_t* idx, float* gate, void* stream);
+
+/*
+ * moe_permute -- expert histogram, prefix sum and stable permutation into
+ * expert-contiguous rows.  [Trinity] examples 2-3; [Olmo] (expert input
+ * buffers, GPU-resident routing); [Beam] sec. 5.4 (counts).
+ * round_mode MOE_ROUND_NEAREST applies token rounding ([SonicMoE] sec. 3):
+ * each expert's count becomes the nearest multiple of `tile` (halves up,
+ * capped at tile*floor(T/tile)); drops remove the pairs with the smallest
+ * score exp(l - LSE_topk), larger token first on ties; additions take the
+ * unassigned tokens with the largest score, smaller token first on ties;
+ * row weights are those scores (kept pairs: their gate).
+ *   idx [T,k], gate [T,k]: from moe_route.  logits [T,E]: read only when
+ *     rounding.
+ *   tile: must be 128 (the grouped-GEMM M tile, also the rounding unit).
+ *   counts [E] out: token count per expert before rounding.
+ *   offsets [E+1] out: segment starts (multiples of tile); offsets[E] = R.
+ *   row_token [cap], row_gate [cap] fp32, row_slot [cap] out: token, weight
+ *     and slot (t*k+j, or -1 for a row added by rounding) of each row;
+ *     padding rows get -1, 0, -1.
+ *   slot_row [T*k] out: row of slot (t,j), or -1 if rounding dropped it.
+ *   extra_row [T,E] out (required when rounding, else may be NULL): row of
+ *     the pair (t,e) added by rounding, or -1.
+ *   ws: workspace of at least moe_permute_workspace_size() bytes.
+ */
+size_t moe_permute_workspace_size(int T, int E, int k, int round_mode);
+int moe_permute(const int32_t* idx, const float* gate, const float* logits,
+                int T, int E, int k, int round_mode, int tile,
+                int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
+                int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
+                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_ffn_fwd -- per-expert SwiGLU FFN on the permuted rows.
+ * [Beam] sec. 2.2/5.3 (expert FFN, grouped instead of looped); [Olmo]
+ * (grouped GEMM).  Experts are SwiGLU:
+ *   H = [x W1_e | x W3_e]  (saved for backward, dtype)
+ *   A = silu(H1) * H3      (transient)
+ *   Y_perm = A W2_e        (transient, dtype)
+ *   x [T,d]; w1, w3 [E,d,f]; w2 [E,f,d]; row_token [cap], offsets [E+1] from
+ *   moe_permute with tile 128.  H [cap,2f] out; Y_perm [cap,d] out.
+ */
+size_t moe_ffn_fwd_workspace_size(int T, int d, int f, int E, int k, int dtype);
+int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void* w2,
+                       const int32_t* row_token, const int32_t* offsets,
+                       int T, int d, int f, int E, int k, int dtype,
+                       void* H, void* Y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine -- routing-weighted unpermute: O_t = sum over token t's rows of
+ * row_gate[row] * Y_perm[row], summed in fp32 in a fixed order (kept slots in
+ * slot order, then rows added by rounding in ascending expert id).
+ * [Beam] sec. 2.2 (weighted sum); [Trinity] example 3 (add back per token).
+ *   Y_perm [cap,d]; row_gate [cap]; slot_row [T*k]; extra_row [T,E] or NULL.
+ *   out [T,d] (dtype).
+ */
+int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_row,
+                const int32_t* extra_row, int T, int d, int E, int k, int dtype,
+                void* out, void* stream);
+
+/*
+ * moe_layer_bwd -- backward of the whole layer from the saved set
+ * {x, idx, gate, plan, H}.  Y is never stored: the router-score gradient is
+ * dS = <dA', A> with dA' = dO W2^T and A recomputed from H ([SonicMoE] sec. 1).
+ *   dA = s dA'; SwiGLU backward gives dH = [dA*H3*silu'(H1) | dA*silu(H1)];
+ *   dW2_e = sum (s A)^T dO;  [dW1|dW3]_e = sum x^T dH;
+ *   dX_perm = dH [W1|W3]^T;  dx_t = sum over t's rows of dX_perm + dlogits_t W_gate^T;
+ *   dlogits_te = [e in F_t] s_te dS_te - [e in K_t] g_te sum_{F_t} s dS
+ *   (F_t: token t's final rows with weights s; K_t: its top-k);
+ *   dW_gate = x^T dlogits.
+ *   router_grad = 0 when the logits did not come from x W_gate (override):
+ *   dW_gate is then zero and dx gets no router term.
+ *   Outputs: dx [T,d] (dtype), dw_gate [d,E] fp32, dw1, dw3 [E,d,f] (dtype),
+ *   dw2 [E,f,d] (dtype), dS [cap] fp32 (may be NULL), dlogits [T,E] fp32
+ *   (may be NULL).  Every output element is written (no accumulation).
+ */
+size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype);
+int moe_layer_bwd(const void* dout, const void* x, const void* w_gate,
+                  const void* w1, const void* w3, const void* w2,
+                  const int32_t* idx, const float* gate, const int32_t* offsets,
+                  const int32_t* row_token, const float* row_gate,
+                  const int32_t* slot_row, const int32_t* extra_row, const void* H,
+                  int T, int d, int f, int E, int k, int dtype, int router_grad,
+                  void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2,
+                  float* dS, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_check_status -- synchronises `stream`, then returns MOE_OK, a CUDA
+ * error (MOE_ERR_CUDA) or MOE_ERR_DEVICE_TIMEOUT if a bounded device wait
+ * expired since the last check (the flag is cleared by this call).
+ */
+int moe_check_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

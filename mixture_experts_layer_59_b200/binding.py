@@ -1,0 +1,216 @@
+"""Python binding of ``libmoe_b200.so`` (ctypes; argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does
+nothing but turn torch tensors into device pointers, allocate outputs the
+caller did not pass, and raise ``MoEError`` on a non-zero return code.  All
+arithmetic happens in the library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ROUND_NONE, MOE_ROUND_NEAREST = 0, 1
+TILE = 128
+
+EXPORTS = [
+    "moe_version", "moe_last_error", "moe_row_capacity", "moe_route",
+    "moe_permute_workspace_size", "moe_permute", "moe_ffn_fwd_workspace_size",
+    "moe_expert_ffn_fwd", "moe_combine", "moe_layer_bwd_workspace_size", "moe_layer_bwd",
+    "moe_check_status",
+]
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"moe error {code}: {msg}")
+        self.code = code
+
+
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+_SIGS = {
+    "moe_version": (_i, []),
+    "moe_last_error": (ctypes.c_char_p, []),
+    "moe_row_capacity": (_sz, [_i, _i, _i, _i]),
+    "moe_route": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_permute_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                         _vp, _sz, _vp]),
+    "moe_ffn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "moe_expert_ffn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp,
+                                _vp, _sz, _vp]),
+    "moe_combine": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "moe_layer_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "moe_layer_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
+    "moe_check_status": (_i, [_vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_59_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(l, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc):
+    if rc != 0:
+        raise MoEError(rc, lib().moe_last_error().decode())
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return MOE_BF16
+    if dt == torch.float32:
+        return MOE_F32
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def moe_version() -> int:
+    return lib().moe_version()
+
+
+def moe_row_capacity(T, E, k, tile=TILE) -> int:
+    return lib().moe_row_capacity(T, E, k, tile)
+
+
+def moe_route(x, w_gate, k, logits_override=None, logit_bias=None, logits=None, idx=None,
+              gate=None, T=None, E=None, stream=None):
+    """logits [T,E] f32, idx [T,k] i32, gate [T,k] f32 (outputs allocated if None)."""
+    if T is None:
+        T = (logits_override if logits_override is not None else x).shape[0]
+    if E is None:
+        E = (logits_override if logits_override is not None else w_gate).shape[1]
+    dev = (logits_override if logits_override is not None else x).device
+    d = x.shape[1] if x is not None else 0
+    dt = dtype_code(x.dtype) if x is not None else MOE_F32
+    logits = logits if logits is not None else torch.empty(T, E, device=dev, dtype=torch.float32)
+    idx = idx if idx is not None else torch.empty(T, k, device=dev, dtype=torch.int32)
+    gate = gate if gate is not None else torch.empty(T, k, device=dev, dtype=torch.float32)
+    _check(lib().moe_route(_p(x), _p(w_gate), T, d, E, k, dt, _p(logits_override), _p(logit_bias),
+                           _p(logits), _p(idx), _p(gate), _stream(stream)))
+    return logits, idx, gate
+
+
+def moe_permute_workspace_size(T, E, k, round_mode) -> int:
+    return lib().moe_permute_workspace_size(T, E, k, round_mode)
+
+
+def moe_permute(idx, gate, logits, E, round_mode=MOE_ROUND_NONE, tile=TILE, out=None, ws=None,
+                stream=None):
+    """Returns dict counts, offsets, row_token, row_gate, row_slot, slot_row, extra_row."""
+    T, k = idx.shape
+    dev = idx.device
+    cap = moe_row_capacity(T, E, k, tile)
+    o = dict(out) if out else {}
+    o.setdefault("counts", torch.empty(E, device=dev, dtype=torch.int32))
+    o.setdefault("offsets", torch.empty(E + 1, device=dev, dtype=torch.int32))
+    o.setdefault("row_token", torch.empty(cap, device=dev, dtype=torch.int32))
+    o.setdefault("row_gate", torch.empty(cap, device=dev, dtype=torch.float32))
+    o.setdefault("row_slot", torch.empty(cap, device=dev, dtype=torch.int32))
+    o.setdefault("slot_row", torch.empty(T * k, device=dev, dtype=torch.int32))
+    if round_mode:
+        o.setdefault("extra_row", torch.empty(T, E, device=dev, dtype=torch.int32))
+    else:
+        o.setdefault("extra_row", None)
+    wsb = moe_permute_workspace_size(T, E, k, round_mode)
+    if ws is None:
+        ws = torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8)
+    _check(lib().moe_permute(_p(idx), _p(gate), _p(logits), T, E, k, round_mode, tile,
+                             _p(o["counts"]), _p(o["offsets"]), _p(o["row_token"]),
+                             _p(o["row_gate"]), _p(o["row_slot"]), _p(o["slot_row"]),
+                             _p(o["extra_row"]), _p(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype) -> int:
+    return lib().moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype)
+
+
+def moe_expert_ffn_fwd(x, w1, w3, w2, row_token, offsets, k, H=None, Y_perm=None, ws=None,
+                       stream=None):
+    T, d = x.shape
+    E, _, f = w1.shape
+    dt = dtype_code(x.dtype)
+    cap = moe_row_capacity(T, E, k)
+    H = H if H is not None else torch.empty(cap, 2 * f, device=x.device, dtype=x.dtype)
+    Y_perm = Y_perm if Y_perm is not None else torch.empty(cap, d, device=x.device, dtype=x.dtype)
+    if ws is None:
+        ws = torch.empty(max(moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), device=x.device,
+                         dtype=torch.uint8)
+    _check(lib().moe_expert_ffn_fwd(_p(x), _p(w1), _p(w3), _p(w2), _p(row_token), _p(offsets), T,
+                                    d, f, E, k, dt, _p(H), _p(Y_perm), _p(ws), ws.numel(),
+                                    _stream(stream)))
+    return H, Y_perm
+
+
+def moe_combine(Y_perm, row_gate, slot_row, extra_row, T, E, k, out=None, stream=None):
+    d = Y_perm.shape[1]
+    out = out if out is not None else torch.empty(T, d, device=Y_perm.device, dtype=Y_perm.dtype)
+    _check(lib().moe_combine(_p(Y_perm), _p(row_gate), _p(slot_row), _p(extra_row), T, d, E, k,
+                             dtype_code(Y_perm.dtype), _p(out), _stream(stream)))
+    return out
+
+
+def moe_layer_bwd_workspace_size(T, d, f, E, k, dtype) -> int:
+    return lib().moe_layer_bwd_workspace_size(T, d, f, E, k, dtype)
+
+
+def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=True, out=None,
+                  ws=None, stream=None):
+    """plan: dict from moe_permute.  Returns dict dx, dw_gate, dw1, dw3, dw2, dS, dlogits."""
+    T, d = x.shape
+    E, _, f = w1.shape
+    k = idx.shape[1]
+    dt = dtype_code(x.dtype)
+    cap = moe_row_capacity(T, E, k)
+    dev = x.device
+    o = dict(out) if out else {}
+    o.setdefault("dx", torch.empty(T, d, device=dev, dtype=x.dtype))
+    o.setdefault("dw_gate", torch.empty(d, E, device=dev, dtype=torch.float32))
+    o.setdefault("dw1", torch.empty_like(w1))
+    o.setdefault("dw3", torch.empty_like(w3))
+    o.setdefault("dw2", torch.empty_like(w2))
+    o.setdefault("dS", torch.empty(cap, device=dev, dtype=torch.float32))
+    o.setdefault("dlogits", torch.empty(T, E, device=dev, dtype=torch.float32))
+    if ws is None:
+        ws = torch.empty(max(moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), device=dev,
+                         dtype=torch.uint8)
+    _check(lib().moe_layer_bwd(
+        _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(idx), _p(gate),
+        _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
+        _p(plan["extra_row"]), _p(H), T, d, f, E, k, dt, 1 if router_grad else 0,
+        _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
+        _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_check_status(stream=None):
+    _check(lib().moe_check_status(_stream(stream)))

@@ -1,0 +1,311 @@
+// extern "C" entry points: argument checks, workspace layout, kernel order.
+#include <cstdio>
+#include <string>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+static thread_local std::string g_err = "";
+
+void set_error(const std::string& msg) { g_err = msg; }
+int fail(int code, const std::string& msg) {
+  g_err = msg;
+  return code;
+}
+int cuda_fail(cudaError_t e, const char* what) {
+  g_err = std::string(what) + ": " + cudaGetErrorString(e);
+  return MOE_ERR_CUDA;
+}
+
+__device__ int g_moe_status = 0;
+
+int* status_ptr() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_status) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+int device_sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 1;
+  }
+  return cache[dev];
+}
+
+// ------------------------------------------------------------ checks
+static int check_common(int T, int E, int k, int dtype) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (k < 1 || k > 8) return fail(MOE_ERR_UNSUPPORTED, "k must be in [1, 8]");
+  if (E < k || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [k, 256]");
+  if (dtype != MOE_F32 && dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "dtype must be MOE_F32 or MOE_BF16");
+  return MOE_OK;
+}
+
+static int check_dims(int d, int f, int dtype) {
+  const int q = dtype == MOE_BF16 ? 128 : 64;
+  if (d <= 0 || d % q) return fail(MOE_ERR_UNSUPPORTED, "d must be a positive multiple of " + std::to_string(q));
+  if (f < 0 || f % q || f == 0) return fail(MOE_ERR_UNSUPPORTED, "f must be a positive multiple of " + std::to_string(q));
+  return MOE_OK;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE_PTR(p)                                                              \
+  do {                                                                              \
+    if ((p) == nullptr) return fail(MOE_ERR_INVALID_ARG, #p " must not be NULL");   \
+  } while (0)
+#define REQUIRE_ALIGNED(p)                                                                 \
+  do {                                                                                     \
+    if (!aligned16(p)) return fail(MOE_ERR_INVALID_ARG, #p " must be 16-byte aligned");     \
+  } while (0)
+
+static size_t esize(int dtype) { return dtype == MOE_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------ workspace layouts
+template <class A>
+struct FwdWs {
+  void* xg = nullptr;
+  void* act = nullptr;
+  void carve(A& a, int T, int d, int f, int E, int k, int dtype) {
+    const size_t cap = (size_t)T * k + (size_t)E * 128;
+    if (dtype == MOE_BF16 && tc_available()) xg = a.template take<uint16_t>(cap * d);
+    act = a.template take<char>(cap * f * esize(dtype));
+  }
+};
+
+template <class A>
+struct BwdWs {
+  void *dog = nullptr, *xg = nullptr, *dH = nullptr, *gact = nullptr, *dxp = nullptr;
+  float *dap = nullptr, *ds = nullptr, *dl = nullptr, *dx_acc = nullptr;
+  int nparts = 1;
+  void carve(A& a, int T, int d, int f, int E, int k, int dtype) {
+    const size_t cap = (size_t)T * k + (size_t)E * 128;
+    const size_t es = esize(dtype);
+    const bool tc = dtype == MOE_BF16 && tc_available();
+    nparts = tc ? tc_num_dS_parts(f) : 1;
+    if (tc) {
+      dog = a.template take<char>(cap * d * es);
+      xg = a.template take<char>(cap * d * es);
+    } else {
+      dap = a.template take<float>(cap * f);
+    }
+    dH = a.template take<char>(cap * 2 * f * es);
+    gact = a.template take<char>(cap * f * es);
+    dxp = a.template take<char>(cap * d * es);
+    ds = a.template take<float>(cap * nparts);
+    dl = a.template take<float>((size_t)T * E + 1);
+    dx_acc = a.template take<float>((size_t)T * d + 1);
+  }
+};
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int moe_version(void) { return 10000; }
+
+const char* moe_last_error(void) { return g_err.c_str(); }
+
+size_t moe_row_capacity(int T, int E, int k, int tile) {
+  if (T < 0 || E < 0 || k < 0 || tile < 0) return 0;
+  return (size_t)T * k + (size_t)E * tile;
+}
+
+int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
+              const float* logits_override, const float* logit_bias, float* logits,
+              int32_t* idx, float* gate, void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (T == 0) return MOE_OK;
+  REQUIRE_PTR(logits);
+  REQUIRE_PTR(idx);
+  REQUIRE_PTR(gate);
+  cudaStream_t s = (cudaStream_t)stream;
+  const float* src = logits_override;
+  if (src == nullptr) {
+    REQUIRE_PTR(x);
+    REQUIRE_PTR(w_gate);
+    if (d <= 0) return fail(MOE_ERR_INVALID_ARG, "d must be > 0");
+    if (int rc = launch_router_logits_simt(x, w_gate, T, d, E, dtype, nullptr, logits, s)) return rc;
+    src = logits;
+  }
+  return launch_topk_softmax(src, logit_bias, logits, T, E, k, idx, gate, s);
+}
+
+size_t moe_permute_workspace_size(int T, int E, int k, int round_mode) {
+  if (T < 0 || E <= 0 || k <= 0) return 0;
+  return permute_ws_bytes(T, E, k, round_mode, 128);
+}
+
+int moe_permute(const int32_t* idx, const float* gate, const float* logits, int T, int E, int k,
+                int round_mode, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
+                float* row_gate, int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
+                void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_common(T, E, k, MOE_F32)) return rc;
+  if (tile != 128)
+    return fail(MOE_ERR_UNSUPPORTED, "tile must be 128 (the grouped-GEMM M tile)");
+  if (round_mode != MOE_ROUND_NONE && round_mode != MOE_ROUND_NEAREST)
+    return fail(MOE_ERR_INVALID_ARG, "round_mode must be MOE_ROUND_NONE or MOE_ROUND_NEAREST");
+  REQUIRE_PTR(counts);
+  REQUIRE_PTR(offsets);
+  if (T > 0) {
+    REQUIRE_PTR(idx);
+    REQUIRE_PTR(gate);
+    REQUIRE_PTR(row_token);
+    REQUIRE_PTR(row_gate);
+    REQUIRE_PTR(row_slot);
+    REQUIRE_PTR(slot_row);
+  }
+  if (round_mode) {
+    REQUIRE_PTR(logits);
+    REQUIRE_PTR(extra_row);
+  }
+  if (ws_bytes < permute_ws_bytes(T, E, k, round_mode, tile))
+    return fail(MOE_ERR_WORKSPACE, "permute workspace smaller than moe_permute_workspace_size()");
+  PermuteWs w;
+  if (int rc = carve_permute_ws(ws, ws_bytes, T, E, k, round_mode, tile, &w)) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (round_mode == MOE_ROUND_NONE)
+    return launch_permute_exact(idx, gate, T, E, k, tile, counts, offsets, row_token, row_gate,
+                                row_slot, slot_row, w, s);
+  return launch_permute_round(idx, gate, logits, T, E, k, tile, counts, offsets, row_token,
+                              row_gate, row_slot, slot_row, extra_row, w, s);
+}
+
+size_t moe_ffn_fwd_workspace_size(int T, int d, int f, int E, int k, int dtype) {
+  if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0) return 0;
+  Sizer z;
+  FwdWs<Sizer> w;
+  w.carve(z, T, d, f, E, k, dtype);
+  return z.used;
+}
+
+int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void* w2,
+                       const int32_t* row_token, const int32_t* offsets, int T, int d, int f, int E,
+                       int k, int dtype, void* H, void* Y_perm, void* ws, size_t ws_bytes,
+                       void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (int rc = check_dims(d, f, dtype)) return rc;
+  REQUIRE_PTR(x); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
+  REQUIRE_PTR(row_token); REQUIRE_PTR(offsets); REQUIRE_PTR(H); REQUIRE_PTR(Y_perm);
+  REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2);
+  REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(Y_perm); REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype))
+    return fail(MOE_ERR_WORKSPACE, "ffn workspace smaller than moe_ffn_fwd_workspace_size()");
+  Carve c(ws, ws_bytes);
+  FwdWs<Carve> w;
+  w.carve(c, T, d, f, E, k, dtype);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "ffn workspace too small");
+  cudaStream_t s = (cudaStream_t)stream;
+  FfnPtrs p{x, w1, w3, w2, row_token, offsets, T, d, f, E, (int)((size_t)T * k + (size_t)E * 128), dtype};
+  if (dtype == MOE_BF16 && tc_available()) {
+    if (int rc = launch_gather_rows(x, row_token, offsets, E, d, dtype, w.xg, s)) return rc;
+    return tc_ffn_fwd(p, w.xg, H, w.act, Y_perm, device_sm_count(), s);
+  }
+  return simt_ffn_fwd(p, H, w.act, Y_perm, s);
+}
+
+int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_row,
+                const int32_t* extra_row, int T, int d, int E, int k, int dtype, void* out,
+                void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (d <= 0 || d % 8) return fail(MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 8");
+  if (T == 0) return MOE_OK;
+  REQUIRE_PTR(Y_perm); REQUIRE_PTR(row_gate); REQUIRE_PTR(slot_row); REQUIRE_PTR(out);
+  REQUIRE_ALIGNED(Y_perm); REQUIRE_ALIGNED(out);
+  return launch_token_reduce(Y_perm, row_gate, slot_row, extra_row, T, d, E, k, dtype, true,
+                             false, out, (cudaStream_t)stream);
+}
+
+size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype) {
+  if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0) return 0;
+  Sizer z;
+  BwdWs<Sizer> w;
+  w.carve(z, T, d, f, E, k, dtype);
+  return z.used;
+}
+
+int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
+                  const void* w3, const void* w2, const int32_t* idx, const float* gate,
+                  const int32_t* offsets, const int32_t* row_token, const float* row_gate,
+                  const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
+                  int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
+                  void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
+                  size_t ws_bytes, void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (int rc = check_dims(d, f, dtype)) return rc;
+  REQUIRE_PTR(dout); REQUIRE_PTR(x); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
+  REQUIRE_PTR(idx); REQUIRE_PTR(gate); REQUIRE_PTR(offsets); REQUIRE_PTR(row_token);
+  REQUIRE_PTR(row_gate); REQUIRE_PTR(slot_row); REQUIRE_PTR(H); REQUIRE_PTR(dx);
+  REQUIRE_PTR(dw_gate); REQUIRE_PTR(dw1); REQUIRE_PTR(dw3); REQUIRE_PTR(dw2);
+  if (router_grad) REQUIRE_PTR(w_gate);
+  REQUIRE_ALIGNED(dout); REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3);
+  REQUIRE_ALIGNED(w2); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(dx); REQUIRE_ALIGNED(dw1);
+  REQUIRE_ALIGNED(dw3); REQUIRE_ALIGNED(dw2); REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_layer_bwd_workspace_size(T, d, f, E, k, dtype))
+    return fail(MOE_ERR_WORKSPACE, "bwd workspace smaller than moe_layer_bwd_workspace_size()");
+  Carve c(ws, ws_bytes);
+  BwdWs<Carve> w;
+  w.carve(c, T, d, f, E, k, dtype);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "bwd workspace too small");
+  cudaStream_t s = (cudaStream_t)stream;
+  FfnPtrs p{x, w1, w3, w2, row_token, offsets, T, d, f, E, (int)((size_t)T * k + (size_t)E * 128), dtype};
+  int rc;
+  if (dtype == MOE_BF16 && tc_available()) {
+    if ((rc = launch_gather_rows(dout, row_token, offsets, E, d, dtype, w.dog, s))) return rc;
+    if ((rc = launch_gather_rows(x, row_token, offsets, E, d, dtype, w.xg, s))) return rc;
+    if ((rc = tc_ffn_bwd(p, w.dog, w.xg, row_gate, H, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2,
+                         device_sm_count(), s)))
+      return rc;
+  } else {
+    if ((rc = simt_ffn_bwd(p, dout, row_gate, H, w.dap, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2, s)))
+      return rc;
+  }
+  float* dl = dlogits ? dlogits : w.dl;
+  if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row, T, E, k,
+                              dl, dS, s)))
+    return rc;
+  if (router_grad) {
+    if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
+                                  true, w.dx_acc, s)))
+      return rc;
+    return simt_router_bwd_gemms(x, w_gate, dl, w.dx_acc, T, d, E, dtype, dw_gate, dx, s);
+  }
+  cudaError_t e = cudaMemsetAsync(dw_gate, 0, (size_t)d * E * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset dw_gate");
+  return launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false, false,
+                             dx, s);
+}
+
+int moe_check_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int flag = 0;
+  e = cudaMemcpyFromSymbol(&flag, g_moe_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status flag");
+  if (flag != 0) {
+    int zero = 0;
+    cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int));
+    char buf[96];
+    snprintf(buf, sizeof(buf), "device-side check failed (code 0x%x)", flag);
+    return fail(MOE_ERR_DEVICE_TIMEOUT, buf);
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Host-side launchers shared between the translation units of the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---------------------------------------------------------------- routing
+int launch_router_logits_simt(const void* x, const void* wg, int T, int d, int E, int dtype,
+                              const float* bias, float* logits, cudaStream_t s);
+int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out,
+                        int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
+
+// ---------------------------------------------------------------- permutation
+struct PermuteWs {
+  int32_t* blockcnt;   // [nb, E]
+  int32_t* blockbase;  // [nb, E]
+  // exact plan (used as input of the rounding pass)
+  int32_t* ex_counts;
+  int32_t* ex_offsets;
+  int32_t* ex_row_token;
+  float* ex_row_gate;
+  int32_t* ex_row_slot;
+  double* lse;         // [T]
+};
+size_t permute_ws_bytes(int T, int E, int k, int round_mode, int tile);
+int carve_permute_ws(void* ws, size_t bytes, int T, int E, int k, int round_mode, int tile,
+                     PermuteWs* out);
+int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, int k, int tile,
+                         int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
+                         int32_t* row_slot, int32_t* slot_row, const PermuteWs& w, cudaStream_t s);
+int launch_permute_round(const int32_t* idx, const float* gate, const float* logits, int T, int E,
+                         int k, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
+                         float* row_gate, int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
+                         const PermuteWs& w, cudaStream_t s);
+
+// ---------------------------------------------------------------- row ops
+int launch_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets, int E,
+                       int width, int dtype, void* dst, cudaStream_t s);
+// out[t] = sum over token t's rows (kept slots in order, then added rows by
+// ascending expert) of (weighted ? row_gate[r] : 1) * src[r]; out fp32 or dtype.
+int launch_token_reduce(const void* src, const float* row_gate, const int32_t* slot_row,
+                        const int32_t* extra_row, int T, int width, int E, int k, int dtype,
+                        bool weighted, bool out_f32, void* out, cudaStream_t s);
+// dlogits and (optionally) the final dS rows from dS partials [cap, nparts].
+int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
+                      const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
+                      int T, int E, int k, float* dlogits, float* dS_out, cudaStream_t s);
+
+// ---------------------------------------------------------------- CUDA-core GEMM path
+struct FfnPtrs {
+  const void *x, *w1, *w3, *w2;
+  const int32_t *row_token, *offsets;
+  int T, d, f, E, cap, dtype;
+};
+int simt_ffn_fwd(const FfnPtrs& p, void* H, void* act, void* Y, cudaStream_t s);
+int simt_ffn_bwd(const FfnPtrs& p, const void* dout, const float* row_gate, const void* H,
+                 float* dap, void* dH, void* gact, float* ds, void* dXp, void* dw1, void* dw3,
+                 void* dw2, cudaStream_t s);
+int simt_router_bwd_gemms(const void* x, const void* wg, const float* dl, const float* dx_acc,
+                          int T, int d, int E, int dtype, float* dw_gate, void* dx, cudaStream_t s);
+
+// ---------------------------------------------------------------- tensor-core path
+bool tc_available();
+int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, int num_sms,
+               cudaStream_t s);
+int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* row_gate,
+               const void* H, void* dH, void* gact, float* ds_part, void* dXp, void* dw1,
+               void* dw3, void* dw2, int num_sms, cudaStream_t s);
+int tc_num_dS_parts(int f);
+
+int device_sm_count();
+
+}  // namespace moe

@@ -1,0 +1,485 @@
+// Router top-k/softmax and the expert permutation (exact and token-rounded).
+//
+// Top-k then softmax over the k logits: Beam article sec. 5.3 / Trinity Large
+// commentary example 1.  Histogram + prefix sum + stable scatter into
+// expert-contiguous rows: Trinity example 2-3, Olmo-core 3 ("row-wise EP puts
+// data straight into expert input buffers", routing kept on the GPU).
+// Token rounding: SonicMoE summary sec. 3.
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+// ============================================================== top-k + softmax
+// One warp per token.  Each lane holds up to 8 of the E <= 256 logits
+// (expert e = lane + 32*i).  k rounds of a warp arg-max (ties: lowest id).
+__global__ void k_topk_softmax(const float* __restrict__ logits_in, const float* __restrict__ bias,
+                               float* __restrict__ logits_out, int T, int E, int k,
+                               int32_t* __restrict__ idx, float* __restrict__ gate) {
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int e = lane + 32 * i;
+      float l = -INFINITY;
+      if (e < E) {
+        l = logits_in[(size_t)t * E + e];
+        if (bias) l += bias[e];
+        if (logits_out != logits_in || bias) logits_out[(size_t)t * E + e] = l;
+      }
+      v[i] = l;
+    }
+    unsigned taken = 0;  // bit i: my element i already selected
+    float top[8];
+    int topi[8];
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        int e = lane + 32 * i;
+        if (e < E && !(taken >> i & 1u)) {
+          if (v[i] > bv || (v[i] == bv && e < bi)) { bv = v[i]; bi = e; }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      top[j] = bv;
+      topi[j] = bi;
+    }
+    if (lane == 0) {
+      float m = top[0], z = 0.f;
+      float ex[8];
+      for (int j = 0; j < k; ++j) { ex[j] = expf(top[j] - m); z += ex[j]; }
+      float inv = 1.0f / z;
+      for (int j = 0; j < k; ++j) {
+        idx[(size_t)t * k + j] = topi[j];
+        gate[(size_t)t * k + j] = ex[j] * inv;
+      }
+    }
+  }
+}
+
+int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out, int T,
+                        int E, int k, int32_t* idx, float* gate, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  int blocks = (T + 7) / 8;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, idx, gate);
+  MOE_CHECK_LAUNCH("topk_softmax");
+  return MOE_OK;
+}
+
+// ============================================================== exact permutation
+// Block b owns tokens [256 b, 256 b + 256); warp w of it owns 32 of them.
+// bits[w][e] has bit `lane` set when token (w, lane) chose expert e, so the
+// rank of a token among the block's tokens of expert e (ascending token id)
+// is sum over earlier warps of popc(bits[w'][e]) + popc(bits[w][e] & lanes below).
+constexpr int PERM_TOK = 256;
+
+__device__ __forceinline__ void build_bits(const int32_t* __restrict__ idx, int T, int E, int k,
+                                           uint32_t* bits, int* status) {
+  for (int i = threadIdx.x; i < 8 * E; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * PERM_TOK + threadIdx.x;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      int e = idx[(size_t)t * k + j];
+      if (e >= 0 && e < E) atomicOr(&bits[w * E + e], 1u << lane);
+      else record_status(status, 0x120);  // invalid expert id: flag it, skip the slot
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void k_perm_count(const int32_t* __restrict__ idx, int T, int E, int k,
+                             int32_t* __restrict__ blockcnt, int* status) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* bits = sm;
+  build_bits(idx, T, E, k, bits, status);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(bits[w * E + e]);
+    blockcnt[(size_t)blockIdx.x * E + e] = c;
+  }
+}
+
+// Single block: per-expert running sums over blocks, padded exclusive scan
+// over experts, padding rows.
+__global__ void k_perm_scan(const int32_t* __restrict__ blockcnt, int nb, int E, int tile,
+                            int32_t* __restrict__ blockbase, int32_t* __restrict__ counts,
+                            int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+                            float* __restrict__ row_gate, int32_t* __restrict__ row_slot) {
+  __shared__ int s_cnt[256];
+  __shared__ int s_off[257];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int b = 0; b < nb; ++b) {
+      blockbase[(size_t)b * E + e] = run;
+      run += blockcnt[(size_t)b * E + e];
+    }
+    s_cnt[e] = run;
+    counts[e] = run;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = acc;
+      acc += (s_cnt[e] + tile - 1) / tile * tile;
+    }
+    s_off[E] = acc;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = s_off[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int o = s_off[e];
+    for (int b = 0; b < nb; ++b) blockbase[(size_t)b * E + e] += o;
+  }
+  // padding rows of every segment
+  for (int e = 0; e < E; ++e) {
+    int lo = s_off[e] + s_cnt[e], hi = s_off[e + 1];
+    for (int r = lo + threadIdx.x; r < hi; r += blockDim.x) {
+      row_token[r] = -1;
+      row_gate[r] = 0.f;
+      row_slot[r] = -1;
+    }
+  }
+}
+
+__global__ void k_perm_scatter(const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                               int T, int E, int k, const int32_t* __restrict__ blockbase,
+                               int32_t* __restrict__ row_token, float* __restrict__ row_gate,
+                               int32_t* __restrict__ row_slot, int32_t* __restrict__ slot_row,
+                               int* status) {
+  extern __shared__ uint32_t sm[];
+  uint32_t* bits = sm;
+  int* wpre = reinterpret_cast<int*>(sm + 8 * E);
+  build_bits(idx, T, E, k, bits, status);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = blockbase[(size_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wpre[w * E + e] = run;
+      run += __popc(bits[w * E + e]);
+    }
+  }
+  __syncthreads();
+  const int t = blockIdx.x * PERM_TOK + threadIdx.x;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const uint32_t below = (1u << lane) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int s = t * k + j;
+    int e = idx[s];
+    if (e < 0 || e >= E) { slot_row[s] = -1; continue; }
+    int row = wpre[w * E + e] + __popc(bits[w * E + e] & below);
+    row_token[row] = t;
+    row_gate[row] = gate[s];
+    row_slot[row] = s;
+    slot_row[s] = row;
+  }
+}
+
+static int perm_blocks(int T) { return (T + PERM_TOK - 1) / PERM_TOK; }
+
+size_t permute_ws_bytes(int T, int E, int k, int round_mode, int tile) {
+  Sizer z;
+  int nb = perm_blocks(T) > 0 ? perm_blocks(T) : 1;
+  z.take<int32_t>((size_t)nb * E);
+  z.take<int32_t>((size_t)nb * E);
+  if (round_mode) {
+    size_t cap = (size_t)T * k + (size_t)E * tile;
+    z.take<int32_t>(E);
+    z.take<int32_t>(E + 1);
+    z.take<int32_t>(cap);
+    z.take<float>(cap);
+    z.take<int32_t>(cap);
+    z.take<double>(T > 0 ? T : 1);
+  }
+  return z.used;
+}
+
+int carve_permute_ws(void* ws, size_t bytes, int T, int E, int k, int round_mode, int tile,
+                     PermuteWs* o) {
+  Carve c(ws, bytes);
+  int nb = perm_blocks(T) > 0 ? perm_blocks(T) : 1;
+  *o = PermuteWs{};
+  o->blockcnt = c.take<int32_t>((size_t)nb * E);
+  o->blockbase = c.take<int32_t>((size_t)nb * E);
+  if (round_mode) {
+    size_t cap = (size_t)T * k + (size_t)E * tile;
+    o->ex_counts = c.take<int32_t>(E);
+    o->ex_offsets = c.take<int32_t>(E + 1);
+    o->ex_row_token = c.take<int32_t>(cap);
+    o->ex_row_gate = c.take<float>(cap);
+    o->ex_row_slot = c.take<int32_t>(cap);
+    o->lse = c.take<double>(T > 0 ? T : 1);
+  }
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "permute workspace too small");
+  return MOE_OK;
+}
+
+int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, int k, int tile,
+                         int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
+                         int32_t* row_slot, int32_t* slot_row, const PermuteWs& w,
+                         cudaStream_t s) {
+  const int nb = perm_blocks(T);
+  const size_t smem_count = (size_t)8 * E * sizeof(uint32_t);
+  if (nb > 0) {
+    k_perm_count<<<nb, PERM_TOK, smem_count, s>>>(idx, T, E, k, w.blockcnt, status_ptr());
+    MOE_CHECK_LAUNCH("perm_count");
+  }
+  k_perm_scan<<<1, 256, 0, s>>>(w.blockcnt, nb, E, tile, w.blockbase, counts, offsets, row_token,
+                                row_gate, row_slot);
+  MOE_CHECK_LAUNCH("perm_scan");
+  if (nb > 0) {
+    k_perm_scatter<<<nb, PERM_TOK, 2 * smem_count, s>>>(idx, gate, T, E, k, w.blockbase,
+                                                        row_token, row_gate, row_slot, slot_row,
+                                                        status_ptr());
+    MOE_CHECK_LAUNCH("perm_scatter");
+  }
+  return MOE_OK;
+}
+
+// ============================================================== token rounding
+// Log-sum-exp of each token's top-k logits, in fp64 so that the ranking key
+// l_te - LSE_t orders pairs the same way on any correctly rounding host.
+__global__ void k_round_lse(const float* __restrict__ logits, const int32_t* __restrict__ idx,
+                            int T, int E, int k, double* __restrict__ lse) {
+  int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  double m = -INFINITY;
+  for (int j = 0; j < k; ++j) m = fmax(m, (double)logits[(size_t)t * E + idx[(size_t)t * k + j]]);
+  double z = 0.0;
+  for (int j = 0; j < k; ++j) z += exp((double)logits[(size_t)t * E + idx[(size_t)t * k + j]] - m);
+  lse[t] = m + log(z);
+}
+
+__device__ __forceinline__ uint64_t order_key(double v) {
+  if (v == 0.0) v = 0.0;  // fold -0 into +0
+  uint64_t u = (uint64_t)__double_as_longlong(v);
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+constexpr int RS_THREADS = 1024;
+
+// Block-wide exclusive scan of one int per thread (1024 threads).
+__device__ __forceinline__ int block_excl_scan(int v, int* s_warp, int* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int y = s_warp[lane];
+    int z = y;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int q = __shfl_up_sync(0xffffffffu, z, o);
+      if (lane >= o) z += q;
+    }
+    s_warp[lane] = z - y;  // exclusive prefix of warp totals
+    if (lane == 31) s_warp[32] = z;
+  }
+  __syncthreads();
+  int r = s_warp[w] + x - v;
+  *total = s_warp[32];
+  __syncthreads();
+  return r;
+}
+
+// One block per expert.  Chooses the final members of expert e's segment and
+// writes the final rows.  `cand` is either the assigned tokens (drop case,
+// candidates = rows of the exact segment) or the unassigned ones (add case).
+__global__ void __launch_bounds__(RS_THREADS)
+k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
+               const int32_t* __restrict__ ex_counts, const int32_t* __restrict__ ex_offsets,
+               const int32_t* __restrict__ ex_row_token, const float* __restrict__ ex_row_gate,
+               const int32_t* __restrict__ ex_row_slot, int T, int E, int tile,
+               int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+               int32_t* __restrict__ row_token, float* __restrict__ row_gate,
+               int32_t* __restrict__ row_slot, int32_t* __restrict__ slot_row,
+               int32_t* __restrict__ extra_row) {
+  extern __shared__ uint32_t bm[];  // membership bitmap of the assigned tokens, T bits
+  __shared__ int s_off[257];
+  __shared__ int s_hist[256];
+  __shared__ int s_warp[33];
+  __shared__ int s_sel, s_rem;
+  const int e = blockIdx.x;
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    const int cap_rows = tile * (T / tile);
+    for (int i = 0; i < E; ++i) {
+      s_off[i] = acc;
+      int c = ex_counts[i];
+      int r = tile * ((c + tile / 2) / tile);
+      acc += r < cap_rows ? r : cap_rows;
+    }
+    s_off[E] = acc;
+  }
+  __syncthreads();
+  if (e == 0) {
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) offsets[i] = s_off[i];
+    for (int i = threadIdx.x; i < E; i += blockDim.x) counts[i] = ex_counts[i];
+  }
+  const int c = ex_counts[e];
+  const int r = s_off[e + 1] - s_off[e];
+  const int in0 = ex_offsets[e];
+  const int out0 = s_off[e];
+
+  if (r == c) {  // nothing to drop or add: copy the segment
+    for (int i = threadIdx.x; i < c; i += blockDim.x) {
+      int s = ex_row_slot[in0 + i];
+      row_token[out0 + i] = ex_row_token[in0 + i];
+      row_gate[out0 + i] = ex_row_gate[in0 + i];
+      row_slot[out0 + i] = s;
+      slot_row[s] = out0 + i;
+    }
+    return;
+  }
+  const bool drop = r < c;
+  const int m = drop ? r : r - c;  // how many candidates to select (largest first)
+  const int ncand = drop ? c : T;
+  const int nwords = (T + 31) / 32;
+  if (!drop) {
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) bm[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < c; i += blockDim.x) {
+      int t = ex_row_token[in0 + i];
+      atomicOr(&bm[t >> 5], 1u << (t & 31));
+    }
+    __syncthreads();
+  }
+  auto cand_token = [&](int i) -> int { return drop ? ex_row_token[in0 + i] : i; };
+  auto is_cand = [&](int i) -> bool { return drop || !((bm[i >> 5] >> (i & 31)) & 1u); };
+  auto cand_key = [&](int t) -> uint64_t {
+    return order_key((double)logits[(size_t)t * E + e] - lse[t]);
+  };
+
+  // radix select of the m-th largest key among the candidates
+  uint64_t prefix = 0, pmask = 0;
+  int rem = m;
+  if (m > 0) {
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < ncand; i += blockDim.x) {
+        if (!is_cand(i)) continue;
+        uint64_t u = cand_key(cand_token(i));
+        if ((u & pmask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255], 1);
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        int cum = 0, sel = 0;
+        for (int dg = 255; dg >= 0; --dg) {
+          if (cum + s_hist[dg] >= rem) { sel = dg; break; }
+          cum += s_hist[dg];
+        }
+        s_sel = sel;
+        s_rem = rem - cum;
+      }
+      __syncthreads();
+      prefix |= (uint64_t)s_sel << shift;
+      pmask |= (uint64_t)255 << shift;
+      rem = s_rem;
+      __syncthreads();
+    }
+  }
+  const uint64_t thr = prefix;  // value of the m-th largest key
+  const int need_eq = rem;      // how many keys equal to thr are selected
+
+  // ordered pass: ties broken by ascending position (= ascending token id)
+  int eq_base = 0, out_base = 0, asg_base = 0;
+  for (int i0 = 0; i0 < ncand; i0 += blockDim.x) {
+    const int i = i0 + threadIdx.x;
+    int t = -1, assigned = 0, cand = 0, eq = 0, gt = 0;
+    uint64_t u = 0;
+    if (i < ncand) {
+      t = cand_token(i);
+      cand = is_cand(i);
+      assigned = drop ? 1 : !cand;
+      if (cand && m > 0) {
+        u = cand_key(t);
+        eq = (u == thr);
+        gt = (u > thr);
+      }
+    }
+    int tot;
+    const int eq_rank = eq_base + block_excl_scan(eq, s_warp, &tot);
+    eq_base += tot;
+    const int selected = cand && m > 0 && (gt || (eq && eq_rank < need_eq));
+    // drop case: members are the selected (kept) candidates;
+    // add case: members are the assigned tokens plus the selected ones
+    const int member = drop ? selected : (assigned || selected);
+    const int pos = out_base + block_excl_scan(member, s_warp, &tot);
+    out_base += tot;
+    const int asg_rank = asg_base + block_excl_scan(assigned, s_warp, &tot);
+    asg_base += tot;
+    if (i < ncand) {
+      const int row = out0 + pos;
+      if (assigned) {
+        const int src = drop ? in0 + i : in0 + asg_rank;
+        const int s = ex_row_slot[src];
+        if (member) {
+          row_token[row] = t;
+          row_gate[row] = ex_row_gate[src];
+          row_slot[row] = s;
+          slot_row[s] = row;
+        } else {
+          slot_row[s] = -1;
+        }
+      } else if (member) {
+        row_token[row] = t;
+        row_gate[row] = (float)exp((double)logits[(size_t)t * E + e] - lse[t]);
+        row_slot[row] = -1;
+        extra_row[(size_t)t * E + e] = row;
+      }
+    }
+  }
+}
+
+int launch_permute_round(const int32_t* idx, const float* gate, const float* logits, int T, int E,
+                         int k, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
+                         float* row_gate, int32_t* row_slot, int32_t* slot_row,
+                         int32_t* extra_row, const PermuteWs& w, cudaStream_t s) {
+  // 1. exact plan into the workspace (its slot_row is scratch: the final
+  //    slot_row is fully rewritten by the selection below)
+  int rc = launch_permute_exact(idx, gate, T, E, k, tile, w.ex_counts, w.ex_offsets,
+                                w.ex_row_token, w.ex_row_gate, w.ex_row_slot, slot_row, w, s);
+  if (rc) return rc;
+  if (T > 0) {
+    k_round_lse<<<(T + 255) / 256, 256, 0, s>>>(logits, idx, T, E, k, w.lse);
+    MOE_CHECK_LAUNCH("round_lse");
+    cudaError_t e = cudaMemsetAsync(extra_row, 0xff, (size_t)T * E * sizeof(int32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "memset extra_row");
+  }
+  const size_t smem = (size_t)((T + 31) / 32 + 1) * sizeof(uint32_t);
+  if (smem > 200 * 1024) return fail(MOE_ERR_UNSUPPORTED, "token rounding supports T <= 1.6M");
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_round_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "round_select smem attribute");
+  }
+  k_round_select<<<E, RS_THREADS, smem, s>>>(logits, w.lse, w.ex_counts, w.ex_offsets,
+                                             w.ex_row_token, w.ex_row_gate, w.ex_row_slot, T, E,
+                                             tile, counts, offsets, row_token, row_gate, row_slot,
+                                             slot_row, extra_row);
+  MOE_CHECK_LAUNCH("round_select");
+  return MOE_OK;
+}
+
+}  // namespace moe

@@ -1,0 +1,68 @@
+"""One MoE layer step (forward + backward) through the C ABI, with every
+buffer allocated once up front so that a step allocates nothing."""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class MoELayerStep:
+    """Buffers and call sequence of one forward+backward pass.
+
+    forward(): moe_route -> moe_permute -> moe_expert_ffn_fwd -> moe_combine
+    backward(): moe_layer_bwd (saved set: x, logits, idx, gate, plan, H)
+    """
+
+    def __init__(self, T, d, f, E, k, dtype=torch.bfloat16, device="cuda",
+                 round_mode=B.MOE_ROUND_NONE):
+        self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
+        self.dtype, self.device, self.round_mode = dtype, device, round_mode
+        dt = B.dtype_code(dtype)
+        cap = B.moe_row_capacity(T, E, k)
+        self.cap = cap
+        e = lambda *s, dt_=torch.float32: torch.empty(*s, device=device, dtype=dt_)
+        self.logits, self.idx, self.gate = e(T, E), e(T, k, dt_=torch.int32), e(T, k)
+        self.plan = dict(counts=e(E, dt_=torch.int32), offsets=e(E + 1, dt_=torch.int32),
+                         row_token=e(cap, dt_=torch.int32), row_gate=e(cap),
+                         row_slot=e(cap, dt_=torch.int32), slot_row=e(T * k, dt_=torch.int32),
+                         extra_row=e(T, E, dt_=torch.int32) if round_mode else None)
+        self.H, self.Y = e(cap, 2 * f, dt_=dtype), e(cap, d, dt_=dtype)
+        self.out = e(T, d, dt_=dtype)
+        self.ws_perm = e(max(B.moe_permute_workspace_size(T, E, k, round_mode), 1), dt_=torch.uint8)
+        self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
+        self.ws_bwd = e(max(B.moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
+        self.grads = dict(dx=e(T, d, dt_=dtype), dw_gate=e(d, E), dw1=e(E, d, f, dt_=dtype),
+                          dw3=e(E, d, f, dt_=dtype), dw2=e(E, f, d, dt_=dtype), dS=e(cap),
+                          dlogits=e(T, E))
+
+    def forward(self, x, w_gate, w1, w3, w2, logits_override=None, logit_bias=None, stream=None):
+        self._saved = (x, w_gate, w1, w3, w2)
+        self.router_grad = logits_override is None
+        B.moe_route(x, w_gate, self.k, logits_override, logit_bias, self.logits, self.idx,
+                    self.gate, T=self.T, E=self.E, stream=stream)
+        B.moe_permute(self.idx, self.gate, self.logits, self.E, self.round_mode, out=self.plan,
+                      ws=self.ws_perm, stream=stream)
+        B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan["row_token"], self.plan["offsets"], self.k,
+                             self.H, self.Y, self.ws_fwd, stream=stream)
+        B.moe_combine(self.Y, self.plan["row_gate"], self.plan["slot_row"],
+                      self.plan["extra_row"], self.T, self.E, self.k, self.out, stream=stream)
+        return self.out
+
+    def backward(self, dout, stream=None):
+        x, w_gate, w1, w3, w2 = self._saved
+        return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
+                               self.H, self.router_grad, out=self.grads, ws=self.ws_bwd,
+                               stream=stream)
+
+    # number of library kernel launches of one step (forward + backward)
+    def launches_per_step(self, tensor_cores: bool) -> int:
+        route = 2 if self.router_grad else 1
+        perm = 3 if not self.round_mode else 5
+        if tensor_cores:
+            fwd = 3 + 1
+            bwd = 2 + 4 + 1 + (3 if self.router_grad else 2)
+        else:
+            fwd = 3 + 1
+            bwd = 5 + 1 + (3 if self.router_grad else 1)
+        return route + perm + fwd + bwd

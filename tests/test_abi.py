@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/moe.h declares, sizes workspaces consistently, and rejects bad
+arguments before launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_59_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s*(moe_[a-z_0-9]+)\s*\(", src, re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    names = _declared()
+    assert "moe_route" in names and "moe_layer_bwd" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(B.EXPORTS) >= set(names)
+
+
+def test_version_and_capacity():
+    assert B.moe_version() >= 10000
+    assert B.moe_row_capacity(16384, 8, 4) == 16384 * 4 + 8 * 128
+
+
+def test_workspace_sizes_monotone():
+    a = B.moe_layer_bwd_workspace_size(1000, 256, 256, 8, 2, B.MOE_BF16)
+    b = B.moe_layer_bwd_workspace_size(2000, 256, 256, 8, 2, B.MOE_BF16)
+    assert 0 < a < b
+    assert B.moe_permute_workspace_size(100, 8, 2, 1) > B.moe_permute_workspace_size(100, 8, 2, 0)
+    assert B.moe_ffn_fwd_workspace_size(100, 256, 256, 8, 2, B.MOE_F32) > 0
+
+
+def _rc_route(**kw):
+    args = dict(x=None, wg=None, T=4, d=128, E=8, k=2, dtype=B.MOE_BF16, lo=None, lb=None,
+                logits=None, idx=None, gate=None, stream=None)
+    args.update(kw)
+    lib = B.lib()
+    return lib.moe_route(args["x"], args["wg"], args["T"], args["d"], args["E"], args["k"],
+                         args["dtype"], args["lo"], args["lb"], args["logits"], args["idx"],
+                         args["gate"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=0), -2), (dict(k=9), -2), (dict(E=1, k=2), -2), (dict(E=300), -2),
+    (dict(dtype=7), -2), (dict(T=-1), -1),
+])
+def test_route_rejects_bad_shapes(kw, code):
+    assert _rc_route(**kw) == code
+    assert len(B.lib().moe_last_error()) > 0
+
+
+def test_route_rejects_null_outputs():
+    assert _rc_route() == -1
+    assert b"NULL" in B.lib().moe_last_error()
+
+
+def test_permute_rejects_tile_and_mode():
+    lib = B.lib()
+    fake = ctypes.c_void_p(16)
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 64, fake, fake, fake, fake, fake, fake,
+                         None, fake, 1 << 20, None)
+    assert rc == -2
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 3, 128, fake, fake, fake, fake, fake, fake,
+                         None, fake, 1 << 20, None)
+    assert rc == -1
+    # rounding needs logits and extra_row
+    rc = lib.moe_permute(fake, fake, None, 4, 8, 2, 1, 128, fake, fake, fake, fake, fake, fake,
+                         None, fake, 1 << 20, None)
+    assert rc == -1
+    # workspace too small
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 128, fake, fake, fake, fake, fake, fake,
+                         None, fake, 8, None)
+    assert rc == -5
+
+
+def test_ffn_rejects_unaligned_dims_and_small_workspace():
+    lib = B.lib()
+    fake = ctypes.c_void_p(256)
+    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, 16, 100, 128, 8, 2,
+                                B.MOE_BF16, fake, fake, fake, 1 << 30, None)
+    assert rc == -2
+    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, 16, 128, 128, 8, 2,
+                                B.MOE_BF16, fake, fake, fake, 16, None)
+    assert rc == -5
+    odd = ctypes.c_void_p(258)
+    rc = lib.moe_expert_ffn_fwd(odd, fake, fake, fake, fake, fake, 16, 128, 128, 8, 2,
+                                B.MOE_BF16, fake, fake, fake, 1 << 30, None)
+    assert rc == -1
+
+
+def test_bwd_rejects_missing_w_gate_with_router_grad():
+    lib = B.lib()
+    f = ctypes.c_void_p(256)
+    args = [f, f, None, f, f, f, f, f, f, f, f, f, None, f, 16, 128, 128, 8, 2, B.MOE_BF16, 1,
+            f, f, f, f, f, None, None, f, 1 << 40, None]
+    assert lib.moe_layer_bwd(*args) == -1
+    assert b"w_gate" in lib.moe_last_error()

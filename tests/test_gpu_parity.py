@@ -1,0 +1,143 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle, element
+by element, on seeded inputs that span several tiles and a ragged tail."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_59_b200 import binding as B
+from mixture_experts_layer_59_b200 import synth
+from oracle import moe_oracle as O
+
+from helpers import (BF16_TOL, F32_TOL, assert_close, compare_layer, compare_plan, f64,
+                     fp32_router_logits, gpu_layer, i64, oracle_layer)
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(T, d, f, E, k, dtype="bf16", routing="learned", std=0.05):
+    return synth.MoEConfig("test", T, d, f, E, k, dtype=dtype, std=std, routing=routing)
+
+
+# ------------------------------------------------------------------ routing
+
+def test_route_learned_logits_and_topk():
+    cfg = _cfg(1000, 256, 128, 16, 4, std=0.05)
+    inp = synth.make_inputs(cfg, seed=3, device="cuda")
+    logits, idx, gate = B.moe_route(inp["x"], inp["w_gate"], cfg.k)
+    torch.cuda.synchronize()
+    ref_logits, ref_idx, _ = O.route(f64(inp["x"]), f64(inp["w_gate"]), cfg.k)
+    scale = np.abs(ref_logits).max()
+    np.testing.assert_allclose(f64(logits), ref_logits, atol=1e-5 * scale, rtol=0)
+    # the top-k set is unique wherever the k-th and (k+1)-th logits are apart
+    srt = -np.sort(-ref_logits, axis=1)
+    margin = srt[:, cfg.k - 1] - srt[:, cfg.k]
+    clear = margin > 1e-4 * scale
+    assert clear.mean() > 0.99
+    np.testing.assert_array_equal(i64(idx)[clear], ref_idx[clear])
+    # and the gate is the softmax of the GPU's own top-k logits
+    g_ref = O.route(None, None, cfg.k, logits_override=f64(logits))[2]
+    np.testing.assert_allclose(f64(gate), g_ref, rtol=1e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 8), (256, 8), (5, 5), (33, 3)])
+def test_route_override_ties_bitexact(E, k):
+    T = 777
+    lo = synth.quantized_logits(T, E, levels=4, seed=E)
+    bias = torch.linspace(-0.5, 0.5, E) if E == 33 else None
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(),
+                                    logit_bias=None if bias is None else bias.cuda(), T=T, E=E)
+    torch.cuda.synchronize()
+    ref_l, ref_idx, ref_g = O.route(None, None, k, logits_override=f64(lo),
+                                    logit_bias=None if bias is None else f64(bias))
+    np.testing.assert_array_equal(i64(idx), ref_idx)
+    np.testing.assert_array_equal(f64(logits), f64(torch.from_numpy(ref_l.astype(np.float32))))
+    np.testing.assert_allclose(f64(gate), ref_g, rtol=1e-6, atol=1e-7)
+
+
+# ------------------------------------------------------------------ permutation
+
+@pytest.mark.parametrize("T,E,k", [(1, 8, 2), (255, 8, 2), (1000, 16, 4), (4097, 64, 8),
+                                   (3000, 256, 8), (300, 4, 4)])
+def test_permute_exact_bitexact(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    lo = torch.randn(T, E, generator=g)
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E)
+    plan_g = B.moe_permute(idx, gate, logits, E, B.MOE_ROUND_NONE)
+    torch.cuda.synchronize()
+    _, ridx, rgate = O.route(None, None, k, logits_override=f64(lo))
+    np.testing.assert_array_equal(i64(idx), ridx)
+    compare_plan(plan_g, O.exact_plan(ridx, rgate, E))
+
+
+@pytest.mark.parametrize("T,E,k,skew", [(1000, 8, 2, 0.0), (1000, 8, 2, 1.5), (5000, 16, 4, 1.1),
+                                        (8192, 64, 8, 1.1), (3000, 256, 8, 1.1), (200, 8, 2, 0.0)])
+def test_permute_rounded_bitexact(T, E, k, skew):
+    g = torch.Generator().manual_seed(7 * T + E)
+    lo = torch.randn(T, E, generator=g)
+    if skew:
+        rank = torch.randperm(E, generator=g).double() + 1
+        lo = lo + (-skew * torch.log(rank)).float()[None, :]
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E)
+    plan_g = B.moe_permute(idx, gate, logits, E, B.MOE_ROUND_NEAREST)
+    torch.cuda.synchronize()
+    _, ridx, _ = O.route(None, None, k, logits_override=f64(lo))
+    plan = O.rounded_plan(ridx, f64(lo), E)
+    assert (plan["dropped"].any() or plan["added"].any()) or T < 256
+    compare_plan(plan_g, plan)
+
+
+# ------------------------------------------------------------------ whole layer
+
+@pytest.mark.parametrize("round_mode", [0, 1])
+def test_layer_bf16_small(round_mode):
+    """Several M tiles per expert, ragged tails, d and f spanning several N tiles."""
+    cfg = _cfg(1000, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=11, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    g = gpu_layer(inp, cfg.k, round_mode, lg)
+    fwd, bwd = oracle_layer(inp, cfg.k, round_mode, lg)
+    compare_layer(g, fwd, bwd, BF16_TOL)
+
+
+def test_layer_bf16_many_experts_empty_segments():
+    """E=64 with T*k=1536: some experts get no tokens (empty segments, zero dW)."""
+    cfg = _cfg(384, 128, 128, 64, 4, std=0.08)
+    inp = synth.make_inputs(cfg, seed=5, device="cuda")
+    bias = torch.zeros(64)
+    bias[40:] = -30.0                     # experts 40..63 are never chosen
+    lg = fp32_router_logits(inp["x"], inp["w_gate"], bias)
+    g = gpu_layer(inp, cfg.k, 0, lg)
+    fwd, bwd = oracle_layer(inp, cfg.k, 0, lg)
+    assert (fwd["plan"]["counts"] == 0).sum() >= 24
+    compare_layer(g, fwd, bwd, BF16_TOL)
+    assert np.all(f64(g["dw1"])[40:] == 0) and np.all(f64(g["dw2"])[40:] == 0)
+
+
+def test_layer_fp32_tiny_config():
+    """The tiny fp32 workload in full (T=256, d=128, f=256, E=8, k=2)."""
+    cfg = synth.CONFIGS["tiny_fp32"]
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    g = gpu_layer(inp, cfg.k, 0, lg)
+    fwd, bwd = oracle_layer(inp, cfg.k, 0, lg, staged=False)
+    compare_layer(g, fwd, bwd, F32_TOL)
+
+
+def test_layer_router_grad_off_with_override():
+    cfg = _cfg(500, 128, 128, 8, 2, routing="uniform")
+    inp = synth.make_inputs(cfg, seed=2, device="cuda")
+    lg = f64(inp["logits_override"]).astype(np.float32)
+    g = gpu_layer(inp, cfg.k, 0, lg, router_grad=False)
+    fwd, bwd = oracle_layer(inp, cfg.k, 0, lg, router_grad=False)
+    compare_layer(g, fwd, bwd, BF16_TOL)
+    assert np.all(f64(g["dw_gate"]) == 0)
+
+
+def test_zero_tokens_is_a_no_op():
+    E, k = 8, 2
+    lo = torch.empty(0, E, device="cuda")
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=0, E=E)
+    plan = B.moe_permute(idx, gate, logits, E)
+    torch.cuda.synchronize()
+    assert i64(plan["offsets"]).tolist() == [0] * (E + 1)
+    assert i64(plan["counts"]).tolist() == [0] * E
