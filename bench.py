@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Benchmark of the token-choice MoE layer, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = route (router GEMM, top-k, softmax) -> permute -> grouped GEMMs with
+fused SwiGLU -> combine -> backward (dS = <dA', A>, dX/dW grouped GEMMs, router
+gradient), on the coarse workload T=16384, d=2048, f=1024, E=8, k=4, bf16,
+learned routing, seeded synthetic inputs resident in HBM.  L2 is flushed
+(512 MiB write) between timed steps, outside the timed events.
+
+With N > 1 (launched by torchrun) every rank runs an independent replica on
+its own GPU: the layer does not shard, so there is no data-path collective;
+`value` is the tokens of all ranks divided by the slowest rank's time.
+
+`--impl reference` times the CPU oracle (test infrastructure) on a bounded
+token sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd+bwd tokens/sec on 1 B200; grouped-GEMM TFLOP/s as % of BF16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="coarse")
+    ap.add_argument("--routing", default=None, help="override the workload's routing variant")
+    ap.add_argument("--round", type=int, default=0, help="1 = token rounding to 128-row tiles")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens of the cpu_baseline sample")
+    ap.add_argument("--ref-sample", type=int, default=256, help="tokens per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer written between steps")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured (MEASURED_PEAKS.json)"
+    return FALLBACK_PEAKS, "fallback (profiling recipe)"
+
+
+# ------------------------------------------------------------------ FLOP model
+def gemm_flops(kind, T, d, f, k):
+    """Algorithmic FLOPs of one launch of each grouped GEMM (live rows only)."""
+    rows = T * k
+    return {
+        "tc_up": 2.0 * rows * d * 2 * f,
+        "tc_down": 2.0 * rows * f * d,
+        "tc_dap": 2.0 * rows * d * f + 2.0 * rows * f,   # + dS = <dA', A>
+        "tc_dx": 2.0 * rows * 2 * f * d,
+        "tc_dw2": 2.0 * rows * f * d,
+        "tc_dw13": 2.0 * rows * d * 2 * f,
+    }.get(kind)
+
+
+def step_flops(T, d, f, E, k, router=True):
+    return 18.0 * T * k * d * f + 2.0 * T * k * f + (6.0 * T * d * E if router else 0.0)
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for fn in ("tc_gemm.cu", "tcgen05.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "mixture_experts_layer_59_b200", "csrc", fn), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source
+    is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    ent = d.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thr = threading.Thread(target=self._read, daemon=True)
+            self.thr.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ts, ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            rows.append((ts, parts))
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.15] or rows
+        sm = [float(p[2]) for _, p in inside if p[2].replace(".", "").isdigit()]
+        smax = [float(p[3]) for _, p in inside if p[3].replace(".", "").isdigit()]
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for _, p in inside:
+            for nm, v in zip(names[1:], p[6:10]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ oracle arms
+def oracle_tokens_per_s(cfg, n_tokens, seed=0, repeats=1):
+    """Time the CPU oracle (as it stands) on the first n_tokens of the workload."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    from mixture_experts_layer_59_b200 import synth
+    from oracle import moe_oracle as O
+
+    inp = synth.make_inputs(cfg.with_(T=n_tokens), seed=seed, device="cpu")
+    f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
+    x, wg, w1, w3, w2, do = (f64(inp[n]) for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    lo, lb = f64(inp["logits_override"]), f64(inp["logit_bias"])
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        fwd = O.layer_fwd(x, wg, w1, w3, w2, cfg.k, logits_override=lo, logit_bias=lb)
+        O.layer_bwd(do, x, wg, w1, w3, w2, fwd, router_grad_on=lo is None)
+        times.append(time.perf_counter() - t0)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return n_tokens, times, threads
+
+
+def run_reference(args, cfg, rank, world):
+    if rank != 0:
+        return 0
+    n, times, threads = oracle_tokens_per_s(cfg, args.ref_sample, repeats=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    total = sum(timed)
+    value = n * len(timed) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(timed), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {n} tokens of the workload per step (full expert weights), "
+                                   f"fwd+bwd, numpy fp64 with bf16 staging"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, args):
+    return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "d_ff": cfg.f, "E": cfg.E,
+            "k": cfg.k, "routing": cfg.routing, "token_rounding": bool(args.round),
+            "l2": f"flushed between timed steps ({args.flush_mb} MiB write)", "replicas": args.gpus}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_59_b200 import binding as B
+    from mixture_experts_layer_59_b200 import synth
+    from mixture_experts_layer_59_b200.layer import MoELayerStep
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    inp = synth.make_inputs(cfg, seed=rank, device=dev)
+    step = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round)
+    flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    lo, lb = inp["logits_override"], inp["logit_bias"]
+
+    def one_step():
+        step.forward(x, wg, w1, w3, w2, lo, lb)
+        step.backward(dout)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    B.moe_check_status()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    B.moe_profile_enable(True)
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        one_step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    B.moe_profile_enable(False)
+    barrier()
+    clocks = sampler.stop(t0, t1)
+    prof = B.moe_profile_report()
+    B.moe_check_status()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.T * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the public API with host buffers
+    x_h = x.cpu().pin_memory()
+    d_h = dout.cpu().pin_memory()
+    out_h = torch.empty_like(step.out, device="cpu").pin_memory()
+    dx_h = torch.empty_like(step.grads["dx"], device="cpu").pin_memory()
+    x_d, d_d = torch.empty_like(x), torch.empty_like(dout)
+    e2e_ms = []
+    for i in range(args.e2e_steps + 2 if args.e2e_steps > 0 else 0):
+        flush.zero_()
+        s_ev, e_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_ev.record()
+        x_d.copy_(x_h, non_blocking=True)
+        d_d.copy_(d_h, non_blocking=True)
+        step.forward(x_d, wg, w1, w3, w2, lo, lb)
+        step.backward(d_d)
+        out_h.copy_(step.out, non_blocking=True)
+        dx_h.copy_(step.grads["dx"], non_blocking=True)
+        e_ev.record()
+        torch.cuda.synchronize()
+        if i >= 2:
+            e2e_ms.append(s_ev.elapsed_time(e_ev))
+    e2e_total = sum(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_value = world * cfg.T * len(e2e_ms) / (e2e_total / 1e3) if e2e_ms else None
+    h2d = x.numel() * x.element_size() + dout.numel() * dout.element_size()
+    d2h = step.out.numel() * step.out.element_size() * 2
+
+    if rank != 0:
+        return 0
+
+    # ---- roofline of the dominant kernel (measured live over the timed region)
+    peaks, peak_src = load_peaks()
+    gemm = {n: v for n, v in prof.items() if n.startswith("tc_")}
+    kernels = {n: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1),
+                   "share": v[1] / max(sum(p[1] for p in prof.values()), 1e-12)}
+               for n, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    launches = sum(v[0] for v in prof.values())
+    roof = None
+    gemm_summary = None
+    if gemm:
+        dom = max(gemm, key=lambda n: gemm[n][1])
+        n_l, tot = gemm[dom]
+        avg_s = tot / n_l / 1e3
+        fl = gemm_flops(dom, cfg.T, cfg.d, cfg.f, cfg.k)
+        achieved = fl / avg_s / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic_for(dom, cfg.name),
+                "peak_source": f"{peak_src}: bf16 sustained",
+                "flops_per_launch": fl, "avg_launch_us": avg_s * 1e6}
+        g_fl = sum(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) * v[0] for n, v in gemm.items())
+        g_ms = sum(v[1] for v in gemm.values())
+        gemm_summary = {"tflops": g_fl / (g_ms / 1e3) / 1e12,
+                        "frac_of_peak": g_fl / (g_ms / 1e3) / 1e12 / peak,
+                        "ms_per_step": g_ms / args.steps}
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        n, times, threads = oracle_tokens_per_s(cfg, args.cpu_sample)
+        cpu = {"value": n / times[0], "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"first {n} of {cfg.T} tokens (full expert weights), one fwd+bwd, "
+                         f"numpy fp64 with bf16 staging, {times[0]:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights N(0,0.02^2), x,dO ~ N(0,1))",
+        "config": workload_config(cfg, args),
+        "tflops_per_gpu": step_flops(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k) / (ms_per_step / 1e3) / 1e12,
+        "gemm": gemm_summary,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_total / len(e2e_ms) if e2e_ms else None},
+        "clocks": clocks,
+        "gpu_launches": launches,
+        "kernels": kernels,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    from mixture_experts_layer_59_b200 import synth
+    cfg = synth.CONFIGS[args.workload]
+    if args.routing:
+        cfg = cfg.with_(routing=args.routing)
+    if args.tokens:
+        cfg = cfg.with_(T=args.tokens)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank, world)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, cfg, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -182,6 +182,18 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate,
  */
 int moe_check_status(void* stream);
 
+/*
+ * Measurement hook (the pages have no counterpart; it serves the benchmark).
+ * moe_profile_enable(1): from now on every kernel the library launches is
+ * bracketed by two CUDA events recorded on the kernel's own stream.
+ * moe_profile_enable(0) stops recording.
+ * moe_profile_report: waits for the recorded events, then writes one line
+ * "<kernel> <launches> <total_ms>" per kernel name into buf (NUL-terminated)
+ * and forgets the records.  Returns MOE_ERR_INVALID_ARG if buf is too small.
+ */
+int moe_profile_enable(int on);
+int moe_profile_report(char* buf, size_t buf_len);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,7 @@ EXPORTS = [
     "moe_version", "moe_last_error", "moe_row_capacity", "moe_route",
     "moe_permute_workspace_size", "moe_permute", "moe_ffn_fwd_workspace_size",
     "moe_expert_ffn_fwd", "moe_combine", "moe_layer_bwd_workspace_size", "moe_layer_bwd",
-    "moe_check_status",
+    "moe_check_status", "moe_profile_enable", "moe_profile_report",
 ]
 
 _lib = None
@@ -52,6 +52,8 @@ _SIGS = {
     "moe_layer_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_layer_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
+    "moe_profile_enable": (_i, [_i]),
+    "moe_profile_report": (_i, [ctypes.c_char_p, _sz]),
 }
 
 
@@ -214,3 +216,19 @@ def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=T
 
 def moe_check_status(stream=None):
     _check(lib().moe_check_status(_stream(stream)))
+
+
+def moe_profile_enable(on: bool = True):
+    _check(lib().moe_profile_enable(1 if on else 0))
+
+
+def moe_profile_report() -> dict:
+    """{kernel name: (launches, total_ms)} of the launches recorded since the
+    last report (waits for their events)."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    _check(lib().moe_profile_report(buf, len(buf)))
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.split()
+        out[name] = (int(n), float(ms))
+    return out

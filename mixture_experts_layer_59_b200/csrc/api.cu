@@ -1,6 +1,10 @@
 // extern "C" entry points: argument checks, workspace layout, kernel order.
 #include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "internal.h"
@@ -31,6 +35,44 @@ int* status_ptr() {
     if (cudaGetSymbolAddress(&p, g_moe_status) == cudaSuccess) cache[dev] = static_cast<int*>(p);
   }
   return cache[dev];
+}
+
+// ------------------------------------------------------------ profiling hook
+namespace {
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+struct ProfRec {
+  std::string name;
+  cudaEvent_t a, b;
+};
+std::vector<ProfRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+
+cudaEvent_t prof_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+ProfScope::ProfScope(const char* n, cudaStream_t s) : name(n), stream(s) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof_on) return;
+  start = prof_event();
+  cudaEventRecord(start, stream);
+}
+
+ProfScope::~ProfScope() {
+  if (start == nullptr) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t stop = prof_event();
+  cudaEventRecord(stop, stream);
+  g_recs.push_back(ProfRec{name, start, stop});
 }
 
 int device_sm_count() {
@@ -290,6 +332,40 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   if (e != cudaSuccess) return cuda_fail(e, "memset dw_gate");
   return launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false, false,
                              dx, s);
+}
+
+int moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return MOE_OK;
+}
+
+int moe_profile_report(char* buf, size_t buf_len) {
+  if (buf == nullptr || buf_len == 0) return fail(MOE_ERR_INVALID_ARG, "buf must not be NULL");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  std::map<std::string, std::pair<int, double>> agg;
+  int rc = MOE_OK;
+  for (auto& r : g_recs) {
+    float ms = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) rc = cuda_fail(e, "profile event");
+    auto& v = agg[r.name];
+    v.first += 1;
+    v.second += ms;
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_recs.clear();
+  std::string out;
+  char line[160];
+  for (auto& kv : agg) {
+    snprintf(line, sizeof(line), "%s %d %.6f\n", kv.first.c_str(), kv.second.first, kv.second.second);
+    out += line;
+  }
+  if (out.size() + 1 > buf_len) return fail(MOE_ERR_INVALID_ARG, "report buffer too small");
+  memcpy(buf, out.c_str(), out.size() + 1);
+  return rc;
 }
 
 int moe_check_status(void* stream) {

@@ -23,6 +23,16 @@ int cuda_fail(cudaError_t e, const char* what);
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Measurement hook: while profiling is enabled (moe_profile_enable), every
+// kernel launch of the library is bracketed by CUDA events on its stream.
+struct ProfScope {
+  const char* name;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr;
+  ProfScope(const char* n, cudaStream_t s);
+  ~ProfScope();
+};
+
 // Bump allocator over a caller workspace.
 struct Carve {
   char* base;

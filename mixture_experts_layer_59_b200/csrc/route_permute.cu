@@ -72,7 +72,10 @@ int launch_topk_softmax(const float* logits_in, const float* bias, float* logits
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, idx, gate);
+  {
+    ProfScope _ps("topk_softmax", s);
+    k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, idx, gate);
+  }
   MOE_CHECK_LAUNCH("topk_softmax");
   return MOE_OK;
 }
@@ -236,16 +239,25 @@ int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, in
   const int nb = perm_blocks(T);
   const size_t smem_count = (size_t)8 * E * sizeof(uint32_t);
   if (nb > 0) {
-    k_perm_count<<<nb, PERM_TOK, smem_count, s>>>(idx, T, E, k, w.blockcnt, status_ptr());
+    {
+      ProfScope _ps("perm_count", s);
+      k_perm_count<<<nb, PERM_TOK, smem_count, s>>>(idx, T, E, k, w.blockcnt, status_ptr());
+    }
     MOE_CHECK_LAUNCH("perm_count");
   }
-  k_perm_scan<<<1, 256, 0, s>>>(w.blockcnt, nb, E, tile, w.blockbase, counts, offsets, row_token,
-                                row_gate, row_slot);
+  {
+    ProfScope _ps("perm_scan", s);
+    k_perm_scan<<<1, 256, 0, s>>>(w.blockcnt, nb, E, tile, w.blockbase, counts, offsets, row_token,
+                                  row_gate, row_slot);
+  }
   MOE_CHECK_LAUNCH("perm_scan");
   if (nb > 0) {
-    k_perm_scatter<<<nb, PERM_TOK, 2 * smem_count, s>>>(idx, gate, T, E, k, w.blockbase,
-                                                        row_token, row_gate, row_slot, slot_row,
-                                                        status_ptr());
+    {
+      ProfScope _ps("perm_scatter", s);
+      k_perm_scatter<<<nb, PERM_TOK, 2 * smem_count, s>>>(idx, gate, T, E, k, w.blockbase,
+                                                          row_token, row_gate, row_slot, slot_row,
+                                                          status_ptr());
+    }
     MOE_CHECK_LAUNCH("perm_scatter");
   }
   return MOE_OK;
@@ -462,7 +474,10 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
                                 w.ex_row_token, w.ex_row_gate, w.ex_row_slot, slot_row, w, s);
   if (rc) return rc;
   if (T > 0) {
-    k_round_lse<<<(T + 255) / 256, 256, 0, s>>>(logits, idx, T, E, k, w.lse);
+    {
+      ProfScope _ps("round_lse", s);
+      k_round_lse<<<(T + 255) / 256, 256, 0, s>>>(logits, idx, T, E, k, w.lse);
+    }
     MOE_CHECK_LAUNCH("round_lse");
     cudaError_t e = cudaMemsetAsync(extra_row, 0xff, (size_t)T * E * sizeof(int32_t), s);
     if (e != cudaSuccess) return cuda_fail(e, "memset extra_row");
@@ -474,10 +489,13 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
                                          (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "round_select smem attribute");
   }
-  k_round_select<<<E, RS_THREADS, smem, s>>>(logits, w.lse, w.ex_counts, w.ex_offsets,
-                                             w.ex_row_token, w.ex_row_gate, w.ex_row_slot, T, E,
-                                             tile, counts, offsets, row_token, row_gate, row_slot,
-                                             slot_row, extra_row);
+  {
+    ProfScope _ps("round_select", s);
+    k_round_select<<<E, RS_THREADS, smem, s>>>(logits, w.lse, w.ex_counts, w.ex_offsets,
+                                               w.ex_row_token, w.ex_row_gate, w.ex_row_slot, T, E,
+                                               tile, counts, offsets, row_token, row_gate, row_slot,
+                                               slot_row, extra_row);
+  }
   MOE_CHECK_LAUNCH("round_select");
   return MOE_OK;
 }

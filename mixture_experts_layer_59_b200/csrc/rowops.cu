@@ -50,12 +50,15 @@ __global__ void k_gather_rows(const T* __restrict__ src, const int32_t* __restri
 int launch_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets, int E,
                        int width, int dtype, void* dst, cudaStream_t s) {
   const int blocks = device_sm_count() * 8;
-  if (dtype == MOE_BF16)
+  if (dtype == MOE_BF16) {
+    ProfScope _ps("gather_rows", s);
     k_gather_rows<__nv_bfloat16><<<blocks, 256, 0, s>>>(
         (const __nv_bfloat16*)src, row_token, offsets, E, width, (__nv_bfloat16*)dst);
-  else
+  } else {
+    ProfScope _ps("gather_rows", s);
     k_gather_rows<float><<<blocks, 256, 0, s>>>((const float*)src, row_token, offsets, E, width,
                                                 (float*)dst);
+  }
   MOE_CHECK_LAUNCH("gather_rows");
   return MOE_OK;
 }
@@ -138,18 +141,24 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
   if (T == 0) return MOE_OK;
   int blocks = T < device_sm_count() * 16 ? T : device_sm_count() * 16;
   if (dtype == MOE_BF16) {
-    if (out_f32)
+    if (out_f32) {
+      ProfScope _ps("token_reduce", s);
       k_token_reduce<__nv_bfloat16, float><<<blocks, 256, 0, s>>>(
           (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
           (float*)out);
-    else
+    } else {
+      ProfScope _ps("token_reduce", s);
       k_token_reduce<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(
           (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
           (__nv_bfloat16*)out);
+    }
   } else {
-    k_token_reduce<float, float><<<blocks, 256, 0, s>>>((const float*)src, row_gate, slot_row,
-                                                        extra_row, T, width, E, k, weighted,
-                                                        (float*)out);
+    {
+      ProfScope _ps("token_reduce", s);
+      k_token_reduce<float, float><<<blocks, 256, 0, s>>>((const float*)src, row_gate, slot_row,
+                                                          extra_row, T, width, E, k, weighted,
+                                                          (float*)out);
+    }
   }
   MOE_CHECK_LAUNCH("token_reduce");
   return MOE_OK;
@@ -216,8 +225,11 @@ int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, cons
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
-  k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row, T,
-                                      E, k, dlogits, dS_out);
+  {
+    ProfScope _ps("router_bwd", s);
+    k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row, T,
+                                        E, k, dlogits, dS_out);
+  }
   MOE_CHECK_LAUNCH("router_bwd");
   return MOE_OK;
 }

@@ -76,11 +76,14 @@ int launch_router_logits_simt(const void* x, const void* wg, int T, int d, int E
   (void)bias;
   if (T == 0) return MOE_OK;
   dim3 grid((T + SB - 1) / SB, (E + SB - 1) / SB);
-  if (dtype == MOE_BF16)
+  if (dtype == MOE_BF16) {
+    ProfScope _ps("router_logits", s);
     k_router_logits<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)x,
                                                         (const __nv_bfloat16*)wg, T, d, E, logits);
-  else
+  } else {
+    ProfScope _ps("router_logits", s);
     k_router_logits<float><<<grid, 256, 0, s>>>((const float*)x, (const float*)wg, T, d, E, logits);
+  }
   MOE_CHECK_LAUNCH("router_logits");
   return MOE_OK;
 }
@@ -282,11 +285,20 @@ static dim3 rows_grid(int cap, int ncols) { return dim3((cap + SB - 1) / SB, nco
 
 template <class T>
 static int ffn_fwd_t(const FfnPtrs& p, T* H, T* act, T* Y, cudaStream_t s) {
-  k_simt_up<T><<<rows_grid(p.cap, 2 * p.f), 256, 0, s>>>(p, H);
+  {
+    ProfScope _ps("simt_up", s);
+    k_simt_up<T><<<rows_grid(p.cap, 2 * p.f), 256, 0, s>>>(p, H);
+  }
   MOE_CHECK_LAUNCH("simt_up");
-  k_simt_swiglu<T><<<device_sm_count() * 8, 256, 0, s>>>(H, p.offsets, p.E, p.f, act);
+  {
+    ProfScope _ps("simt_swiglu", s);
+    k_simt_swiglu<T><<<device_sm_count() * 8, 256, 0, s>>>(H, p.offsets, p.E, p.f, act);
+  }
   MOE_CHECK_LAUNCH("simt_swiglu");
-  k_simt_down<T><<<rows_grid(p.cap, p.d), 256, 0, s>>>(p, act, Y);
+  {
+    ProfScope _ps("simt_down", s);
+    k_simt_down<T><<<rows_grid(p.cap, p.d), 256, 0, s>>>(p, act, Y);
+  }
   MOE_CHECK_LAUNCH("simt_down");
   return MOE_OK;
 }
@@ -301,16 +313,31 @@ template <class T>
 static int ffn_bwd_t(const FfnPtrs& p, const T* dout, const float* row_gate, const T* H,
                      float* dap, T* dH, T* gact, float* ds, T* dxp, T* dw1, T* dw3, T* dw2,
                      cudaStream_t s) {
-  k_simt_dap<T><<<rows_grid(p.cap, p.f), 256, 0, s>>>(p, dout, dap);
+  {
+    ProfScope _ps("simt_dap", s);
+    k_simt_dap<T><<<rows_grid(p.cap, p.f), 256, 0, s>>>(p, dout, dap);
+  }
   MOE_CHECK_LAUNCH("simt_dap");
-  k_simt_dap_epi<T><<<device_sm_count() * 8, 256, 0, s>>>(dap, H, row_gate, p.offsets, p.E, p.f,
-                                                          dH, gact, ds);
+  {
+    ProfScope _ps("simt_dap_epi", s);
+    k_simt_dap_epi<T><<<device_sm_count() * 8, 256, 0, s>>>(dap, H, row_gate, p.offsets, p.E, p.f,
+                                                            dH, gact, ds);
+  }
   MOE_CHECK_LAUNCH("simt_dap_epi");
-  k_simt_dx<T><<<rows_grid(p.cap, p.d), 256, 0, s>>>(p, dH, dxp);
+  {
+    ProfScope _ps("simt_dx", s);
+    k_simt_dx<T><<<rows_grid(p.cap, p.d), 256, 0, s>>>(p, dH, dxp);
+  }
   MOE_CHECK_LAUNCH("simt_dx");
-  k_simt_dw2<T><<<dim3(p.f / SB, p.d / SB, p.E), 256, 0, s>>>(p, dout, gact, dw2);
+  {
+    ProfScope _ps("simt_dw2", s);
+    k_simt_dw2<T><<<dim3(p.f / SB, p.d / SB, p.E), 256, 0, s>>>(p, dout, gact, dw2);
+  }
   MOE_CHECK_LAUNCH("simt_dw2");
-  k_simt_dw13<T><<<dim3(p.d / SB, 2 * p.f / SB, p.E), 256, 0, s>>>(p, dH, dw1, dw3);
+  {
+    ProfScope _ps("simt_dw13", s);
+    k_simt_dw13<T><<<dim3(p.d / SB, 2 * p.f / SB, p.E), 256, 0, s>>>(p, dH, dw1, dw3);
+  }
   MOE_CHECK_LAUNCH("simt_dw13");
   return MOE_OK;
 }
@@ -330,10 +357,16 @@ int simt_ffn_bwd(const FfnPtrs& p, const void* dout, const float* row_gate, cons
 template <class T>
 static int router_bwd_t(const T* x, const T* wg, const float* dl, const float* dx_acc, int T_,
                         int d, int E, float* dwg, T* dx, cudaStream_t s) {
-  k_simt_dwg<T><<<dim3(d / SB, (E + SB - 1) / SB), 256, 0, s>>>(x, dl, T_, d, E, dwg);
+  {
+    ProfScope _ps("simt_dwg", s);
+    k_simt_dwg<T><<<dim3(d / SB, (E + SB - 1) / SB), 256, 0, s>>>(x, dl, T_, d, E, dwg);
+  }
   MOE_CHECK_LAUNCH("simt_dwg");
   if (T_ > 0) {
-    k_simt_dx_router<T><<<dim3((T_ + SB - 1) / SB, d / SB), 256, 0, s>>>(dl, wg, dx_acc, T_, d, E, dx);
+    {
+      ProfScope _ps("simt_dx_router", s);
+      k_simt_dx_router<T><<<dim3((T_ + SB - 1) / SB, d / SB), 256, 0, s>>>(dl, wg, dx_acc, T_, d, E, dx);
+    }
     MOE_CHECK_LAUNCH("simt_dx_router");
   }
   return MOE_OK;

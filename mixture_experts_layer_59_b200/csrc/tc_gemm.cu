@@ -461,7 +461,11 @@ static int launch(const TcArgs& a, int grid, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<KIND, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return cuda_fail(e, "tc gemm smem attribute");
-  k_tc_gemm<KIND, BN><<<grid, 192, C::SMEM, s>>>(a);
+  static const char* kNames[6] = {"tc_up", "tc_down", "tc_dap", "tc_dx", "tc_dw2", "tc_dw13"};
+  {
+    ProfScope _ps(kNames[KIND], s);
+    k_tc_gemm<KIND, BN><<<grid, 192, C::SMEM, s>>>(a);
+  }
   MOE_CHECK_LAUNCH("tc_gemm");
   return MOE_OK;
 }
