@@ -122,6 +122,29 @@ int moe_permute(const int32_t* idx, const float* gate, const float* logits,
                 void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_permute_noalloc -- moe_permute without rounding, for callers that
+ * cannot allocate device memory at call time: plugin hosts that pass a
+ * kernel nothing but its input and output buffers and own every allocation,
+ * and step loops that must not call cudaMalloc between launches because it
+ * can synchronise the whole device.  The pages have no counterpart of this
+ * entry point; it computes exactly what moe_permute (round_mode
+ * MOE_ROUND_NONE) computes, with the same arguments minus logits, extra_row
+ * and the workspace.
+ *   Scratch: a static device array of 512 KiB (per-block expert counts and
+ *   bases) that every device which loads the library keeps until exit.
+ *   Limit: T <= 65536 (and E <= 256); larger T returns MOE_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address (a
+ *   one-time set-up with that device current); make that first call before
+ *   any stream capture.  Calls share the array, so calls whose kernels
+ *   overlap on the GPU (different streams or host threads) race and must be
+ *   ordered by the caller.  Nothing in it needs clearing between calls.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+int moe_permute_noalloc(const int32_t* idx, const float* gate, int T, int E, int k, int tile,
+                        int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
+                        int32_t* row_slot, int32_t* slot_row, void* stream);
+
+/*
  * moe_expert_ffn_fwd -- per-expert SwiGLU FFN on the permuted rows.
  * [Beam] sec. 2.2/5.3 (expert FFN, grouped instead of looped); [Olmo]
  * (grouped GEMM).  Experts are SwiGLU:

@@ -23,7 +23,7 @@ EXPORTS = [
     "moe_version", "moe_last_error", "moe_row_capacity", "moe_route",
     "moe_permute_workspace_size", "moe_permute", "moe_ffn_fwd_workspace_size",
     "moe_expert_ffn_fwd", "moe_combine", "moe_layer_bwd_workspace_size", "moe_layer_bwd",
-    "moe_check_status", "moe_profile_enable", "moe_profile_report",
+    "moe_check_status", "moe_profile_enable", "moe_profile_report", "moe_permute_noalloc",
 ]
 
 _lib = None
@@ -53,6 +53,7 @@ _SIGS = {
     "moe_layer_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
     "moe_profile_enable": (_i, [_i]),
+    "moe_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_profile_report": (_i, [ctypes.c_char_p, _sz]),
 }
 
@@ -232,3 +233,23 @@ def moe_profile_report() -> dict:
         name, n, ms = line.split()
         out[name] = (int(n), float(ms))
     return out
+
+
+def moe_permute_noalloc(idx, gate, E, tile=TILE, out=None, stream=None):
+    """moe_permute without rounding and without a workspace (static device
+    scratch, T <= 65536).  Output buffers are allocated here if not passed."""
+    T, k = idx.shape
+    dev = idx.device
+    cap = moe_row_capacity(T, E, k, tile)
+    o = dict(out) if out else {}
+    o.setdefault("counts", torch.empty(E, device=dev, dtype=torch.int32))
+    o.setdefault("offsets", torch.empty(E + 1, device=dev, dtype=torch.int32))
+    o.setdefault("row_token", torch.empty(cap, device=dev, dtype=torch.int32))
+    o.setdefault("row_gate", torch.empty(cap, device=dev, dtype=torch.float32))
+    o.setdefault("row_slot", torch.empty(cap, device=dev, dtype=torch.int32))
+    o.setdefault("slot_row", torch.empty(T * k, device=dev, dtype=torch.int32))
+    o.setdefault("extra_row", None)
+    _check(lib().moe_permute_noalloc(_p(idx), _p(gate), T, E, k, tile, _p(o["counts"]),
+                                     _p(o["offsets"]), _p(o["row_token"]), _p(o["row_gate"]),
+                                     _p(o["row_slot"]), _p(o["slot_row"]), _stream(stream)))
+    return o

@@ -501,3 +501,76 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
 }
 
 }  // namespace moe
+
+// ============================================================== allocation-free permute
+// Some callers cannot allocate device memory at call time: plugin hosts that
+// hand a kernel only its input and output buffers and own every allocation,
+// and step loops that must not call cudaMalloc between launches (it can
+// synchronise the whole device).  moe_permute_noalloc serves them: the exact
+// permutation with its per-block scratch (expert counts and bases of each
+// 256-token block) kept in the static array below instead of a workspace.
+//
+// Limits: T <= 65536 and E <= 256, i.e. 2 * 256 blocks * 256 experts * 4 B
+// = 512 KiB, held by every device that loads the library until exit.
+// Every call shares this array and overwrites each word it later reads, so
+// nothing needs clearing between calls; calls whose kernels overlap on the
+// GPU (other streams, other host threads) race on it and must be ordered by
+// the caller.
+namespace moe {
+namespace {
+constexpr int NOALLOC_MAX_T = 65536;
+constexpr int NOALLOC_MAX_E = 256;
+constexpr int NOALLOC_BLOCKS = NOALLOC_MAX_T / PERM_TOK;
+constexpr size_t NOALLOC_WORDS = (size_t)2 * NOALLOC_BLOCKS * NOALLOC_MAX_E;
+}  // namespace
+
+static __device__ __align__(256) int32_t g_permute_scratch[NOALLOC_WORDS];
+
+// Device address of g_permute_scratch on the current device.  The host-side
+// name of a __device__ array is only a stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+static int permute_scratch_address(int32_t** out) {
+  static int32_t* cache[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(permute scratch)");
+    cache[dev] = static_cast<int32_t*>(p);
+  }
+  *out = cache[dev];
+  return MOE_OK;
+}
+
+}  // namespace moe
+
+extern "C" int moe_permute_noalloc(const int32_t* idx, const float* gate, int T, int E, int k,
+                                   int tile, int32_t* counts, int32_t* offsets,
+                                   int32_t* row_token, float* row_gate, int32_t* row_slot,
+                                   int32_t* slot_row, void* stream) {
+  using namespace moe;
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (k < 1 || k > 8) return fail(MOE_ERR_UNSUPPORTED, "k must be in [1, 8]");
+  if (E < k || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [k, 256]");
+  if (tile != 128) return fail(MOE_ERR_UNSUPPORTED, "tile must be 128 (the grouped-GEMM M tile)");
+  if (T > NOALLOC_MAX_T)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_permute_noalloc: T = " + std::to_string(T) +
+                    " exceeds the static scratch limit of 65536 tokens; use moe_permute");
+  if (counts == nullptr || offsets == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "counts and offsets must not be NULL");
+  if (T > 0 && (idx == nullptr || gate == nullptr || row_token == nullptr ||
+                row_gate == nullptr || row_slot == nullptr || slot_row == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "idx, gate and the row maps must not be NULL");
+  int32_t* scratch = nullptr;
+  if (int rc = permute_scratch_address(&scratch)) return rc;
+  const int nb = perm_blocks(T) > 0 ? perm_blocks(T) : 1;
+  PermuteWs w{};
+  w.blockcnt = scratch;
+  w.blockbase = scratch + (size_t)nb * E;
+  return launch_permute_exact(idx, gate, T, E, k, tile, counts, offsets, row_token, row_gate,
+                              row_slot, slot_row, w, (cudaStream_t)stream);
+}
