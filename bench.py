@@ -306,7 +306,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel (measured live over the timed region)
     peaks, peak_src = load_peaks()
-    gemm = {n: v for n, v in prof.items() if n.startswith("tc_")}
+    gemm = {n: v for n, v in prof.items() if gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k)}
     kernels = {n: {"launches": v[0], "avg_us": 1e3 * v[1] / max(v[0], 1),
                    "share": v[1] / max(sum(p[1] for p in prof.values()), 1e-12)}
                for n, v in sorted(prof.items(), key=lambda kv: -kv[1][1])}

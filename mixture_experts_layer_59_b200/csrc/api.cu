@@ -132,7 +132,8 @@ struct FwdWs {
 template <class A>
 struct BwdWs {
   void *dog = nullptr, *xg = nullptr, *dH = nullptr, *gact = nullptr, *dxp = nullptr;
-  float *dap = nullptr, *ds = nullptr, *dl = nullptr, *dx_acc = nullptr;
+  float *dap = nullptr, *ds = nullptr, *dl = nullptr, *dx_acc = nullptr, *dwg_part = nullptr;
+  void *dl_hi = nullptr, *dl_lo = nullptr;
   int nparts = 1;
   void carve(A& a, int T, int d, int f, int E, int k, int dtype) {
     const size_t cap = (size_t)T * k + (size_t)E * 128;
@@ -151,6 +152,13 @@ struct BwdWs {
     ds = a.template take<float>(cap * nparts);
     dl = a.template take<float>((size_t)T * E + 1);
     dx_acc = a.template take<float>((size_t)T * d + 1);
+    if (tc && tc_router_ok(E)) {
+      int chunk = 0;
+      const int splits = tc_dwg_splits(T, d, &chunk);
+      dl_hi = a.template take<uint16_t>((size_t)T * E + 8);
+      dl_lo = a.template take<uint16_t>((size_t)T * E + 8);
+      dwg_part = a.template take<float>((size_t)splits * d * E);
+    }
   }
 };
 
@@ -183,6 +191,13 @@ int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int
     REQUIRE_PTR(x);
     REQUIRE_PTR(w_gate);
     if (d <= 0) return fail(MOE_ERR_INVALID_ARG, "d must be > 0");
+    if (dtype == MOE_BF16 && d % 64 == 0 && tc_router_ok(E)) {
+      // tensor-core router GEMM with the bias, top-k and softmax in its epilogue
+      REQUIRE_ALIGNED(x);
+      REQUIRE_ALIGNED(w_gate);
+      return tc_router_fwd(x, w_gate, logit_bias, T, d, E, k, logits, idx, gate,
+                           device_sm_count(), s);
+    }
     if (int rc = launch_router_logits_simt(x, w_gate, T, d, E, dtype, nullptr, logits, s)) return rc;
     src = logits;
   }
@@ -319,9 +334,25 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
       return rc;
   }
   float* dl = dlogits ? dlogits : w.dl;
+  const bool tc_router = router_grad && w.dl_hi != nullptr;
   if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row, T, E, k,
-                              dl, dS, s)))
+                              dl, dS, tc_router ? w.dl_hi : nullptr,
+                              tc_router ? w.dl_lo : nullptr, s)))
     return rc;
+  if (tc_router) {
+    // dW_gate and the router term of dx on the tensor cores; the unpermute-sum
+    // of dX_perm is fused into the dx epilogue (rows of added pairs, present
+    // only with token rounding, go through an fp32 row sum first)
+    const float* acc = nullptr;
+    if (extra_row != nullptr) {
+      if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype,
+                                    false, true, w.dx_acc, s)))
+        return rc;
+      acc = w.dx_acc;
+    }
+    return tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate, w.dxp,
+                         slot_row, acc, dx, device_sm_count(), s);
+  }
   if (router_grad) {
     if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
                                   true, w.dx_acc, s)))

@@ -44,9 +44,11 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
                         const int32_t* extra_row, int T, int width, int E, int k, int dtype,
                         bool weighted, bool out_f32, void* out, cudaStream_t s);
 // dlogits and (optionally) the final dS rows from dS partials [cap, nparts].
+// Optionally also writes dlogits split as bf16 hi + bf16 lo (tensor-core router GEMMs).
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      int T, int E, int k, float* dlogits, float* dS_out, cudaStream_t s);
+                      int T, int E, int k, float* dlogits, float* dS_out, void* dl_hi,
+                      void* dl_lo, cudaStream_t s);
 
 // ---------------------------------------------------------------- CUDA-core GEMM path
 struct FfnPtrs {
@@ -69,6 +71,14 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
                const void* H, void* dH, void* gact, float* ds_part, void* dXp, void* dw1,
                void* dw3, void* dw2, int num_sms, cudaStream_t s);
 int tc_num_dS_parts(int f);
+bool tc_router_ok(int E);
+int tc_dwg_splits(int T, int d, int* chunk);
+int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
+                  float* logits, int32_t* idx, float* gate, int num_sms, cudaStream_t s);
+int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
+                  int d, int E, int k, float* dwg_part, float* dw_gate, const void* dxp,
+                  const int32_t* slot_row, const float* dx_acc, void* dx, int num_sms,
+                  cudaStream_t s);
 
 int device_sm_count();
 

@@ -63,75 +63,74 @@ int launch_gather_rows(const void* src, const int32_t* row_token, const int32_t*
   return MOE_OK;
 }
 
-// ============================================================== token rows
-// Rows of token t: kept slots in slot order, then rows added by token
-// rounding in ascending expert id.  Built in shared memory by one block.
-// Returns the count; rows[] and (optionally) wts[] are filled.
-__device__ int token_row_list(int t, const int32_t* __restrict__ slot_row,
-                              const int32_t* __restrict__ extra_row, const float* __restrict__ row_gate,
-                              int E, int k, int* rows, float* wts, int* s_cnt) {
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j < k; ++j) {
-      int r = slot_row[(size_t)t * k + j];
-      if (r >= 0) rows[n++] = r;
-    }
-    *s_cnt = n;
-  }
-  __syncthreads();
-  int n = *s_cnt;
-  if (extra_row != nullptr) {
-    // ordered compaction of extra_row[t, 0..E) over the first E threads
-    __shared__ int s_wc[8];
-    const int e = threadIdx.x;
-    const int r = (e < E) ? extra_row[(size_t)t * E + e] : -1;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const unsigned bal = __ballot_sync(0xffffffffu, r >= 0);
-    if (lane == 0 && w < 8) s_wc[w] = __popc(bal);
-    __syncthreads();
-    int base = n;
-    for (int i = 0; i < w && i < 8; ++i) base += s_wc[i];
-    if (r >= 0 && e < E) rows[base + __popc(bal & ((1u << lane) - 1u))] = r;
-    int tot = 0;
-    for (int i = 0; i < 8; ++i) tot += s_wc[i];
-    n += tot;
-    __syncthreads();
-  }
-  if (wts != nullptr)
-    for (int i = threadIdx.x; i < n; i += blockDim.x) wts[i] = row_gate[rows[i]];
-  __syncthreads();
-  return n;
-}
+// out[t, :] = sum_rows (weighted ? row_gate[r] : 1) * src[r, :].
+// One warp per token: the warp first lists the token's rows in shared memory
+// (kept slots in slot order, then added rows by ascending expert), then each
+// lane sums 16-byte vectors of up to 8 rows at a time, issuing the loads of
+// all those rows before accumulating, in fixed row order.
+constexpr int TR_WARPS = 8;
 
-// out[t, :] = sum_rows (weighted ? row_gate[r] : 1) * src[r, :]; one block per token.
 template <class T, class OutT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(TR_WARPS * 32)
 k_token_reduce(const T* __restrict__ src, const float* __restrict__ row_gate,
                const int32_t* __restrict__ slot_row, const int32_t* __restrict__ extra_row,
                int T_, int width, int E, int k, bool weighted, OutT* __restrict__ out) {
-  __shared__ int rows[8 + 256];
-  __shared__ float wts[8 + 256];
-  __shared__ int s_cnt;
+  __shared__ int s_rows[TR_WARPS][8 + 256];
+  __shared__ float s_wts[TR_WARPS][8 + 256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int* rows = s_rows[w];
+  float* wts = s_wts[w];
   const int nvec = width / Vec<T>::N;
-  for (int t = blockIdx.x; t < T_; t += gridDim.x) {
-    const int n = token_row_list(t, slot_row, extra_row, row_gate, E, k, rows,
-                                 weighted ? wts : nullptr, &s_cnt);
-    for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+  for (int t = blockIdx.x * TR_WARPS + w; t < T_; t += gridDim.x * TR_WARPS) {
+    // kept slots: ordered compaction of slot_row[t, 0..k)
+    const int rs = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    unsigned bal = __ballot_sync(0xffffffffu, rs >= 0);
+    int n = __popc(bal);
+    if (rs >= 0) rows[__popc(bal & ((1u << lane) - 1u))] = rs;
+    if (extra_row != nullptr) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int re = (e0 + lane < E) ? extra_row[(size_t)t * E + e0 + lane] : -1;
+        bal = __ballot_sync(0xffffffffu, re >= 0);
+        if (re >= 0) rows[n + __popc(bal & ((1u << lane) - 1u))] = re;
+        n += __popc(bal);
+      }
+    }
+    __syncwarp();
+    if (weighted)
+      for (int j = lane; j < n; j += 32) wts[j] = row_gate[rows[j]];
+    __syncwarp();
+    for (int i = lane; i < nvec; i += 32) {
       float acc[Vec<T>::N];
 #pragma unroll
       for (int q = 0; q < Vec<T>::N; ++q) acc[q] = 0.f;
-      for (int j = 0; j < n; ++j) {
-        Vec<T> v;
-        v.v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)rows[j] * width) + i);
-        const float w = weighted ? wts[j] : 1.0f;
+      for (int j0 = 0; j0 < n; j0 += 8) {
+        Vec<T> v[8];
 #pragma unroll
-        for (int q = 0; q < Vec<T>::N; ++q) acc[q] = fmaf(w, v.get(q), acc[q]);
+        for (int j = 0; j < 8; ++j)
+          if (j0 + j < n)
+            v[j].v = __ldg(reinterpret_cast<const uint4*>(src + (size_t)rows[j0 + j] * width) + i);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j0 + j < n) {
+            const float wt = weighted ? wts[j0 + j] : 1.0f;
+#pragma unroll
+            for (int q = 0; q < Vec<T>::N; ++q) acc[q] = fmaf(wt, v[j].get(q), acc[q]);
+          }
+        }
       }
       OutT* o = out + (size_t)t * width + (size_t)i * Vec<T>::N;
+      if constexpr (sizeof(OutT) == 2) {
+        Vec<T> r;
 #pragma unroll
-      for (int q = 0; q < Vec<T>::N; ++q) o[q] = from_f<OutT>(acc[q]);
+        for (int q = 0; q < Vec<T>::N; ++q) r.set(q, acc[q]);
+        *reinterpret_cast<uint4*>(o) = r.v;
+      } else {
+#pragma unroll
+        for (int q = 0; q < Vec<T>::N; q += 4)
+          *reinterpret_cast<float4*>(o + q) = make_float4(acc[q], acc[q + 1], acc[q + 2], acc[q + 3]);
+      }
     }
-    __syncthreads();
+    __syncwarp();
   }
 }
 
@@ -139,23 +138,24 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
                         const int32_t* extra_row, int T, int width, int E, int k, int dtype,
                         bool weighted, bool out_f32, void* out, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  int blocks = T < device_sm_count() * 16 ? T : device_sm_count() * 16;
+  int blocks = (T + TR_WARPS - 1) / TR_WARPS;
+  if (blocks > device_sm_count() * 32) blocks = device_sm_count() * 32;
   if (dtype == MOE_BF16) {
     if (out_f32) {
       ProfScope _ps("token_reduce", s);
-      k_token_reduce<__nv_bfloat16, float><<<blocks, 256, 0, s>>>(
+      k_token_reduce<__nv_bfloat16, float><<<blocks, TR_WARPS * 32, 0, s>>>(
           (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
           (float*)out);
     } else {
       ProfScope _ps("token_reduce", s);
-      k_token_reduce<__nv_bfloat16, __nv_bfloat16><<<blocks, 256, 0, s>>>(
+      k_token_reduce<__nv_bfloat16, __nv_bfloat16><<<blocks, TR_WARPS * 32, 0, s>>>(
           (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
           (__nv_bfloat16*)out);
     }
   } else {
     {
       ProfScope _ps("token_reduce", s);
-      k_token_reduce<float, float><<<blocks, 256, 0, s>>>((const float*)src, row_gate, slot_row,
+      k_token_reduce<float, float><<<blocks, TR_WARPS * 32, 0, s>>>((const float*)src, row_gate, slot_row,
                                                           extra_row, T, width, E, k, weighted,
                                                           (float*)out);
     }
@@ -172,7 +172,8 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
                              const int32_t* __restrict__ idx, const float* __restrict__ gate,
                              const float* __restrict__ row_gate, const int32_t* __restrict__ slot_row,
                              const int32_t* __restrict__ extra_row, int T, int E, int k,
-                             float* __restrict__ dlogits, float* __restrict__ dS_out) {
+                             float* __restrict__ dlogits, float* __restrict__ dS_out,
+                             __nv_bfloat16* __restrict__ dl_hi, __nv_bfloat16* __restrict__ dl_lo) {
   __shared__ float s_dl[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float* dl = s_dl[w];
@@ -214,21 +215,32 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
       dl[e] -= gate[(size_t)t * k + lane] * part;
     }
     __syncwarp();
-    for (int e = lane; e < E; e += 32) dlogits[(size_t)t * E + e] = dl[e];
+    for (int e = lane; e < E; e += 32) {
+      const float v = dl[e];
+      dlogits[(size_t)t * E + e] = v;
+      if (dl_hi != nullptr) {
+        // v = hi + lo with hi = bf16(v), lo = bf16(v - hi): ~16 significant bits
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        dl_hi[(size_t)t * E + e] = h;
+        dl_lo[(size_t)t * E + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+      }
+    }
     __syncwarp();
   }
 }
 
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      int T, int E, int k, float* dlogits, float* dS_out, cudaStream_t s) {
+                      int T, int E, int k, float* dlogits, float* dS_out, void* dl_hi,
+                      void* dl_lo, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
   {
     ProfScope _ps("router_bwd", s);
     k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row, T,
-                                        E, k, dlogits, dS_out);
+                                        E, k, dlogits, dS_out, (__nv_bfloat16*)dl_hi,
+                                        (__nv_bfloat16*)dl_lo);
   }
   MOE_CHECK_LAUNCH("router_bwd");
   return MOE_OK;

@@ -13,15 +13,24 @@
 //   DX    dXp = dH [W1_e | W3_e]^T   varlen-M, K = 2f
 //   DW2   dW2_e = (sA)^T dOg         varlen-K (K = rows of e)
 //   DW13  [dW1_e | dW3_e] = Xg^T dH  varlen-K
+//   RT    logits = x W_gate (+bias)  one group, N = E padded to 64; epilogue:
+//                                    top-k (ties: lowest id) and softmax over
+//                                    the k logits (Beam sec. 5.3 / Trinity ex. 1)
+//   DWG   dW_gate = x^T dlogits      split-K over tokens; dlogits enters as a
+//                                    bf16 hi part plus a bf16 lo remainder,
+//                                    accumulated in the same fp32 accumulator
+//   DXR   dx = sum of the token's dX_perm rows + dlogits W_gate^T
+//                                    (router term and unpermute-sum fused)
 // The grouped GEMM replaces the per-expert loop of the Beam article's
 // MoELayer (sec. 5.3); Olmo-core 3 names grouped GEMM for the same purpose;
 // dS = <dA', A> without a stored Y is the SonicMoE summary's sec. 1.
 //
-// CTA layout (192 threads, one CTA per SM):
+// CTA layout (320 threads, one CTA per SM):
 //   warp 0      TMA producer (one lane): A and B tiles into a ring of stages
 //   warp 1      TMEM allocator + MMA issuer (one lane): 128 x BN x 16 UMMAs
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, fused math,
-//               16-byte global stores
+//   warps 2..9  epilogue: tcgen05.ld of the fp32 accumulator, fused math,
+//               16-byte global stores.  Warp w reads TMEM lanes 32*(w%4)..+31
+//               (the rows it may access); warps w and w+4 split the columns.
 // The accumulator is double-buffered in TMEM (2 x BN columns) so that the
 // epilogue of tile i overlaps the main loop of tile i+1.  Tiles are assigned
 // round-robin to the CTAs; the row count R and the per-expert segments are
@@ -38,18 +47,29 @@ namespace moe {
 
 using namespace tc;
 
-enum Kind : int { K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5 };
+enum Kind : int {
+  K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8
+};
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
 constexpr int ATOM = 8192;             // one 64 x 64 bf16 TMA box
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
+constexpr int THREADS = 320;           // 2 control warps + 8 epilogue warps
+constexpr int EPI_THREADS = 256;
+
+// Sigmoid for the tensor-core epilogues (fast exponential and division; the
+// results are rounded to bf16 afterwards).
+__device__ __forceinline__ float sigmoid_fast(float z) {
+  return __fdividef(1.0f, 1.0f + __expf(-z));
+}
 
 struct TcArgs {
   CUtensorMap mA;    // A operand
-  CUtensorMap mB0;   // B operand (W1 / W2 / activation)
-  CUtensorMap mB1;   // second B source (W3) where the kind has one
+  CUtensorMap mA1;   // second A source (DXR: dlogits lo part)
+  CUtensorMap mB0;   // B operand (W1 / W2 / activation / W_gate / dlogits hi)
+  CUtensorMap mB1;   // second B source (W3, dlogits lo) where the kind has one
   const int32_t* offsets;
   int E, d, f;
   int M, N, K;       // varlen-M: N, K fixed; varlen-K: M, N fixed
@@ -62,18 +82,31 @@ struct TcArgs {
   float* ds_part;            // DAP: [cap, nparts]
   int nparts;
   int* status;
+  // router kinds
+  int T, k, splits, chunk;
+  const float* bias;         // RT: [E] or null
+  float* logits;             // RT: [T, E]
+  int32_t* idx;              // RT: [T, k]
+  float* gate;               // RT: [T, k]
+  float* dwg_part;           // DWG: [splits, d, E]
+  const __nv_bfloat16* dxp;  // DXR: [cap, d]
+  const int32_t* slot_row;   // DXR: [T, k]
+  const float* dx_acc;       // DXR: [T, d] fp32 row sums (used instead of dxp when set)
+  __nv_bfloat16* dx;         // DXR: [T, d]
 };
 
 template <int KIND> struct KT {
   static constexpr bool VARLEN_K = (KIND == K_DW2 || KIND == K_DW13);
-  static constexpr bool A_MN = VARLEN_K;
-  static constexpr bool B_MN = (KIND == K_UP || KIND == K_DOWN || VARLEN_K);
+  static constexpr bool A_MN = VARLEN_K || KIND == K_DWG;
+  static constexpr bool B_MN = (KIND == K_UP || KIND == K_DOWN || VARLEN_K || KIND == K_RT ||
+                                KIND == K_DWG);
+  static constexpr bool ROUTER = (KIND == K_RT || KIND == K_DWG || KIND == K_DXR);
 };
 
 template <int BN> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int SMEM = STAGES * STAGE + 1024;
   static constexpr int TMEM_COLS = 2 * BN;
 };
@@ -87,7 +120,32 @@ __device__ __forceinline__ bool tile_info(int t, const TcArgs& a, const int* s_o
                                           TileInfo& ti) {
   if (t >= total) return false;
   const int ntiles = a.N / BN;
-  if constexpr (KT<KIND>::VARLEN_K) {
+  if constexpr (KIND == K_RT) {
+    ti.e = 0;
+    ti.m0 = t * BM;
+    ti.ntile = 0;
+    ti.n0 = 0;
+    ti.krow0 = 0;
+    ti.kb_count = a.K / BK;
+  } else if constexpr (KIND == K_DWG) {
+    const int mtiles = a.M / BM;
+    const int sp = t / mtiles;          // split of the token range
+    ti.e = sp;
+    ti.m0 = (t - sp * mtiles) * BM;
+    ti.ntile = 0;
+    ti.n0 = 0;
+    ti.krow0 = sp * a.chunk;
+    const int rows = min(a.chunk, a.T - ti.krow0);
+    ti.kb_count = 2 * ((rows + BK - 1) / BK);   // hi pass, then lo pass
+  } else if constexpr (KIND == K_DXR) {
+    const int mt = t / ntiles;
+    ti.e = 0;
+    ti.ntile = t - mt * ntiles;
+    ti.m0 = mt * BM;
+    ti.n0 = ti.ntile * BN;
+    ti.krow0 = 0;
+    ti.kb_count = 2 * ((a.E + BK - 1) / BK);    // hi pass, then lo pass
+  } else if constexpr (KT<KIND>::VARLEN_K) {
     const int per = (a.M / BM) * ntiles;
     ti.e = t / per;
     const int rem = t - ti.e * per;
@@ -160,7 +218,7 @@ __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
 }
 
 template <int KIND, int BN>
-__global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ TcArgs a) {
   using C = Cfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
@@ -174,7 +232,8 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_off[i] = a.offsets[i];
+  if (a.offsets != nullptr)
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_off[i] = a.offsets[i];
   if (threadIdx.x == 0) {
     s_abort = 0;
     for (int s = 0; s < C::STAGES; ++s) {
@@ -183,12 +242,13 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&tfull_bar[s], 1);
-      mbar_init(&tempty_bar[s], 128);
+      mbar_init(&tempty_bar[s], EPI_THREADS);
     }
     fence_mbar_init();
     prefetch_tmap(&a.mA);
     prefetch_tmap(&a.mB0);
-    if (KIND == K_UP || KIND == K_DX) prefetch_tmap(&a.mB1);
+    if (KIND == K_UP || KIND == K_DX || KIND == K_DWG) prefetch_tmap(&a.mB1);
+    if (KIND == K_DXR) prefetch_tmap(&a.mA1);
   }
   if (warp == 1) {
     tmem_alloc(&s_tmem, C::TMEM_COLS);
@@ -200,7 +260,10 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
   const uint32_t tmem_base = s_tmem;
 
   int total;
-  if constexpr (KT<KIND>::VARLEN_K) total = a.E * (a.M / BM) * (a.N / BN);
+  if constexpr (KIND == K_RT) total = (a.T + BM - 1) / BM;
+  else if constexpr (KIND == K_DWG) total = (a.M / BM) * a.splits;
+  else if constexpr (KIND == K_DXR) total = ((a.T + BM - 1) / BM) * (a.N / BN);
+  else if constexpr (KT<KIND>::VARLEN_K) total = a.E * (a.M / BM) * (a.N / BN);
   else total = (s_off[a.E] / BM) * (a.N / BN);
 
   if (warp == 0) {
@@ -236,6 +299,27 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
             if (k0 < a.f) tma_load_3d(sB, &a.mB0, &full_bar[stage], k0, ti.n0, ti.e);
             else tma_load_3d(sB, &a.mB1, &full_bar[stage], k0 - a.f, ti.n0, ti.e);
+          } else if constexpr (KIND == K_RT) {
+            tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h)
+              tma_load_2d(sB + h * ATOM, &a.mB0, &full_bar[stage], 64 * h, k0);
+          } else if constexpr (KIND == K_DWG) {
+            const int nkb = ti.kb_count / 2;
+            const int pass = kb >= nkb;
+            const int r = ti.krow0 + (kb - pass * nkb) * BK;
+            tma_load_2d(sA, &a.mA, &full_bar[stage], ti.m0, r);
+            tma_load_2d(sA + ATOM, &a.mA, &full_bar[stage], ti.m0 + 64, r);
+            const CUtensorMap* mb = pass ? &a.mB1 : &a.mB0;
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h)
+              tma_load_2d(sB + h * ATOM, mb, &full_bar[stage], 64 * h, r);
+          } else if constexpr (KIND == K_DXR) {
+            const int nkb = ti.kb_count / 2;
+            const int pass = kb >= nkb;
+            const int kk = (kb - pass * nkb) * BK;
+            tma_load_2d(sA, pass ? &a.mA1 : &a.mA, &full_bar[stage], kk, ti.m0);
+            tma_load_2d(sB, &a.mB0, &full_bar[stage], kk, ti.n0);
           } else {  // varlen-K: A and B are row-space activations, MN-major
             const int r = ti.krow0 + k0;
             tma_load_2d(sA, &a.mA, &full_bar[stage], ti.m0, r);
@@ -287,6 +371,7 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                      // TMEM lane quarter of this warp
+    const int half = (warp - 2) >> 2;            // which half of the tile's columns
     const int rloc = q * 32 + lane;              // row of the tile owned by this thread
     int it = 0;
     TileInfo ti;
@@ -302,7 +387,7 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
       if constexpr (KIND == K_UP) {
         const int f = a.f, nf = ti.ntile * (BN / 2);
         float h3[32];
-        for (int c = 0; c < BN / 2; c += 32) {
+        for (int c = half * (BN / 4); c < (half + 1) * (BN / 4); c += 32) {
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
 #pragma unroll
@@ -315,11 +400,14 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
           st_bf16x32(hrow + nf + c, v);
           st_bf16x32(hrow + f + nf + c, h3);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = silu_f(bf16_round(v[i])) * bf16_round(h3[i]);
+          for (int i = 0; i < 32; ++i) {
+            const float h1 = bf16_round(v[i]);
+            v[i] = h1 * sigmoid_fast(h1) * bf16_round(h3[i]);
+          }
           st_bf16x32(a.out1 + (size_t)row * f + nf + c, v);
         }
       } else if constexpr (KIND == K_DOWN || KIND == K_DX) {
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
 #pragma unroll
@@ -331,7 +419,7 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
         const float g = a.row_gate[row];
         float ds = 0.f;
         float h1[32], h3[32];
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           tmem_ld32(tbase + c, r);
           const __nv_bfloat16* hrow = a.hin + (size_t)row * 2 * f;
           ld_bf16x32(hrow + ti.n0 + c, h1);
@@ -341,7 +429,7 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float dap = __uint_as_float(r[i]);
-            const float sg = sigmoid_f(h1[i]);
+            const float sg = sigmoid_fast(h1[i]);
             const float sl = h1[i] * sg;
             const float av = bf16_round(sl * h3[i]);
             ds = fmaf(dap, av, ds);
@@ -355,10 +443,93 @@ __global__ void __launch_bounds__(192, 1) k_tc_gemm(const __grid_constant__ TcAr
           st_bf16x32(drow + f + ti.n0 + c, da3);
           st_bf16x32(a.out2 + (size_t)row * f + ti.n0 + c, ga);
         }
-        a.ds_part[(size_t)row * a.nparts + ti.ntile] = ds;
+        a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
+      } else if constexpr (KIND == K_RT) {
+        const int t = row;
+        const bool valid = t < a.T && half == 0;
+        float tv[8];
+        int tix[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; tix[j] = 0x7fffffff; }
+        for (int c = 0; half == 0 && c < a.E; c += 32) {
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int e = c + i;
+            if (e < a.E) {
+              float l = __uint_as_float(r[i]);
+              if (a.bias) l += a.bias[e];
+              if (valid) a.logits[(size_t)t * a.E + e] = l;
+              // insertion into the descending top-k list; equal values keep
+              // the lower expert id first because ids arrive in ascending order
+              if (l > tv[a.k - 1]) {
+                int j = a.k - 1;
+                while (j > 0 && l > tv[j - 1]) { tv[j] = tv[j - 1]; tix[j] = tix[j - 1]; --j; }
+                tv[j] = l;
+                tix[j] = e;
+              }
+            }
+          }
+        }
+        if (valid) {
+          const float m = tv[0];
+          float z = 0.f, ex[8];
+          for (int j = 0; j < a.k; ++j) { ex[j] = expf(tv[j] - m); z += ex[j]; }
+          const float inv = 1.0f / z;
+          for (int j = 0; j < a.k; ++j) {
+            a.idx[(size_t)t * a.k + j] = tix[j];
+            a.gate[(size_t)t * a.k + j] = ex[j] * inv;
+          }
+        }
+      } else if constexpr (KIND == K_DWG) {
+        // row = d index; partial sums of split ti.e
+        float* dst = a.dwg_part + ((size_t)ti.e * a.M + row) * a.E;
+        for (int c = half * (BN / 2); c < a.E && c < (half + 1) * (BN / 2); c += 32) {
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c + i < a.E) dst[c + i] = __uint_as_float(r[i]);
+        }
+      } else if constexpr (KIND == K_DXR) {
+        const int t = row;
+        const bool valid = t < a.T;
+        int rows8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          rows8[j] = (valid && a.dx_acc == nullptr && j < a.k) ? a.slot_row[(size_t)t * a.k + j] : -1;
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+          tmem_ld32(tbase + c, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          if (valid) {
+            const int col = ti.n0 + c;
+            if (a.dx_acc != nullptr) {
+              const float4* s4 = reinterpret_cast<const float4*>(a.dx_acc + (size_t)t * a.N + col);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 u = s4[q];
+                v[4 * q] += u.x; v[4 * q + 1] += u.y; v[4 * q + 2] += u.z; v[4 * q + 3] += u.w;
+              }
+            } else {
+              float h[32];
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (rows8[j] >= 0) {
+                  ld_bf16x32(a.dxp + (size_t)rows8[j] * a.N + col, h);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) v[i] += h[i];
+                }
+              }
+            }
+            st_bf16x32(a.dx + (size_t)t * a.N + col, v);
+          }
+        }
       } else {  // DW2 / DW13: output row m = row of dW_e
         const size_t ebase = (size_t)ti.e * a.M * (KIND == K_DW2 ? a.N : a.f);
-        for (int c = 0; c < BN; c += 32) {
+        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           if (ti.kb_count > 0) {
             tmem_ld32(tbase + c, r);
             tmem_ld_wait();
@@ -421,7 +592,8 @@ bool tc_available() {
   return major == 10;
 }
 
-int tc_num_dS_parts(int f) { return (f % 256 == 0) ? f / 256 : f / 128; }
+// dS partial sums per row: one per N tile of the DAP GEMM and column half.
+int tc_num_dS_parts(int f) { return 2 * ((f % 256 == 0) ? f / 256 : f / 128); }
 
 // bf16 row-major [outer, inner] viewed in boxes of box_outer x box_inner.
 static int make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
@@ -461,10 +633,12 @@ static int launch(const TcArgs& a, int grid, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<KIND, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return cuda_fail(e, "tc gemm smem attribute");
-  static const char* kNames[6] = {"tc_up", "tc_down", "tc_dap", "tc_dx", "tc_dw2", "tc_dw13"};
+  static const char* kNames[9] = {"tc_up",   "tc_down",   "tc_dap",      "tc_dx",    "tc_dw2",
+                                  "tc_dw13", "tc_router", "tc_router_dw", "tc_dx_router"};
+  static_assert(KIND >= 0 && KIND < 9, "kind out of range");
   {
     ProfScope _ps(kNames[KIND], s);
-    k_tc_gemm<KIND, BN><<<grid, 192, C::SMEM, s>>>(a);
+    k_tc_gemm<KIND, BN><<<grid, THREADS, C::SMEM, s>>>(a);
   }
   MOE_CHECK_LAUNCH("tc_gemm");
   return MOE_OK;
@@ -473,8 +647,12 @@ static int launch(const TcArgs& a, int grid, cudaStream_t s) {
 template <int KIND>
 static int launch_bn(const TcArgs& a, int bn, int grid, cudaStream_t s) {
   if (bn == 256) return launch<KIND, 256>(a, grid, s);
+  if (bn == 64) return launch<KIND, 64>(a, grid, s);
   return launch<KIND, 128>(a, grid, s);
 }
+
+// N tile covering E router columns: 64, 128 or 256.
+static int router_bn(int E) { return E <= 64 ? 64 : (E <= 128 ? 128 : 256); }
 
 static int pick_bn(int n) { return n % 256 == 0 ? 256 : 128; }
 
@@ -487,6 +665,102 @@ static TcArgs base_args(const FfnPtrs& p) {
   a.f = p.f;
   a.status = status_ptr();
   return a;
+}
+
+// ------------------------------------------------------------ router
+bool tc_router_ok(int E) { return E % 8 == 0 && E <= 256 && tc_available(); }
+
+int tc_dwg_splits(int T, int d, int* chunk) {
+  const int mtiles = d / BM;
+  int splits = (160 + mtiles - 1) / mtiles;
+  const int max_splits = (T + BK - 1) / BK;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int c = (T + splits - 1) / splits;
+  c = (c + BK - 1) / BK * BK;
+  if (c < BK) c = BK;
+  *chunk = c;
+  return (T + c - 1) / c > 0 ? (T + c - 1) / c : 1;
+}
+
+int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
+                  float* logits, int32_t* idx, float* gate, int num_sms, cudaStream_t s) {
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.E = E;
+  a.d = d;
+  a.K = d;
+  a.N = router_bn(E);
+  a.T = T;
+  a.k = k;
+  a.bias = bias;
+  a.logits = logits;
+  a.idx = idx;
+  a.gate = gate;
+  a.status = status_ptr();
+  int rc;
+  if ((rc = make_map_2d(&a.mA, x, d, T, 64, BM))) return rc;
+  if ((rc = make_map_2d(&a.mB0, wg, E, d, 64, 64))) return rc;
+  const int tiles = (T + BM - 1) / BM;
+  return launch_bn<K_RT>(a, a.N, tiles < num_sms ? tiles : num_sms, s);
+}
+
+__global__ void k_dwg_reduce(const float* __restrict__ part, int splits, int n,
+                             float* __restrict__ out) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int sp = 0; sp < splits; ++sp) acc += part[(size_t)sp * n + i];
+    out[i] = acc;
+  }
+}
+
+int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
+                  int d, int E, int k, float* dwg_part, float* dw_gate, const void* dxp,
+                  const int32_t* slot_row, const float* dx_acc, void* dx, int num_sms,
+                  cudaStream_t s) {
+  int rc;
+  {  // dW_gate = x^T (dl_hi + dl_lo), split over tokens, then a fixed-order sum
+    TcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.E = E;
+    a.d = d;
+    a.M = d;
+    a.N = router_bn(E);
+    a.T = T;
+    a.status = status_ptr();
+    a.splits = tc_dwg_splits(T, d, &a.chunk);
+    a.dwg_part = dwg_part;
+    if ((rc = make_map_2d(&a.mA, x, d, T, 64, 64))) return rc;
+    if ((rc = make_map_2d(&a.mB0, dl_hi, E, T, 64, 64))) return rc;
+    if ((rc = make_map_2d(&a.mB1, dl_lo, E, T, 64, 64))) return rc;
+    const int tiles = (d / BM) * a.splits;
+    if ((rc = launch_bn<K_DWG>(a, a.N, tiles < num_sms ? tiles : num_sms, s))) return rc;
+    {
+      ProfScope _ps("dwg_reduce", s);
+      k_dwg_reduce<<<num_sms * 4, 256, 0, s>>>(dwg_part, a.splits, d * E, dw_gate);
+    }
+    MOE_CHECK_LAUNCH("dwg_reduce");
+  }
+  {  // dx = unpermute-sum of dX_perm (or the fp32 row sums) + dl W_gate^T
+    TcArgs a;
+    memset(&a, 0, sizeof(a));
+    a.E = E;
+    a.d = d;
+    a.N = d;
+    a.T = T;
+    a.k = k;
+    a.status = status_ptr();
+    a.dxp = (const __nv_bfloat16*)dxp;
+    a.slot_row = slot_row;
+    a.dx_acc = dx_acc;
+    a.dx = (__nv_bfloat16*)dx;
+    const int bn = pick_bn(d);
+    if ((rc = make_map_2d(&a.mA, dl_hi, E, T, 64, BM))) return rc;
+    if ((rc = make_map_2d(&a.mA1, dl_lo, E, T, 64, BM))) return rc;
+    if ((rc = make_map_2d(&a.mB0, wg, E, d, 64, bn))) return rc;
+    if ((rc = launch_bn<K_DXR>(a, bn, num_sms, s))) return rc;
+  }
+  return MOE_OK;
 }
 
 int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, int num_sms,
@@ -534,7 +808,7 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     a.out1 = (__nv_bfloat16*)dH;
     a.out2 = (__nv_bfloat16*)gact;
     a.ds_part = ds_part;
-    a.nparts = f / bn;
+    a.nparts = 2 * (f / bn);
     if (a.nparts != tc_num_dS_parts(f)) return fail(MOE_ERR_UNSUPPORTED, "dS partition mismatch");
     if ((rc = launch_bn<K_DAP>(a, bn, num_sms, s))) return rc;
   }
