@@ -297,12 +297,14 @@ def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
     """Forward (and, given dout, backward) quantities of the listed rows.
 
     Rows are grouped by the expert that owns them; padding rows give zeros.
+    w1, w3, w2 may be arrays or any object whose [e] gives expert e's matrix
+    (weights are read one expert at a time).
     Returns a dict of arrays aligned with ``rows``: H [n,2f], A [n,f],
     Y [n,d] and, with dout, dS [n], dH [n,2f], gA [n,f], dXp [n,d].
     """
     rows = np.asarray(rows, np.int64)
-    x, w1, w3, w2 = map(_f64, (x, w1, w3, w2))
-    n, d, f = len(rows), x.shape[1], w1.shape[2]
+    x = _f64(x)
+    n, d, f = len(rows), x.shape[1], np.shape(w1[0])[1]
     res = dict(H=np.zeros((n, 2 * f)), A=np.zeros((n, f)), Y=np.zeros((n, d)))
     if dout is not None:
         dout = _f64(dout)
@@ -313,12 +315,13 @@ def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
     for e in np.unique(es[toks_all >= 0]):
         sel = np.nonzero((es == e) & (toks_all >= 0))[0]
         toks = toks_all[sel]
-        h1, h3, a, y = expert_rows_forward(x[toks], w1[e], w3[e], w2[e], staged)
+        w1e, w3e, w2e = _f64(w1[e]), _f64(w3[e]), _f64(w2[e])
+        h1, h3, a, y = expert_rows_forward(x[toks], w1e, w3e, w2e, staged)
         res["H"][sel, :f], res["H"][sel, f:], res["A"][sel], res["Y"][sel] = h1, h3, a, y
         if dout is not None:
             g = plan["row_gate"][rows[sel]]
             ds, da1, da3, ga, dxp = expert_rows_backward(
-                dout[toks], g, h1, h3, w1[e], w3[e], w2[e], staged)
+                dout[toks], g, h1, h3, w1e, w3e, w2e, staged)
             res["dS"][sel] = ds
             res["dH"][sel, :f], res["dH"][sel, f:] = da1, da3
             res["gA"][sel] = ga
@@ -405,17 +408,21 @@ def sampled_tokens(tokens, dout, x, w_gate, w1, w3, w2, fwd, staged=True, router
     these depends on nothing but the token itself and its experts' weights,
     so the values equal those of the full layer."""
     plan = fwd["plan"]
-    dout, x, w_gate = map(_f64, (dout, x, w_gate))
+    dout, x, w_gate = _f64(dout), _f64(x), _f64(w_gate)
+    per_tok = [token_rows(plan, t) for t in tokens]
+    all_rows = [r for tr in per_tok for r in tr]
+    res = rows_compute(all_rows, plan, x, w1, w3, w2, dout, staged)
     out, dx, dl, dS = {}, {}, {}, {}
-    for t in tokens:
-        tr = token_rows(plan, t)
-        res = rows_compute(tr, plan, x, w1, w3, w2, dout, staged)
-        out[t] = (plan["row_gate"][tr][:, None] * res["Y"]).sum(axis=0)
-        dl[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"])
-        dx[t] = res["dXp"].sum(axis=0)
+    pos = 0
+    for t, tr in zip(tokens, per_tok):
+        sl = slice(pos, pos + len(tr))
+        pos += len(tr)
+        out[t] = (plan["row_gate"][tr][:, None] * res["Y"][sl]).sum(axis=0)
+        dl[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][sl])
+        dx[t] = res["dXp"][sl].sum(axis=0)
         if router_grad_on:
             dx[t] = dx[t] + dl[t] @ w_gate.T
-        for r, v in zip(tr, res["dS"]):
+        for r, v in zip(tr, res["dS"][sl]):
             dS[r] = v
     return dict(out=out, dx=dx, dlogits=dl, dS=dS)
 
@@ -424,7 +431,7 @@ def sampled_expert_grads(experts, dout, x, w1, w3, w2, fwd, staged=True):
     """dW1, dW3, dW2 of the listed experts (sums over that expert's rows)."""
     plan = fwd["plan"]
     dout, x = _f64(dout), _f64(x)
-    f = np.shape(w1)[2]
+    f = np.shape(w1[0])[1]
     out = {}
     for e in experts:
         lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
@@ -436,3 +443,32 @@ def sampled_expert_grads(experts, dout, x, w1, w3, w2, fwd, staged=True):
         out[e] = dict(dw2=res["gA"].T @ dout[tk], dw1=x[tk].T @ res["dH"][:, :f],
                       dw3=x[tk].T @ res["dH"][:, f:])
     return out
+
+
+def expert_grad_slices(e, cols, dout, x, w1e, w3e, w2e, fwd, staged=True):
+    """Selected columns of dW1_e and dW3_e (all d rows) and the same-numbered
+    rows of dW2_e (all d columns), from expert e's rows.
+
+    Column c of H1/H3/A/dH involves only column c of W1_e, W3_e and row c of
+    W2_e, so these slices follow from the per-element formulas of
+    expert_rows_forward / expert_rows_backward restricted to those columns.
+    """
+    plan = fwd["plan"]
+    dout, x = _f64(dout), _f64(x)
+    cols = np.asarray(cols)
+    lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
+    toks = plan["row_token"][lo:hi]
+    live = toks >= 0
+    tk = toks[live]
+    g = plan["row_gate"][lo:hi][live]
+    xr, dor = x[tk], dout[tk]
+    w1c, w3c, w2r = _f64(w1e)[:, cols], _f64(w3e)[:, cols], _f64(w2e)[cols, :]
+    h1 = _stage(xr @ w1c, staged)
+    h3 = _stage(xr @ w3c, staged)
+    a = _stage(silu(h1) * h3, staged)
+    dap = dor @ w2r.T
+    da = g[:, None] * dap
+    da3 = _stage(da * silu(h1), staged)
+    da1 = _stage(da * h3 * silu_grad(h1), staged)
+    ga = _stage(g[:, None] * a, staged)
+    return dict(dw1=xr.T @ da1, dw3=xr.T @ da3, dw2=ga.T @ dor)

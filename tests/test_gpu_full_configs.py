@@ -1,0 +1,126 @@
+"""GPU parity at the full workload sizes (coarse, pool, fine, sparse, and
+sparse with token rounding), in the launch configuration bench.py times.
+
+The oracle cannot run whole layers of this size in float64 in seconds, so it
+checks what it can compute one by one, exactly:
+  * the routing plan (counts, offsets, every row map) in full, bit-exact;
+  * out, dx, dlogits and dS of sampled tokens (each depends only on the token
+    and its experts' weights);
+  * sampled columns of dW1/dW3 and rows of dW2 for the most and least loaded
+    experts and one more;
+  * dW_gate through the property dW_gate = x^T dlogits, which holds at any size.
+Expert weights are copied to the host one expert at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_59_b200 import binding as B
+from mixture_experts_layer_59_b200 import synth
+from oracle import moe_oracle as O
+
+from helpers import (BF16_TOL, assert_close, compare_plan, f64, fp32_router_logits, gpu_layer,
+                     i64)
+
+pytestmark = pytest.mark.gpu
+
+
+class DeviceExperts:
+    """fp64 host copy of expert e of an [E, a, b] device tensor, on demand."""
+
+    def __init__(self, t, keep=16):
+        self.t, self.keep, self.cache = t, keep, {}
+
+    def __getitem__(self, e):
+        e = int(e)
+        if e not in self.cache:
+            if len(self.cache) >= self.keep:
+                self.cache.pop(next(iter(self.cache)))
+            self.cache[e] = self.t[e].to("cpu", torch.float64).numpy()
+        return self.cache[e]
+
+
+CASES = [
+    ("coarse", "learned", 0, 64),
+    ("coarse", "uniform", 0, 64),
+    ("pool", "uniform", 0, 64),
+    ("pool", "gauss", 0, 64),
+    ("fine", "learned", 0, 64),
+    ("sparse", "zipf", 0, 12),
+    ("sparse", "zipf", 1, 12),
+]
+
+
+@pytest.mark.parametrize("name,routing,round_mode,n_tok", CASES,
+                         ids=[f"{c[0]}-{c[1]}-round{c[2]}" for c in CASES])
+def test_full_size_layer(name, routing, round_mode, n_tok):
+    cfg = synth.CONFIGS[name].with_(routing=routing)
+    T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    router_grad = inp["logits_override"] is None
+    x64, wg64 = f64(inp["x"]), f64(inp["w_gate"])
+    if router_grad:
+        logits32 = fp32_router_logits(x64, wg64, inp["logit_bias"])
+        # the tensor-core router itself, against the oracle's logits
+        lg, idx_g, _ = B.moe_route(inp["x"], inp["w_gate"], k, logit_bias=inp["logit_bias"])
+        torch.cuda.synchronize()
+        lg = f64(lg)
+        scale = np.abs(logits32).max()
+        assert np.abs(lg - logits32).max() <= 1e-5 * scale
+        srt = -np.sort(-logits32.astype(np.float64), axis=1)
+        gaps = srt[:, :k] - srt[:, 1:k + 1]
+        clear = gaps[:, k - 1] > 1e-4 * scale          # top-k set is unique
+        ordered = np.all(gaps > 1e-4 * scale, axis=1)  # and so is its order
+        ref_idx = O.route(None, None, k, logits_override=logits32.astype(np.float64))[1]
+        np.testing.assert_array_equal(np.sort(i64(idx_g)[clear], 1), np.sort(ref_idx[clear], 1))
+        np.testing.assert_array_equal(i64(idx_g)[ordered], ref_idx[ordered])
+        del lg, idx_g
+    else:
+        logits32 = f64(inp["logits_override"]).astype(np.float32)
+
+    g = gpu_layer(inp, k, round_mode, logits32, router_grad=router_grad)
+
+    # routing plan, in full
+    lg64 = logits32.astype(np.float64)
+    _, idx, gate = O.route(None, None, k, logits_override=lg64)
+    plan = O.exact_plan(idx, gate, E) if round_mode == 0 else O.rounded_plan(idx, lg64, E)
+    np.testing.assert_array_equal(i64(g["idx"]), idx)
+    compare_plan(g["plan"], plan)
+    if round_mode:
+        assert plan["R"] < O.exact_plan(idx, gate, E)["R"]   # rounding removed padding rows
+    fwd = dict(logits=lg64, idx=idx, gate=gate, plan=plan)
+
+    W1, W3, W2 = DeviceExperts(inp["w1"]), DeviceExperts(inp["w3"]), DeviceExperts(inp["w2"])
+    dout64 = f64(inp["dout"])
+    rng = np.random.default_rng(1234)
+    tokens = sorted(set([0, T - 1] + list(rng.choice(T, n_tok - 2, replace=False))))
+    s = O.sampled_tokens(tokens, dout64, x64, wg64, W1, W3, W2, fwd, router_grad_on=router_grad)
+    out_g, dx_g, dl_g = f64(g["out"]), f64(g["dx"]), f64(g["dlogits"])
+    assert_close(out_g[tokens], np.stack([s["out"][t] for t in tokens]), "out", BF16_TOL)
+    assert_close(dx_g[tokens], np.stack([s["dx"][t] for t in tokens]), "dx", BF16_TOL)
+    assert_close(dl_g[tokens], np.stack([s["dlogits"][t] for t in tokens]), "dlogits", BF16_TOL)
+    rows = sorted(s["dS"])
+    assert_close(f64(g["dS"])[rows], np.array([s["dS"][r] for r in rows]), "dS", BF16_TOL)
+
+    # weight gradients: sampled columns of the most / least loaded and one more expert
+    counts = np.diff(plan["offsets"])
+    live = np.nonzero(counts > 0)[0]
+    experts = sorted({int(live[np.argmax(counts[live])]), int(live[np.argmin(counts[live])]),
+                      int(rng.choice(live))})
+    cols = sorted(rng.choice(f, 16, replace=False))
+    dw1, dw3, dw2 = g["dw1"], g["dw3"], g["dw2"]
+    for e in experts:
+        ref = O.expert_grad_slices(e, cols, dout64, x64, W1[e], W3[e], W2[e], fwd)
+        assert_close(f64(dw1[e][:, cols]), ref["dw1"], f"dw1[{e}]", BF16_TOL)
+        assert_close(f64(dw3[e][:, cols]), ref["dw3"], f"dw3[{e}]", BF16_TOL)
+        assert_close(f64(dw2[e][cols, :]), ref["dw2"], f"dw2[{e}]", BF16_TOL)
+    empty = np.nonzero(counts == 0)[0]
+    if len(empty):
+        e0 = int(empty[0])
+        assert float(dw1[e0].abs().max()) == 0.0 and float(dw2[e0].abs().max()) == 0.0
+
+    # dW_gate = x^T dlogits (property at any size), or zero without a router gradient
+    if router_grad:
+        assert_close(g["dw_gate"], x64.T @ dl_g, "dw_gate", BF16_TOL)
+    else:
+        assert float(g["dw_gate"].abs().max()) == 0.0

@@ -377,3 +377,35 @@ def test_rounded_plan_drop_tie_takes_largest_token():
     plan = O.rounded_plan(idx, logits, E, tile)
     assert list(plan["row_token"][0:4]) == [0, 1, 2, 3]
     assert plan["slot_row"][4] == -1 and plan["dropped"][4, 0]
+
+
+def test_expert_grad_slices_equal_full_grads():
+    rng = np.random.default_rng(15)
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, 60, 8, 12, 3, scale=0.3)
+    for rm in (0, 1):
+        fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4, round_mode=rm)
+        bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd)
+        cols = [0, 5, 11]
+        for e in range(3):
+            sl = O.expert_grad_slices(e, cols, dout, x, w1[e], w3[e], w2[e], fwd)
+            np.testing.assert_allclose(sl["dw1"], bwd["dw1"][e][:, cols], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(sl["dw3"], bwd["dw3"][e][:, cols], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(sl["dw2"], bwd["dw2"][e][cols, :], rtol=1e-12, atol=1e-14)
+
+
+def test_rows_compute_accepts_per_expert_weight_access():
+    rng = np.random.default_rng(16)
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, 30, 8, 6, 4, scale=0.3)
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=2, tile=4)
+
+    class Lazy:
+        def __init__(self, a):
+            self.a = a
+
+        def __getitem__(self, e):
+            return self.a[e].astype(np.float32)
+
+    s1 = O.sampled_tokens([3, 9], dout, x, wg, w1, w3, w2, fwd)
+    s2 = O.sampled_tokens([3, 9], dout, x, wg, Lazy(w1), Lazy(w3), Lazy(w2), fwd)
+    for t in (3, 9):
+        np.testing.assert_allclose(s1["dx"][t], s2["dx"][t], rtol=1e-6, atol=1e-9)
