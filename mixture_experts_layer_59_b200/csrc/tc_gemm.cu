@@ -70,13 +70,13 @@ struct TcArgs {
   CUtensorMap mA1;   // second A source (DXR: dlogits lo part)
   CUtensorMap mB0;   // B operand (W1 / W2 / activation / W_gate / dlogits hi)
   CUtensorMap mB1;   // second B source (W3, dlogits lo) where the kind has one
+  CUtensorMap sO0;   // bf16 outputs written by TMA stores (32 x 32 boxes, 64-byte swizzle)
+  CUtensorMap sO1;
+  CUtensorMap sO2;
   const int32_t* offsets;
   int E, d, f;
   int M, N, K;       // varlen-M: N, K fixed; varlen-K: M, N fixed
-  // epilogue operands
-  __nv_bfloat16* out0;   // H / Y / dXp / dW2 / dW1
-  __nv_bfloat16* out1;   // A (UP) / dH (DAP) / dW3 (DW13)
-  __nv_bfloat16* out2;   // s*A (DAP)
+  // epilogue operands (bf16 outputs go through the sO* store maps)
   const __nv_bfloat16* hin;  // H (DAP)
   const float* row_gate;     // DAP
   float* ds_part;            // DAP: [cap, nparts]
@@ -92,7 +92,6 @@ struct TcArgs {
   const __nv_bfloat16* dxp;  // DXR: [cap, d]
   const int32_t* slot_row;   // DXR: [T, k]
   const float* dx_acc;       // DXR: [T, d] fp32 row sums (used instead of dxp when set)
-  __nv_bfloat16* dx;         // DXR: [T, d]
 };
 
 template <int KIND> struct KT {
@@ -107,7 +106,8 @@ template <int BN> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int SMEM = STAGES * STAGE + 1024;
+  static constexpr int OUT_BYTES = 8 * 2048;   // one 32 x 32 bf16 staging tile per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE + OUT_BYTES + 1024;
   static constexpr int TMEM_COLS = 2 * BN;
 };
 
@@ -188,19 +188,6 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   }
 }
 
-__device__ __forceinline__ void st_bf16x32(__nv_bfloat16* dst, const float* v) {
-  uint4* p = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u;
-    __nv_bfloat162 h[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
-    memcpy(&u, h, 16);
-    p[q] = u;
-  }
-}
-
 __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
   const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -214,6 +201,33 @@ __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
       v[q * 8 + 2 * i] = f2.x;
       v[q * 8 + 2 * i + 1] = f2.y;
     }
+  }
+}
+
+// Stage one warp's 32 rows x 32 columns (row = lane) in its 2 KB shared tile
+// (64-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
+// and store it with one TMA tile store at (col, row0).  The previous store from
+// the same tile must have finished reading it first.
+__device__ __forceinline__ void stage_store(uint8_t* tile, const float* v, const CUtensorMap* map,
+                                            int col, int row0, int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  uint8_t* rowp = tile + lane * 64;
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+    uint4 u;
+    memcpy(&u, h, 16);
+    *reinterpret_cast<uint4*>(rowp + ((q ^ sw) << 4)) = u;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, tile, col, row0);
+    bulk_commit();
   }
 }
 
@@ -384,6 +398,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       const int row = ti.m0 + rloc;
       float v[32];
       uint32_t r[32];
+      uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * 2048;
+      const int row0 = ti.m0 + q * 32;           // first row of this warp's 32-row slab
       if constexpr (KIND == K_UP) {
         const int f = a.f, nf = ti.ntile * (BN / 2);
         float h3[32];
@@ -396,15 +412,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) h3[i] = __uint_as_float(r[i]);
-          __nv_bfloat16* hrow = a.out0 + (size_t)row * 2 * f;
-          st_bf16x32(hrow + nf + c, v);
-          st_bf16x32(hrow + f + nf + c, h3);
+          stage_store(otile, v, &a.sO0, nf + c, row0, lane);        // H1
+          stage_store(otile, h3, &a.sO0, f + nf + c, row0, lane);   // H3
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float h1 = bf16_round(v[i]);
             v[i] = h1 * sigmoid_fast(h1) * bf16_round(h3[i]);
           }
-          st_bf16x32(a.out1 + (size_t)row * f + nf + c, v);
+          stage_store(otile, v, &a.sO1, nf + c, row0, lane);        // A
         }
       } else if constexpr (KIND == K_DOWN || KIND == K_DX) {
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
@@ -412,7 +427,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          st_bf16x32(a.out0 + (size_t)row * a.N + ti.n0 + c, v);
+          stage_store(otile, v, &a.sO0, ti.n0 + c, row0, lane);
         }
       } else if constexpr (KIND == K_DAP) {
         const int f = a.f;
@@ -425,7 +440,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           ld_bf16x32(hrow + ti.n0 + c, h1);
           ld_bf16x32(hrow + f + ti.n0 + c, h3);
           tmem_ld_wait();
-          float da3[32], ga[32];
+          float da3[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float dap = __uint_as_float(r[i]);
@@ -436,12 +451,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             const float da = g * dap;
             v[i] = da * h3[i] * (sg * (1.0f + h1[i] * (1.0f - sg)));
             da3[i] = da * sl;
-            ga[i] = g * av;
+            h1[i] = g * av;                                           // s * A
           }
-          __nv_bfloat16* drow = a.out1 + (size_t)row * 2 * f;
-          st_bf16x32(drow + ti.n0 + c, v);
-          st_bf16x32(drow + f + ti.n0 + c, da3);
-          st_bf16x32(a.out2 + (size_t)row * f + ti.n0 + c, ga);
+          stage_store(otile, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
+          stage_store(otile, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
+          stage_store(otile, h1, &a.sO1, ti.n0 + c, row0, lane);      // s * A
         }
         a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
       } else if constexpr (KIND == K_RT) {
@@ -504,8 +518,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          const int col = ti.n0 + c;
           if (valid) {
-            const int col = ti.n0 + c;
             if (a.dx_acc != nullptr) {
               const float4* s4 = reinterpret_cast<const float4*>(a.dx_acc + (size_t)t * a.N + col);
 #pragma unroll
@@ -524,11 +538,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
                 }
               }
             }
-            st_bf16x32(a.dx + (size_t)t * a.N + col, v);
           }
+          // rows at or beyond T are clipped by the tensor map
+          stage_store(otile, v, &a.sO0, col, row0, lane);
         }
-      } else {  // DW2 / DW13: output row m = row of dW_e
-        const size_t ebase = (size_t)ti.e * a.M * (KIND == K_DW2 ? a.N : a.f);
+      } else {  // DW2 / DW13: output row m = row of dW_e (maps view dW as [E*M, N])
+        const int orow0 = ti.e * a.M + row0;
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           if (ti.kb_count > 0) {
             tmem_ld32(tbase + c, r);
@@ -541,10 +556,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           }
           const int col = ti.n0 + c;
           if constexpr (KIND == K_DW2) {
-            st_bf16x32(a.out0 + ebase + (size_t)row * a.N + col, v);
+            stage_store(otile, v, &a.sO0, col, orow0, lane);
           } else {
-            if (col < a.f) st_bf16x32(a.out0 + ebase + (size_t)row * a.f + col, v);
-            else st_bf16x32(a.out1 + ebase + (size_t)row * a.f + col - a.f, v);
+            if (col < a.f) stage_store(otile, v, &a.sO0, col, orow0, lane);
+            else stage_store(otile, v, &a.sO1, col - a.f, orow0, lane);
           }
         }
       }
@@ -552,6 +567,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       mbar_arrive(&tempty_bar[acc]);
     }
   }
+
+  // the epilogue's bulk stores must finish before the CTA exits
+  if (warp >= 2 && lane == 0) bulk_wait_all();
 
   // on an aborted run give in-flight TMA copies and MMAs time to land
   if (s_abort) {
@@ -597,7 +615,8 @@ int tc_num_dS_parts(int f) { return 2 * ((f % 256 == 0) ? f / 256 : f / 128); }
 
 // bf16 row-major [outer, inner] viewed in boxes of box_outer x box_inner.
 static int make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
-                       uint32_t box_inner, uint32_t box_outer) {
+                       uint32_t box_inner, uint32_t box_outer,
+                       CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, outer};
@@ -605,10 +624,15 @@ static int make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (2d) failed: " + std::to_string((int)r));
   return MOE_OK;
+}
+
+// Output map of the epilogue's TMA stores: 32 x 32 boxes, 64-byte swizzle.
+static int make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer) {
+  return make_map_2d(m, ptr, inner, outer, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // bf16 [d2, d1, d0] (d0 innermost) viewed in boxes of box1 x box0.
@@ -753,8 +777,8 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
     a.dxp = (const __nv_bfloat16*)dxp;
     a.slot_row = slot_row;
     a.dx_acc = dx_acc;
-    a.dx = (__nv_bfloat16*)dx;
     const int bn = pick_bn(d);
+    if ((rc = make_store_map(&a.sO0, dx, d, T))) return rc;
     if ((rc = make_map_2d(&a.mA, dl_hi, E, T, 64, BM))) return rc;
     if ((rc = make_map_2d(&a.mA1, dl_lo, E, T, 64, BM))) return rc;
     if ((rc = make_map_2d(&a.mB0, wg, E, d, 64, bn))) return rc;
@@ -774,8 +798,8 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
     if ((rc = make_map_2d(&a.mA, xg, d, cap, 64, BM))) return rc;
     if ((rc = make_map_3d(&a.mB0, p.w1, f, d, E, 64, 64))) return rc;
     if ((rc = make_map_3d(&a.mB1, p.w3, f, d, E, 64, 64))) return rc;
-    a.out0 = (__nv_bfloat16*)H;
-    a.out1 = (__nv_bfloat16*)act;
+    if ((rc = make_store_map(&a.sO0, H, 2 * f, cap))) return rc;
+    if ((rc = make_store_map(&a.sO1, act, f, cap))) return rc;
     if ((rc = launch<K_UP, 256>(a, num_sms, s))) return rc;
   }
   {  // DOWN: Y = A W2
@@ -785,7 +809,7 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
     const int bn = pick_bn(d);
     if ((rc = make_map_2d(&a.mA, act, f, cap, 64, BM))) return rc;
     if ((rc = make_map_3d(&a.mB0, p.w2, d, f, E, 64, 64))) return rc;
-    a.out0 = (__nv_bfloat16*)Y;
+    if ((rc = make_store_map(&a.sO0, Y, d, cap))) return rc;
     if ((rc = launch_bn<K_DOWN>(a, bn, num_sms, s))) return rc;
   }
   return MOE_OK;
@@ -805,8 +829,8 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if ((rc = make_map_3d(&a.mB0, p.w2, d, f, E, 64, bn))) return rc;
     a.hin = (const __nv_bfloat16*)H;
     a.row_gate = row_gate;
-    a.out1 = (__nv_bfloat16*)dH;
-    a.out2 = (__nv_bfloat16*)gact;
+    if ((rc = make_store_map(&a.sO0, dH, 2 * f, cap))) return rc;
+    if ((rc = make_store_map(&a.sO1, gact, f, cap))) return rc;
     a.ds_part = ds_part;
     a.nparts = 2 * (f / bn);
     if (a.nparts != tc_num_dS_parts(f)) return fail(MOE_ERR_UNSUPPORTED, "dS partition mismatch");
@@ -820,7 +844,7 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if ((rc = make_map_2d(&a.mA, dH, 2 * f, cap, 64, BM))) return rc;
     if ((rc = make_map_3d(&a.mB0, p.w1, f, d, E, 64, bn))) return rc;
     if ((rc = make_map_3d(&a.mB1, p.w3, f, d, E, 64, bn))) return rc;
-    a.out0 = (__nv_bfloat16*)dXp;
+    if ((rc = make_store_map(&a.sO0, dXp, d, cap))) return rc;
     if ((rc = launch_bn<K_DX>(a, bn, num_sms, s))) return rc;
   }
   {  // DW2: dW2_e = (sA)^T dOg
@@ -830,7 +854,7 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     const int bn = pick_bn(d);
     if ((rc = make_map_2d(&a.mA, gact, f, cap, 64, 64))) return rc;
     if ((rc = make_map_2d(&a.mB0, dog, d, cap, 64, 64))) return rc;
-    a.out0 = (__nv_bfloat16*)dw2;
+    if ((rc = make_store_map(&a.sO0, dw2, d, (uint64_t)E * f))) return rc;
     if ((rc = launch_bn<K_DW2>(a, bn, num_sms, s))) return rc;
   }
   {  // DW13: [dW1 | dW3]_e = Xg^T dH
@@ -840,8 +864,8 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     const int bn = pick_bn(2 * f);
     if ((rc = make_map_2d(&a.mA, xg, d, cap, 64, 64))) return rc;
     if ((rc = make_map_2d(&a.mB0, dH, 2 * f, cap, 64, 64))) return rc;
-    a.out0 = (__nv_bfloat16*)dw1;
-    a.out1 = (__nv_bfloat16*)dw3;
+    if ((rc = make_store_map(&a.sO0, dw1, f, (uint64_t)E * d))) return rc;
+    if ((rc = make_store_map(&a.sO1, dw3, f, (uint64_t)E * d))) return rc;
     if ((rc = launch_bn<K_DW13>(a, bn, num_sms, s))) return rc;
   }
   return MOE_OK;
