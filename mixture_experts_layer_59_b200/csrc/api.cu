@@ -340,18 +340,13 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
                               tc_router ? w.dl_lo : nullptr, s)))
     return rc;
   if (tc_router) {
-    // dW_gate and the router term of dx on the tensor cores; the unpermute-sum
-    // of dX_perm is fused into the dx epilogue (rows of added pairs, present
-    // only with token rounding, go through an fp32 row sum first)
-    const float* acc = nullptr;
-    if (extra_row != nullptr) {
-      if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype,
-                                    false, true, w.dx_acc, s)))
-        return rc;
-      acc = w.dx_acc;
-    }
-    return tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate, w.dxp,
-                         slot_row, acc, dx, device_sm_count(), s);
+    // dx = (warp-per-token fp32 sum of the token's dX_perm rows) + the router
+    // term dl W_gate^T from the tensor cores; dW_gate on the tensor cores too
+    if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
+                                  true, w.dx_acc, s)))
+      return rc;
+    return tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate, w.dx_acc,
+                         dx, device_sm_count(), s);
   }
   if (router_grad) {
     if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,

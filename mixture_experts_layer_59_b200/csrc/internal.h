@@ -76,9 +76,8 @@ int tc_dwg_splits(int T, int d, int* chunk);
 int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
                   float* logits, int32_t* idx, float* gate, int num_sms, cudaStream_t s);
 int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
-                  int d, int E, int k, float* dwg_part, float* dw_gate, const void* dxp,
-                  const int32_t* slot_row, const float* dx_acc, void* dx, int num_sms,
-                  cudaStream_t s);
+                  int d, int E, int k, float* dwg_part, float* dw_gate, const float* dx_acc,
+                  void* dx, int num_sms, cudaStream_t s);
 
 int device_sm_count();
 

@@ -19,8 +19,7 @@
 //   DWG   dW_gate = x^T dlogits      split-K over tokens; dlogits enters as a
 //                                    bf16 hi part plus a bf16 lo remainder,
 //                                    accumulated in the same fp32 accumulator
-//   DXR   dx = sum of the token's dX_perm rows + dlogits W_gate^T
-//                                    (router term and unpermute-sum fused)
+//   DXR   dx = (fp32 sum of the token's dX_perm rows) + dlogits W_gate^T
 // The grouped GEMM replaces the per-expert loop of the Beam article's
 // MoELayer (sec. 5.3); Olmo-core 3 names grouped GEMM for the same purpose;
 // dS = <dA', A> without a stored Y is the SonicMoE summary's sec. 1.
@@ -89,9 +88,7 @@ struct TcArgs {
   int32_t* idx;              // RT: [T, k]
   float* gate;               // RT: [T, k]
   float* dwg_part;           // DWG: [splits, d, E]
-  const __nv_bfloat16* dxp;  // DXR: [cap, d]
-  const int32_t* slot_row;   // DXR: [T, k]
-  const float* dx_acc;       // DXR: [T, d] fp32 row sums (used instead of dxp when set)
+  const float* dx_acc;       // DXR: [T, d] fp32 sums of each token's dX_perm rows
 };
 
 template <int KIND> struct KT {
@@ -106,8 +103,8 @@ template <int BN> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int OUT_BYTES = 8 * 2048;   // one 32 x 32 bf16 staging tile per epilogue warp
-  static constexpr int SMEM = STAGES * STAGE + OUT_BYTES + 1024;
+  static constexpr int OUT_BYTES = 8 * 2 * 2048;  // two 32 x 32 bf16 staging tiles per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE + OUT_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
 };
 
@@ -204,13 +201,16 @@ __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
   }
 }
 
-// Stage one warp's 32 rows x 32 columns (row = lane) in its 2 KB shared tile
-// (64-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
-// and store it with one TMA tile store at (col, row0).  The previous store from
-// the same tile must have finished reading it first.
-__device__ __forceinline__ void stage_store(uint8_t* tile, const float* v, const CUtensorMap* map,
-                                            int col, int row0, int lane) {
-  if (lane == 0) bulk_wait_read_all();
+// Stage one warp's 32 rows x 32 columns (row = lane) in one of its two 2 KB
+// shared tiles (64-byte swizzle: 16-byte chunk c of row r sits at chunk
+// c ^ ((r >> 1) & 3)) and store it with one TMA tile store at (col, row0).
+// The tiles alternate; before a tile is rewritten, the store issued from it
+// two calls ago must have finished reading it.
+__device__ __forceinline__ void stage_store(uint8_t* tiles, int& which, const float* v,
+                                            const CUtensorMap* map, int col, int row0, int lane) {
+  uint8_t* tile = tiles + which * 2048;
+  which ^= 1;
+  if (lane == 0) bulk_wait_read_1();
   __syncwarp();
   uint8_t* rowp = tile + lane * 64;
   const int sw = (lane >> 1) & 3;
@@ -243,8 +243,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
   __shared__ int s_off[257];
   __shared__ volatile int s_abort;
 
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // 128-byte swizzled tiles need a 1024-byte aligned base: refuse to run otherwise
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) record_status(a.status, 0x2ff);
+    return;
+  }
 
   if (a.offsets != nullptr)
     for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_off[i] = a.offsets[i];
@@ -387,6 +392,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const int half = (warp - 2) >> 2;            // which half of the tile's columns
     const int rloc = q * 32 + lane;              // row of the tile owned by this thread
+    int obuf = 0;                                // staging tile used by the next store
     int it = 0;
     TileInfo ti;
     for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x, ++it) {
@@ -398,7 +404,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       const int row = ti.m0 + rloc;
       float v[32];
       uint32_t r[32];
-      uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * 2048;
+      uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * 4096;
       const int row0 = ti.m0 + q * 32;           // first row of this warp's 32-row slab
       if constexpr (KIND == K_UP) {
         const int f = a.f, nf = ti.ntile * (BN / 2);
@@ -412,14 +418,14 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) h3[i] = __uint_as_float(r[i]);
-          stage_store(otile, v, &a.sO0, nf + c, row0, lane);        // H1
-          stage_store(otile, h3, &a.sO0, f + nf + c, row0, lane);   // H3
+          stage_store(otile, obuf, v, &a.sO0, nf + c, row0, lane);        // H1
+          stage_store(otile, obuf, h3, &a.sO0, f + nf + c, row0, lane);   // H3
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float h1 = bf16_round(v[i]);
             v[i] = h1 * sigmoid_fast(h1) * bf16_round(h3[i]);
           }
-          stage_store(otile, v, &a.sO1, nf + c, row0, lane);        // A
+          stage_store(otile, obuf, v, &a.sO1, nf + c, row0, lane);        // A
         }
       } else if constexpr (KIND == K_DOWN || KIND == K_DX) {
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
@@ -427,7 +433,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          stage_store(otile, v, &a.sO0, ti.n0 + c, row0, lane);
+          stage_store(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);
         }
       } else if constexpr (KIND == K_DAP) {
         const int f = a.f;
@@ -453,47 +459,66 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             da3[i] = da * sl;
             h1[i] = g * av;                                           // s * A
           }
-          stage_store(otile, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
-          stage_store(otile, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
-          stage_store(otile, h1, &a.sO1, ti.n0 + c, row0, lane);      // s * A
+          stage_store(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
+          stage_store(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
+          stage_store(otile, obuf, h1, &a.sO1, ti.n0 + c, row0, lane);      // s * A
         }
         a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
       } else if constexpr (KIND == K_RT) {
-        const int t = row;
-        const bool valid = t < a.T && half == 0;
-        float tv[8];
-        int tix[8];
+        // logits (+bias) and a running top-8 list kept sorted in registers;
+        // equal values keep the lower expert id first (ids arrive ascending)
+        if (half == 0) {
+          const int t = row;
+          const bool valid = t < a.T;
+          float tv[8];
+          int tix[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; tix[j] = 0x7fffffff; }
-        for (int c = 0; half == 0 && c < a.E; c += 32) {
-          tmem_ld32(tbase + c, r);
-          tmem_ld_wait();
+          for (int j = 0; j < 8; ++j) { tv[j] = -INFINITY; tix[j] = 0x7fffffff; }
+          for (int c = 0; c < a.E; c += 32) {
+            tmem_ld32(tbase + c, r);
+            tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = c + i;
-            if (e < a.E) {
-              float l = __uint_as_float(r[i]);
-              if (a.bias) l += a.bias[e];
-              if (valid) a.logits[(size_t)t * a.E + e] = l;
-              // insertion into the descending top-k list; equal values keep
-              // the lower expert id first because ids arrive in ascending order
-              if (l > tv[a.k - 1]) {
-                int j = a.k - 1;
-                while (j > 0 && l > tv[j - 1]) { tv[j] = tv[j - 1]; tix[j] = tix[j - 1]; --j; }
-                tv[j] = l;
-                tix[j] = e;
+            for (int i = 0; i < 32; ++i) {
+              v[i] = __uint_as_float(r[i]);
+              if (a.bias && c + i < a.E) v[i] += a.bias[c + i];
+            }
+            if (valid) {
+              float4* dst = reinterpret_cast<float4*>(a.logits + (size_t)t * a.E + c);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                if (c + 4 * q < a.E) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (c + i < a.E && v[i] > tv[7]) {
+                tv[7] = v[i];
+                tix[7] = c + i;
+#pragma unroll
+                for (int j = 7; j > 0; --j) {
+                  if (tv[j] > tv[j - 1]) {
+                    const float fv = tv[j]; tv[j] = tv[j - 1]; tv[j - 1] = fv;
+                    const int iv = tix[j]; tix[j] = tix[j - 1]; tix[j - 1] = iv;
+                  }
+                }
               }
             }
           }
-        }
-        if (valid) {
-          const float m = tv[0];
-          float z = 0.f, ex[8];
-          for (int j = 0; j < a.k; ++j) { ex[j] = expf(tv[j] - m); z += ex[j]; }
-          const float inv = 1.0f / z;
-          for (int j = 0; j < a.k; ++j) {
-            a.idx[(size_t)t * a.k + j] = tix[j];
-            a.gate[(size_t)t * a.k + j] = ex[j] * inv;
+          if (valid) {
+            const float m = tv[0];
+            float z = 0.f, ex[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              ex[j] = j < a.k ? expf(tv[j] - m) : 0.f;
+              z += ex[j];
+            }
+            const float inv = 1.0f / z;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (j < a.k) {
+                a.idx[(size_t)t * a.k + j] = tix[j];
+                a.gate[(size_t)t * a.k + j] = ex[j] * inv;
+              }
+            }
           }
         }
       } else if constexpr (KIND == K_DWG) {
@@ -509,10 +534,6 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       } else if constexpr (KIND == K_DXR) {
         const int t = row;
         const bool valid = t < a.T;
-        int rows8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          rows8[j] = (valid && a.dx_acc == nullptr && j < a.k) ? a.slot_row[(size_t)t * a.k + j] : -1;
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
@@ -520,27 +541,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           const int col = ti.n0 + c;
           if (valid) {
-            if (a.dx_acc != nullptr) {
-              const float4* s4 = reinterpret_cast<const float4*>(a.dx_acc + (size_t)t * a.N + col);
+            const float4* s4 = reinterpret_cast<const float4*>(a.dx_acc + (size_t)t * a.N + col);
 #pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const float4 u = s4[q];
-                v[4 * q] += u.x; v[4 * q + 1] += u.y; v[4 * q + 2] += u.z; v[4 * q + 3] += u.w;
-              }
-            } else {
-              float h[32];
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                if (rows8[j] >= 0) {
-                  ld_bf16x32(a.dxp + (size_t)rows8[j] * a.N + col, h);
-#pragma unroll
-                  for (int i = 0; i < 32; ++i) v[i] += h[i];
-                }
-              }
+            for (int q = 0; q < 8; ++q) {
+              const float4 u = s4[q];
+              v[4 * q] += u.x; v[4 * q + 1] += u.y; v[4 * q + 2] += u.z; v[4 * q + 3] += u.w;
             }
           }
           // rows at or beyond T are clipped by the tensor map
-          stage_store(otile, v, &a.sO0, col, row0, lane);
+          stage_store(otile, obuf, v, &a.sO0, col, row0, lane);
         }
       } else {  // DW2 / DW13: output row m = row of dW_e (maps view dW as [E*M, N])
         const int orow0 = ti.e * a.M + row0;
@@ -556,10 +565,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           }
           const int col = ti.n0 + c;
           if constexpr (KIND == K_DW2) {
-            stage_store(otile, v, &a.sO0, col, orow0, lane);
+            stage_store(otile, obuf, v, &a.sO0, col, orow0, lane);
           } else {
-            if (col < a.f) stage_store(otile, v, &a.sO0, col, orow0, lane);
-            else stage_store(otile, v, &a.sO1, col - a.f, orow0, lane);
+            if (col < a.f) stage_store(otile, obuf, v, &a.sO0, col, orow0, lane);
+            else stage_store(otile, obuf, v, &a.sO1, col - a.f, orow0, lane);
           }
         }
       }
@@ -739,9 +748,8 @@ __global__ void k_dwg_reduce(const float* __restrict__ part, int splits, int n,
 }
 
 int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
-                  int d, int E, int k, float* dwg_part, float* dw_gate, const void* dxp,
-                  const int32_t* slot_row, const float* dx_acc, void* dx, int num_sms,
-                  cudaStream_t s) {
+                  int d, int E, int k, float* dwg_part, float* dw_gate, const float* dx_acc,
+                  void* dx, int num_sms, cudaStream_t s) {
   int rc;
   {  // dW_gate = x^T (dl_hi + dl_lo), split over tokens, then a fixed-order sum
     TcArgs a;
@@ -765,7 +773,7 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
     }
     MOE_CHECK_LAUNCH("dwg_reduce");
   }
-  {  // dx = unpermute-sum of dX_perm (or the fp32 row sums) + dl W_gate^T
+  {  // dx = fp32 unpermute-sum of dX_perm + dl W_gate^T
     TcArgs a;
     memset(&a, 0, sizeof(a));
     a.E = E;
@@ -774,8 +782,6 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
     a.T = T;
     a.k = k;
     a.status = status_ptr();
-    a.dxp = (const __nv_bfloat16*)dxp;
-    a.slot_row = slot_row;
     a.dx_acc = dx_acc;
     const int bn = pick_bn(d);
     if ((rc = make_store_map(&a.sO0, dx, d, T))) return rc;
