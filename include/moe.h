@@ -147,16 +147,19 @@ int moe_permute_noalloc(const int32_t* idx, const float* gate, int T, int E, int
 /*
  * moe_expert_ffn_fwd -- per-expert SwiGLU FFN on the permuted rows.
  * [Beam] sec. 2.2/5.3 (expert FFN, grouped instead of looped); [Olmo]
- * (grouped GEMM).  Experts are SwiGLU:
+ * (grouped GEMM; rows placed straight into expert input buffers).  Experts
+ * are SwiGLU:
  *   H = [x W1_e | x W3_e]  (saved for backward, dtype)
  *   A = silu(H1) * H3      (transient)
  *   Y_perm = A W2_e        (transient, dtype)
- *   x [T,d]; w1, w3 [E,d,f]; w2 [E,f,d]; row_token [cap], offsets [E+1] from
+ *   x [T,d]; w1, w3 [E,d,f]; w2 [E,f,d]; row_token [cap], offsets [E+1],
+ *   slot_row [T*k] and extra_row [T,E] (NULL without rounding) from
  *   moe_permute with tile 128.  H [cap,2f] out; Y_perm [cap,d] out.
  */
 size_t moe_ffn_fwd_workspace_size(int T, int d, int f, int E, int k, int dtype);
 int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void* w2,
                        const int32_t* row_token, const int32_t* offsets,
+                       const int32_t* slot_row, const int32_t* extra_row,
                        int T, int d, int f, int E, int k, int dtype,
                        void* H, void* Y_perm, void* ws, size_t ws_bytes, void* stream);
 

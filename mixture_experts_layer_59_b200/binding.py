@@ -46,8 +46,8 @@ _SIGS = {
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                          _vp, _sz, _vp]),
     "moe_ffn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
-    "moe_expert_ffn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp,
-                                _vp, _sz, _vp]),
+    "moe_expert_ffn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_layer_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_layer_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
@@ -157,8 +157,8 @@ def moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype) -> int:
     return lib().moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype)
 
 
-def moe_expert_ffn_fwd(x, w1, w3, w2, row_token, offsets, k, H=None, Y_perm=None, ws=None,
-                       stream=None):
+def moe_expert_ffn_fwd(x, w1, w3, w2, plan, k, H=None, Y_perm=None, ws=None, stream=None):
+    """plan: dict from moe_permute (row_token, offsets, slot_row, extra_row)."""
     T, d = x.shape
     E, _, f = w1.shape
     dt = dtype_code(x.dtype)
@@ -168,9 +168,10 @@ def moe_expert_ffn_fwd(x, w1, w3, w2, row_token, offsets, k, H=None, Y_perm=None
     if ws is None:
         ws = torch.empty(max(moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), device=x.device,
                          dtype=torch.uint8)
-    _check(lib().moe_expert_ffn_fwd(_p(x), _p(w1), _p(w3), _p(w2), _p(row_token), _p(offsets), T,
-                                    d, f, E, k, dt, _p(H), _p(Y_perm), _p(ws), ws.numel(),
-                                    _stream(stream)))
+    _check(lib().moe_expert_ffn_fwd(_p(x), _p(w1), _p(w3), _p(w2), _p(plan["row_token"]),
+                                    _p(plan["offsets"]), _p(plan["slot_row"]),
+                                    _p(plan.get("extra_row")), T, d, f, E, k, dt, _p(H),
+                                    _p(Y_perm), _p(ws), ws.numel(), _stream(stream)))
     return H, Y_perm
 
 

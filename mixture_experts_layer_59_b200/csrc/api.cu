@@ -253,13 +253,14 @@ size_t moe_ffn_fwd_workspace_size(int T, int d, int f, int E, int k, int dtype) 
 }
 
 int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void* w2,
-                       const int32_t* row_token, const int32_t* offsets, int T, int d, int f, int E,
-                       int k, int dtype, void* H, void* Y_perm, void* ws, size_t ws_bytes,
-                       void* stream) {
+                       const int32_t* row_token, const int32_t* offsets, const int32_t* slot_row,
+                       const int32_t* extra_row, int T, int d, int f, int E, int k, int dtype,
+                       void* H, void* Y_perm, void* ws, size_t ws_bytes, void* stream) {
   if (int rc = check_common(T, E, k, dtype)) return rc;
   if (int rc = check_dims(d, f, dtype)) return rc;
   REQUIRE_PTR(x); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
   REQUIRE_PTR(row_token); REQUIRE_PTR(offsets); REQUIRE_PTR(H); REQUIRE_PTR(Y_perm);
+  if (T > 0) REQUIRE_PTR(slot_row);
   REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2);
   REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(Y_perm); REQUIRE_ALIGNED(ws);
   if (ws_bytes < moe_ffn_fwd_workspace_size(T, d, f, E, k, dtype))
@@ -271,7 +272,9 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
   cudaStream_t s = (cudaStream_t)stream;
   FfnPtrs p{x, w1, w3, w2, row_token, offsets, T, d, f, E, (int)((size_t)T * k + (size_t)E * 128), dtype};
   if (dtype == MOE_BF16 && tc_available()) {
-    if (int rc = launch_gather_rows(x, row_token, offsets, E, d, dtype, w.xg, s)) return rc;
+    if (int rc = launch_scatter_rows(x, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
+                                     w.xg, s))
+      return rc;
     return tc_ffn_fwd(p, w.xg, H, w.act, Y_perm, device_sm_count(), s);
   }
   return simt_ffn_fwd(p, H, w.act, Y_perm, s);
@@ -324,8 +327,12 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   FfnPtrs p{x, w1, w3, w2, row_token, offsets, T, d, f, E, (int)((size_t)T * k + (size_t)E * 128), dtype};
   int rc;
   if (dtype == MOE_BF16 && tc_available()) {
-    if ((rc = launch_gather_rows(dout, row_token, offsets, E, d, dtype, w.dog, s))) return rc;
-    if ((rc = launch_gather_rows(x, row_token, offsets, E, d, dtype, w.xg, s))) return rc;
+    if ((rc = launch_scatter_rows(dout, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
+                                  w.dog, s)))
+      return rc;
+    if ((rc = launch_scatter_rows(x, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
+                                  w.xg, s)))
+      return rc;
     if ((rc = tc_ffn_bwd(p, w.dog, w.xg, row_gate, H, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2,
                          device_sm_count(), s)))
       return rc;
@@ -340,8 +347,15 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
                               tc_router ? w.dl_lo : nullptr, s)))
     return rc;
   if (tc_router) {
-    // dx = (warp-per-token fp32 sum of the token's dX_perm rows) + the router
-    // term dl W_gate^T from the tensor cores; dW_gate on the tensor cores too
+    // dW_gate on the tensor cores (split-K, hi/lo dlogits); dx = unpermute-sum
+    // of dX_perm + dl W_gate^T: one CUDA-core pass when W_gate fits in shared
+    // memory, otherwise fp32 row sums + the tensor-core router term
+    if (dx_fused_ok(d, E)) {
+      if ((rc = tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate,
+                              nullptr, nullptr, device_sm_count(), s)))
+        return rc;
+      return launch_dx_fused(w.dxp, slot_row, extra_row, dl, w_gate, T, d, E, k, dx, s);
+    }
     if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
                                   true, w.dx_acc, s)))
       return rc;

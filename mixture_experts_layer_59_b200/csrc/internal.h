@@ -36,8 +36,16 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
                          const PermuteWs& w, cudaStream_t s);
 
 // ---------------------------------------------------------------- row ops
-int launch_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets, int E,
-                       int width, int dtype, void* dst, cudaStream_t s);
+// dst[row] = src[token of row] for every row (token-order scatter: each source
+// row read once); padding rows (token -1) zeroed.
+int launch_scatter_rows(const void* src, const int32_t* slot_row, const int32_t* extra_row,
+                        const int32_t* row_token, const int32_t* offsets, int T, int width, int E,
+                        int k, int dtype, void* dst, cudaStream_t s);
+// dx = bf16(sum of the token's dX_perm rows + dl W_gate^T), W_gate staged in smem.
+bool dx_fused_ok(int d, int E);
+int launch_dx_fused(const void* dxp, const int32_t* slot_row, const int32_t* extra_row,
+                    const float* dl, const void* wg, int T, int d, int E, int k, void* dx,
+                    cudaStream_t s);
 // out[t] = sum over token t's rows (kept slots in order, then added rows by
 // ascending expert) of (weighted ? row_gate[r] : 1) * src[r]; out fp32 or dtype.
 int launch_token_reduce(const void* src, const float* row_gate, const int32_t* slot_row,

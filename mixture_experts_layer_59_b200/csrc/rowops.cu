@@ -30,36 +30,191 @@ template <> struct Vec<float> {
   __device__ __forceinline__ void set(int i, float f) { reinterpret_cast<float*>(&v)[i] = f; }
 };
 
-// ============================================================== gather rows
-// dst[r, :] = src[row_token[r], :] for live rows, 0 for padding rows; r < R.
+// ============================================================== scatter rows
+// dst[row, :] = src[t, :] for every row of token t (its kept slots, then the
+// rows added by token rounding); rows that hold no pair (padding, token -1)
+// are zeroed.  Blocks [0, nbt) own tokens, one warp per token, so each source
+// row is read once and written to its k rows with coalesced 16-byte stores;
+// the remaining blocks zero the padding rows.
 template <class T>
-__global__ void k_gather_rows(const T* __restrict__ src, const int32_t* __restrict__ row_token,
-                              const int32_t* __restrict__ offsets, int E, int width,
-                              T* __restrict__ dst) {
-  const int R = offsets[E];
+__global__ void __launch_bounds__(256)
+k_scatter_rows(const T* __restrict__ src, const int32_t* __restrict__ slot_row,
+               const int32_t* __restrict__ extra_row, const int32_t* __restrict__ row_token,
+               const int32_t* __restrict__ offsets, int T_, int width, int E, int k, int nbt,
+               T* __restrict__ dst) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nvec = width / Vec<T>::N;
-  const int warps = blockDim.x >> 5, lane = threadIdx.x & 31;
-  for (int r = blockIdx.x * warps + (threadIdx.x >> 5); r < R; r += gridDim.x * warps) {
-    const int t = row_token[r];
-    const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)(t < 0 ? 0 : t) * width);
-    uint4* o = reinterpret_cast<uint4*>(dst + (size_t)r * width);
-    for (int i = lane; i < nvec; i += 32) o[i] = t >= 0 ? __ldg(s + i) : make_uint4(0, 0, 0, 0);
+  if ((int)blockIdx.x < nbt) {
+    const int t = blockIdx.x * 8 + w;
+    if (t >= T_) return;
+    const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    int rk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
+    const uint4* s4 = reinterpret_cast<const uint4*>(src + (size_t)t * width);
+    for (int i = lane; i < nvec; i += 32) {
+      const uint4 v = __ldg(s4 + i);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (rk[j] >= 0) reinterpret_cast<uint4*>(dst + (size_t)rk[j] * width)[i] = v;
+    }
+    if (extra_row != nullptr) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int re = e0 + lane < E ? extra_row[(size_t)t * E + e0 + lane] : -1;
+        unsigned bal = __ballot_sync(0xffffffffu, re >= 0);
+        while (bal) {
+          const int b = __ffs(bal) - 1;
+          bal &= bal - 1;
+          const int r = __shfl_sync(0xffffffffu, re, b);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * width);
+          for (int i = lane; i < nvec; i += 32) d4[i] = __ldg(s4 + i);
+        }
+      }
+    }
+  } else {
+    const int R = offsets[E];
+    const int nb = gridDim.x - nbt;
+    for (int r = (blockIdx.x - nbt) * 8 + w; r < R; r += nb * 8) {
+      if (row_token[r] >= 0) continue;
+      uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * width);
+      for (int i = lane; i < nvec; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
-int launch_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets, int E,
-                       int width, int dtype, void* dst, cudaStream_t s) {
-  const int blocks = device_sm_count() * 8;
+int launch_scatter_rows(const void* src, const int32_t* slot_row, const int32_t* extra_row,
+                        const int32_t* row_token, const int32_t* offsets, int T, int width, int E,
+                        int k, int dtype, void* dst, cudaStream_t s) {
+  const int nbt = (T + 7) / 8;
+  const int blocks = nbt + device_sm_count() * 2;
   if (dtype == MOE_BF16) {
-    ProfScope _ps("gather_rows", s);
-    k_gather_rows<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        (const __nv_bfloat16*)src, row_token, offsets, E, width, (__nv_bfloat16*)dst);
+    ProfScope _ps("scatter_rows", s);
+    k_scatter_rows<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        (const __nv_bfloat16*)src, slot_row, extra_row, row_token, offsets, T, width, E, k, nbt,
+        (__nv_bfloat16*)dst);
   } else {
-    ProfScope _ps("gather_rows", s);
-    k_gather_rows<float><<<blocks, 256, 0, s>>>((const float*)src, row_token, offsets, E, width,
-                                                (float*)dst);
+    ProfScope _ps("scatter_rows", s);
+    k_scatter_rows<float><<<blocks, 256, 0, s>>>((const float*)src, slot_row, extra_row, row_token,
+                                                 offsets, T, width, E, k, nbt, (float*)dst);
   }
-  MOE_CHECK_LAUNCH("gather_rows");
+  MOE_CHECK_LAUNCH("scatter_rows");
+  return MOE_OK;
+}
+
+// ============================================================== fused dx (small router)
+// dx[t, :] = bf16( sum over t's rows of dX_perm[row, :] + sum_e dl[t, e] W_gate[:, e] )
+// for routers whose W_gate fits in shared memory (E <= 32, d*E*2 <= 48 KB).
+// One warp per token; a lane owns 8 consecutive columns per step and loads the
+// next step's rows before summing the current ones.
+__device__ __forceinline__ void load_rows8(const __nv_bfloat16* __restrict__ dxp, const int (&rk)[8],
+                                           int d, int i, uint4 (&raw)[8]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    raw[j] = rk[j] >= 0 ? __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)rk[j] * d) + i)
+                        : make_uint4(0, 0, 0, 0);
+}
+
+__global__ void __launch_bounds__(256)
+k_dx_fused(const __nv_bfloat16* __restrict__ dxp, const int32_t* __restrict__ slot_row,
+           const int32_t* __restrict__ extra_row, const float* __restrict__ dl,
+           const __nv_bfloat16* __restrict__ wg, int T_, int d, int E, int k,
+           __nv_bfloat16* __restrict__ dx) {
+  extern __shared__ __align__(16) uint8_t smem_wg[];
+  // W_gate transposed to [E][d] (bf16): a lane's 8 consecutive columns of one
+  // expert are one conflict-free 16-byte shared load.  Staged once per block
+  // (persistent grid); each thread owns whole columns.
+  __nv_bfloat16* w_t = reinterpret_cast<__nv_bfloat16*>(smem_wg);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    for (int e0 = 0; e0 < E; e0 += 8) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)c * E + e0));
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) w_t[(size_t)(e0 + q) * d + c] = h[q];
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nvec = d / 8;
+  for (int t = blockIdx.x * 8 + w; t < T_; t += gridDim.x * 8) {
+    float dlr[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) dlr[e] = e < E ? dl[(size_t)t * E + e] : 0.f;
+    const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    int rk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
+    uint4 nxt[8];
+    if (lane < nvec) load_rows8(dxp, rk, d, lane, nxt);
+    for (int i = lane; i < nvec; i += 32) {
+      uint4 raw[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) raw[j] = nxt[j];
+      if (i + 32 < nvec) load_rows8(dxp, rk, d, i + 32, nxt);
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rk[j] >= 0) {
+          Vec<__nv_bfloat16> v;
+          v.v = raw[j];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] += v.get(q);
+        }
+      }
+      if (extra_row != nullptr) {
+        for (int e0 = 0; e0 < E; e0 += 32) {
+          const int re = e0 + lane < E ? extra_row[(size_t)t * E + e0 + lane] : -1;
+          unsigned bal = __ballot_sync(__activemask(), re >= 0);
+          while (bal) {
+            const int b = __ffs(bal) - 1;
+            bal &= bal - 1;
+            const int r = __shfl_sync(__activemask(), re, b);
+            Vec<__nv_bfloat16> v;
+            v.v = __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)r * d) + i);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] += v.get(q);
+          }
+        }
+      }
+      // router term: columns 8i..8i+7 of every expert column of W_gate
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        if (e < E) {
+          Vec<__nv_bfloat16> wv;
+          wv.v = reinterpret_cast<const uint4*>(w_t + (size_t)e * d)[i];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[q] = fmaf(dlr[e], wv.get(q), acc[q]);
+        }
+      }
+      Vec<__nv_bfloat16> o;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) o.set(q, acc[q]);
+      reinterpret_cast<uint4*>(dx + (size_t)t * d)[i] = o.v;
+    }
+  }
+}
+
+bool dx_fused_ok(int d, int E) { return E <= 32 && E % 8 == 0 && (size_t)d * E * 2 <= 48 * 1024; }
+
+int launch_dx_fused(const void* dxp, const int32_t* slot_row, const int32_t* extra_row,
+                    const float* dl, const void* wg, int T, int d, int E, int k, void* dx,
+                    cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const size_t smem = (size_t)d * E * 2;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(k_dx_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "dx_fused smem attribute");
+  }
+  int blocks = (T + 7) / 8;
+  const int per_sm = (int)(200 * 1024 / (smem + 1024)) < 8 ? (int)(200 * 1024 / (smem + 1024)) : 8;
+  if (blocks > device_sm_count() * per_sm) blocks = device_sm_count() * per_sm;
+  {
+    ProfScope _ps("dx_fused", s);
+    k_dx_fused<<<blocks, 256, smem, s>>>((const __nv_bfloat16*)dxp, slot_row, extra_row, dl,
+                                         (const __nv_bfloat16*)wg, T, d, E, k, (__nv_bfloat16*)dx);
+  }
+  MOE_CHECK_LAUNCH("dx_fused");
   return MOE_OK;
 }
 

@@ -185,6 +185,12 @@ __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// Element i of 32 bf16 values packed in four uint4, as fp32.
+__device__ __forceinline__ float bf16_lane(const uint4 (&p)[4], int i) {
+  const uint32_t w = reinterpret_cast<const uint32_t*>(&p[i >> 3])[(i >> 1) & 3];
+  return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
 __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
   const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -398,6 +404,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
     for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      // DAP: the first chunk of H does not depend on the accumulator, so its
+      // loads are issued before waiting for the main loop
+      uint4 hn1[4], hn3[4];
+      const __nv_bfloat16* hrow = nullptr;
+      if constexpr (KIND == K_DAP) {
+        hrow = a.hin + (size_t)(ti.m0 + rloc) * 2 * a.f;
+        const uint4* s1 = reinterpret_cast<const uint4*>(hrow + ti.n0 + half * (BN / 2));
+        const uint4* s3 = reinterpret_cast<const uint4*>(hrow + a.f + ti.n0 + half * (BN / 2));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) { hn1[q] = s1[q]; hn3[q] = s3[q]; }
+      }
       if (!bounded_wait(&tfull_bar[acc], acc_phase, &s_abort, a.status, 4)) break;
       fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
@@ -439,29 +456,39 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
         const int f = a.f;
         const float g = a.row_gate[row];
         float ds = 0.f;
-        float h1[32], h3[32];
-        for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+        const int c_end = (half + 1) * (BN / 2);
+        for (int c = half * (BN / 2); c < c_end; c += 32) {
           tmem_ld32(tbase + c, r);
-          const __nv_bfloat16* hrow = a.hin + (size_t)row * 2 * f;
-          ld_bf16x32(hrow + ti.n0 + c, h1);
-          ld_bf16x32(hrow + f + ti.n0 + c, h3);
+          // this chunk's H (prefetched), then the next chunk's loads in flight
+          uint4 p1[4], p3[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) { p1[q] = hn1[q]; p3[q] = hn3[q]; }
+          if (c + 32 < c_end) {
+            const uint4* s1 = reinterpret_cast<const uint4*>(hrow + ti.n0 + c + 32);
+            const uint4* s3 = reinterpret_cast<const uint4*>(hrow + f + ti.n0 + c + 32);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) { hn1[q] = s1[q]; hn3[q] = s3[q]; }
+          }
           tmem_ld_wait();
           float da3[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
+            const float h1 = bf16_lane(p1, i), h3 = bf16_lane(p3, i);
             const float dap = __uint_as_float(r[i]);
-            const float sg = sigmoid_fast(h1[i]);
-            const float sl = h1[i] * sg;
-            const float av = bf16_round(sl * h3[i]);
+            const float sg = sigmoid_fast(h1);
+            const float sl = h1 * sg;
+            const float av = bf16_round(sl * h3);
             ds = fmaf(dap, av, ds);
             const float da = g * dap;
-            v[i] = da * h3[i] * (sg * (1.0f + h1[i] * (1.0f - sg)));
+            v[i] = da * h3 * (sg * (1.0f + h1 * (1.0f - sg)));
             da3[i] = da * sl;
-            h1[i] = g * av;                                           // s * A
+            r[i] = __float_as_uint(g * av);                           // s * A
           }
           stage_store(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
           stage_store(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
-          stage_store(otile, obuf, h1, &a.sO1, ti.n0 + c, row0, lane);      // s * A
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+          stage_store(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);      // s * A
         }
         a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
       } else if constexpr (KIND == K_RT) {
@@ -773,7 +800,7 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
     }
     MOE_CHECK_LAUNCH("dwg_reduce");
   }
-  {  // dx = fp32 unpermute-sum of dX_perm + dl W_gate^T
+  if (dx != nullptr) {  // dx = fp32 unpermute-sum of dX_perm + dl W_gate^T
     TcArgs a;
     memset(&a, 0, sizeof(a));
     a.E = E;

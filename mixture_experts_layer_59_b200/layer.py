@@ -43,8 +43,8 @@ class MoELayerStep:
                     self.gate, T=self.T, E=self.E, stream=stream)
         B.moe_permute(self.idx, self.gate, self.logits, self.E, self.round_mode, out=self.plan,
                       ws=self.ws_perm, stream=stream)
-        B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan["row_token"], self.plan["offsets"], self.k,
-                             self.H, self.Y, self.ws_fwd, stream=stream)
+        B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan, self.k, self.H, self.Y, self.ws_fwd,
+                             stream=stream)
         B.moe_combine(self.Y, self.plan["row_gate"], self.plan["slot_row"],
                       self.plan["extra_row"], self.T, self.E, self.k, self.out, stream=stream)
         return self.out

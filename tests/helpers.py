@@ -56,7 +56,7 @@ def gpu_layer(inp, k, round_mode, logits32, router_grad=True, dev="cuda"):
     T, E = lo.shape
     logits, idx, gate = B.moe_route(x, wg, k, logits_override=lo)
     plan = B.moe_permute(idx, gate, logits, E, round_mode)
-    H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan["row_token"], plan["offsets"], k)
+    H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
     out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)
     g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H, router_grad=router_grad)
     B.moe_check_status()

@@ -90,14 +90,14 @@ def test_permute_rejects_tile_and_mode():
 def test_ffn_rejects_unaligned_dims_and_small_workspace():
     lib = B.lib()
     fake = ctypes.c_void_p(256)
-    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, 16, 100, 128, 8, 2,
+    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, fake, None, 16, 100, 128, 8, 2,
                                 B.MOE_BF16, fake, fake, fake, 1 << 30, None)
     assert rc == -2
-    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, 16, 128, 128, 8, 2,
+    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, fake, None, 16, 128, 128, 8, 2,
                                 B.MOE_BF16, fake, fake, fake, 16, None)
     assert rc == -5
     odd = ctypes.c_void_p(258)
-    rc = lib.moe_expert_ffn_fwd(odd, fake, fake, fake, fake, fake, 16, 128, 128, 8, 2,
+    rc = lib.moe_expert_ffn_fwd(odd, fake, fake, fake, fake, fake, fake, None, 16, 128, 128, 8, 2,
                                 B.MOE_BF16, fake, fake, fake, 1 << 30, None)
     assert rc == -1
 
@@ -109,3 +109,11 @@ def test_bwd_rejects_missing_w_gate_with_router_grad():
             f, f, f, f, f, None, None, f, 1 << 40, None]
     assert lib.moe_layer_bwd(*args) == -1
     assert b"w_gate" in lib.moe_last_error()
+
+
+def test_ffn_requires_slot_row():
+    lib = B.lib()
+    fake = ctypes.c_void_p(256)
+    rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, None, None, 16, 128, 128, 8, 2,
+                                B.MOE_BF16, fake, fake, fake, 1 << 30, None)
+    assert rc == -1 and b"slot_row" in lib.moe_last_error()
