@@ -23,6 +23,9 @@ Sources (cited by page title and section):
   [Olmo]     Olmo-core 3 news piece -- "row-wise expert parallelism puts data
              straight into expert input buffers", GPU-resident routing,
              grouped GEMM.
+  [KJ]       "Breaking the hundred-billion-parameter barrier: how MoE reshapes
+             distributed training" -- challenge 1, solution 1: load-balance
+             loss L = lambda * CV(mean over the batch of G_i)^2.
 
 Readings taken where the pages are silent (each also listed in the design doc):
   * top-k then softmax over the k selected logits (sec. 5.3 / example 1); ties
@@ -40,6 +43,10 @@ Readings taken where the pages are silent (each also listed in the design doc):
     top-k logits); drops take the smallest keys (ties: larger token first),
     additions take the largest keys among unassigned tokens (ties: smaller
     token first); final weights are s_te without renormalisation.
+  * balance loss: G_i is token i's routing distribution over the E experts
+    (its top-k gates, zeros elsewhere); CV is the population coefficient of
+    variation over experts (std / mean); count statistics use the top-k
+    choices before any rounding.
 
 parity pins: tests/test_oracle_pins.py (brute force, dense masked evaluation,
 closed-form 2-expert example, central finite differences, the 145 -> 128
@@ -365,7 +372,8 @@ def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
                 A=res["A"], Y=res["Y"], out=out)
 
 
-def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True):
+def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True,
+              extra_dlogits=None):
     """Full backward from the saved set {x, logits, idx, gate, plan, H}.
 
     dW2_e = sum_rows (g A)^T dO,  [dW1|dW3]_e = sum_rows x^T dH,
@@ -395,6 +403,8 @@ def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True
         dlogits[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][tr])
         for r in tr:
             dx[t] += res["dXp"][r]
+    if extra_dlogits is not None:      # gradient of auxiliary router losses
+        dlogits = dlogits + np.asarray(extra_dlogits, np.float64)
     dw_gate = np.zeros((d, E))
     if router_grad_on:
         dx += dlogits @ w_gate.T
@@ -472,3 +482,50 @@ def expert_grad_slices(e, cols, dout, x, w1e, w3e, w2e, fwd, staged=True):
     da1 = _stage(da * h3 * silu_grad(h1), staged)
     ga = _stage(g[:, None] * a, staged)
     return dict(dw1=xr.T @ da1, dw3=xr.T @ da3, dw2=ga.T @ dor)
+
+
+# --------------------------------------------------------------------------
+# load-balance loss and routing statistics  ([KJ] challenge 1; [Trinity]
+# example 2; [Beam] sec. 2.3 / 5.4)
+# --------------------------------------------------------------------------
+
+def balance_loss(idx, gate, E, lam):
+    """L = lam * CV(importance)^2 with importance_e = mean over tokens of the
+    token's routing weight on expert e (0 if e is not among its top-k).
+
+    Returns dict(loss, importance [E], dgate [T,k] = dL/dgate, counts [E],
+    max_share, count_cv2, count_mse) where the count statistics follow the
+    per-expert token histogram: max share of all assignments, CV^2 of the
+    counts and the mean squared deviation of the counts from their mean.
+    """
+    idx = np.asarray(idx)
+    gate = np.asarray(gate, np.float64)
+    T, k = idx.shape
+    G = np.zeros((T, E))
+    G[np.arange(T)[:, None], idx] = gate
+    imp = G.mean(axis=0)
+    m = imp.mean()
+    var = ((imp - m) ** 2).mean()
+    loss = lam * var / m ** 2
+    # d(var/m^2)/d imp_e = (2/E)(imp_e - m)/m^2 - 2 var/(E m^3)
+    dimp = lam * (2.0 / E * (imp - m) / m ** 2 - 2.0 * var / (E * m ** 3))
+    dgate = dimp[idx] / T
+    counts = np.bincount(idx.ravel(), minlength=E).astype(np.float64)
+    cm = counts.mean()
+    return dict(loss=loss, importance=imp, dgate=dgate, counts=counts,
+                max_share=counts.max() / counts.sum(),
+                count_cv2=((counts - cm) ** 2).mean() / cm ** 2,
+                count_mse=((counts - cm) ** 2).mean())
+
+
+def gate_grad_to_logits(idx, gate, dgate, E):
+    """dlogits from a gradient on the top-k gates (softmax over the k logits):
+    dl_t,idx_j = g_j (a_j - sum_i g_i a_i) with a = dgate; zero elsewhere."""
+    idx = np.asarray(idx)
+    gate = np.asarray(gate, np.float64)
+    dgate = np.asarray(dgate, np.float64)
+    T, k = idx.shape
+    dl = np.zeros((T, E))
+    tot = (gate * dgate).sum(axis=1, keepdims=True)
+    dl[np.arange(T)[:, None], idx] = gate * (dgate - tot)
+    return dl

@@ -409,3 +409,86 @@ def test_rows_compute_accepts_per_expert_weight_access():
     s2 = O.sampled_tokens([3, 9], dout, x, wg, Lazy(w1), Lazy(w3), Lazy(w2), fwd)
     for t in (3, 9):
         np.testing.assert_allclose(s1["dx"][t], s2["dx"][t], rtol=1e-6, atol=1e-9)
+
+
+# ---------------------------------------------------------------- balance loss
+
+def test_balance_loss_closed_form_uniform_and_collapsed():
+    # perfectly balanced routing: every expert gets the same importance -> 0
+    T, E, k = 8, 4, 1
+    idx = np.array([[t % E] for t in range(T)])
+    gate = np.ones((T, k))
+    r = O.balance_loss(idx, gate, E, lam=0.5)
+    assert r["loss"] == 0 and r["count_mse"] == 0 and r["max_share"] == 0.25
+    # every token on expert 0: importance = [1,0,0,0], mean 1/4, var 3/16,
+    # CV^2 = (3/16)/(1/16) = 3 = E - 1
+    idx = np.zeros((T, 1), int)
+    r = O.balance_loss(idx, gate, E, lam=2.0)
+    assert abs(r["loss"] - 2.0 * 3) < 1e-12
+    assert r["max_share"] == 1.0 and abs(r["count_cv2"] - 3) < 1e-12
+    # counts [8,0,0,0]: mean 2, squared deviations 36,4,4,4 -> mse 12
+    assert abs(r["count_mse"] - 12) < 1e-12
+
+
+def test_balance_loss_matches_torch_autograd():
+    rng = np.random.default_rng(17)
+    T, E, k = 20, 6, 2
+    logits = rng.standard_normal((T, E))
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    r = O.balance_loss(idx, gate, E, lam=0.3)
+    g = torch.tensor(gate, requires_grad=True)
+    G = torch.zeros(T, E, dtype=torch.float64).scatter(1, torch.tensor(idx, dtype=torch.int64), g)
+    imp = G.mean(0)
+    loss = 0.3 * imp.var(unbiased=False) / imp.mean() ** 2
+    loss.backward()
+    assert abs(loss.item() - r["loss"]) < 1e-12
+    np.testing.assert_allclose(r["dgate"], g.grad.numpy(), rtol=1e-10, atol=1e-14)
+    np.testing.assert_allclose(r["importance"], imp.detach().numpy(), rtol=1e-12)
+
+
+def test_gate_grad_to_logits_matches_finite_differences():
+    rng = np.random.default_rng(18)
+    T, E, k = 6, 5, 3
+    logits = rng.standard_normal((T, E))
+    _, idx, gate = O.route(None, None, k, logits_override=logits)
+    a = rng.standard_normal((T, k))
+    dl = O.gate_grad_to_logits(idx, gate, a, E)
+    h = 1e-6
+    for t in range(T):
+        for e in range(E):
+            lp, lm = logits.copy(), logits.copy()
+            lp[t, e] += h
+            lm[t, e] -= h
+            gp = O.route(None, None, k, logits_override=lp)[2]
+            gm = O.route(None, None, k, logits_override=lm)[2]
+            num = ((gp - gm) * a).sum() / (2 * h)
+            assert abs(num - dl[t, e]) < 1e-7
+
+
+def test_layer_with_balance_loss_matches_central_differences():
+    """Total loss = <dO, O> + lambda CV^2: gradients through both terms."""
+    rng = np.random.default_rng(19)
+    T, d, f, E, k, tile, lam = 9, 4, 3, 4, 2, 4, 0.7
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, T, d, f, E)
+
+    def total(xx, wgg):
+        fwd = O.layer_fwd(xx, wgg, w1, w3, w2, k=k, tile=tile, staged=False)
+        return float(np.sum(fwd["out"] * dout)) + O.balance_loss(fwd["idx"], fwd["gate"], E, lam)["loss"], fwd
+
+    _, fwd = total(x, wg)
+    bl = O.balance_loss(fwd["idx"], fwd["gate"], E, lam)
+    extra = O.gate_grad_to_logits(fwd["idx"], fwd["gate"], bl["dgate"], E)
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False, extra_dlogits=extra)
+    h = 1e-6
+    for p, g in ((x, bwd["dx"]), (wg, bwd["dw_gate"])):
+        num = np.zeros_like(p)
+        for i in np.ndindex(p.shape):
+            old = p[i]
+            p[i] = old + h
+            lp, fp = total(x, wg)
+            p[i] = old - h
+            lm, fm = total(x, wg)
+            p[i] = old
+            assert np.array_equal(fp["idx"], fwd["idx"]) and np.array_equal(fm["idx"], fwd["idx"])
+            num[i] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-7)
