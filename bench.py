@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
     ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer written between steps")
+    ap.add_argument("--balance-loss", type=float, default=None,
+                    help="add the load-balance loss (this lambda) and its gradient to every step")
     return ap.parse_args()
 
 
@@ -208,6 +210,7 @@ def run_reference(args, cfg, rank, world):
 def workload_config(cfg, args):
     return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "d_ff": cfg.f, "E": cfg.E,
             "k": cfg.k, "routing": cfg.routing, "token_rounding": bool(args.round),
+            "balance_loss_lambda": args.balance_loss,
             "l2": f"flushed between timed steps ({args.flush_mb} MiB write)", "replicas": args.gpus}
 
 
@@ -223,7 +226,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(cfg, seed=rank, device=dev)
-    step = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round)
+    step = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round,
+                        balance_lambda=args.balance_loss)
     flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
     x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo, lb = inp["logits_override"], inp["logit_bias"]

@@ -187,6 +187,9 @@ int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_r
  *   dW_gate = x^T dlogits.
  *   router_grad = 0 when the logits did not come from x W_gate (override):
  *   dW_gate is then zero and dx gets no router term.
+ *   gate_grad [T,k] fp32 or NULL: gradient of auxiliary losses with respect
+ *   to the gates (e.g. from moe_balance_loss); it enters dlogits through the
+ *   softmax over the k logits: dl_t,idx_j += g_j (a_j - sum_i g_i a_i).
  *   Outputs: dx [T,d] (dtype), dw_gate [d,E] fp32, dw1, dw3 [E,d,f] (dtype),
  *   dw2 [E,f,d] (dtype), dS [cap] fp32 (may be NULL), dlogits [T,E] fp32
  *   (may be NULL).  Every output element is written (no accumulation).
@@ -194,12 +197,34 @@ int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_r
 size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype);
 int moe_layer_bwd(const void* dout, const void* x, const void* w_gate,
                   const void* w1, const void* w3, const void* w2,
-                  const int32_t* idx, const float* gate, const int32_t* offsets,
+                  const int32_t* idx, const float* gate, const float* gate_grad,
+                  const int32_t* offsets,
                   const int32_t* row_token, const float* row_gate,
                   const int32_t* slot_row, const int32_t* extra_row, const void* H,
                   int T, int d, int f, int E, int k, int dtype, int router_grad,
                   void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2,
                   float* dS, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_balance_loss -- load-balance loss and routing statistics.
+ * ["Breaking the hundred-billion-parameter barrier: how MoE reshapes
+ * distributed training", challenge 1, solution 1]: L = lambda * CV(m)^2 with
+ * m_e = (1/T) sum_t G_te the mean routing distribution (G_t: token t's top-k
+ * gates, zero elsewhere) and CV the population coefficient of variation over
+ * the E experts.  Statistics of the expert token counts: [Trinity] example 2
+ * (bincount, squared deviation from the mean), [Beam] sec. 5.4 (share of the
+ * busiest expert).
+ *   idx [T,k], gate [T,k] from moe_route (T >= 1).
+ *   stats [4] fp32 out: loss, max share of assignments, CV^2 of the counts,
+ *     mean squared deviation of the counts from their mean.
+ *   importance [E] fp32 out: m.
+ *   dgate [T,k] fp32 out or NULL: dL/dgate, to pass to moe_layer_bwd.
+ *   All sums run in a fixed order (deterministic).
+ */
+size_t moe_balance_loss_workspace_size(int T, int E, int k);
+int moe_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k, float lambda,
+                     float* stats, float* importance, float* dgate, void* ws, size_t ws_bytes,
+                     void* stream);
 
 /*
  * moe_check_status -- synchronises `stream`, then returns MOE_OK, a CUDA

@@ -24,6 +24,7 @@ EXPORTS = [
     "moe_permute_workspace_size", "moe_permute", "moe_ffn_fwd_workspace_size",
     "moe_expert_ffn_fwd", "moe_combine", "moe_layer_bwd_workspace_size", "moe_layer_bwd",
     "moe_check_status", "moe_profile_enable", "moe_profile_report", "moe_permute_noalloc",
+    "moe_balance_loss_workspace_size", "moe_balance_loss",
 ]
 
 _lib = None
@@ -50,7 +51,9 @@ _SIGS = {
                                 _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_layer_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
-    "moe_layer_bwd": (_i, [_vp] * 14 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
+    "moe_layer_bwd": (_i, [_vp] * 15 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
+    "moe_balance_loss_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
     "moe_profile_enable": (_i, [_i]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -188,7 +191,7 @@ def moe_layer_bwd_workspace_size(T, d, f, E, k, dtype) -> int:
 
 
 def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=True, out=None,
-                  ws=None, stream=None):
+                  ws=None, stream=None, gate_grad=None):
     """plan: dict from moe_permute.  Returns dict dx, dw_gate, dw1, dw3, dw2, dS, dlogits."""
     T, d = x.shape
     E, _, f = w1.shape
@@ -208,7 +211,7 @@ def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=T
         ws = torch.empty(max(moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), device=dev,
                          dtype=torch.uint8)
     _check(lib().moe_layer_bwd(
-        _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(idx), _p(gate),
+        _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(idx), _p(gate), _p(gate_grad),
         _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
         _p(plan["extra_row"]), _p(H), T, d, f, E, k, dt, 1 if router_grad else 0,
         _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
@@ -254,3 +257,19 @@ def moe_permute_noalloc(idx, gate, E, tile=TILE, out=None, stream=None):
                                      _p(o["offsets"]), _p(o["row_token"]), _p(o["row_gate"]),
                                      _p(o["row_slot"]), _p(o["slot_row"]), _stream(stream)))
     return o
+
+
+def moe_balance_loss(idx, gate, E, lam, dgate=True, ws=None, stream=None):
+    """Returns dict(stats [4] = loss, max share, count CV^2, count MSE;
+    importance [E]; dgate [T,k] or None)."""
+    T, k = idx.shape
+    dev = idx.device
+    stats = torch.empty(4, device=dev, dtype=torch.float32)
+    imp = torch.empty(E, device=dev, dtype=torch.float32)
+    dg = torch.empty(T, k, device=dev, dtype=torch.float32) if dgate else None
+    if ws is None:
+        ws = torch.empty(max(lib().moe_balance_loss_workspace_size(T, E, k), 1), device=dev,
+                         dtype=torch.uint8)
+    _check(lib().moe_balance_loss(_p(idx), _p(gate), T, E, k, float(lam), _p(stats), _p(imp),
+                                  _p(dg), _p(ws), ws.numel(), _stream(stream)))
+    return dict(stats=stats, importance=imp, dgate=dg)

@@ -302,7 +302,7 @@ size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype
 
 int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
                   const void* w3, const void* w2, const int32_t* idx, const float* gate,
-                  const int32_t* offsets, const int32_t* row_token, const float* row_gate,
+                  const float* gate_grad, const int32_t* offsets, const int32_t* row_token, const float* row_gate,
                   const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
                   int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
                   void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
@@ -342,8 +342,8 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   }
   float* dl = dlogits ? dlogits : w.dl;
   const bool tc_router = router_grad && w.dl_hi != nullptr;
-  if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row, T, E, k,
-                              dl, dS, tc_router ? w.dl_hi : nullptr,
+  if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row,
+                              gate_grad, T, E, k, dl, dS, tc_router ? w.dl_hi : nullptr,
                               tc_router ? w.dl_lo : nullptr, s)))
     return rc;
   if (tc_router) {
@@ -406,6 +406,24 @@ int moe_profile_report(char* buf, size_t buf_len) {
   if (out.size() + 1 > buf_len) return fail(MOE_ERR_INVALID_ARG, "report buffer too small");
   memcpy(buf, out.c_str(), out.size() + 1);
   return rc;
+}
+
+size_t moe_balance_loss_workspace_size(int T, int E, int k) {
+  (void)k;
+  if (T < 0 || E <= 0) return 0;
+  return balance_ws_bytes(T, E);
+}
+
+int moe_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k, float lambda,
+                     float* stats, float* importance, float* dgate, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (int rc = check_common(T, E, k, MOE_F32)) return rc;
+  if (T == 0) return fail(MOE_ERR_INVALID_ARG, "the balance loss needs T >= 1");
+  REQUIRE_PTR(idx); REQUIRE_PTR(gate); REQUIRE_PTR(stats); REQUIRE_PTR(importance);
+  if (ws_bytes < balance_ws_bytes(T, E))
+    return fail(MOE_ERR_WORKSPACE, "balance workspace smaller than moe_balance_loss_workspace_size()");
+  return launch_balance_loss(idx, gate, T, E, k, lambda, stats, importance, dgate, ws, ws_bytes,
+                             (cudaStream_t)stream);
 }
 
 int moe_check_status(void* stream) {

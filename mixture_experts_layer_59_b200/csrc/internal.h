@@ -55,8 +55,13 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
 // Optionally also writes dlogits split as bf16 hi + bf16 lo (tensor-core router GEMMs).
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      int T, int E, int k, float* dlogits, float* dS_out, void* dl_hi,
-                      void* dl_lo, cudaStream_t s);
+                      const float* gate_grad, int T, int E, int k, float* dlogits, float* dS_out,
+                      void* dl_hi, void* dl_lo, cudaStream_t s);
+// Load-balance loss lambda*CV^2, routing statistics and dL/dgate.
+size_t balance_ws_bytes(int T, int E);
+int launch_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k, float lam,
+                        float* stats, float* importance, float* dgate, void* ws, size_t ws_bytes,
+                        cudaStream_t s);
 
 // ---------------------------------------------------------------- CUDA-core GEMM path
 struct FfnPtrs {

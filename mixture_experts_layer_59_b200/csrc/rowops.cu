@@ -319,6 +319,135 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
   return MOE_OK;
 }
 
+// ============================================================== load-balance loss
+// importance_e = (1/T) sum_t G_te, G_t = token t's top-k gates (zero elsewhere);
+// L = lambda * CV(importance)^2 with the population CV over the E experts
+// ("Breaking the hundred-billion-parameter barrier" article, challenge 1);
+// token counts per expert give the routing statistics (Trinity commentary
+// example 2, Beam article sec. 5.4).  All sums run in a fixed order.
+constexpr int BAL_TOK = 256;
+
+__global__ void __launch_bounds__(256)
+k_balance_partial(const int32_t* __restrict__ idx, const float* __restrict__ gate, int T, int E,
+                  int k, float* __restrict__ psum, int32_t* __restrict__ pcnt) {
+  __shared__ int s_key[BAL_TOK * 8];
+  __shared__ float s_val[BAL_TOK * 8];
+  const int t0 = blockIdx.x * BAL_TOK;
+  const int n = min(BAL_TOK, T - t0) * k;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    s_key[i] = idx[(size_t)t0 * k + i];
+    s_val[i] = gate[(size_t)t0 * k + i];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float acc = 0.f;
+    int c = 0;
+    for (int i = 0; i < n; ++i) {
+      if (s_key[i] == e) { acc += s_val[i]; ++c; }
+    }
+    psum[(size_t)blockIdx.x * E + e] = acc;
+    pcnt[(size_t)blockIdx.x * E + e] = c;
+  }
+}
+
+// One block: reduce the partials, then loss, statistics and dL/dimportance.
+__global__ void __launch_bounds__(256)
+k_balance_final(const float* __restrict__ psum, const int32_t* __restrict__ pcnt, int nb, int T,
+                int E, float lam, float* __restrict__ stats, float* __restrict__ importance,
+                float* __restrict__ dimp) {
+  __shared__ float s_imp[256];
+  __shared__ float s_cnt[256];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    float acc = 0.f;
+    int c = 0;
+    for (int b = 0; b < nb; ++b) {
+      acc += psum[(size_t)b * E + e];
+      c += pcnt[(size_t)b * E + e];
+    }
+    s_imp[e] = acc / (float)T;
+    s_cnt[e] = (float)c;
+    importance[e] = acc / (float)T;
+  }
+  __syncthreads();
+  __shared__ float s_m, s_var, s_cm, s_cvar, s_cmax, s_ctot;
+  if (threadIdx.x == 0) {
+    double m = 0, cm = 0, cmax = 0, ctot = 0;
+    for (int e = 0; e < E; ++e) {
+      m += s_imp[e];
+      cm += s_cnt[e];
+      cmax = fmax(cmax, (double)s_cnt[e]);
+    }
+    ctot = cm;
+    m /= E;
+    cm /= E;
+    double var = 0, cvar = 0;
+    for (int e = 0; e < E; ++e) {
+      var += (s_imp[e] - m) * (s_imp[e] - m);
+      cvar += (s_cnt[e] - cm) * (s_cnt[e] - cm);
+    }
+    var /= E;
+    cvar /= E;
+    s_m = (float)m;
+    s_var = (float)var;
+    stats[0] = (float)(lam * var / (m * m));
+    stats[1] = ctot > 0 ? (float)(cmax / ctot) : 0.f;
+    stats[2] = cm > 0 ? (float)(cvar / (cm * cm)) : 0.f;
+    stats[3] = (float)cvar;
+  }
+  __syncthreads();
+  // d(var/m^2)/d imp_e = (2/E)(imp_e - m)/m^2 - 2 var/(E m^3)
+  const float m = s_m, var = s_var;
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    dimp[e] = lam * (2.0f / E * (s_imp[e] - m) / (m * m) - 2.0f * var / (E * m * m * m));
+}
+
+__global__ void k_balance_dgate(const int32_t* __restrict__ idx, const float* __restrict__ dimp,
+                                int n, float inv_T, float* __restrict__ dgate) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    dgate[i] = dimp[idx[i]] * inv_T;
+}
+
+size_t balance_ws_bytes(int T, int E) {
+  Sizer z;
+  const int nb = (T + BAL_TOK - 1) / BAL_TOK;
+  z.take<float>((size_t)nb * E);
+  z.take<int32_t>((size_t)nb * E);
+  z.take<float>(E);
+  return z.used;
+}
+
+int launch_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k, float lam,
+                        float* stats, float* importance, float* dgate, void* ws, size_t ws_bytes,
+                        cudaStream_t s) {
+  Carve c(ws, ws_bytes);
+  const int nb = (T + BAL_TOK - 1) / BAL_TOK;
+  float* psum = c.take<float>((size_t)nb * E);
+  int32_t* pcnt = c.take<int32_t>((size_t)nb * E);
+  float* dimp = c.take<float>(E);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "balance-loss workspace too small");
+  {
+    ProfScope _ps("balance_partial", s);
+    k_balance_partial<<<nb, 256, 0, s>>>(idx, gate, T, E, k, psum, pcnt);
+  }
+  MOE_CHECK_LAUNCH("balance_partial");
+  {
+    ProfScope _ps("balance_final", s);
+    k_balance_final<<<1, 256, 0, s>>>(psum, pcnt, nb, T, E, lam, stats, importance, dimp);
+  }
+  MOE_CHECK_LAUNCH("balance_final");
+  if (dgate != nullptr) {
+    const int n = T * k;
+    int blocks = (n + 255) / 256;
+    if (blocks > device_sm_count() * 4) blocks = device_sm_count() * 4;
+    {
+      ProfScope _ps("balance_dgate", s);
+      k_balance_dgate<<<blocks, 256, 0, s>>>(idx, dimp, n, 1.0f / (float)T, dgate);
+    }
+    MOE_CHECK_LAUNCH("balance_dgate");
+  }
+  return MOE_OK;
+}
+
 // ============================================================== router backward
 // One warp per token.  dS of a row = sum of its partials (fixed order).
 //   v_r = row_gate[r] * dS[r] for every row r of token t (expert e_r)
@@ -326,9 +455,10 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
 __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
                              const int32_t* __restrict__ idx, const float* __restrict__ gate,
                              const float* __restrict__ row_gate, const int32_t* __restrict__ slot_row,
-                             const int32_t* __restrict__ extra_row, int T, int E, int k,
-                             float* __restrict__ dlogits, float* __restrict__ dS_out,
-                             __nv_bfloat16* __restrict__ dl_hi, __nv_bfloat16* __restrict__ dl_lo) {
+                             const int32_t* __restrict__ extra_row, const float* __restrict__ gate_grad,
+                             int T, int E, int k, float* __restrict__ dlogits,
+                             float* __restrict__ dS_out, __nv_bfloat16* __restrict__ dl_hi,
+                             __nv_bfloat16* __restrict__ dl_lo) {
   __shared__ float s_dl[8][256];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   float* dl = s_dl[w];
@@ -365,9 +495,22 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     __syncwarp();
+    // gradient of auxiliary router losses on the gates, through the
+    // softmax over the k logits: g_j (a_j - sum_i g_i a_i)
+    float ga = 0.f, aj = 0.f;
+    if (gate_grad != nullptr && lane < k) {
+      aj = gate_grad[(size_t)t * k + lane];
+      ga = gate[(size_t)t * k + lane] * aj;
+    }
+    if (gate_grad != nullptr) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, o);
+    }
     if (lane < k) {
       const int e = idx[(size_t)t * k + lane];
-      dl[e] -= gate[(size_t)t * k + lane] * part;
+      const float gj = gate[(size_t)t * k + lane];
+      dl[e] -= gj * part;
+      if (gate_grad != nullptr) dl[e] += gj * (aj - ga);
     }
     __syncwarp();
     for (int e = lane; e < E; e += 32) {
@@ -386,15 +529,15 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
 
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      int T, int E, int k, float* dlogits, float* dS_out, void* dl_hi,
-                      void* dl_lo, cudaStream_t s) {
+                      const float* gate_grad, int T, int E, int k, float* dlogits, float* dS_out,
+                      void* dl_hi, void* dl_lo, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
   {
     ProfScope _ps("router_bwd", s);
-    k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row, T,
-                                        E, k, dlogits, dS_out, (__nv_bfloat16*)dl_hi,
+    k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row,
+                                        gate_grad, T, E, k, dlogits, dS_out, (__nv_bfloat16*)dl_hi,
                                         (__nv_bfloat16*)dl_lo);
   }
   MOE_CHECK_LAUNCH("router_bwd");

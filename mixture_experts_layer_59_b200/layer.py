@@ -15,7 +15,7 @@ class MoELayerStep:
     """
 
     def __init__(self, T, d, f, E, k, dtype=torch.bfloat16, device="cuda",
-                 round_mode=B.MOE_ROUND_NONE):
+                 round_mode=B.MOE_ROUND_NONE, balance_lambda=None):
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         self.dtype, self.device, self.round_mode = dtype, device, round_mode
         dt = B.dtype_code(dtype)
@@ -32,6 +32,10 @@ class MoELayerStep:
         self.ws_perm = e(max(B.moe_permute_workspace_size(T, E, k, round_mode), 1), dt_=torch.uint8)
         self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
         self.ws_bwd = e(max(B.moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
+        self.balance_lambda = balance_lambda
+        if balance_lambda is not None:
+            self.ws_bal = e(max(B.lib().moe_balance_loss_workspace_size(T, E, k), 1), dt_=torch.uint8)
+        self.balance = None
         self.grads = dict(dx=e(T, d, dt_=dtype), dw_gate=e(d, E), dw1=e(E, d, f, dt_=dtype),
                           dw3=e(E, d, f, dt_=dtype), dw2=e(E, f, d, dt_=dtype), dS=e(cap),
                           dlogits=e(T, E))
@@ -43,6 +47,9 @@ class MoELayerStep:
                     self.gate, T=self.T, E=self.E, stream=stream)
         B.moe_permute(self.idx, self.gate, self.logits, self.E, self.round_mode, out=self.plan,
                       ws=self.ws_perm, stream=stream)
+        if self.balance_lambda is not None:
+            self.balance = B.moe_balance_loss(self.idx, self.gate, self.E, self.balance_lambda,
+                                              ws=self.ws_bal, stream=stream)
         B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan, self.k, self.H, self.Y, self.ws_fwd,
                              stream=stream)
         B.moe_combine(self.Y, self.plan["row_gate"], self.plan["slot_row"],
@@ -53,16 +60,5 @@ class MoELayerStep:
         x, w_gate, w1, w3, w2 = self._saved
         return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
                                self.H, self.router_grad, out=self.grads, ws=self.ws_bwd,
-                               stream=stream)
-
-    # number of library kernel launches of one step (forward + backward)
-    def launches_per_step(self, tensor_cores: bool) -> int:
-        route = 2 if self.router_grad else 1
-        perm = 3 if not self.round_mode else 5
-        if tensor_cores:
-            fwd = 3 + 1
-            bwd = 2 + 4 + 1 + (3 if self.router_grad else 2)
-        else:
-            fwd = 3 + 1
-            bwd = 5 + 1 + (3 if self.router_grad else 1)
-        return route + perm + fwd + bwd
+                               stream=stream,
+                               gate_grad=self.balance["dgate"] if self.balance else None)

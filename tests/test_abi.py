@@ -105,7 +105,7 @@ def test_ffn_rejects_unaligned_dims_and_small_workspace():
 def test_bwd_rejects_missing_w_gate_with_router_grad():
     lib = B.lib()
     f = ctypes.c_void_p(256)
-    args = [f, f, None, f, f, f, f, f, f, f, f, f, None, f, 16, 128, 128, 8, 2, B.MOE_BF16, 1,
+    args = [f, f, None, f, f, f, f, f, None, f, f, f, f, None, f, 16, 128, 128, 8, 2, B.MOE_BF16, 1,
             f, f, f, f, f, None, None, f, 1 << 40, None]
     assert lib.moe_layer_bwd(*args) == -1
     assert b"w_gate" in lib.moe_last_error()
@@ -117,3 +117,10 @@ def test_ffn_requires_slot_row():
     rc = lib.moe_expert_ffn_fwd(fake, fake, fake, fake, fake, fake, None, None, 16, 128, 128, 8, 2,
                                 B.MOE_BF16, fake, fake, fake, 1 << 30, None)
     assert rc == -1 and b"slot_row" in lib.moe_last_error()
+
+
+def test_balance_loss_rejects_empty_batch_and_small_workspace():
+    lib = B.lib()
+    f = ctypes.c_void_p(256)
+    assert lib.moe_balance_loss(f, f, 0, 8, 2, 0.1, f, f, None, f, 1 << 20, None) == -1
+    assert lib.moe_balance_loss(f, f, 100, 8, 2, 0.1, f, f, None, f, 4, None) == -5

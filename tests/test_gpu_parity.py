@@ -143,3 +143,43 @@ def test_zero_tokens_is_a_no_op():
     torch.cuda.synchronize()
     assert i64(plan["offsets"]).tolist() == [0] * (E + 1)
     assert i64(plan["counts"]).tolist() == [0] * E
+
+
+# ------------------------------------------------------------------ load-balance loss
+
+@pytest.mark.parametrize("T,E,k,skew", [(1000, 8, 2, 0.0), (4097, 64, 8, 1.1), (3000, 256, 8, 1.5)])
+def test_balance_loss_and_stats(T, E, k, skew):
+    g = torch.Generator().manual_seed(T + E)
+    lo = torch.randn(T, E, generator=g)
+    if skew:
+        rank = torch.randperm(E, generator=g).double() + 1
+        lo = lo + (-skew * torch.log(rank)).float()[None, :]
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E)
+    r = B.moe_balance_loss(idx, gate, E, lam=0.01)
+    torch.cuda.synchronize()
+    ref = O.balance_loss(i64(idx), f64(gate), E, 0.01)
+    st = f64(r["stats"])
+    np.testing.assert_allclose(st[0], ref["loss"], rtol=1e-5)
+    np.testing.assert_allclose(st[1:], [ref["max_share"], ref["count_cv2"], ref["count_mse"]], rtol=1e-5)
+    np.testing.assert_allclose(f64(r["importance"]), ref["importance"], rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(f64(r["dgate"]), ref["dgate"], rtol=1e-4, atol=1e-9 * np.abs(ref["dgate"]).max())
+
+
+def test_layer_with_balance_loss_gradient():
+    cfg = _cfg(1000, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=13, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    logits, idx, gate = B.moe_route(x, wg, cfg.k, logits_override=torch.from_numpy(lg).cuda())
+    plan = B.moe_permute(idx, gate, logits, cfg.E)
+    H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, cfg.k)
+    bl = B.moe_balance_loss(idx, gate, cfg.E, lam=0.05)
+    gr = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H, gate_grad=bl["dgate"])
+    B.moe_check_status()
+    torch.cuda.synchronize()
+    fwd, _ = oracle_layer(inp, cfg.k, 0, lg)
+    rb = O.balance_loss(fwd["idx"], fwd["gate"], cfg.E, 0.05)
+    extra = O.gate_grad_to_logits(fwd["idx"], fwd["gate"], rb["dgate"], cfg.E)
+    bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd, extra_dlogits=extra)
+    for n in ("dlogits", "dw_gate", "dx", "dw1"):
+        assert_close(gr[n], bwd[n], n, BF16_TOL)
