@@ -106,9 +106,12 @@ def silu_grad(z):
 # router: logits, top-k, softmax over the top-k  ([Beam] 2.2, 5.3; [Trinity] ex. 1)
 # --------------------------------------------------------------------------
 
-def route(x, w_gate, k, logits_override=None, logit_bias=None):
+def route(x, w_gate, k, logits_override=None, logit_bias=None, gate_mode=0):
     """Router logits l = x W_gate (+ optional per-expert bias), the k largest
-    logits of each token (ties: lowest expert id first), and their softmax.
+    logits of each token (ties: lowest expert id first), and their gates:
+    gate_mode 0: softmax over the k selected logits ([Beam] 5.3, [Trinity] ex. 1);
+    gate_mode 1: softmax over all E logits, the k largest kept without
+    renormalisation ([Beam] 2.2 formula, [Trinity] challenge 1).
 
     Returns (logits [T,E] f64, idx [T,k] int32, gate [T,k] f64).
     """
@@ -121,8 +124,13 @@ def route(x, w_gate, k, logits_override=None, logit_bias=None):
     # a stable sort of the negated logits keeps equal values in ascending id
     idx = np.argsort(-logits, axis=1, kind="stable")[:, :k]
     top = np.take_along_axis(logits, idx, axis=1)
-    ex = np.exp(top - top[:, :1])
-    gate = ex / ex.sum(axis=1, keepdims=True)
+    if gate_mode == 0:
+        ex = np.exp(top - top[:, :1])
+        gate = ex / ex.sum(axis=1, keepdims=True)
+    else:
+        m = logits.max(axis=1, keepdims=True)
+        z = np.exp(logits - m).sum(axis=1, keepdims=True)
+        gate = np.exp(top - m) / z
     return logits, idx.astype(np.int32), gate
 
 
@@ -182,26 +190,42 @@ def rounded_target(counts, T, tile=TILE):
     return np.minimum(r, tile * (T // tile))
 
 
-def rounding_keys(logits, idx):
-    """Log-domain ranking key l_te - LSE_{j in top-k(t)} l_tj for every
-    (token, expert) pair; exp(key) is the routing weight of a selected pair."""
+def rounding_keys(logits, idx, gate_mode=0):
+    """Log-domain ranking key of every (token, expert) pair: the log of the
+    weight the pair has (or would have) as a routed pair, i.e.
+    l_te - LSE over the token's top-k logits (gate_mode 0) or over all E
+    logits (gate_mode 1)."""
     logits = np.asarray(logits, np.float64)
-    top = np.take_along_axis(logits, np.asarray(idx), axis=1)
+    if gate_mode == 0:
+        top = np.take_along_axis(logits, np.asarray(idx), axis=1)
+    else:
+        top = logits
     m = top.max(axis=1)
     lse = m + np.log(np.exp(top - m[:, None]).sum(axis=1))
     return logits - lse[:, None]
 
 
-def rounded_plan(idx, logits, E, tile=TILE):
+def capacity_target(counts, capacity):
+    """Capacity factor ([Beam] sec. 2.3): at most `capacity` tokens per expert."""
+    return np.minimum(np.asarray(counts, np.int64), capacity)
+
+
+def rounded_plan(idx, logits, E, tile=TILE, gate_mode=0, capacity=None):
     """Token-rounded permutation ([SonicMoE] sec. 3 with the readings in the
-    module docstring).  Adds ``extra_row[T,E]`` (row of an added pair, else -1)
-    and ``dropped``/``added`` masks for checking."""
+    module docstring), or with ``capacity`` the capacity-factor permutation
+    ([Beam] sec. 2.3: experts above capacity drop their lowest-scoring pairs,
+    ties dropping the larger token first; no pairs are added; segments are
+    padded to the tile).  Adds ``extra_row[T,E]`` (row of an added pair, else
+    -1) and ``dropped``/``added`` masks for checking."""
     idx = np.asarray(idx)
     T, k = idx.shape
     cap = row_capacity(T, E, k, tile)
     counts = np.bincount(idx.ravel(), minlength=E).astype(np.int64)
-    target = rounded_target(counts, T, tile)
-    key = rounding_keys(logits, idx)
+    if capacity is None:
+        target = rounded_target(counts, T, tile)
+    else:
+        target = capacity_target(counts, capacity)
+    key = rounding_keys(logits, idx, gate_mode)
     assigned = np.zeros((T, E), bool)
     assigned[np.arange(T)[:, None], idx] = True
     final = assigned.copy()
@@ -217,7 +241,7 @@ def rounded_plan(idx, logits, E, tile=TILE):
             order = cand[np.lexsort((cand, -key[cand, e]))]
             final[order[:target[e] - counts[e]], e] = True
     offsets = np.zeros(E + 1, np.int64)
-    offsets[1:] = np.cumsum(target)
+    offsets[1:] = np.cumsum(_pad(target, tile))
     row_token = np.full(cap, -1, np.int64)
     row_slot = np.full(cap, -1, np.int64)
     row_gate = np.zeros(cap, np.float64)
@@ -235,11 +259,11 @@ def rounded_plan(idx, logits, E, tile=TILE):
         kept = s >= 0
         slot_row[s[kept]] = rows[kept]
         extra_row[members[~kept], e] = rows[~kept]
-    return dict(mode="rounded", T=T, E=E, k=k, tile=tile, cap=cap, counts=counts,
-                target=target, offsets=offsets, row_token=row_token,
+    return dict(mode="rounded" if capacity is None else "capacity", T=T, E=E, k=k, tile=tile,
+                cap=cap, counts=counts, target=target, offsets=offsets, row_token=row_token,
                 row_slot=row_slot, row_gate=row_gate, slot_row=slot_row,
-                extra_row=extra_row, dropped=assigned & ~final,
-                added=final & ~assigned, R=int(offsets[-1]), key=key)
+                extra_row=extra_row if capacity is None else None, dropped=assigned & ~final,
+                added=final & ~assigned, R=int(offsets[-1]), key=key, gate_mode=gate_mode)
 
 
 def token_rows(plan, t):
@@ -336,32 +360,52 @@ def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
     return res
 
 
-def token_router_grad(plan, idx, gate, t, rows, dS_rows):
+def token_router_grad(plan, idx, gate, t, rows, dS_rows, logits=None):
     """dlogits of token t from the router-score gradients of its rows.
 
-    With F_t the final rows of token t (weights s), K_t its top-k experts and
-    p = softmax over K_t:
+    F_t: the final rows of token t with weights s; K_t: its top-k experts.
+    gate_mode 0 (p = softmax over K_t):
         dl_te = [e in F_t] s_te dS_te - [e in K_t] p_te * sum_{e' in F_t} s_te' dS_te'.
-    For the dropless plan F_t = K_t and s = p = g, giving g_e (dS_e - sum g dS).
+    gate_mode 1 (p = softmax over all E, s_te = p_te):
+        dl_te = [e in F_t] p_te dS_te - p_te * sum_{e' in F_t} p_te' dS_te'   (every e).
+    For the dropless plan and gate_mode 0 this is g_e (dS_e - sum g dS).
     """
     E, k = plan["E"], plan["k"]
+    mode = plan.get("gate_mode", 0)
     dl = np.zeros(E)
     tot = 0.0
     for r, ds, e in zip(rows, dS_rows, row_expert(plan, rows)):
         v = plan["row_gate"][r] * ds
         dl[e] += v
         tot += v
-    for j in range(k):
-        dl[idx[t, j]] -= gate[t, j] * tot
+    if mode == 0:
+        for j in range(k):
+            dl[idx[t, j]] -= gate[t, j] * tot
+    else:
+        lt = np.asarray(logits[t], np.float64)
+        p = np.exp(lt - lt.max())
+        p /= p.sum()
+        dl -= p * tot
     return dl
 
 
+def make_plan(idx, gate, logits, E, tile=TILE, round_mode=0, gate_mode=0, capacity=None):
+    """round_mode 0: dropless; 1: token rounding; 2: capacity factor."""
+    if round_mode == 0:
+        plan = exact_plan(idx, gate, E, tile)
+        plan["gate_mode"] = gate_mode
+        return plan
+    if round_mode == 1:
+        return rounded_plan(idx, logits, E, tile, gate_mode)
+    return rounded_plan(idx, logits, E, tile, gate_mode, capacity=capacity)
+
+
 def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
-              logits_override=None, logit_bias=None, staged=True):
+              logits_override=None, logit_bias=None, staged=True, gate_mode=0, capacity=None):
     """Full forward: route, permute, expert FFN on every row, combine."""
-    logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias)
+    logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias, gate_mode)
     T, E = logits.shape
-    plan = exact_plan(idx, gate, E, tile) if round_mode == 0 else rounded_plan(idx, logits, E, tile)
+    plan = make_plan(idx, gate, logits, E, tile, round_mode, gate_mode, capacity)
     rows = np.arange(plan["R"])
     res = rows_compute(rows, plan, x, w1, w3, w2, None, staged)
     out = np.zeros((T, np.shape(x)[1]))
@@ -400,7 +444,8 @@ def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True
     dx = np.zeros((T, d))
     for t in range(T):
         tr = token_rows(plan, t)
-        dlogits[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][tr])
+        dlogits[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][tr],
+                                       fwd["logits"])
         for r in tr:
             dx[t] += res["dXp"][r]
     if extra_dlogits is not None:      # gradient of auxiliary router losses
@@ -428,7 +473,8 @@ def sampled_tokens(tokens, dout, x, w_gate, w1, w3, w2, fwd, staged=True, router
         sl = slice(pos, pos + len(tr))
         pos += len(tr)
         out[t] = (plan["row_gate"][tr][:, None] * res["Y"][sl]).sum(axis=0)
-        dl[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][sl])
+        dl[t] = token_router_grad(plan, fwd["idx"], fwd["gate"], t, tr, res["dS"][sl],
+                                  fwd["logits"])
         dx[t] = res["dXp"][sl].sum(axis=0)
         if router_grad_on:
             dx[t] = dx[t] + dl[t] @ w_gate.T
@@ -518,14 +564,22 @@ def balance_loss(idx, gate, E, lam):
                 count_mse=((counts - cm) ** 2).mean())
 
 
-def gate_grad_to_logits(idx, gate, dgate, E):
-    """dlogits from a gradient on the top-k gates (softmax over the k logits):
-    dl_t,idx_j = g_j (a_j - sum_i g_i a_i) with a = dgate; zero elsewhere."""
+def gate_grad_to_logits(idx, gate, dgate, E, gate_mode=0, logits=None):
+    """dlogits from a gradient a = dgate on the top-k gates:
+    gate_mode 0: dl_t,idx_j = g_j (a_j - sum_i g_i a_i), zero elsewhere;
+    gate_mode 1: dl_te = [e in K_t] p_e a_e - p_e sum_i g_i a_i (every e)."""
     idx = np.asarray(idx)
     gate = np.asarray(gate, np.float64)
     dgate = np.asarray(dgate, np.float64)
     T, k = idx.shape
     dl = np.zeros((T, E))
     tot = (gate * dgate).sum(axis=1, keepdims=True)
-    dl[np.arange(T)[:, None], idx] = gate * (dgate - tot)
+    if gate_mode == 0:
+        dl[np.arange(T)[:, None], idx] = gate * (dgate - tot)
+    else:
+        lg = np.asarray(logits, np.float64)
+        p = np.exp(lg - lg.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        dl = -p * tot
+        dl[np.arange(T)[:, None], idx] += gate * dgate
     return dl

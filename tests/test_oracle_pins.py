@@ -293,19 +293,21 @@ def test_two_expert_hand_example():
     assert abs(bwd["dx"][0, 0] - want["dx"]) < 1e-9
 
 
-def _loss(params, dout, k, tile, round_mode):
+def _loss(params, dout, k, tile, round_mode, gate_mode=0, capacity=None):
     x, wg, w1, w3, w2 = params
-    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=k, tile=tile, round_mode=round_mode, staged=False)
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k=k, tile=tile, round_mode=round_mode, staged=False,
+                      gate_mode=gate_mode, capacity=capacity)
     return float(np.sum(fwd["out"] * dout)), fwd
 
 
-@pytest.mark.parametrize("round_mode", [0, 1])
-def test_backward_matches_central_differences(round_mode):
-    rng = np.random.default_rng(11 + round_mode)
+@pytest.mark.parametrize("round_mode,gate_mode,capacity", [
+    (0, 0, None), (1, 0, None), (0, 1, None), (1, 1, None), (2, 0, 3), (2, 1, 3)])
+def test_backward_matches_central_differences(round_mode, gate_mode, capacity):
+    rng = np.random.default_rng(11 + round_mode + 10 * gate_mode)
     T, d, f, E, k, tile = 9, 4, 3, 4, 2, 4
     x, wg, w1, w3, w2, dout = _rand_layer(rng, T, d, f, E)
     params = [x, wg, w1, w3, w2]
-    _, fwd = _loss(params, dout, k, tile, round_mode)
+    _, fwd = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
     if round_mode:
         assert fwd["plan"]["dropped"].any() or fwd["plan"]["added"].any()
     bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
@@ -316,12 +318,13 @@ def test_backward_matches_central_differences(round_mode):
         for i in np.ndindex(p.shape):
             old = p[i]
             p[i] = old + h
-            lp, fp = _loss(params, dout, k, tile, round_mode)
+            lp, fp = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
             p[i] = old - h
-            lm, fm = _loss(params, dout, k, tile, round_mode)
+            lm, fm = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
             p[i] = old
             # the discrete routing must not change under the probe
             assert np.array_equal(fp["idx"], fwd["idx"]) and np.array_equal(fm["idx"], fwd["idx"])
+            assert np.array_equal(fp["plan"]["row_token"], fwd["plan"]["row_token"])
             num[i] = (lp - lm) / (2 * h)
         np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-7)
 
@@ -492,3 +495,66 @@ def test_layer_with_balance_loss_matches_central_differences():
             assert np.array_equal(fp["idx"], fwd["idx"]) and np.array_equal(fm["idx"], fwd["idx"])
             num[i] = (lp - lm) / (2 * h)
         np.testing.assert_allclose(g, num, rtol=1e-5, atol=1e-7)
+
+
+
+# ---------------------------------------------------------------- routing variants
+
+def test_route_softmax_then_topk_matches_library():
+    """Gate mode 1: softmax over all E logits, then the k largest without
+    renormalisation (the gating of the Trinity commentary's challenge 1)."""
+    rng = np.random.default_rng(20)
+    x, wg = rng.standard_normal((30, 16)), rng.standard_normal((16, 4))
+    _, idx, gate = O.route(x, wg, 2, gate_mode=1)
+    p = torch.softmax(torch.from_numpy(x @ wg), -1)
+    v, i = torch.topk(p, 2, dim=-1)
+    np.testing.assert_array_equal(idx, i.numpy())
+    np.testing.assert_allclose(gate, v.numpy(), rtol=1e-13)
+    assert np.all(gate.sum(1) < 1.0)
+
+
+def test_capacity_plan_brute_force_subsets():
+    rng = np.random.default_rng(21)
+    T, E, k, tile = 12, 3, 2, 4
+    for trial in range(20):
+        for gate_mode in (0, 1):
+            logits = rng.standard_normal((T, E))
+            _, idx, gate = O.route(None, None, k, logits_override=logits, gate_mode=gate_mode)
+            C = 5
+            plan = O.make_plan(idx, gate, logits, E, tile, round_mode=2, gate_mode=gate_mode,
+                               capacity=C)
+            counts = np.bincount(idx.ravel(), minlength=E)
+            key = O.rounding_keys(logits, idx, gate_mode)
+            assert not plan["added"].any()
+            for e in range(E):
+                lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
+                assert lo % tile == 0 and hi % tile == 0
+                members = [int(t) for t in plan["row_token"][lo:hi] if t >= 0]
+                assigned = [t for t in range(T) if e in idx[t]]
+                keep = min(counts[e], C)
+                assert len(members) == keep
+                best = max(itertools.combinations(assigned, keep), key=lambda s: sum(key[t, e] for t in s))
+                assert set(members) == set(best)
+                for r in range(lo, hi):
+                    t = plan["row_token"][r]
+                    if t >= 0:
+                        j = list(idx[t]).index(e)
+                        assert abs(plan["row_gate"][r] - gate[t, j]) <= 1e-12 * gate[t, j]
+
+
+def test_gate_grad_to_logits_mode1_matches_finite_differences():
+    rng = np.random.default_rng(22)
+    T, E, k = 5, 6, 2
+    logits = rng.standard_normal((T, E))
+    _, idx, gate = O.route(None, None, k, logits_override=logits, gate_mode=1)
+    a = rng.standard_normal((T, k))
+    dl = O.gate_grad_to_logits(idx, gate, a, E, gate_mode=1, logits=logits)
+    h = 1e-6
+    for t in range(T):
+        for e in range(E):
+            lp, lm = logits.copy(), logits.copy()
+            lp[t, e] += h
+            lm[t, e] -= h
+            gp = O.route(None, None, k, logits_override=lp, gate_mode=1)[2]
+            gm = O.route(None, None, k, logits_override=lm, gate_mode=1)[2]
+            assert abs(((gp - gm) * a).sum() / (2 * h) - dl[t, e]) < 1e-7
