@@ -44,7 +44,12 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="coarse")
     ap.add_argument("--routing", default=None, help="override the workload's routing variant")
-    ap.add_argument("--round", type=int, default=0, help="1 = token rounding to 128-row tiles")
+    ap.add_argument("--round", type=int, default=0, choices=[0, 1, 2],
+                    help="1 = token rounding to 128-row tiles, 2 = capacity factor")
+    ap.add_argument("--capacity-factor", type=float, default=1.0,
+                    help="tokens per expert = ceil(factor * T * k / E) with --round 2")
+    ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1],
+                    help="0 = softmax over the top-k logits, 1 = softmax over all E then top-k")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens of the cpu_baseline sample")
     ap.add_argument("--ref-sample", type=int, default=256, help="tokens per reference-arm step")
@@ -162,7 +167,12 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle arms
-def oracle_tokens_per_s(cfg, n_tokens, seed=0, repeats=1):
+def _capacity(T, E, k, args):
+    import math
+    return int(math.ceil(args.capacity_factor * T * k / E)) if args.round == 2 else None
+
+
+def oracle_tokens_per_s(cfg, n_tokens, args, seed=0, repeats=1):
     """Time the CPU oracle (as it stands) on the first n_tokens of the workload."""
     import numpy as np
     import torch
@@ -178,7 +188,9 @@ def oracle_tokens_per_s(cfg, n_tokens, seed=0, repeats=1):
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
-        fwd = O.layer_fwd(x, wg, w1, w3, w2, cfg.k, logits_override=lo, logit_bias=lb)
+        fwd = O.layer_fwd(x, wg, w1, w3, w2, cfg.k, logits_override=lo, logit_bias=lb,
+                          round_mode=args.round, gate_mode=args.gate_mode,
+                          capacity=_capacity(n_tokens, cfg.E, cfg.k, args))
         O.layer_bwd(do, x, wg, w1, w3, w2, fwd, router_grad_on=lo is None)
         times.append(time.perf_counter() - t0)
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -188,7 +200,8 @@ def oracle_tokens_per_s(cfg, n_tokens, seed=0, repeats=1):
 def run_reference(args, cfg, rank, world):
     if rank != 0:
         return 0
-    n, times, threads = oracle_tokens_per_s(cfg, args.ref_sample, repeats=args.warmup + args.steps)
+    n, times, threads = oracle_tokens_per_s(cfg, args.ref_sample, args,
+                                            repeats=args.warmup + args.steps)
     timed = times[args.warmup:]
     total = sum(timed)
     value = n * len(timed) / total
@@ -209,7 +222,9 @@ def run_reference(args, cfg, rank, world):
 
 def workload_config(cfg, args):
     return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "d_ff": cfg.f, "E": cfg.E,
-            "k": cfg.k, "routing": cfg.routing, "token_rounding": bool(args.round),
+            "k": cfg.k, "routing": cfg.routing, "token_rounding": args.round == 1,
+            "capacity_factor": args.capacity_factor if args.round == 2 else None,
+            "gate": "softmax_then_topk" if args.gate_mode else "topk_then_softmax",
             "balance_loss_lambda": args.balance_loss,
             "l2": f"flushed between timed steps ({args.flush_mb} MiB write)", "replicas": args.gpus}
 
@@ -227,7 +242,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.set_device(dev)
     inp = synth.make_inputs(cfg, seed=rank, device=dev)
     step = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round,
-                        balance_lambda=args.balance_loss)
+                        balance_lambda=args.balance_loss, gate_mode=args.gate_mode,
+                        capacity_factor=args.capacity_factor if args.round == 2 else None)
     flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
     x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo, lb = inp["logits_override"], inp["logit_bias"]
@@ -335,7 +351,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                         "ms_per_step": g_ms / args.steps}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        n, times, threads = oracle_tokens_per_s(cfg, args.cpu_sample)
+        n, times, threads = oracle_tokens_per_s(cfg, args.cpu_sample, args)
         cpu = {"value": n / times[0], "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"first {n} of {cfg.T} tokens (full expert weights), one fwd+bwd, "
                          f"numpy fp64 with bf16 staging, {times[0]:.1f} s"}

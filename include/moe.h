@@ -66,6 +66,10 @@ extern "C" {
 
 #define MOE_ROUND_NONE 0
 #define MOE_ROUND_NEAREST 1
+#define MOE_ROUND_CAPACITY 2
+
+#define MOE_GATE_TOPK_SOFTMAX 0
+#define MOE_GATE_SOFTMAX_TOPK 1
 
 /* Library version (major*10000 + minor*100 + patch). */
 int moe_version(void);
@@ -77,18 +81,23 @@ const char* moe_last_error(void);
 size_t moe_row_capacity(int T, int E, int k, int tile);
 
 /*
- * moe_route -- router logits, top-k and softmax over the top-k.
+ * moe_route -- router logits, top-k and the gates of the k chosen experts.
  * [Beam] sec. 2.2 and 5.3; [Trinity] example 1.
  *   x [T,d] (dtype), w_gate [d,E] (dtype).
+ *   gate_mode MOE_GATE_TOPK_SOFTMAX: gates = softmax of the k chosen logits
+ *     ([Beam] sec. 5.3, [Trinity] example 1).  MOE_GATE_SOFTMAX_TOPK: gates =
+ *     softmax over all E logits, the k largest kept without renormalising
+ *     ([Beam] sec. 2.2 formula, [Trinity] challenge 1).  The choice of
+ *     experts is the same in both modes.
  *   logits_override [T,E] fp32 or NULL: when given, x and w_gate are not read
  *     and these values replace x W_gate (random-routing workloads).
  *   logit_bias [E] fp32 or NULL: added to every token's logits.
  *   logits [T,E] fp32 out; idx [T,k] int32 out: the k largest logits in
  *   descending order, ties to the lowest expert id; gate [T,k] fp32 out:
- *   softmax of those k logits.
+ *   the gates of those k experts (per gate_mode).
  */
 int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
-              const float* logits_override, const float* logit_bias,
+              int gate_mode, const float* logits_override, const float* logit_bias,
               float* logits, int32_t* idx, float* gate, void* stream);
 
 /*
@@ -98,25 +107,38 @@ int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int
  * round_mode MOE_ROUND_NEAREST applies token rounding ([SonicMoE] sec. 3):
  * each expert's count becomes the nearest multiple of `tile` (halves up,
  * capped at tile*floor(T/tile)); drops remove the pairs with the smallest
- * score exp(l - LSE_topk), larger token first on ties; additions take the
+ * score exp(l - LSE), larger token first on ties; additions take the
  * unassigned tokens with the largest score, smaller token first on ties;
- * row weights are those scores (kept pairs: their gate).
+ * row weights are those scores (kept pairs: their gate).  LSE is the
+ * log-sum-exp of the token's k chosen logits (gate_mode
+ * MOE_GATE_TOPK_SOFTMAX) or of all its E logits (MOE_GATE_SOFTMAX_TOPK), so
+ * the score is the gate the pair has or would have.
+ * round_mode MOE_ROUND_CAPACITY applies a capacity factor ([Beam] sec. 2.3):
+ * an expert chosen by more than `capacity` tokens keeps the `capacity` pairs
+ * with the largest score (the same score and tie rule as rounding drops) and
+ * drops the rest; no pair is added, segments are padded to the tile with
+ * empty rows.  A dropped slot contributes nothing to its token's output.
  *   idx [T,k], gate [T,k]: from moe_route.  logits [T,E]: read only when
- *     rounding.
+ *     rounding or dropping (round_mode != MOE_ROUND_NONE).
+ *   gate_mode: the mode moe_route used (read only when round_mode !=
+ *     MOE_ROUND_NONE).
+ *   capacity: tokens per expert for MOE_ROUND_CAPACITY (>= 0; e.g.
+ *     ceil(capacity_factor * T * k / E)); ignored otherwise.
  *   tile: must be 128 (the grouped-GEMM M tile, also the rounding unit).
  *   counts [E] out: token count per expert before rounding.
  *   offsets [E+1] out: segment starts (multiples of tile); offsets[E] = R.
  *   row_token [cap], row_gate [cap] fp32, row_slot [cap] out: token, weight
  *     and slot (t*k+j, or -1 for a row added by rounding) of each row;
  *     padding rows get -1, 0, -1.
- *   slot_row [T*k] out: row of slot (t,j), or -1 if rounding dropped it.
- *   extra_row [T,E] out (required when rounding, else may be NULL): row of
- *     the pair (t,e) added by rounding, or -1.
+ *   slot_row [T*k] out: row of slot (t,j), or -1 if rounding or the
+ *     capacity dropped it.
+ *   extra_row [T,E] out (required with MOE_ROUND_NEAREST, else may be NULL
+ *     and is not written): row of the pair (t,e) added by rounding, or -1.
  *   ws: workspace of at least moe_permute_workspace_size() bytes.
  */
 size_t moe_permute_workspace_size(int T, int E, int k, int round_mode);
 int moe_permute(const int32_t* idx, const float* gate, const float* logits,
-                int T, int E, int k, int round_mode, int tile,
+                int T, int E, int k, int round_mode, int tile, int gate_mode, int capacity,
                 int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
                 int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
                 void* ws, size_t ws_bytes, void* stream);
@@ -183,13 +205,19 @@ int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_r
  *   dW2_e = sum (s A)^T dO;  [dW1|dW3]_e = sum x^T dH;
  *   dX_perm = dH [W1|W3]^T;  dx_t = sum over t's rows of dX_perm + dlogits_t W_gate^T;
  *   dlogits_te = [e in F_t] s_te dS_te - [e in K_t] g_te sum_{F_t} s dS
- *   (F_t: token t's final rows with weights s; K_t: its top-k);
+ *   (F_t: token t's final rows with weights s; K_t: its top-k) with
+ *   gate_mode MOE_GATE_TOPK_SOFTMAX; with MOE_GATE_SOFTMAX_TOPK the gates
+ *   are p = softmax over all E logits and every expert gets the second term:
+ *   dlogits_te = [e in F_t] p_te dS_te - p_te sum_{F_t} p dS;
  *   dW_gate = x^T dlogits.
+ *   logits [T,E] fp32 (from moe_route): read only with MOE_GATE_SOFTMAX_TOPK
+ *   (may be NULL otherwise).  gate_mode: the mode moe_route used.
  *   router_grad = 0 when the logits did not come from x W_gate (override):
  *   dW_gate is then zero and dx gets no router term.
  *   gate_grad [T,k] fp32 or NULL: gradient of auxiliary losses with respect
  *   to the gates (e.g. from moe_balance_loss); it enters dlogits through the
- *   softmax over the k logits: dl_t,idx_j += g_j (a_j - sum_i g_i a_i).
+ *   softmax over the k logits: dl_t,idx_j += g_j (a_j - sum_i g_i a_i)
+ *   (MOE_GATE_SOFTMAX_TOPK: dl_te += [e in K_t] p_e a_e - p_e sum_i g_i a_i).
  *   Outputs: dx [T,d] (dtype), dw_gate [d,E] fp32, dw1, dw3 [E,d,f] (dtype),
  *   dw2 [E,f,d] (dtype), dS [cap] fp32 (may be NULL), dlogits [T,E] fp32
  *   (may be NULL).  Every output element is written (no accumulation).
@@ -198,7 +226,7 @@ size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype
 int moe_layer_bwd(const void* dout, const void* x, const void* w_gate,
                   const void* w1, const void* w3, const void* w2,
                   const int32_t* idx, const float* gate, const float* gate_grad,
-                  const int32_t* offsets,
+                  const float* logits, int gate_mode, const int32_t* offsets,
                   const int32_t* row_token, const float* row_gate,
                   const int32_t* slot_row, const int32_t* extra_row, const void* H,
                   int T, int d, int f, int E, int k, int dtype, int router_grad,

@@ -8,6 +8,7 @@ arithmetic happens in the library's CUDA kernels; there is no fallback.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -16,7 +17,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_F32, MOE_BF16 = 0, 1
-MOE_ROUND_NONE, MOE_ROUND_NEAREST = 0, 1
+MOE_ROUND_NONE, MOE_ROUND_NEAREST, MOE_ROUND_CAPACITY = 0, 1, 2
+MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
 TILE = 128
 
 EXPORTS = [
@@ -42,16 +44,16 @@ _SIGS = {
     "moe_version": (_i, []),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_row_capacity": (_sz, [_i, _i, _i, _i]),
-    "moe_route": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_route": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i, _i, _i]),
-    "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
-                         _vp, _sz, _vp]),
+    "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                         _vp, _vp, _vp, _sz, _vp]),
     "moe_ffn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_expert_ffn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                 _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "moe_layer_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
-    "moe_layer_bwd": (_i, [_vp] * 15 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
+    "moe_layer_bwd": (_i, [_vp] * 10 + [_i] + [_vp] * 6 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
     "moe_balance_loss_workspace_size": (_sz, [_i, _i, _i]),
     "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
@@ -108,8 +110,10 @@ def moe_row_capacity(T, E, k, tile=TILE) -> int:
 
 
 def moe_route(x, w_gate, k, logits_override=None, logit_bias=None, logits=None, idx=None,
-              gate=None, T=None, E=None, stream=None):
-    """logits [T,E] f32, idx [T,k] i32, gate [T,k] f32 (outputs allocated if None)."""
+              gate=None, T=None, E=None, stream=None, gate_mode=MOE_GATE_TOPK_SOFTMAX):
+    """logits [T,E] f32, idx [T,k] i32, gate [T,k] f32 (outputs allocated if None).
+    gate_mode: MOE_GATE_TOPK_SOFTMAX (softmax over the k chosen logits) or
+    MOE_GATE_SOFTMAX_TOPK (softmax over all E, the k largest kept)."""
     if T is None:
         T = (logits_override if logits_override is not None else x).shape[0]
     if E is None:
@@ -120,7 +124,8 @@ def moe_route(x, w_gate, k, logits_override=None, logit_bias=None, logits=None, 
     logits = logits if logits is not None else torch.empty(T, E, device=dev, dtype=torch.float32)
     idx = idx if idx is not None else torch.empty(T, k, device=dev, dtype=torch.int32)
     gate = gate if gate is not None else torch.empty(T, k, device=dev, dtype=torch.float32)
-    _check(lib().moe_route(_p(x), _p(w_gate), T, d, E, k, dt, _p(logits_override), _p(logit_bias),
+    _check(lib().moe_route(_p(x), _p(w_gate), T, d, E, k, dt, gate_mode, _p(logits_override),
+                           _p(logit_bias),
                            _p(logits), _p(idx), _p(gate), _stream(stream)))
     return logits, idx, gate
 
@@ -129,9 +134,16 @@ def moe_permute_workspace_size(T, E, k, round_mode) -> int:
     return lib().moe_permute_workspace_size(T, E, k, round_mode)
 
 
+def capacity_from_factor(T, E, k, factor) -> int:
+    """Tokens per expert for a capacity factor: ceil(factor * T * k / E)."""
+    return int(math.ceil(factor * T * k / E))
+
+
 def moe_permute(idx, gate, logits, E, round_mode=MOE_ROUND_NONE, tile=TILE, out=None, ws=None,
-                stream=None):
-    """Returns dict counts, offsets, row_token, row_gate, row_slot, slot_row, extra_row."""
+                stream=None, gate_mode=MOE_GATE_TOPK_SOFTMAX, capacity=-1):
+    """Returns dict counts, offsets, row_token, row_gate, row_slot, slot_row, extra_row
+    (extra_row only with MOE_ROUND_NEAREST, else None).  capacity: tokens per
+    expert with MOE_ROUND_CAPACITY."""
     T, k = idx.shape
     dev = idx.device
     cap = moe_row_capacity(T, E, k, tile)
@@ -142,7 +154,7 @@ def moe_permute(idx, gate, logits, E, round_mode=MOE_ROUND_NONE, tile=TILE, out=
     o.setdefault("row_gate", torch.empty(cap, device=dev, dtype=torch.float32))
     o.setdefault("row_slot", torch.empty(cap, device=dev, dtype=torch.int32))
     o.setdefault("slot_row", torch.empty(T * k, device=dev, dtype=torch.int32))
-    if round_mode:
+    if round_mode == MOE_ROUND_NEAREST:
         o.setdefault("extra_row", torch.empty(T, E, device=dev, dtype=torch.int32))
     else:
         o.setdefault("extra_row", None)
@@ -150,6 +162,7 @@ def moe_permute(idx, gate, logits, E, round_mode=MOE_ROUND_NONE, tile=TILE, out=
     if ws is None:
         ws = torch.empty(max(wsb, 1), device=dev, dtype=torch.uint8)
     _check(lib().moe_permute(_p(idx), _p(gate), _p(logits), T, E, k, round_mode, tile,
+                             gate_mode, capacity,
                              _p(o["counts"]), _p(o["offsets"]), _p(o["row_token"]),
                              _p(o["row_gate"]), _p(o["row_slot"]), _p(o["slot_row"]),
                              _p(o["extra_row"]), _p(ws), ws.numel(), _stream(stream)))
@@ -191,8 +204,10 @@ def moe_layer_bwd_workspace_size(T, d, f, E, k, dtype) -> int:
 
 
 def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=True, out=None,
-                  ws=None, stream=None, gate_grad=None):
-    """plan: dict from moe_permute.  Returns dict dx, dw_gate, dw1, dw3, dw2, dS, dlogits."""
+                  ws=None, stream=None, gate_grad=None, logits=None,
+                  gate_mode=MOE_GATE_TOPK_SOFTMAX):
+    """plan: dict from moe_permute.  Returns dict dx, dw_gate, dw1, dw3, dw2, dS, dlogits.
+    logits (from moe_route) are needed with MOE_GATE_SOFTMAX_TOPK."""
     T, d = x.shape
     E, _, f = w1.shape
     k = idx.shape[1]
@@ -212,8 +227,8 @@ def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=T
                          dtype=torch.uint8)
     _check(lib().moe_layer_bwd(
         _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(idx), _p(gate), _p(gate_grad),
-        _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
-        _p(plan["extra_row"]), _p(H), T, d, f, E, k, dt, 1 if router_grad else 0,
+        _p(logits), gate_mode, _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
+        _p(plan.get("extra_row")), _p(H), T, d, f, E, k, dt, 1 if router_grad else 0,
         _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
         _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
     return o

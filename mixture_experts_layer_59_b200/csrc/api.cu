@@ -178,9 +178,11 @@ size_t moe_row_capacity(int T, int E, int k, int tile) {
 }
 
 int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
-              const float* logits_override, const float* logit_bias, float* logits,
-              int32_t* idx, float* gate, void* stream) {
+              int gate_mode, const float* logits_override, const float* logit_bias,
+              float* logits, int32_t* idx, float* gate, void* stream) {
   if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (gate_mode != MOE_GATE_TOPK_SOFTMAX && gate_mode != MOE_GATE_SOFTMAX_TOPK)
+    return fail(MOE_ERR_INVALID_ARG, "gate_mode must be MOE_GATE_TOPK_SOFTMAX or MOE_GATE_SOFTMAX_TOPK");
   if (T == 0) return MOE_OK;
   REQUIRE_PTR(logits);
   REQUIRE_PTR(idx);
@@ -195,13 +197,13 @@ int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int
       // tensor-core router GEMM with the bias, top-k and softmax in its epilogue
       REQUIRE_ALIGNED(x);
       REQUIRE_ALIGNED(w_gate);
-      return tc_router_fwd(x, w_gate, logit_bias, T, d, E, k, logits, idx, gate,
+      return tc_router_fwd(x, w_gate, logit_bias, T, d, E, k, gate_mode, logits, idx, gate,
                            device_sm_count(), s);
     }
     if (int rc = launch_router_logits_simt(x, w_gate, T, d, E, dtype, nullptr, logits, s)) return rc;
     src = logits;
   }
-  return launch_topk_softmax(src, logit_bias, logits, T, E, k, idx, gate, s);
+  return launch_topk_softmax(src, logit_bias, logits, T, E, k, gate_mode, idx, gate, s);
 }
 
 size_t moe_permute_workspace_size(int T, int E, int k, int round_mode) {
@@ -210,14 +212,20 @@ size_t moe_permute_workspace_size(int T, int E, int k, int round_mode) {
 }
 
 int moe_permute(const int32_t* idx, const float* gate, const float* logits, int T, int E, int k,
-                int round_mode, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
-                float* row_gate, int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
-                void* ws, size_t ws_bytes, void* stream) {
+                int round_mode, int tile, int gate_mode, int capacity, int32_t* counts,
+                int32_t* offsets, int32_t* row_token, float* row_gate, int32_t* row_slot,
+                int32_t* slot_row, int32_t* extra_row, void* ws, size_t ws_bytes, void* stream) {
   if (int rc = check_common(T, E, k, MOE_F32)) return rc;
   if (tile != 128)
     return fail(MOE_ERR_UNSUPPORTED, "tile must be 128 (the grouped-GEMM M tile)");
-  if (round_mode != MOE_ROUND_NONE && round_mode != MOE_ROUND_NEAREST)
-    return fail(MOE_ERR_INVALID_ARG, "round_mode must be MOE_ROUND_NONE or MOE_ROUND_NEAREST");
+  if (round_mode != MOE_ROUND_NONE && round_mode != MOE_ROUND_NEAREST &&
+      round_mode != MOE_ROUND_CAPACITY)
+    return fail(MOE_ERR_INVALID_ARG,
+                "round_mode must be MOE_ROUND_NONE, MOE_ROUND_NEAREST or MOE_ROUND_CAPACITY");
+  if (gate_mode != MOE_GATE_TOPK_SOFTMAX && gate_mode != MOE_GATE_SOFTMAX_TOPK)
+    return fail(MOE_ERR_INVALID_ARG, "gate_mode must be MOE_GATE_TOPK_SOFTMAX or MOE_GATE_SOFTMAX_TOPK");
+  if (round_mode == MOE_ROUND_CAPACITY && capacity < 0)
+    return fail(MOE_ERR_INVALID_ARG, "capacity must be >= 0 with MOE_ROUND_CAPACITY");
   REQUIRE_PTR(counts);
   REQUIRE_PTR(offsets);
   if (T > 0) {
@@ -228,10 +236,8 @@ int moe_permute(const int32_t* idx, const float* gate, const float* logits, int 
     REQUIRE_PTR(row_slot);
     REQUIRE_PTR(slot_row);
   }
-  if (round_mode) {
-    REQUIRE_PTR(logits);
-    REQUIRE_PTR(extra_row);
-  }
+  if (round_mode != MOE_ROUND_NONE) REQUIRE_PTR(logits);
+  if (round_mode == MOE_ROUND_NEAREST) REQUIRE_PTR(extra_row);
   if (ws_bytes < permute_ws_bytes(T, E, k, round_mode, tile))
     return fail(MOE_ERR_WORKSPACE, "permute workspace smaller than moe_permute_workspace_size()");
   PermuteWs w;
@@ -240,8 +246,11 @@ int moe_permute(const int32_t* idx, const float* gate, const float* logits, int 
   if (round_mode == MOE_ROUND_NONE)
     return launch_permute_exact(idx, gate, T, E, k, tile, counts, offsets, row_token, row_gate,
                                 row_slot, slot_row, w, s);
-  return launch_permute_round(idx, gate, logits, T, E, k, tile, counts, offsets, row_token,
-                              row_gate, row_slot, slot_row, extra_row, w, s);
+  // capacity mode adds no pairs, so it never writes extra_row
+  return launch_permute_round(idx, gate, logits, T, E, k, tile, gate_mode,
+                              round_mode == MOE_ROUND_CAPACITY ? capacity : -1, counts, offsets,
+                              row_token, row_gate, row_slot, slot_row,
+                              round_mode == MOE_ROUND_CAPACITY ? nullptr : extra_row, w, s);
 }
 
 size_t moe_ffn_fwd_workspace_size(int T, int d, int f, int E, int k, int dtype) {
@@ -302,7 +311,8 @@ size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype
 
 int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
                   const void* w3, const void* w2, const int32_t* idx, const float* gate,
-                  const float* gate_grad, const int32_t* offsets, const int32_t* row_token, const float* row_gate,
+                  const float* gate_grad, const float* logits, int gate_mode,
+                  const int32_t* offsets, const int32_t* row_token, const float* row_gate,
                   const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
                   int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
                   void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
@@ -314,6 +324,9 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   REQUIRE_PTR(row_gate); REQUIRE_PTR(slot_row); REQUIRE_PTR(H); REQUIRE_PTR(dx);
   REQUIRE_PTR(dw_gate); REQUIRE_PTR(dw1); REQUIRE_PTR(dw3); REQUIRE_PTR(dw2);
   if (router_grad) REQUIRE_PTR(w_gate);
+  if (gate_mode != MOE_GATE_TOPK_SOFTMAX && gate_mode != MOE_GATE_SOFTMAX_TOPK)
+    return fail(MOE_ERR_INVALID_ARG, "gate_mode must be MOE_GATE_TOPK_SOFTMAX or MOE_GATE_SOFTMAX_TOPK");
+  if (gate_mode == MOE_GATE_SOFTMAX_TOPK) REQUIRE_PTR(logits);
   REQUIRE_ALIGNED(dout); REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3);
   REQUIRE_ALIGNED(w2); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(dx); REQUIRE_ALIGNED(dw1);
   REQUIRE_ALIGNED(dw3); REQUIRE_ALIGNED(dw2); REQUIRE_ALIGNED(ws);
@@ -343,7 +356,8 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   float* dl = dlogits ? dlogits : w.dl;
   const bool tc_router = router_grad && w.dl_hi != nullptr;
   if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row,
-                              gate_grad, T, E, k, dl, dS, tc_router ? w.dl_hi : nullptr,
+                              gate_grad, logits, gate_mode, T, E, k, dl, dS,
+                              tc_router ? w.dl_hi : nullptr,
                               tc_router ? w.dl_lo : nullptr, s)))
     return rc;
   if (tc_router) {

@@ -10,7 +10,8 @@ namespace moe {
 int launch_router_logits_simt(const void* x, const void* wg, int T, int d, int E, int dtype,
                               const float* bias, float* logits, cudaStream_t s);
 int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out,
-                        int T, int E, int k, int32_t* idx, float* gate, cudaStream_t s);
+                        int T, int E, int k, int gate_mode, int32_t* idx, float* gate,
+                        cudaStream_t s);
 
 // ---------------------------------------------------------------- permutation
 struct PermuteWs {
@@ -30,10 +31,12 @@ int carve_permute_ws(void* ws, size_t bytes, int T, int E, int k, int round_mode
 int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, int k, int tile,
                          int32_t* counts, int32_t* offsets, int32_t* row_token, float* row_gate,
                          int32_t* row_slot, int32_t* slot_row, const PermuteWs& w, cudaStream_t s);
+// Token rounding (capacity < 0) or capacity-factor dropping (capacity >= 0).
 int launch_permute_round(const int32_t* idx, const float* gate, const float* logits, int T, int E,
-                         int k, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
-                         float* row_gate, int32_t* row_slot, int32_t* slot_row, int32_t* extra_row,
-                         const PermuteWs& w, cudaStream_t s);
+                         int k, int tile, int gate_mode, int capacity, int32_t* counts,
+                         int32_t* offsets, int32_t* row_token, float* row_gate, int32_t* row_slot,
+                         int32_t* slot_row, int32_t* extra_row, const PermuteWs& w,
+                         cudaStream_t s);
 
 // ---------------------------------------------------------------- row ops
 // dst[row] = src[token of row] for every row (token-order scatter: each source
@@ -55,8 +58,9 @@ int launch_token_reduce(const void* src, const float* row_gate, const int32_t* s
 // Optionally also writes dlogits split as bf16 hi + bf16 lo (tensor-core router GEMMs).
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      const float* gate_grad, int T, int E, int k, float* dlogits, float* dS_out,
-                      void* dl_hi, void* dl_lo, cudaStream_t s);
+                      const float* gate_grad, const float* logits, int gate_mode, int T, int E,
+                      int k, float* dlogits, float* dS_out, void* dl_hi, void* dl_lo,
+                      cudaStream_t s);
 // Load-balance loss lambda*CV^2, routing statistics and dL/dgate.
 size_t balance_ws_bytes(int T, int E);
 int launch_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k, float lam,
@@ -87,7 +91,8 @@ int tc_num_dS_parts(int f);
 bool tc_router_ok(int E);
 int tc_dwg_splits(int T, int d, int* chunk);
 int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
-                  float* logits, int32_t* idx, float* gate, int num_sms, cudaStream_t s);
+                  int gate_mode, float* logits, int32_t* idx, float* gate, int num_sms,
+                  cudaStream_t s);
 int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
                   int d, int E, int k, float* dwg_part, float* dw_gate, const float* dx_acc,
                   void* dx, int num_sms, cudaStream_t s);

@@ -14,7 +14,7 @@ namespace moe {
 // One warp per token.  Each lane holds up to 8 of the E <= 256 logits
 // (expert e = lane + 32*i).  k rounds of a warp arg-max (ties: lowest id).
 __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float* __restrict__ bias,
-                               float* __restrict__ logits_out, int T, int E, int k,
+                               float* __restrict__ logits_out, int T, int E, int k, int gate_mode,
                                int32_t* __restrict__ idx, float* __restrict__ gate) {
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
@@ -54,11 +54,20 @@ __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float*
       top[j] = bv;
       topi[j] = bi;
     }
+    // gate_mode 1: normaliser over all E logits (max = top[0])
+    float zall = 0.f;
+    if (gate_mode == 1) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) zall += expf(v[i] - top[0]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zall += __shfl_xor_sync(0xffffffffu, zall, o);
+    }
     if (lane == 0) {
       float m = top[0], z = 0.f;
       float ex[8];
       for (int j = 0; j < k; ++j) { ex[j] = expf(top[j] - m); z += ex[j]; }
-      float inv = 1.0f / z;
+      float inv = 1.0f / (gate_mode == 1 ? zall : z);
       for (int j = 0; j < k; ++j) {
         idx[(size_t)t * k + j] = topi[j];
         gate[(size_t)t * k + j] = ex[j] * inv;
@@ -68,13 +77,14 @@ __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float*
 }
 
 int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out, int T,
-                        int E, int k, int32_t* idx, float* gate, cudaStream_t s) {
+                        int E, int k, int gate_mode, int32_t* idx, float* gate, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
   {
     ProfScope _ps("topk_softmax", s);
-    k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, idx, gate);
+    k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, gate_mode, idx,
+                                          gate);
   }
   MOE_CHECK_LAUNCH("topk_softmax");
   return MOE_OK;
@@ -266,14 +276,19 @@ int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, in
 // ============================================================== token rounding
 // Log-sum-exp of each token's top-k logits, in fp64 so that the ranking key
 // l_te - LSE_t orders pairs the same way on any correctly rounding host.
+// gate_mode 0: over the token's top-k logits; gate_mode 1: over all E logits.
 __global__ void k_round_lse(const float* __restrict__ logits, const int32_t* __restrict__ idx,
-                            int T, int E, int k, double* __restrict__ lse) {
+                            int T, int E, int k, int gate_mode, double* __restrict__ lse) {
   int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= T) return;
+  const int n = gate_mode == 1 ? E : k;
+  auto lg = [&](int j) -> double {
+    return (double)logits[(size_t)t * E + (gate_mode == 1 ? j : idx[(size_t)t * k + j])];
+  };
   double m = -INFINITY;
-  for (int j = 0; j < k; ++j) m = fmax(m, (double)logits[(size_t)t * E + idx[(size_t)t * k + j]]);
+  for (int j = 0; j < n; ++j) m = fmax(m, lg(j));
   double z = 0.0;
-  for (int j = 0; j < k; ++j) z += exp((double)logits[(size_t)t * E + idx[(size_t)t * k + j]] - m);
+  for (int j = 0; j < n; ++j) z += exp(lg(j) - m);
   lse[t] = m + log(z);
 }
 
@@ -321,7 +336,7 @@ __global__ void __launch_bounds__(RS_THREADS)
 k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
                const int32_t* __restrict__ ex_counts, const int32_t* __restrict__ ex_offsets,
                const int32_t* __restrict__ ex_row_token, const float* __restrict__ ex_row_gate,
-               const int32_t* __restrict__ ex_row_slot, int T, int E, int tile,
+               const int32_t* __restrict__ ex_row_slot, int T, int E, int tile, int capacity,
                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                int32_t* __restrict__ row_token, float* __restrict__ row_gate,
                int32_t* __restrict__ row_slot, int32_t* __restrict__ slot_row,
@@ -330,16 +345,25 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
   __shared__ int s_off[257];
   __shared__ int s_hist[256];
   __shared__ int s_warp[33];
-  __shared__ int s_sel, s_rem;
+  __shared__ int s_sel, s_rem, s_r;
   const int e = blockIdx.x;
   if (threadIdx.x == 0) {
+    // target rows per expert: nearest multiple of the tile (capacity < 0), or
+    // at most `capacity` (capacity factor); segments start at tile multiples
     int acc = 0;
     const int cap_rows = tile * (T / tile);
     for (int i = 0; i < E; ++i) {
       s_off[i] = acc;
-      int c = ex_counts[i];
-      int r = tile * ((c + tile / 2) / tile);
-      acc += r < cap_rows ? r : cap_rows;
+      const int c = ex_counts[i];
+      int r;
+      if (capacity < 0) {
+        r = tile * ((c + tile / 2) / tile);
+        r = r < cap_rows ? r : cap_rows;
+      } else {
+        r = c < capacity ? c : capacity;
+      }
+      if (i == e) s_r = r;
+      acc += (r + tile - 1) / tile * tile;
     }
     s_off[E] = acc;
   }
@@ -349,9 +373,15 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
     for (int i = threadIdx.x; i < E; i += blockDim.x) counts[i] = ex_counts[i];
   }
   const int c = ex_counts[e];
-  const int r = s_off[e + 1] - s_off[e];
+  const int r = s_r;
   const int in0 = ex_offsets[e];
   const int out0 = s_off[e];
+  // padding rows after the r members (capacity mode; none with rounding)
+  for (int i = out0 + r + threadIdx.x; i < s_off[e + 1]; i += blockDim.x) {
+    row_token[i] = -1;
+    row_gate[i] = 0.f;
+    row_slot[i] = -1;
+  }
 
   if (r == c) {  // nothing to drop or add: copy the segment
     for (int i = threadIdx.x; i < c; i += blockDim.x) {
@@ -465,9 +495,10 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
 }
 
 int launch_permute_round(const int32_t* idx, const float* gate, const float* logits, int T, int E,
-                         int k, int tile, int32_t* counts, int32_t* offsets, int32_t* row_token,
-                         float* row_gate, int32_t* row_slot, int32_t* slot_row,
-                         int32_t* extra_row, const PermuteWs& w, cudaStream_t s) {
+                         int k, int tile, int gate_mode, int capacity, int32_t* counts,
+                         int32_t* offsets, int32_t* row_token, float* row_gate, int32_t* row_slot,
+                         int32_t* slot_row, int32_t* extra_row, const PermuteWs& w,
+                         cudaStream_t s) {
   // 1. exact plan into the workspace (its slot_row is scratch: the final
   //    slot_row is fully rewritten by the selection below)
   int rc = launch_permute_exact(idx, gate, T, E, k, tile, w.ex_counts, w.ex_offsets,
@@ -476,11 +507,13 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
   if (T > 0) {
     {
       ProfScope _ps("round_lse", s);
-      k_round_lse<<<(T + 255) / 256, 256, 0, s>>>(logits, idx, T, E, k, w.lse);
+      k_round_lse<<<(T + 255) / 256, 256, 0, s>>>(logits, idx, T, E, k, gate_mode, w.lse);
     }
     MOE_CHECK_LAUNCH("round_lse");
-    cudaError_t e = cudaMemsetAsync(extra_row, 0xff, (size_t)T * E * sizeof(int32_t), s);
-    if (e != cudaSuccess) return cuda_fail(e, "memset extra_row");
+    if (extra_row != nullptr) {
+      cudaError_t e = cudaMemsetAsync(extra_row, 0xff, (size_t)T * E * sizeof(int32_t), s);
+      if (e != cudaSuccess) return cuda_fail(e, "memset extra_row");
+    }
   }
   const size_t smem = (size_t)((T + 31) / 32 + 1) * sizeof(uint32_t);
   if (smem > 200 * 1024) return fail(MOE_ERR_UNSUPPORTED, "token rounding supports T <= 1.6M");
@@ -493,8 +526,8 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
     ProfScope _ps("round_select", s);
     k_round_select<<<E, RS_THREADS, smem, s>>>(logits, w.lse, w.ex_counts, w.ex_offsets,
                                                w.ex_row_token, w.ex_row_gate, w.ex_row_slot, T, E,
-                                               tile, counts, offsets, row_token, row_gate, row_slot,
-                                               slot_row, extra_row);
+                                               tile, capacity, counts, offsets, row_token, row_gate,
+                                               row_slot, slot_row, extra_row);
   }
   MOE_CHECK_LAUNCH("round_select");
   return MOE_OK;

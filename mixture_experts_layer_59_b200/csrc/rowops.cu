@@ -456,6 +456,7 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
                              const int32_t* __restrict__ idx, const float* __restrict__ gate,
                              const float* __restrict__ row_gate, const int32_t* __restrict__ slot_row,
                              const int32_t* __restrict__ extra_row, const float* __restrict__ gate_grad,
+                             const float* __restrict__ logits, int gate_mode,
                              int T, int E, int k, float* __restrict__ dlogits,
                              float* __restrict__ dS_out, __nv_bfloat16* __restrict__ dl_hi,
                              __nv_bfloat16* __restrict__ dl_lo) {
@@ -506,11 +507,33 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ga += __shfl_xor_sync(0xffffffffu, ga, o);
     }
-    if (lane < k) {
-      const int e = idx[(size_t)t * k + lane];
-      const float gj = gate[(size_t)t * k + lane];
-      dl[e] -= gj * part;
-      if (gate_grad != nullptr) dl[e] += gj * (aj - ga);
+    if (gate_mode == 0) {
+      if (lane < k) {
+        const int e = idx[(size_t)t * k + lane];
+        const float gj = gate[(size_t)t * k + lane];
+        dl[e] -= gj * part;
+        if (gate_grad != nullptr) dl[e] += gj * (aj - ga);
+      }
+    } else {
+      // gates are softmax probabilities over all E logits: every expert gets
+      // -p_e * (sum of s dS over the rows + sum of g a over the slots)
+      float mx = -INFINITY;
+      for (int e = lane; e < E; e += 32) mx = fmaxf(mx, logits[(size_t)t * E + e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float z = 0.f;
+      for (int e = lane; e < E; e += 32) z += expf(logits[(size_t)t * E + e] - mx);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      const float inv = 1.0f / z;
+      __syncwarp();
+      if (gate_grad != nullptr && lane < k) {
+        const int e = idx[(size_t)t * k + lane];
+        dl[e] += gate[(size_t)t * k + lane] * aj;
+      }
+      __syncwarp();
+      for (int e = lane; e < E; e += 32)
+        dl[e] -= expf(logits[(size_t)t * E + e] - mx) * inv * (part + ga);
     }
     __syncwarp();
     for (int e = lane; e < E; e += 32) {
@@ -529,15 +552,17 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
 
 int launch_router_bwd(const float* ds_part, int nparts, const int32_t* idx, const float* gate,
                       const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
-                      const float* gate_grad, int T, int E, int k, float* dlogits, float* dS_out,
-                      void* dl_hi, void* dl_lo, cudaStream_t s) {
+                      const float* gate_grad, const float* logits, int gate_mode, int T, int E,
+                      int k, float* dlogits, float* dS_out, void* dl_hi, void* dl_lo,
+                      cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > device_sm_count() * 16) blocks = device_sm_count() * 16;
   {
     ProfScope _ps("router_bwd", s);
     k_router_bwd<<<blocks, 256, 0, s>>>(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row,
-                                        gate_grad, T, E, k, dlogits, dS_out, (__nv_bfloat16*)dl_hi,
+                                        gate_grad, logits, gate_mode, T, E, k, dlogits, dS_out,
+                                        (__nv_bfloat16*)dl_hi,
                                         (__nv_bfloat16*)dl_lo);
   }
   MOE_CHECK_LAUNCH("router_bwd");

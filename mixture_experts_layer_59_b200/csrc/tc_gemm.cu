@@ -83,6 +83,7 @@ struct TcArgs {
   int* status;
   // router kinds
   int T, k, splits, chunk;
+  int gate_mode;             // RT: 0 softmax over the top-k, 1 softmax over all E
   const float* bias;         // RT: [E] or null
   float* logits;             // RT: [T, E]
   int32_t* idx;              // RT: [T, k]
@@ -530,6 +531,19 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
               }
             }
           }
+          // gate_mode 1: normaliser over all E logits, from a second pass over
+          // the accumulator (every lane of the warp takes part in the loads)
+          float zall = 0.f;
+          if (a.gate_mode == 1) {
+            for (int c = 0; c < a.E; c += 32) {
+              tmem_ld32(tbase + c, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c + i < a.E)
+                  zall += expf(__uint_as_float(r[i]) + (a.bias ? a.bias[c + i] : 0.f) - tv[0]);
+            }
+          }
           if (valid) {
             const float m = tv[0];
             float z = 0.f, ex[8];
@@ -538,6 +552,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
               ex[j] = j < a.k ? expf(tv[j] - m) : 0.f;
               z += ex[j];
             }
+            if (a.gate_mode == 1) z = zall;
             const float inv = 1.0f / z;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -744,9 +759,11 @@ int tc_dwg_splits(int T, int d, int* chunk) {
 }
 
 int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
-                  float* logits, int32_t* idx, float* gate, int num_sms, cudaStream_t s) {
+                  int gate_mode, float* logits, int32_t* idx, float* gate, int num_sms,
+                  cudaStream_t s) {
   TcArgs a;
   memset(&a, 0, sizeof(a));
+  a.gate_mode = gate_mode;
   a.E = E;
   a.d = d;
   a.K = d;

@@ -15,9 +15,17 @@ class MoELayerStep:
     """
 
     def __init__(self, T, d, f, E, k, dtype=torch.bfloat16, device="cuda",
-                 round_mode=B.MOE_ROUND_NONE, balance_lambda=None):
+                 round_mode=B.MOE_ROUND_NONE, balance_lambda=None,
+                 gate_mode=B.MOE_GATE_TOPK_SOFTMAX, capacity_factor=None):
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         self.dtype, self.device, self.round_mode = dtype, device, round_mode
+        self.gate_mode = gate_mode
+        if round_mode == B.MOE_ROUND_CAPACITY:
+            if capacity_factor is None:
+                raise ValueError("MOE_ROUND_CAPACITY needs capacity_factor")
+            self.capacity = B.capacity_from_factor(T, E, k, capacity_factor)
+        else:
+            self.capacity = -1
         dt = B.dtype_code(dtype)
         cap = B.moe_row_capacity(T, E, k)
         self.cap = cap
@@ -26,7 +34,8 @@ class MoELayerStep:
         self.plan = dict(counts=e(E, dt_=torch.int32), offsets=e(E + 1, dt_=torch.int32),
                          row_token=e(cap, dt_=torch.int32), row_gate=e(cap),
                          row_slot=e(cap, dt_=torch.int32), slot_row=e(T * k, dt_=torch.int32),
-                         extra_row=e(T, E, dt_=torch.int32) if round_mode else None)
+                         extra_row=e(T, E, dt_=torch.int32)
+                         if round_mode == B.MOE_ROUND_NEAREST else None)
         self.H, self.Y = e(cap, 2 * f, dt_=dtype), e(cap, d, dt_=dtype)
         self.out = e(T, d, dt_=dtype)
         self.ws_perm = e(max(B.moe_permute_workspace_size(T, E, k, round_mode), 1), dt_=torch.uint8)
@@ -44,9 +53,10 @@ class MoELayerStep:
         self._saved = (x, w_gate, w1, w3, w2)
         self.router_grad = logits_override is None
         B.moe_route(x, w_gate, self.k, logits_override, logit_bias, self.logits, self.idx,
-                    self.gate, T=self.T, E=self.E, stream=stream)
+                    self.gate, T=self.T, E=self.E, stream=stream, gate_mode=self.gate_mode)
         B.moe_permute(self.idx, self.gate, self.logits, self.E, self.round_mode, out=self.plan,
-                      ws=self.ws_perm, stream=stream)
+                      ws=self.ws_perm, stream=stream, gate_mode=self.gate_mode,
+                      capacity=self.capacity)
         if self.balance_lambda is not None:
             self.balance = B.moe_balance_loss(self.idx, self.gate, self.E, self.balance_lambda,
                                               ws=self.ws_bal, stream=stream)
@@ -61,4 +71,5 @@ class MoELayerStep:
         return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
                                self.H, self.router_grad, out=self.grads, ws=self.ws_bwd,
                                stream=stream,
-                               gate_grad=self.balance["dgate"] if self.balance else None)
+                               gate_grad=self.balance["dgate"] if self.balance else None,
+                               logits=self.logits, gate_mode=self.gate_mode)

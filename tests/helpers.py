@@ -29,6 +29,8 @@ def assert_close(gpu, ref, name, tol=BF16_TOL):
     gpu, ref = f64(gpu), f64(ref)
     assert gpu.shape == ref.shape, (name, gpu.shape, ref.shape)
     assert np.all(np.isfinite(gpu)), f"{name}: non-finite values"
+    if ref.size == 0:
+        return
     diff = np.abs(gpu - ref)
     scale = np.abs(ref).max()
     mx = diff.max() if diff.size else 0.0
@@ -49,25 +51,29 @@ def fp32_router_logits(x, w_gate, logit_bias=None):
     return lg.astype(np.float32)
 
 
-def gpu_layer(inp, k, round_mode, logits32, router_grad=True, dev="cuda"):
+def gpu_layer(inp, k, round_mode, logits32, router_grad=True, dev="cuda", gate_mode=0,
+              capacity=-1):
     """Forward + backward through the C ABI with the routing logits given."""
     x, wg, w1, w3, w2, dout = (inp[n].to(dev) for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo = torch.from_numpy(np.ascontiguousarray(logits32)).to(dev)
     T, E = lo.shape
-    logits, idx, gate = B.moe_route(x, wg, k, logits_override=lo)
-    plan = B.moe_permute(idx, gate, logits, E, round_mode)
+    logits, idx, gate = B.moe_route(x, wg, k, logits_override=lo, gate_mode=gate_mode)
+    plan = B.moe_permute(idx, gate, logits, E, round_mode, gate_mode=gate_mode, capacity=capacity)
     H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
     out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)
-    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H, router_grad=router_grad)
+    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H, router_grad=router_grad,
+                        logits=logits, gate_mode=gate_mode)
     B.moe_check_status()
     torch.cuda.synchronize()
     return dict(logits=logits, idx=idx, gate=gate, plan=plan, H=H, Y=Y, out=out, **g)
 
 
-def oracle_layer(inp, k, round_mode, logits32, staged=True, router_grad=True):
+def oracle_layer(inp, k, round_mode, logits32, staged=True, router_grad=True, gate_mode=0,
+                 capacity=None):
     x, wg, w1, w3, w2, dout = (f64(inp[n]) for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     fwd = O.layer_fwd(x, wg, w1, w3, w2, k, round_mode=round_mode,
-                      logits_override=np.asarray(logits32, np.float64), staged=staged)
+                      logits_override=np.asarray(logits32, np.float64), staged=staged,
+                      gate_mode=gate_mode, capacity=capacity)
     bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=staged, router_grad_on=router_grad)
     return fwd, bwd
 

@@ -45,18 +45,19 @@ def test_workspace_sizes_monotone():
 
 
 def _rc_route(**kw):
-    args = dict(x=None, wg=None, T=4, d=128, E=8, k=2, dtype=B.MOE_BF16, lo=None, lb=None,
+    args = dict(x=None, wg=None, T=4, d=128, E=8, k=2, dtype=B.MOE_BF16, gm=0, lo=None, lb=None,
                 logits=None, idx=None, gate=None, stream=None)
     args.update(kw)
     lib = B.lib()
     return lib.moe_route(args["x"], args["wg"], args["T"], args["d"], args["E"], args["k"],
-                         args["dtype"], args["lo"], args["lb"], args["logits"], args["idx"],
+                         args["dtype"], args["gm"], args["lo"], args["lb"], args["logits"],
+                         args["idx"],
                          args["gate"], args["stream"])
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(k=0), -2), (dict(k=9), -2), (dict(E=1, k=2), -2), (dict(E=300), -2),
-    (dict(dtype=7), -2), (dict(T=-1), -1),
+    (dict(dtype=7), -2), (dict(T=-1), -1), (dict(gm=2), -1),
 ])
 def test_route_rejects_bad_shapes(kw, code):
     assert _rc_route(**kw) == code
@@ -71,18 +72,26 @@ def test_route_rejects_null_outputs():
 def test_permute_rejects_tile_and_mode():
     lib = B.lib()
     fake = ctypes.c_void_p(16)
-    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 64, fake, fake, fake, fake, fake, fake,
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 64, 0, -1, fake, fake, fake, fake, fake, fake,
                          None, fake, 1 << 20, None)
     assert rc == -2
-    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 3, 128, fake, fake, fake, fake, fake, fake,
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 3, 128, 0, -1, fake, fake, fake, fake, fake, fake,
                          None, fake, 1 << 20, None)
     assert rc == -1
     # rounding needs logits and extra_row
-    rc = lib.moe_permute(fake, fake, None, 4, 8, 2, 1, 128, fake, fake, fake, fake, fake, fake,
+    rc = lib.moe_permute(fake, fake, None, 4, 8, 2, 1, 128, 0, -1, fake, fake, fake, fake, fake, fake,
                          None, fake, 1 << 20, None)
     assert rc == -1
+    # capacity mode: a capacity is required, extra_row is not
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 2, 128, 0, -1, fake, fake, fake, fake, fake,
+                         fake, None, fake, 1 << 20, None)
+    assert rc == -1 and b"capacity" in lib.moe_last_error()
+    # gate_mode out of range
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 1, 128, 5, -1, fake, fake, fake, fake, fake,
+                         fake, fake, fake, 1 << 20, None)
+    assert rc == -1 and b"gate_mode" in lib.moe_last_error()
     # workspace too small
-    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 128, fake, fake, fake, fake, fake, fake,
+    rc = lib.moe_permute(fake, fake, fake, 4, 8, 2, 0, 128, 0, -1, fake, fake, fake, fake, fake, fake,
                          None, fake, 8, None)
     assert rc == -5
 
@@ -105,10 +114,19 @@ def test_ffn_rejects_unaligned_dims_and_small_workspace():
 def test_bwd_rejects_missing_w_gate_with_router_grad():
     lib = B.lib()
     f = ctypes.c_void_p(256)
-    args = [f, f, None, f, f, f, f, f, None, f, f, f, f, None, f, 16, 128, 128, 8, 2, B.MOE_BF16, 1,
-            f, f, f, f, f, None, None, f, 1 << 40, None]
+    args = [f, f, None, f, f, f, f, f, None, None, 0, f, f, f, f, None, f, 16, 128, 128, 8, 2,
+            B.MOE_BF16, 1, f, f, f, f, f, None, None, f, 1 << 40, None]
     assert lib.moe_layer_bwd(*args) == -1
     assert b"w_gate" in lib.moe_last_error()
+
+
+def test_bwd_softmax_topk_gates_need_logits():
+    lib = B.lib()
+    f = ctypes.c_void_p(256)
+    args = [f, f, f, f, f, f, f, f, None, None, B.MOE_GATE_SOFTMAX_TOPK, f, f, f, f, None, f, 16,
+            128, 128, 8, 2, B.MOE_BF16, 1, f, f, f, f, f, None, None, f, 1 << 40, None]
+    assert lib.moe_layer_bwd(*args) == -1
+    assert b"logits" in lib.moe_last_error()
 
 
 def test_ffn_requires_slot_row():

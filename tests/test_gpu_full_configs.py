@@ -40,29 +40,35 @@ class DeviceExperts:
         return self.cache[e]
 
 
+# (workload, routing, round_mode, sampled tokens, gate_mode, capacity factor)
 CASES = [
-    ("coarse", "learned", 0, 64),
-    ("coarse", "uniform", 0, 64),
-    ("pool", "uniform", 0, 64),
-    ("pool", "gauss", 0, 64),
-    ("fine", "learned", 0, 64),
-    ("sparse", "zipf", 0, 12),
-    ("sparse", "zipf", 1, 12),
+    ("coarse", "learned", 0, 64, 0, None),
+    ("coarse", "uniform", 0, 64, 0, None),
+    ("pool", "uniform", 0, 64, 0, None),
+    ("pool", "gauss", 0, 64, 0, None),
+    ("fine", "learned", 0, 64, 0, None),
+    ("sparse", "zipf", 0, 12, 0, None),
+    ("sparse", "zipf", 1, 12, 0, None),
+    ("coarse", "learned", 2, 64, 1, 1.0),     # softmax over all E, capacity factor 1
+    ("fine", "learned", 1, 64, 1, None),      # softmax over all E, token rounding
+    ("sparse", "zipf", 2, 12, 0, 1.25),
 ]
 
 
-@pytest.mark.parametrize("name,routing,round_mode,n_tok", CASES,
-                         ids=[f"{c[0]}-{c[1]}-round{c[2]}" for c in CASES])
-def test_full_size_layer(name, routing, round_mode, n_tok):
+@pytest.mark.parametrize("name,routing,round_mode,n_tok,gate_mode,cf", CASES,
+                         ids=[f"{c[0]}-{c[1]}-round{c[2]}-gate{c[4]}" for c in CASES])
+def test_full_size_layer(name, routing, round_mode, n_tok, gate_mode, cf):
     cfg = synth.CONFIGS[name].with_(routing=routing)
     T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    cap = B.capacity_from_factor(T, E, k, cf) if round_mode == 2 else -1
     inp = synth.make_inputs(cfg, seed=0, device="cuda")
     router_grad = inp["logits_override"] is None
     x64, wg64 = f64(inp["x"]), f64(inp["w_gate"])
     if router_grad:
         logits32 = fp32_router_logits(x64, wg64, inp["logit_bias"])
         # the tensor-core router itself, against the oracle's logits
-        lg, idx_g, _ = B.moe_route(inp["x"], inp["w_gate"], k, logit_bias=inp["logit_bias"])
+        lg, idx_g, gate_g = B.moe_route(inp["x"], inp["w_gate"], k, logit_bias=inp["logit_bias"],
+                                        gate_mode=gate_mode)
         torch.cuda.synchronize()
         lg = f64(lg)
         scale = np.abs(logits32).max()
@@ -74,20 +80,28 @@ def test_full_size_layer(name, routing, round_mode, n_tok):
         ref_idx = O.route(None, None, k, logits_override=logits32.astype(np.float64))[1]
         np.testing.assert_array_equal(np.sort(i64(idx_g)[clear], 1), np.sort(ref_idx[clear], 1))
         np.testing.assert_array_equal(i64(idx_g)[ordered], ref_idx[ordered])
-        del lg, idx_g
+        # gates: the oracle's gate rule applied to the GPU's own logits and choice
+        g_ref = O.route(None, None, k, logits_override=lg, gate_mode=gate_mode)[2]
+        same = np.all(i64(idx_g) == O.route(None, None, k, logits_override=lg)[1], axis=1)
+        np.testing.assert_allclose(f64(gate_g)[same], g_ref[same], rtol=5e-6, atol=1e-7)
+        del lg, idx_g, gate_g
     else:
         logits32 = f64(inp["logits_override"]).astype(np.float32)
 
-    g = gpu_layer(inp, k, round_mode, logits32, router_grad=router_grad)
+    g = gpu_layer(inp, k, round_mode, logits32, router_grad=router_grad, gate_mode=gate_mode,
+                  capacity=cap)
 
     # routing plan, in full
     lg64 = logits32.astype(np.float64)
-    _, idx, gate = O.route(None, None, k, logits_override=lg64)
-    plan = O.exact_plan(idx, gate, E) if round_mode == 0 else O.rounded_plan(idx, lg64, E)
+    _, idx, gate = O.route(None, None, k, logits_override=lg64, gate_mode=gate_mode)
+    plan = O.make_plan(idx, gate, lg64, E, round_mode=round_mode, gate_mode=gate_mode,
+                       capacity=cap if round_mode == 2 else None)
     np.testing.assert_array_equal(i64(g["idx"]), idx)
     compare_plan(g["plan"], plan)
-    if round_mode:
+    if round_mode == 1:
         assert plan["R"] < O.exact_plan(idx, gate, E)["R"]   # rounding removed padding rows
+    if round_mode == 2:
+        assert plan["dropped"].any()
     fwd = dict(logits=lg64, idx=idx, gate=gate, plan=plan)
 
     W1, W3, W2 = DeviceExperts(inp["w1"]), DeviceExperts(inp["w3"]), DeviceExperts(inp["w2"])

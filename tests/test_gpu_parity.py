@@ -183,3 +183,118 @@ def test_layer_with_balance_loss_gradient():
     bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd, extra_dlogits=extra)
     for n in ("dlogits", "dw_gate", "dx", "dw1"):
         assert_close(gr[n], bwd[n], n, BF16_TOL)
+
+
+# ------------------------------------------------------------------ routing variants
+
+@pytest.mark.parametrize("E,k", [(8, 2), (64, 8), (256, 8), (33, 3)])
+def test_route_softmax_then_topk_gates(E, k):
+    """Gates = softmax over all E logits, the k largest kept; same expert choice."""
+    T = 777
+    lo = synth.quantized_logits(T, E, levels=4, seed=E + 1)
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E,
+                                    gate_mode=B.MOE_GATE_SOFTMAX_TOPK)
+    torch.cuda.synchronize()
+    _, ref_idx, ref_g = O.route(None, None, k, logits_override=f64(lo), gate_mode=1)
+    np.testing.assert_array_equal(i64(idx), ref_idx)
+    np.testing.assert_allclose(f64(gate), ref_g, rtol=2e-6, atol=1e-7)
+    assert np.all(f64(gate).sum(1) <= 1 + 1e-6)
+
+
+def test_route_softmax_then_topk_tensor_core_router():
+    """The tensor-core router epilogue's normaliser over all E logits."""
+    cfg = _cfg(1000, 256, 128, 64, 8, std=0.05)
+    inp = synth.make_inputs(cfg, seed=4, device="cuda")
+    bias = torch.linspace(-0.3, 0.3, cfg.E, device="cuda")
+    logits, idx, gate = B.moe_route(inp["x"], inp["w_gate"], cfg.k, logit_bias=bias,
+                                    gate_mode=B.MOE_GATE_SOFTMAX_TOPK)
+    torch.cuda.synchronize()
+    # gates against the oracle fed the GPU's own logits and choice
+    lg = f64(logits)
+    p = np.exp(lg - lg.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    np.testing.assert_allclose(f64(gate), np.take_along_axis(p, i64(idx), 1), rtol=2e-6, atol=1e-7)
+    _, ref_idx, _ = O.route(None, None, cfg.k, logits_override=lg, gate_mode=1)
+    np.testing.assert_array_equal(i64(idx), ref_idx)
+
+
+@pytest.mark.parametrize("T,E,k,skew,gate_mode,cf", [
+    (1000, 8, 2, 1.5, 0, 1.0), (1000, 8, 2, 1.5, 1, 1.25), (5000, 16, 4, 1.1, 0, 1.0),
+    (8192, 64, 8, 1.1, 1, 1.0), (3000, 256, 8, 1.1, 0, 2.0), (200, 8, 2, 0.0, 0, 0.0),
+    (300, 4, 4, 0.0, 1, 1.0)])
+def test_permute_capacity_bitexact(T, E, k, skew, gate_mode, cf):
+    """Capacity-factor dropping: every row map bit-exact (cf 0 drops every pair)."""
+    g = torch.Generator().manual_seed(5 * T + E)
+    lo = torch.randn(T, E, generator=g)
+    if skew:
+        rank = torch.randperm(E, generator=g).double() + 1
+        lo = lo + (-skew * torch.log(rank)).float()[None, :]
+    cap = B.capacity_from_factor(T, E, k, cf)
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E,
+                                    gate_mode=gate_mode)
+    plan_g = B.moe_permute(idx, gate, logits, E, B.MOE_ROUND_CAPACITY, gate_mode=gate_mode,
+                           capacity=cap)
+    torch.cuda.synchronize()
+    _, ridx, rgate = O.route(None, None, k, logits_override=f64(lo), gate_mode=gate_mode)
+    plan = O.make_plan(ridx, rgate, f64(lo), E, round_mode=2, gate_mode=gate_mode, capacity=cap)
+    assert plan_g["extra_row"] is None
+    if skew and cf <= 1.0:                 # uneven load: the busiest experts drop
+        assert plan["dropped"].any()
+    compare_plan(plan_g, plan)
+
+
+@pytest.mark.parametrize("T,E,k,skew", [(1000, 8, 2, 1.5), (8192, 64, 8, 1.1), (3000, 256, 8, 1.1)])
+def test_permute_rounded_softmax_then_topk_bitexact(T, E, k, skew):
+    """Token rounding with scores from the softmax over all E logits."""
+    g = torch.Generator().manual_seed(11 * T + E)
+    lo = torch.randn(T, E, generator=g)
+    rank = torch.randperm(E, generator=g).double() + 1
+    lo = lo + (-skew * torch.log(rank)).float()[None, :]
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E,
+                                    gate_mode=1)
+    plan_g = B.moe_permute(idx, gate, logits, E, B.MOE_ROUND_NEAREST, gate_mode=1)
+    torch.cuda.synchronize()
+    _, ridx, rgate = O.route(None, None, k, logits_override=f64(lo), gate_mode=1)
+    plan = O.make_plan(ridx, rgate, f64(lo), E, round_mode=1, gate_mode=1)
+    assert plan["added"].any() or plan["dropped"].any()
+    compare_plan(plan_g, plan)
+
+
+@pytest.mark.parametrize("round_mode,gate_mode,cf", [(0, 1, None), (1, 1, None), (2, 0, 1.0),
+                                                    (2, 1, 1.25), (2, 0, 0.0)])
+def test_layer_bf16_routing_variants(round_mode, gate_mode, cf):
+    """The whole layer under each routing variant, against the oracle."""
+    cfg = _cfg(1000, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=17, device="cuda")
+    bias = torch.tensor([0.6, 0.4, 0.2, 0.0, 0.0, -0.2, -0.4, -0.6])   # uneven load
+    lg = fp32_router_logits(inp["x"], inp["w_gate"], bias)
+    cap = B.capacity_from_factor(cfg.T, cfg.E, cfg.k, cf) if round_mode == 2 else -1
+    g = gpu_layer(inp, cfg.k, round_mode, lg, gate_mode=gate_mode, capacity=cap)
+    fwd, bwd = oracle_layer(inp, cfg.k, round_mode, lg, gate_mode=gate_mode,
+                            capacity=cap if round_mode == 2 else None)
+    if round_mode == 2:
+        assert fwd["plan"]["dropped"].any()
+    compare_layer(g, fwd, bwd, BF16_TOL)
+
+
+def test_layer_softmax_then_topk_with_balance_loss_gradient():
+    cfg = _cfg(1000, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=19, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    logits, idx, gate = B.moe_route(x, wg, cfg.k, logits_override=torch.from_numpy(lg).cuda(),
+                                    gate_mode=1)
+    plan = B.moe_permute(idx, gate, logits, cfg.E)
+    H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, cfg.k)
+    bl = B.moe_balance_loss(idx, gate, cfg.E, lam=0.05)
+    gr = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H, gate_grad=bl["dgate"],
+                         logits=logits, gate_mode=1)
+    B.moe_check_status()
+    torch.cuda.synchronize()
+    fwd, _ = oracle_layer(inp, cfg.k, 0, lg, gate_mode=1)
+    rb = O.balance_loss(fwd["idx"], fwd["gate"], cfg.E, 0.05)
+    extra = O.gate_grad_to_logits(fwd["idx"], fwd["gate"], rb["dgate"], cfg.E, gate_mode=1,
+                                  logits=fwd["logits"])
+    bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd, extra_dlogits=extra)
+    for n in ("dlogits", "dw_gate", "dx", "dw1"):
+        assert_close(gr[n], bwd[n], n, BF16_TOL)
