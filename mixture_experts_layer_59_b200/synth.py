@@ -59,7 +59,7 @@ CONFIGS = {
 # One stream id per drawn tensor, so that changing one tensor's shape never
 # changes another tensor's values.
 _STREAMS = {"x": 1, "w_gate": 2, "w1": 3, "w3": 4, "w2": 5, "dout": 6,
-            "logits": 7, "zipf_rank": 8}
+            "logits": 7, "zipf_rank": 8, "noise": 9}
 
 
 def _gen(seed: int, stream: str, device) -> torch.Generator:
@@ -118,3 +118,9 @@ def quantized_logits(T: int, E: int, levels: int, seed: int = 0) -> torch.Tensor
     occur; used to exercise the lowest-expert-id tie rule."""
     g = _gen(seed, "logits", "cpu")
     return torch.randint(0, levels, (T, E), generator=g).to(torch.float32) * 0.25
+
+
+def logit_noise(T: int, E: int, std: float, seed: int = 0, device="cpu") -> torch.Tensor:
+    """Gaussian routing noise eps ~ N(0, std^2) [T,E] fp32 for noisy top-k
+    gating: the random numbers the method draws, handed to both sides."""
+    return _normal((T, E), std, torch.float32, seed, "noise", device)

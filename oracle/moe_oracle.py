@@ -43,6 +43,11 @@ Readings taken where the pages are silent (each also listed in the design doc):
     top-k logits); drops take the smallest keys (ties: larger token first),
     additions take the largest keys among unassigned tokens (ties: smaller
     token first); final weights are s_te without renormalisation.
+  * noisy top-k gating ([Beam] sec. 3.3, second point: noise added to the
+    routing scores in training): the caller draws the noise eps [T,E] and
+    passes it in; routing (choice, gates, rounding scores) uses l + eps, and
+    the gradient reaches the clean logits unchanged because eps depends on
+    no parameter.
   * balance loss: G_i is token i's routing distribution over the E experts
     (its top-k gates, zeros elsewhere); CV is the population coefficient of
     variation over experts (std / mean); count statistics use the top-k
@@ -106,9 +111,11 @@ def silu_grad(z):
 # router: logits, top-k, softmax over the top-k  ([Beam] 2.2, 5.3; [Trinity] ex. 1)
 # --------------------------------------------------------------------------
 
-def route(x, w_gate, k, logits_override=None, logit_bias=None, gate_mode=0):
-    """Router logits l = x W_gate (+ optional per-expert bias), the k largest
-    logits of each token (ties: lowest expert id first), and their gates:
+def route(x, w_gate, k, logits_override=None, logit_bias=None, gate_mode=0, logit_noise=None):
+    """Router logits l = x W_gate (+ optional per-expert bias, + optional
+    noise eps [T,E] drawn by the caller: noisy top-k gating, [Beam] 3.3), the
+    k largest logits of each token (ties: lowest expert id first), and their
+    gates:
     gate_mode 0: softmax over the k selected logits ([Beam] 5.3, [Trinity] ex. 1);
     gate_mode 1: softmax over all E logits, the k largest kept without
     renormalisation ([Beam] 2.2 formula, [Trinity] challenge 1).
@@ -121,6 +128,8 @@ def route(x, w_gate, k, logits_override=None, logit_bias=None, gate_mode=0):
         logits = np.asarray(x, np.float64) @ np.asarray(w_gate, np.float64)
     if logit_bias is not None:
         logits = logits + np.asarray(logit_bias, np.float64)[None, :]
+    if logit_noise is not None:
+        logits = logits + np.asarray(logit_noise, np.float64)
     # a stable sort of the negated logits keeps equal values in ascending id
     idx = np.argsort(-logits, axis=1, kind="stable")[:, :k]
     top = np.take_along_axis(logits, idx, axis=1)
@@ -401,9 +410,10 @@ def make_plan(idx, gate, logits, E, tile=TILE, round_mode=0, gate_mode=0, capaci
 
 
 def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
-              logits_override=None, logit_bias=None, staged=True, gate_mode=0, capacity=None):
+              logits_override=None, logit_bias=None, staged=True, gate_mode=0, capacity=None,
+              logit_noise=None):
     """Full forward: route, permute, expert FFN on every row, combine."""
-    logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias, gate_mode)
+    logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias, gate_mode, logit_noise)
     T, E = logits.shape
     plan = make_plan(idx, gate, logits, E, tile, round_mode, gate_mode, capacity)
     rows = np.arange(plan["R"])

@@ -293,21 +293,26 @@ def test_two_expert_hand_example():
     assert abs(bwd["dx"][0, 0] - want["dx"]) < 1e-9
 
 
-def _loss(params, dout, k, tile, round_mode, gate_mode=0, capacity=None):
+def _loss(params, dout, k, tile, round_mode, gate_mode=0, capacity=None, noise=None):
     x, wg, w1, w3, w2 = params
     fwd = O.layer_fwd(x, wg, w1, w3, w2, k=k, tile=tile, round_mode=round_mode, staged=False,
-                      gate_mode=gate_mode, capacity=capacity)
+                      gate_mode=gate_mode, capacity=capacity, logit_noise=noise)
     return float(np.sum(fwd["out"] * dout)), fwd
 
 
-@pytest.mark.parametrize("round_mode,gate_mode,capacity", [
-    (0, 0, None), (1, 0, None), (0, 1, None), (1, 1, None), (2, 0, 3), (2, 1, 3)])
-def test_backward_matches_central_differences(round_mode, gate_mode, capacity):
-    rng = np.random.default_rng(11 + round_mode + 10 * gate_mode)
+@pytest.mark.parametrize("round_mode,gate_mode,capacity,noisy", [
+    (0, 0, None, 0), (1, 0, None, 0), (0, 1, None, 0), (1, 1, None, 0), (2, 0, 3, 0), (2, 1, 3, 0),
+    (0, 0, None, 1), (1, 1, None, 1)])
+def test_backward_matches_central_differences(round_mode, gate_mode, capacity, noisy):
+    rng = np.random.default_rng(11 + round_mode + 10 * gate_mode + 100 * noisy)
     T, d, f, E, k, tile = 9, 4, 3, 4, 2, 4
     x, wg, w1, w3, w2, dout = _rand_layer(rng, T, d, f, E)
     params = [x, wg, w1, w3, w2]
-    _, fwd = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
+    noise = rng.standard_normal((T, E)) if noisy else None
+    _, fwd = _loss(params, dout, k, tile, round_mode, gate_mode, capacity, noise)
+    if noisy:   # the noise changes the routing of some token
+        assert not np.array_equal(fwd["idx"], _loss(params, dout, k, tile, round_mode,
+                                                     gate_mode, capacity)[1]["idx"])
     if round_mode:
         assert fwd["plan"]["dropped"].any() or fwd["plan"]["added"].any()
     bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
@@ -318,9 +323,9 @@ def test_backward_matches_central_differences(round_mode, gate_mode, capacity):
         for i in np.ndindex(p.shape):
             old = p[i]
             p[i] = old + h
-            lp, fp = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
+            lp, fp = _loss(params, dout, k, tile, round_mode, gate_mode, capacity, noise)
             p[i] = old - h
-            lm, fm = _loss(params, dout, k, tile, round_mode, gate_mode, capacity)
+            lm, fm = _loss(params, dout, k, tile, round_mode, gate_mode, capacity, noise)
             p[i] = old
             # the discrete routing must not change under the probe
             assert np.array_equal(fp["idx"], fwd["idx"]) and np.array_equal(fm["idx"], fwd["idx"])
@@ -558,3 +563,26 @@ def test_gate_grad_to_logits_mode1_matches_finite_differences():
             gp = O.route(None, None, k, logits_override=lp, gate_mode=1)[2]
             gm = O.route(None, None, k, logits_override=lm, gate_mode=1)[2]
             assert abs(((gp - gm) * a).sum() / (2 * h) - dl[t, e]) < 1e-7
+
+
+def test_noisy_routing_special_cases():
+    """Zero noise is no noise; a dominant noise on one expert makes every token
+    choose it first, with gate -> 1 under the all-E softmax, and leaves the
+    choice of the other k-1 experts to the clean logits."""
+    rng = np.random.default_rng(23)
+    T, d, E, k = 40, 8, 6, 3
+    x, wg = rng.standard_normal((T, d)), rng.standard_normal((d, E))
+    base = O.route(x, wg, k)
+    zero = O.route(x, wg, k, logit_noise=np.zeros((T, E)))
+    for a, b in zip(base, zero):
+        np.testing.assert_array_equal(a, b)
+    eps = np.zeros((T, E))
+    eps[:, 4] = 80.0
+    lg, idx, gate = O.route(x, wg, k, gate_mode=1, logit_noise=eps)
+    assert np.all(idx[:, 0] == 4)
+    np.testing.assert_allclose(gate[:, 0], 1.0, rtol=1e-12)
+    clean = x @ wg
+    for t in range(T):
+        rest = [e for e in np.argsort(-clean[t], kind="stable") if e != 4][:k - 1]
+        assert list(idx[t, 1:]) == rest
+    np.testing.assert_allclose(lg, clean + eps, rtol=1e-15)
