@@ -48,6 +48,8 @@ def parse_args():
                     help="1 = token rounding to 128-row tiles, 2 = capacity factor")
     ap.add_argument("--capacity-factor", type=float, default=1.0,
                     help="tokens per expert = ceil(factor * T * k / E) with --round 2")
+    ap.add_argument("--noise-std", type=float, default=0.0,
+                    help="noisy top-k gating: Gaussian routing noise of this std on the scores")
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1],
                     help="0 = softmax over the top-k logits, 1 = softmax over all E then top-k")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -185,11 +187,13 @@ def oracle_tokens_per_s(cfg, n_tokens, args, seed=0, repeats=1):
     f64 = lambda t: None if t is None else t.to(torch.float64).numpy()
     x, wg, w1, w3, w2, do = (f64(inp[n]) for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo, lb = f64(inp["logits_override"]), f64(inp["logit_bias"])
+    eps = (f64(synth.logit_noise(n_tokens, cfg.E, args.noise_std, seed=seed))
+           if args.noise_std else None)
     times = []
     for _ in range(repeats):
         t0 = time.perf_counter()
         fwd = O.layer_fwd(x, wg, w1, w3, w2, cfg.k, logits_override=lo, logit_bias=lb,
-                          round_mode=args.round, gate_mode=args.gate_mode,
+                          round_mode=args.round, gate_mode=args.gate_mode, logit_noise=eps,
                           capacity=_capacity(n_tokens, cfg.E, cfg.k, args))
         O.layer_bwd(do, x, wg, w1, w3, w2, fwd, router_grad_on=lo is None)
         times.append(time.perf_counter() - t0)
@@ -225,6 +229,7 @@ def workload_config(cfg, args):
             "k": cfg.k, "routing": cfg.routing, "token_rounding": args.round == 1,
             "capacity_factor": args.capacity_factor if args.round == 2 else None,
             "gate": "softmax_then_topk" if args.gate_mode else "topk_then_softmax",
+            "routing_noise_std": args.noise_std or None,
             "balance_loss_lambda": args.balance_loss,
             "l2": f"flushed between timed steps ({args.flush_mb} MiB write)", "replicas": args.gpus}
 
@@ -247,9 +252,11 @@ def run_ours(args, cfg, rank, world, local_rank):
     flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
     x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo, lb = inp["logits_override"], inp["logit_bias"]
+    noise = (synth.logit_noise(cfg.T, cfg.E, args.noise_std, seed=rank, device=dev)
+             if args.noise_std else None)
 
     def one_step():
-        step.forward(x, wg, w1, w3, w2, lo, lb)
+        step.forward(x, wg, w1, w3, w2, lo, lb, logit_noise=noise)
         step.backward(dout)
 
     for _ in range(args.warmup):
@@ -304,7 +311,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         s_ev.record()
         x_d.copy_(x_h, non_blocking=True)
         d_d.copy_(d_h, non_blocking=True)
-        step.forward(x_d, wg, w1, w3, w2, lo, lb)
+        step.forward(x_d, wg, w1, w3, w2, lo, lb, logit_noise=noise)
         step.backward(d_d)
         out_h.copy_(step.out, non_blocking=True)
         dx_h.copy_(step.grads["dx"], non_blocking=True)

@@ -92,13 +92,19 @@ size_t moe_row_capacity(int T, int E, int k, int tile);
  *   logits_override [T,E] fp32 or NULL: when given, x and w_gate are not read
  *     and these values replace x W_gate (random-routing workloads).
  *   logit_bias [E] fp32 or NULL: added to every token's logits.
+ *   logit_noise [T,E] fp32 or NULL: noisy top-k gating ([Beam] sec. 3.3,
+ *     noise on the routing scores in training): added after the bias
+ *     (fp32 adds in that order); the caller draws it.  Choice, gates and the
+ *     returned logits are those of the noisy scores; the gradient
+ *     moe_layer_bwd returns for the logits is also that of the clean ones.
  *   logits [T,E] fp32 out; idx [T,k] int32 out: the k largest logits in
  *   descending order, ties to the lowest expert id; gate [T,k] fp32 out:
  *   the gates of those k experts (per gate_mode).
  */
 int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
               int gate_mode, const float* logits_override, const float* logit_bias,
-              float* logits, int32_t* idx, float* gate, void* stream);
+              const float* logit_noise, float* logits, int32_t* idx, float* gate,
+              void* stream);
 
 /*
  * moe_permute -- expert histogram, prefix sum and stable permutation into

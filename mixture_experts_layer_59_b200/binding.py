@@ -44,7 +44,7 @@ _SIGS = {
     "moe_version": (_i, []),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_row_capacity": (_sz, [_i, _i, _i, _i]),
-    "moe_route": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_route": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i, _i, _i]),
     "moe_permute": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
                          _vp, _vp, _vp, _sz, _vp]),
@@ -110,10 +110,12 @@ def moe_row_capacity(T, E, k, tile=TILE) -> int:
 
 
 def moe_route(x, w_gate, k, logits_override=None, logit_bias=None, logits=None, idx=None,
-              gate=None, T=None, E=None, stream=None, gate_mode=MOE_GATE_TOPK_SOFTMAX):
+              gate=None, T=None, E=None, stream=None, gate_mode=MOE_GATE_TOPK_SOFTMAX,
+              logit_noise=None):
     """logits [T,E] f32, idx [T,k] i32, gate [T,k] f32 (outputs allocated if None).
     gate_mode: MOE_GATE_TOPK_SOFTMAX (softmax over the k chosen logits) or
-    MOE_GATE_SOFTMAX_TOPK (softmax over all E, the k largest kept)."""
+    MOE_GATE_SOFTMAX_TOPK (softmax over all E, the k largest kept).
+    logit_noise [T,E] f32: routing noise added to the scores (noisy top-k)."""
     if T is None:
         T = (logits_override if logits_override is not None else x).shape[0]
     if E is None:
@@ -125,7 +127,7 @@ def moe_route(x, w_gate, k, logits_override=None, logit_bias=None, logits=None, 
     idx = idx if idx is not None else torch.empty(T, k, device=dev, dtype=torch.int32)
     gate = gate if gate is not None else torch.empty(T, k, device=dev, dtype=torch.float32)
     _check(lib().moe_route(_p(x), _p(w_gate), T, d, E, k, dt, gate_mode, _p(logits_override),
-                           _p(logit_bias),
+                           _p(logit_bias), _p(logit_noise),
                            _p(logits), _p(idx), _p(gate), _stream(stream)))
     return logits, idx, gate
 

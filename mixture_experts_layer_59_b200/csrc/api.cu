@@ -179,7 +179,8 @@ size_t moe_row_capacity(int T, int E, int k, int tile) {
 
 int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int dtype,
               int gate_mode, const float* logits_override, const float* logit_bias,
-              float* logits, int32_t* idx, float* gate, void* stream) {
+              const float* logit_noise, float* logits, int32_t* idx, float* gate,
+              void* stream) {
   if (int rc = check_common(T, E, k, dtype)) return rc;
   if (gate_mode != MOE_GATE_TOPK_SOFTMAX && gate_mode != MOE_GATE_SOFTMAX_TOPK)
     return fail(MOE_ERR_INVALID_ARG, "gate_mode must be MOE_GATE_TOPK_SOFTMAX or MOE_GATE_SOFTMAX_TOPK");
@@ -197,13 +198,14 @@ int moe_route(const void* x, const void* w_gate, int T, int d, int E, int k, int
       // tensor-core router GEMM with the bias, top-k and softmax in its epilogue
       REQUIRE_ALIGNED(x);
       REQUIRE_ALIGNED(w_gate);
-      return tc_router_fwd(x, w_gate, logit_bias, T, d, E, k, gate_mode, logits, idx, gate,
-                           device_sm_count(), s);
+      return tc_router_fwd(x, w_gate, logit_bias, logit_noise, T, d, E, k, gate_mode, logits,
+                           idx, gate, device_sm_count(), s);
     }
     if (int rc = launch_router_logits_simt(x, w_gate, T, d, E, dtype, nullptr, logits, s)) return rc;
     src = logits;
   }
-  return launch_topk_softmax(src, logit_bias, logits, T, E, k, gate_mode, idx, gate, s);
+  return launch_topk_softmax(src, logit_bias, logit_noise, logits, T, E, k, gate_mode, idx, gate,
+                             s);
 }
 
 size_t moe_permute_workspace_size(int T, int E, int k, int round_mode) {

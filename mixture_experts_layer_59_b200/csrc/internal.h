@@ -9,9 +9,9 @@ namespace moe {
 // ---------------------------------------------------------------- routing
 int launch_router_logits_simt(const void* x, const void* wg, int T, int d, int E, int dtype,
                               const float* bias, float* logits, cudaStream_t s);
-int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out,
-                        int T, int E, int k, int gate_mode, int32_t* idx, float* gate,
-                        cudaStream_t s);
+int launch_topk_softmax(const float* logits_in, const float* bias, const float* noise,
+                        float* logits_out, int T, int E, int k, int gate_mode, int32_t* idx,
+                        float* gate, cudaStream_t s);
 
 // ---------------------------------------------------------------- permutation
 struct PermuteWs {
@@ -90,9 +90,9 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
 int tc_num_dS_parts(int f);
 bool tc_router_ok(int E);
 int tc_dwg_splits(int T, int d, int* chunk);
-int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
-                  int gate_mode, float* logits, int32_t* idx, float* gate, int num_sms,
-                  cudaStream_t s);
+int tc_router_fwd(const void* x, const void* wg, const float* bias, const float* noise, int T,
+                  int d, int E, int k, int gate_mode, float* logits, int32_t* idx, float* gate,
+                  int num_sms, cudaStream_t s);
 int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* dl_lo, int T,
                   int d, int E, int k, float* dwg_part, float* dw_gate, const float* dx_acc,
                   void* dx, int num_sms, cudaStream_t s);

@@ -14,8 +14,9 @@ namespace moe {
 // One warp per token.  Each lane holds up to 8 of the E <= 256 logits
 // (expert e = lane + 32*i).  k rounds of a warp arg-max (ties: lowest id).
 __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float* __restrict__ bias,
-                               float* __restrict__ logits_out, int T, int E, int k, int gate_mode,
-                               int32_t* __restrict__ idx, float* __restrict__ gate) {
+                               const float* __restrict__ noise, float* __restrict__ logits_out,
+                               int T, int E, int k, int gate_mode, int32_t* __restrict__ idx,
+                               float* __restrict__ gate) {
   const int lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   for (int t = blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += gridDim.x * warps) {
@@ -27,7 +28,8 @@ __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float*
       if (e < E) {
         l = logits_in[(size_t)t * E + e];
         if (bias) l += bias[e];
-        if (logits_out != logits_in || bias) logits_out[(size_t)t * E + e] = l;
+        if (noise) l += noise[(size_t)t * E + e];
+        if (logits_out != logits_in || bias || noise) logits_out[(size_t)t * E + e] = l;
       }
       v[i] = l;
     }
@@ -76,15 +78,16 @@ __global__ void k_topk_softmax(const float* __restrict__ logits_in, const float*
   }
 }
 
-int launch_topk_softmax(const float* logits_in, const float* bias, float* logits_out, int T,
-                        int E, int k, int gate_mode, int32_t* idx, float* gate, cudaStream_t s) {
+int launch_topk_softmax(const float* logits_in, const float* bias, const float* noise,
+                        float* logits_out, int T, int E, int k, int gate_mode, int32_t* idx,
+                        float* gate, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + 7) / 8;
   if (blocks > 148 * 16) blocks = 148 * 16;
   {
     ProfScope _ps("topk_softmax", s);
-    k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, logits_out, T, E, k, gate_mode, idx,
-                                          gate);
+    k_topk_softmax<<<blocks, 256, 0, s>>>(logits_in, bias, noise, logits_out, T, E, k, gate_mode,
+                                          idx, gate);
   }
   MOE_CHECK_LAUNCH("topk_softmax");
   return MOE_OK;

@@ -85,6 +85,7 @@ struct TcArgs {
   int T, k, splits, chunk;
   int gate_mode;             // RT: 0 softmax over the top-k, 1 softmax over all E
   const float* bias;         // RT: [E] or null
+  const float* noise;        // RT: [T, E] routing noise or null
   float* logits;             // RT: [T, E]
   int32_t* idx;              // RT: [T, k]
   float* gate;               // RT: [T, k]
@@ -509,6 +510,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             for (int i = 0; i < 32; ++i) {
               v[i] = __uint_as_float(r[i]);
               if (a.bias && c + i < a.E) v[i] += a.bias[c + i];
+              if (a.noise && valid && c + i < a.E) v[i] += a.noise[(size_t)t * a.E + c + i];
             }
             if (valid) {
               float4* dst = reinterpret_cast<float4*>(a.logits + (size_t)t * a.E + c);
@@ -540,8 +542,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
               tmem_ld_wait();
 #pragma unroll
               for (int i = 0; i < 32; ++i)
-                if (c + i < a.E)
-                  zall += expf(__uint_as_float(r[i]) + (a.bias ? a.bias[c + i] : 0.f) - tv[0]);
+                if (c + i < a.E) {
+                  float l = __uint_as_float(r[i]);
+                  if (a.bias) l += a.bias[c + i];
+                  if (a.noise && valid) l += a.noise[(size_t)t * a.E + c + i];
+                  zall += expf(l - tv[0]);
+                }
             }
           }
           if (valid) {
@@ -758,9 +764,9 @@ int tc_dwg_splits(int T, int d, int* chunk) {
   return (T + c - 1) / c > 0 ? (T + c - 1) / c : 1;
 }
 
-int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d, int E, int k,
-                  int gate_mode, float* logits, int32_t* idx, float* gate, int num_sms,
-                  cudaStream_t s) {
+int tc_router_fwd(const void* x, const void* wg, const float* bias, const float* noise, int T,
+                  int d, int E, int k, int gate_mode, float* logits, int32_t* idx, float* gate,
+                  int num_sms, cudaStream_t s) {
   TcArgs a;
   memset(&a, 0, sizeof(a));
   a.gate_mode = gate_mode;
@@ -771,6 +777,7 @@ int tc_router_fwd(const void* x, const void* wg, const float* bias, int T, int d
   a.T = T;
   a.k = k;
   a.bias = bias;
+  a.noise = noise;
   a.logits = logits;
   a.idx = idx;
   a.gate = gate;

@@ -49,11 +49,13 @@ class MoELayerStep:
                           dw3=e(E, d, f, dt_=dtype), dw2=e(E, f, d, dt_=dtype), dS=e(cap),
                           dlogits=e(T, E))
 
-    def forward(self, x, w_gate, w1, w3, w2, logits_override=None, logit_bias=None, stream=None):
+    def forward(self, x, w_gate, w1, w3, w2, logits_override=None, logit_bias=None, stream=None,
+                logit_noise=None):
         self._saved = (x, w_gate, w1, w3, w2)
         self.router_grad = logits_override is None
         B.moe_route(x, w_gate, self.k, logits_override, logit_bias, self.logits, self.idx,
-                    self.gate, T=self.T, E=self.E, stream=stream, gate_mode=self.gate_mode)
+                    self.gate, T=self.T, E=self.E, stream=stream, gate_mode=self.gate_mode,
+                    logit_noise=logit_noise)
         B.moe_permute(self.idx, self.gate, self.logits, self.E, self.round_mode, out=self.plan,
                       ws=self.ws_perm, stream=stream, gate_mode=self.gate_mode,
                       capacity=self.capacity)

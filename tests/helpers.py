@@ -52,12 +52,13 @@ def fp32_router_logits(x, w_gate, logit_bias=None):
 
 
 def gpu_layer(inp, k, round_mode, logits32, router_grad=True, dev="cuda", gate_mode=0,
-              capacity=-1):
+              capacity=-1, noise=None):
     """Forward + backward through the C ABI with the routing logits given."""
     x, wg, w1, w3, w2, dout = (inp[n].to(dev) for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
     lo = torch.from_numpy(np.ascontiguousarray(logits32)).to(dev)
     T, E = lo.shape
-    logits, idx, gate = B.moe_route(x, wg, k, logits_override=lo, gate_mode=gate_mode)
+    logits, idx, gate = B.moe_route(x, wg, k, logits_override=lo, gate_mode=gate_mode,
+                                    logit_noise=None if noise is None else noise.to(dev))
     plan = B.moe_permute(idx, gate, logits, E, round_mode, gate_mode=gate_mode, capacity=capacity)
     H, Y = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
     out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)

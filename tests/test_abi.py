@@ -46,11 +46,12 @@ def test_workspace_sizes_monotone():
 
 def _rc_route(**kw):
     args = dict(x=None, wg=None, T=4, d=128, E=8, k=2, dtype=B.MOE_BF16, gm=0, lo=None, lb=None,
-                logits=None, idx=None, gate=None, stream=None)
+                ln=None, logits=None, idx=None, gate=None, stream=None)
     args.update(kw)
     lib = B.lib()
     return lib.moe_route(args["x"], args["wg"], args["T"], args["d"], args["E"], args["k"],
-                         args["dtype"], args["gm"], args["lo"], args["lb"], args["logits"],
+                         args["dtype"], args["gm"], args["lo"], args["lb"], args["ln"],
+                         args["logits"],
                          args["idx"],
                          args["gate"], args["stream"])
 

@@ -298,3 +298,54 @@ def test_layer_softmax_then_topk_with_balance_loss_gradient():
     bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd, extra_dlogits=extra)
     for n in ("dlogits", "dw_gate", "dx", "dw1"):
         assert_close(gr[n], bwd[n], n, BF16_TOL)
+
+
+# ------------------------------------------------------------------ noisy top-k gating
+
+@pytest.mark.parametrize("E,k,gate_mode", [(8, 2, 0), (64, 8, 1), (256, 8, 0)])
+def test_route_noisy_scores_bitexact(E, k, gate_mode):
+    """Routing noise is added after the bias in fp32; the oracle routes the
+    same fp32 scores."""
+    T = 999
+    lo = torch.randn(T, E, generator=torch.Generator().manual_seed(E))
+    bias = torch.linspace(-0.5, 0.5, E)
+    eps = synth.logit_noise(T, E, 1.0, seed=E)
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), logit_bias=bias.cuda(),
+                                    T=T, E=E, gate_mode=gate_mode, logit_noise=eps.cuda())
+    torch.cuda.synchronize()
+    scores = (lo + bias[None, :]) + eps                     # the same two fp32 adds
+    _, ref_idx, ref_g = O.route(None, None, k, logits_override=f64(scores), gate_mode=gate_mode)
+    np.testing.assert_array_equal(f64(logits), f64(scores))
+    np.testing.assert_array_equal(i64(idx), ref_idx)
+    np.testing.assert_allclose(f64(gate), ref_g, rtol=2e-6, atol=1e-7)
+    clean = O.route(None, None, k, logits_override=f64(lo + bias[None, :]))[1]
+    assert (i64(idx) != clean).any()                       # the noise changed some choices
+
+
+@pytest.mark.parametrize("gate_mode", [0, 1])
+def test_route_noisy_tensor_core_router(gate_mode):
+    cfg = _cfg(1000, 256, 128, 64, 8, std=0.05)
+    inp = synth.make_inputs(cfg, seed=8, device="cuda")
+    eps = synth.logit_noise(cfg.T, cfg.E, 0.5, seed=8, device="cuda")
+    logits, idx, gate = B.moe_route(inp["x"], inp["w_gate"], cfg.k, gate_mode=gate_mode,
+                                    logit_noise=eps)
+    torch.cuda.synchronize()
+    ref = f64(inp["x"]) @ f64(inp["w_gate"]) + f64(eps)
+    scale = np.abs(ref).max()
+    np.testing.assert_allclose(f64(logits), ref, atol=1e-5 * scale, rtol=0)
+    # the choice and gates follow the GPU's own noisy scores exactly
+    _, own_idx, own_g = O.route(None, None, cfg.k, logits_override=f64(logits), gate_mode=gate_mode)
+    np.testing.assert_array_equal(i64(idx), own_idx)
+    np.testing.assert_allclose(f64(gate), own_g, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("round_mode,gate_mode", [(0, 0), (1, 1)])
+def test_layer_noisy_routing(round_mode, gate_mode):
+    cfg = _cfg(1000, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=23, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    eps = synth.logit_noise(cfg.T, cfg.E, 0.02, seed=23)
+    g = gpu_layer(inp, cfg.k, round_mode, lg, gate_mode=gate_mode, noise=eps)
+    noisy32 = (torch.from_numpy(lg) + eps).numpy()          # the scores the GPU routed on
+    fwd, bwd = oracle_layer(inp, cfg.k, round_mode, noisy32, gate_mode=gate_mode)
+    compare_layer(g, fwd, bwd, BF16_TOL)
