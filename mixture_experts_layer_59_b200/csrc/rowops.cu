@@ -106,15 +106,21 @@ int launch_scatter_rows(const void* src, const int32_t* slot_row, const int32_t*
 // for routers whose W_gate fits in shared memory (E <= 32, d*E*2 <= 48 KB).
 // One warp per token; a lane owns 8 consecutive columns per step and loads the
 // next step's rows before summing the current ones.
-__device__ __forceinline__ void load_rows8(const __nv_bfloat16* __restrict__ dxp, const int (&rk)[8],
-                                           int d, int i, uint4 (&raw)[8]) {
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    raw[j] = rk[j] >= 0 ? __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)rk[j] * d) + i)
-                        : make_uint4(0, 0, 0, 0);
-}
+// dx_t = sum over token t's rows of dX_perm + dl_t W_gate^T, for small
+// routers (E <= 32): one warp per token; each lane owns 8 consecutive columns
+// per vector and handles two vectors per pass, issuing the loads of all the
+// token's rows for both before any arithmetic.  The row sum runs in fp32 in
+// slot order, then the rows added by rounding in ascending expert id, then the
+// router term in ascending expert id.
+template <int MAXE, int MAXK> struct DxfTraits {
+  // vectors per lane per pass (loads in flight) and resident blocks per SM,
+  // chosen so that the registers fit without spilling
+  static constexpr int V = MAXK <= 4 ? 2 : 1;
+  static constexpr int MINB = (MAXE * MAXK <= 32 || (MAXE <= 16 && MAXK <= 2)) ? 4 : 2;
+};
 
-__global__ void __launch_bounds__(256)
+template <int MAXE, int MAXK>
+__global__ void __launch_bounds__(256, (DxfTraits<MAXE, MAXK>::MINB))
 k_dx_fused(const __nv_bfloat16* __restrict__ dxp, const int32_t* __restrict__ slot_row,
            const int32_t* __restrict__ extra_row, const float* __restrict__ dl,
            const __nv_bfloat16* __restrict__ wg, int T_, int d, int E, int k,
@@ -122,8 +128,9 @@ k_dx_fused(const __nv_bfloat16* __restrict__ dxp, const int32_t* __restrict__ sl
   extern __shared__ __align__(16) uint8_t smem_wg[];
   // W_gate transposed to [E][d] (bf16): a lane's 8 consecutive columns of one
   // expert are one conflict-free 16-byte shared load.  Staged once per block
-  // (persistent grid); each thread owns whole columns.
+  // (persistent grid).
   __nv_bfloat16* w_t = reinterpret_cast<__nv_bfloat16*>(smem_wg);
+  __shared__ int s_extra[8][32];  // rows added by rounding, per warp (E <= 32)
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     for (int e0 = 0; e0 < E; e0 += 8) {
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(wg + (size_t)c * E + e0));
@@ -136,84 +143,121 @@ k_dx_fused(const __nv_bfloat16* __restrict__ dxp, const int32_t* __restrict__ sl
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nvec = d / 8;
   for (int t = blockIdx.x * 8 + w; t < T_; t += gridDim.x * 8) {
-    float dlr[32];
+    // the token's added rows, in ascending expert id (whole warp)
+    int n_extra = 0;
+    if (extra_row != nullptr) {
+      const int re = lane < E ? extra_row[(size_t)t * E + lane] : -1;
+      const unsigned bal = __ballot_sync(0xffffffffu, re >= 0);
+      if (re >= 0) s_extra[w][__popc(bal & ((1u << lane) - 1u))] = re;
+      n_extra = __popc(bal);
+      __syncwarp();
+    }
+    float dlr[MAXE];
 #pragma unroll
-    for (int e = 0; e < 32; ++e) dlr[e] = e < E ? dl[(size_t)t * E + e] : 0.f;
+    for (int e = 0; e < MAXE; ++e) dlr[e] = e < E ? dl[(size_t)t * E + e] : 0.f;
     const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
-    int rk[8];
+    int rk[MAXK];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
-    uint4 nxt[8];
-    if (lane < nvec) load_rows8(dxp, rk, d, lane, nxt);
-    for (int i = lane; i < nvec; i += 32) {
-      uint4 raw[8];
+    for (int j = 0; j < MAXK; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
+    constexpr int V = DxfTraits<MAXE, MAXK>::V;
+    for (int i0 = lane; i0 < nvec; i0 += 32 * V) {
+      uint4 raw[V][MAXK];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) raw[j] = nxt[j];
-      if (i + 32 < nvec) load_rows8(dxp, rk, d, i + 32, nxt);
-      float acc[8];
+      for (int v = 0; v < V; ++v) {
+        const int i = i0 + 32 * v;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (rk[j] >= 0) {
-          Vec<__nv_bfloat16> v;
-          v.v = raw[j];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc[q] += v.get(q);
-        }
+        for (int j = 0; j < MAXK; ++j)
+          raw[v][j] = (i < nvec && rk[j] >= 0)
+                          ? __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)rk[j] * d) + i)
+                          : make_uint4(0, 0, 0, 0);
       }
-      if (extra_row != nullptr) {
-        for (int e0 = 0; e0 < E; e0 += 32) {
-          const int re = e0 + lane < E ? extra_row[(size_t)t * E + e0 + lane] : -1;
-          unsigned bal = __ballot_sync(__activemask(), re >= 0);
-          while (bal) {
-            const int b = __ffs(bal) - 1;
-            bal &= bal - 1;
-            const int r = __shfl_sync(__activemask(), re, b);
-            Vec<__nv_bfloat16> v;
-            v.v = __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)r * d) + i);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[q] += v.get(q);
+      for (int v = 0; v < V; ++v) {
+        const int i = i0 + 32 * v;
+        if (i >= nvec) break;
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+        for (int j = 0; j < MAXK; ++j) {
+          if (rk[j] >= 0) {
+            Vec<__nv_bfloat16> u;
+            u.v = raw[v][j];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] += u.get(q);
           }
         }
-      }
-      // router term: columns 8i..8i+7 of every expert column of W_gate
+        for (int j = 0; j < n_extra; ++j) {
+          Vec<__nv_bfloat16> u;
+          u.v = __ldg(reinterpret_cast<const uint4*>(dxp + (size_t)s_extra[w][j] * d) + i);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        if (e < E) {
-          Vec<__nv_bfloat16> wv;
-          wv.v = reinterpret_cast<const uint4*>(w_t + (size_t)e * d)[i];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc[q] = fmaf(dlr[e], wv.get(q), acc[q]);
+          for (int q = 0; q < 8; ++q) acc[q] += u.get(q);
         }
-      }
-      Vec<__nv_bfloat16> o;
+        // router term: columns 8i..8i+7 of every expert column of W_gate
 #pragma unroll
-      for (int q = 0; q < 8; ++q) o.set(q, acc[q]);
-      reinterpret_cast<uint4*>(dx + (size_t)t * d)[i] = o.v;
+        for (int e = 0; e < MAXE; ++e) {
+          if (e < E) {
+            Vec<__nv_bfloat16> wv;
+            wv.v = reinterpret_cast<const uint4*>(w_t + (size_t)e * d)[i];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(dlr[e], wv.get(q), acc[q]);
+          }
+        }
+        Vec<__nv_bfloat16> o;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) o.set(q, acc[q]);
+        reinterpret_cast<uint4*>(dx + (size_t)t * d)[i] = o.v;
+      }
     }
+    __syncwarp();
   }
 }
 
 bool dx_fused_ok(int d, int E) { return E <= 32 && E % 8 == 0 && (size_t)d * E * 2 <= 48 * 1024; }
+
+template <int MAXE, int MAXK>
+static void dx_fused_go(int blocks, size_t smem, cudaStream_t s, const void* dxp,
+                        const int32_t* slot_row, const int32_t* extra_row, const float* dl,
+                        const void* wg, int T, int d, int E, int k, void* dx) {
+  k_dx_fused<MAXE, MAXK><<<blocks, 256, smem, s>>>((const __nv_bfloat16*)dxp, slot_row, extra_row,
+                                                   dl, (const __nv_bfloat16*)wg, T, d, E, k,
+                                                   (__nv_bfloat16*)dx);
+}
+
+template <int MAXE>
+static int dx_fused_k(int blocks, size_t smem, cudaStream_t s, const void* dxp,
+                      const int32_t* slot_row, const int32_t* extra_row, const float* dl,
+                      const void* wg, int T, int d, int E, int k, void* dx) {
+  if (smem > 48 * 1024) {
+    cudaError_t e;
+    if (k <= 2) e = cudaFuncSetAttribute(k_dx_fused<MAXE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    else if (k <= 4) e = cudaFuncSetAttribute(k_dx_fused<MAXE, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    else e = cudaFuncSetAttribute(k_dx_fused<MAXE, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "dx_fused smem attribute");
+  }
+  if (k <= 2) dx_fused_go<MAXE, 2>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
+  else if (k <= 4) dx_fused_go<MAXE, 4>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
+  else dx_fused_go<MAXE, 8>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
+  return MOE_OK;
+}
 
 int launch_dx_fused(const void* dxp, const int32_t* slot_row, const int32_t* extra_row,
                     const float* dl, const void* wg, int T, int d, int E, int k, void* dx,
                     cudaStream_t s) {
   if (T == 0) return MOE_OK;
   const size_t smem = (size_t)d * E * 2;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(k_dx_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "dx_fused smem attribute");
-  }
   int blocks = (T + 7) / 8;
-  const int per_sm = (int)(200 * 1024 / (smem + 1024)) < 8 ? (int)(200 * 1024 / (smem + 1024)) : 8;
+  const int fit = (int)(220 * 1024 / (smem + 2048));
+  const int per_sm = fit < 4 ? (fit > 0 ? fit : 1) : 4;
   if (blocks > device_sm_count() * per_sm) blocks = device_sm_count() * per_sm;
+  int rc;
   {
     ProfScope _ps("dx_fused", s);
-    k_dx_fused<<<blocks, 256, smem, s>>>((const __nv_bfloat16*)dxp, slot_row, extra_row, dl,
-                                         (const __nv_bfloat16*)wg, T, d, E, k, (__nv_bfloat16*)dx);
+    if (E <= 8) rc = dx_fused_k<8>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
+    else if (E <= 16) rc = dx_fused_k<16>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
+    else rc = dx_fused_k<32>(blocks, smem, s, dxp, slot_row, extra_row, dl, wg, T, d, E, k, dx);
   }
+  if (rc) return rc;
   MOE_CHECK_LAUNCH("dx_fused");
   return MOE_OK;
 }

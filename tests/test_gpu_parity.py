@@ -349,3 +349,19 @@ def test_layer_noisy_routing(round_mode, gate_mode):
     noisy32 = (torch.from_numpy(lg) + eps).numpy()          # the scores the GPU routed on
     fwd, bwd = oracle_layer(inp, cfg.k, round_mode, noisy32, gate_mode=gate_mode)
     compare_layer(g, fwd, bwd, BF16_TOL)
+
+
+@pytest.mark.parametrize("d,E,k,round_mode", [(384, 32, 4, 1), (128, 16, 2, 1), (640, 24, 8, 0),
+                                              (896, 8, 3, 1)])
+def test_layer_bf16_fused_dx_shapes(d, E, k, round_mode):
+    """Shapes of the fused dx pass (E <= 32) whose row width is not a multiple
+    of 32 vectors, with rows added by rounding, and k of every size class."""
+    cfg = _cfg(700, d, 128, E, k, std=0.05)
+    inp = synth.make_inputs(cfg, seed=d + E, device="cuda")
+    bias = torch.linspace(1.0, -1.0, E)                 # uneven load: rounding adds rows
+    lg = fp32_router_logits(inp["x"], inp["w_gate"], bias)
+    g = gpu_layer(inp, cfg.k, round_mode, lg)
+    fwd, bwd = oracle_layer(inp, cfg.k, round_mode, lg)
+    if round_mode:
+        assert fwd["plan"]["added"].any()
+    compare_layer(g, fwd, bwd, BF16_TOL)
