@@ -55,7 +55,9 @@ Readings taken where the pages are silent (each also listed in the design doc):
 
 parity pins: tests/test_oracle_pins.py (brute force, dense masked evaluation,
 closed-form 2-expert example, central finite differences, the 145 -> 128
-rounding example, invariants).  No function here is unpinned.
+rounding example, invariants; MXFP8 against torch's float8_e4m3fn conversion,
+the 256-code table, closed-form scales and saturation).  No function here is
+unpinned.
 """
 from __future__ import annotations
 
@@ -291,13 +293,112 @@ def row_expert(plan, rows):
 
 
 # --------------------------------------------------------------------------
+# MXFP8: the OCP Microscaling (MX) v1.0 format with E4M3 elements -- blocks of
+# 32 consecutive elements share one power-of-two scale X = 2^e (an E8M0 code
+# e + 127).  The pages name the format (Olmo-core 3 news piece: "MXFP8
+# low-precision switch"; SonicMoE summary, future work) without defining it;
+# this is the public definition.  Blocks run along the contraction dimension
+# of each GEMM, the only direction in which the scales factor out of a dot
+# product.
+# --------------------------------------------------------------------------
+MX_BLOCK = 32
+E4M3_MAX = 448.0       # 1.75 * 2^8, the largest finite E4M3 value
+E4M3_EMAX = 8          # exponent of that value
+E4M3_EMIN = -6         # exponent of the smallest normal value
+
+
+def e4m3_round(v):
+    """Nearest E4M3 value (ties to the even mantissa), saturated to +-448.
+
+    A value of binade 2^e (e >= -6) is rounded on the grid 2^(e-3) (three
+    mantissa bits); below 2^-6 the grid is the subnormal step 2^-9."""
+    v = np.asarray(v, np.float64)
+    a = np.abs(v)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))       # a = m 2^ex, m in [0.5, 1)
+    e = np.maximum(ex - 1, E4M3_EMIN)
+    step = np.ldexp(1.0, e - 3)
+    q = np.minimum(np.round(a / step) * step, E4M3_MAX)   # np.round: half to even
+    return np.where(np.signbit(v), -q, q)
+
+
+def e4m3_encode(q):
+    """uint8 codes of values already on the E4M3 grid (sign, 4-bit exponent
+    with bias 7, 3-bit mantissa; -0 keeps its sign bit)."""
+    q = np.asarray(q, np.float64)
+    a = np.abs(q)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    e = ex - 1
+    normal = (a > 0) & (e >= E4M3_EMIN)
+    exp_field = np.where(normal, e + 7, 0)
+    mant = np.where(normal, a / np.ldexp(1.0, e) - 1.0, a / 2.0 ** -9) * np.where(normal, 8, 1)
+    code = (exp_field.astype(np.int64) << 3) | np.rint(mant).astype(np.int64)
+    return (code | (np.signbit(q).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def e4m3_decode(code):
+    """Values of uint8 E4M3 codes (0x7F and 0xFF are NaN)."""
+    c = np.asarray(code, np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    ef, mf = (c >> 3) & 0xF, c & 7
+    val = np.where(ef == 0, mf * 2.0 ** -9, (1.0 + mf / 8.0) * np.ldexp(1.0, ef - 7))
+    return np.where((c & 0x7F) == 0x7F, np.nan, sign * val)
+
+
+def mx_shared_exp(amax):
+    """Shared exponent of a block: floor(log2 amax) - 8 (so that the block's
+    largest element lands in [256, 512) before rounding), clamped to the E8M0
+    range [-127, 127]; -127 for an all-zero block."""
+    amax = np.asarray(amax, np.float64)
+    _, ex = np.frexp(np.where(amax > 0, amax, 1.0))
+    return np.where(amax > 0, np.clip(ex - 1 - E4M3_EMAX, -127, 127), -127).astype(np.int64)
+
+
+def mx_quantize(a, axis):
+    """MXFP8 quantisation of ``a`` in blocks of 32 along ``axis``.
+
+    Returns (q, se): q the E4M3 element values (on the E4M3 grid, shape of
+    ``a``) and se the shared exponents (one per block, the block axis in place
+    of ``axis``); the represented value is q * 2^se."""
+    a = np.moveaxis(np.asarray(a, np.float64), axis, -1)
+    n = a.shape[-1]
+    assert n % MX_BLOCK == 0
+    blk = a.reshape(a.shape[:-1] + (n // MX_BLOCK, MX_BLOCK))
+    se = mx_shared_exp(np.abs(blk).max(axis=-1))
+    q = e4m3_round(blk / np.ldexp(1.0, se)[..., None])
+    return (np.moveaxis(q.reshape(a.shape), -1, axis), np.moveaxis(se, -1, axis))
+
+
+def mx_dequantize(q, se, axis):
+    q = np.moveaxis(np.asarray(q, np.float64), axis, -1)
+    se = np.moveaxis(np.asarray(se), axis, -1)
+    x = q * np.repeat(np.ldexp(1.0, se), MX_BLOCK, axis=-1)
+    return np.moveaxis(x, -1, axis)
+
+
+def mx_fake_quant(a, axis):
+    """The values MXFP8 represents for ``a`` (blocks of 32 along ``axis``)."""
+    return mx_dequantize(*mx_quantize(a, axis), axis)
+
+
+# --------------------------------------------------------------------------
 # expert SwiGLU FFN on the rows of one expert
 # --------------------------------------------------------------------------
 
-def expert_rows_forward(xr, w1e, w3e, w2e, staged):
+def expert_rows_forward(xr, w1e, w3e, w2e, staged, precision="bf16"):
     """H = [x W1 | x W3] (bf16-staged if ``staged``), A = silu(h1) * h3,
-    Y = A W2, for the rows ``xr`` [n,d] routed to one expert."""
+    Y = A W2, for the rows ``xr`` [n,d] routed to one expert.
+
+    precision "mxfp8": both GEMMs take MXFP8 operands -- x and W1/W3 in blocks
+    along d, A (after its bf16 staging) and W2 in blocks along f -- with exact
+    products and sums of the represented values."""
     xr = np.asarray(xr, np.float64)
+    if precision == "mxfp8":
+        xq = mx_fake_quant(xr, 1)
+        h1 = _stage(xq @ mx_fake_quant(w1e, 0), staged)
+        h3 = _stage(xq @ mx_fake_quant(w3e, 0), staged)
+        a = _stage(silu(h1) * h3, staged)
+        y = _stage(mx_fake_quant(a, 1) @ mx_fake_quant(w2e, 0), staged)
+        return h1, h3, a, y
     h1 = _stage(xr @ w1e, staged)
     h3 = _stage(xr @ w3e, staged)
     a = _stage(silu(h1) * h3, staged)
@@ -333,8 +434,12 @@ def _f64(a):
     return np.asarray(a, dtype=np.float64)
 
 
-def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
+def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True, precision="bf16"):
     """Forward (and, given dout, backward) quantities of the listed rows.
+
+    With precision "mxfp8" the forward GEMMs take MXFP8 operands; the backward
+    uses that forward's H and the unquantised x and weights (the quantisers
+    pass gradients straight through).
 
     Rows are grouped by the expert that owns them; padding rows give zeros.
     w1, w3, w2 may be arrays or any object whose [e] gives expert e's matrix
@@ -356,7 +461,7 @@ def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True):
         sel = np.nonzero((es == e) & (toks_all >= 0))[0]
         toks = toks_all[sel]
         w1e, w3e, w2e = _f64(w1[e]), _f64(w3[e]), _f64(w2[e])
-        h1, h3, a, y = expert_rows_forward(x[toks], w1e, w3e, w2e, staged)
+        h1, h3, a, y = expert_rows_forward(x[toks], w1e, w3e, w2e, staged, precision)
         res["H"][sel, :f], res["H"][sel, f:], res["A"][sel], res["Y"][sel] = h1, h3, a, y
         if dout is not None:
             g = plan["row_gate"][rows[sel]]
@@ -411,19 +516,20 @@ def make_plan(idx, gate, logits, E, tile=TILE, round_mode=0, gate_mode=0, capaci
 
 def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
               logits_override=None, logit_bias=None, staged=True, gate_mode=0, capacity=None,
-              logit_noise=None):
-    """Full forward: route, permute, expert FFN on every row, combine."""
+              logit_noise=None, precision="bf16"):
+    """Full forward: route, permute, expert FFN on every row, combine.
+    precision "mxfp8": the expert GEMMs take MXFP8 operands (expert_rows_forward)."""
     logits, idx, gate = route(x, w_gate, k, logits_override, logit_bias, gate_mode, logit_noise)
     T, E = logits.shape
     plan = make_plan(idx, gate, logits, E, tile, round_mode, gate_mode, capacity)
     rows = np.arange(plan["R"])
-    res = rows_compute(rows, plan, x, w1, w3, w2, None, staged)
+    res = rows_compute(rows, plan, x, w1, w3, w2, None, staged, precision)
     out = np.zeros((T, np.shape(x)[1]))
     for t in range(T):
         for r in token_rows(plan, t):
             out[t] += plan["row_gate"][r] * res["Y"][r]
     return dict(logits=logits, idx=idx, gate=gate, plan=plan, H=res["H"],
-                A=res["A"], Y=res["Y"], out=out)
+                A=res["A"], Y=res["Y"], out=out, precision=precision)
 
 
 def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True,
@@ -440,7 +546,7 @@ def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True
     E, _, f = w1.shape
     R = plan["R"]
     rows = np.arange(R)
-    res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged)
+    res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged, fwd.get("precision", "bf16"))
     dw1, dw3, dw2 = np.zeros_like(w1), np.zeros_like(w3), np.zeros_like(w2)
     for e in range(E):
         lo, hi = plan["offsets"][e], plan["offsets"][e + 1]
@@ -476,7 +582,7 @@ def sampled_tokens(tokens, dout, x, w_gate, w1, w3, w2, fwd, staged=True, router
     dout, x, w_gate = _f64(dout), _f64(x), _f64(w_gate)
     per_tok = [token_rows(plan, t) for t in tokens]
     all_rows = [r for tr in per_tok for r in tr]
-    res = rows_compute(all_rows, plan, x, w1, w3, w2, dout, staged)
+    res = rows_compute(all_rows, plan, x, w1, w3, w2, dout, staged, fwd.get("precision", "bf16"))
     out, dx, dl, dS = {}, {}, {}, {}
     pos = 0
     for t, tr in zip(tokens, per_tok):
@@ -504,7 +610,7 @@ def sampled_expert_grads(experts, dout, x, w1, w3, w2, fwd, staged=True):
         toks = plan["row_token"][lo:hi]
         live = toks >= 0
         rows = np.arange(lo, hi)[live]
-        res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged)
+        res = rows_compute(rows, plan, x, w1, w3, w2, dout, staged, fwd.get("precision", "bf16"))
         tk = toks[live]
         out[e] = dict(dw2=res["gA"].T @ dout[tk], dw1=x[tk].T @ res["dH"][:, :f],
                       dw3=x[tk].T @ res["dH"][:, f:])
@@ -529,8 +635,14 @@ def expert_grad_slices(e, cols, dout, x, w1e, w3e, w2e, fwd, staged=True):
     g = plan["row_gate"][lo:hi][live]
     xr, dor = x[tk], dout[tk]
     w1c, w3c, w2r = _f64(w1e)[:, cols], _f64(w3e)[:, cols], _f64(w2e)[cols, :]
-    h1 = _stage(xr @ w1c, staged)
-    h3 = _stage(xr @ w3c, staged)
+    if fwd.get("precision", "bf16") == "mxfp8":
+        # H from MXFP8 operands (blocks along d: columns quantise independently)
+        xq = mx_fake_quant(xr, 1)
+        h1 = _stage(xq @ mx_fake_quant(w1c, 0), staged)
+        h3 = _stage(xq @ mx_fake_quant(w3c, 0), staged)
+    else:
+        h1 = _stage(xr @ w1c, staged)
+        h3 = _stage(xr @ w3c, staged)
     a = _stage(silu(h1) * h3, staged)
     dap = dor @ w2r.T
     da = g[:, None] * dap

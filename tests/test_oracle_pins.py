@@ -586,3 +586,111 @@ def test_noisy_routing_special_cases():
         rest = [e for e in np.argsort(-clean[t], kind="stable") if e != 4][:k - 1]
         assert list(idx[t, 1:]) == rest
     np.testing.assert_allclose(lg, clean + eps, rtol=1e-15)
+
+
+# ---------------------------------------------------------------- MXFP8 (OCP MX, E4M3 elements)
+
+def _e4m3_torch(v):
+    t = torch.from_numpy(np.asarray(v, np.float32))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_round_matches_torch_below_overflow():
+    """Round-to-nearest-even on the E4M3 grid, against torch's float8_e4m3fn
+    conversion, for normal, subnormal and exact-midpoint inputs (|v| < 464,
+    where rounding never overflows)."""
+    rng = np.random.default_rng(30)
+    mant = rng.uniform(1.0, 2.0, 4000)
+    ex = rng.integers(-12, 9, 4000)
+    v = (mant * np.ldexp(1.0, ex)).astype(np.float32).astype(np.float64)
+    v *= np.where(rng.random(4000) < 0.5, -1.0, 1.0)
+    grid = np.unique(np.abs(O.e4m3_decode(np.arange(0, 0x7F))))
+    mids = (grid[1:] + grid[:-1]) / 2                    # exact ties
+    v = np.concatenate([v, mids, -mids])
+    v = v[np.abs(v) < 464]
+    np.testing.assert_array_equal(O.e4m3_round(v), _e4m3_torch(v))
+
+
+def test_e4m3_code_table():
+    """All 256 codes: decode agrees with torch's float8_e4m3fn bit pattern,
+    encode inverts decode, and the extremes are the format's."""
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    dec = O.e4m3_decode(codes)
+    np.testing.assert_array_equal(np.isnan(dec), np.isnan(ref))
+    ok = ~np.isnan(dec)
+    np.testing.assert_array_equal(dec[ok], ref[ok])
+    np.testing.assert_array_equal(O.e4m3_encode(dec[ok]), codes[ok])
+    assert O.e4m3_decode(0x7E) == 448 and O.e4m3_decode(0x08) == 2.0 ** -6
+    assert O.e4m3_decode(0x01) == 2.0 ** -9 and O.e4m3_decode(0x80) == 0 and np.signbit(O.e4m3_decode(0x80))
+
+
+def test_e4m3_saturates_to_448():
+    v = np.array([448, 463.99, 464, 465, 479.9, 480, 512, 1e6, 3e38])
+    np.testing.assert_array_equal(O.e4m3_round(v), np.minimum(_e4m3_torch(np.minimum(v, 448)), 448))
+    np.testing.assert_array_equal(O.e4m3_round(v), np.full(v.shape, 448.0))
+    np.testing.assert_array_equal(O.e4m3_round(-v), np.full(v.shape, -448.0))
+
+
+def test_mx_shared_exponent_closed_form():
+    """2^se is the largest power of two with amax / 2^se >= 256 (so the block
+    maximum scales into [256, 512)); all-zero blocks and tiny maxima take the
+    E8M0 floor -127, huge maxima its ceiling 127."""
+    rng = np.random.default_rng(31)
+    amax = np.exp(rng.uniform(-60, 60, 2000))
+    se = O.mx_shared_exp(amax)
+    r = amax / np.ldexp(1.0, se)
+    assert np.all((r >= 256) & (r < 512))
+    assert np.all(se == np.floor(np.log2(amax / 256.0)))
+    np.testing.assert_array_equal(O.mx_shared_exp(np.array([0.0, 2.0 ** -140, 2.0 ** 140])),
+                                  [-127, -127, 127])
+    np.testing.assert_array_equal(O.mx_shared_exp(np.array([1.0, 256.0, 511.999, 512.0])),
+                                  [-8, 0, 0, 1])
+
+
+def test_mx_quantize_error_bound_and_idempotence():
+    """Each element is the E4M3 rounding of v / 2^se: error <= 2^-4 |v| in the
+    normal range, <= 2^(se-10) in the subnormal range, and only elements
+    that scale to >= 464 saturate.  Blocks run along the requested axis."""
+    rng = np.random.default_rng(32)
+    a = rng.standard_normal((6, 96)) * np.exp(rng.uniform(-8, 8, (6, 1)))
+    a[2, 32:64] = 0.0                                     # an all-zero block
+    a[3, :5] *= 1e-6                                      # subnormal-range elements
+    for axis, arr in ((1, a), (0, a.T.copy())):
+        q, se = O.mx_quantize(arr, axis)
+        assert se.shape == ((6, 3) if axis == 1 else (3, 6))
+        deq = O.mx_dequantize(q, se, axis)
+        scale = np.repeat(np.ldexp(1.0, se), 32, axis=axis)
+        s = arr / scale
+        err = np.abs(deq - arr) / scale
+        sat = np.abs(s) >= 464
+        assert np.all(err[~sat] <= np.maximum(np.abs(s[~sat]) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-12))
+        assert np.all(np.abs(q[sat]) == 448)
+        np.testing.assert_array_equal(O.mx_fake_quant(deq, axis), deq)   # idempotent
+    q, se = O.mx_quantize(a, 1)
+    assert se[2, 1] == -127 and np.all(q[2, 32:64] == 0)
+
+
+def test_mxfp8_layer_equals_bf16_layer_on_the_mx_grid():
+    """With x, W1, W3 already on the MXFP8 grid the quantised up-projection is
+    exact, so H equals the unquantised layer's; Y then uses the MXFP8 image of
+    A and W2; the backward reads the MXFP8 forward's H."""
+    rng = np.random.default_rng(33)
+    T, d, f, E, k = 24, 64, 64, 4, 2
+    x, wg, w1, w3, w2, dout = _rand_layer(rng, T, d, f, E)
+    x, w1, w3 = O.mx_fake_quant(x, 1), O.mx_fake_quant(w1, 1), O.mx_fake_quant(w3, 1)
+    a = O.layer_fwd(x, wg, w1, w3, w2, k, tile=4, staged=False)
+    b = O.layer_fwd(x, wg, w1, w3, w2, k, tile=4, staged=False, precision="mxfp8")
+    np.testing.assert_array_equal(a["H"], b["H"])
+    R = b["plan"]["R"]
+    for r in range(R):
+        e, t = O.row_expert(b["plan"], [r])[0], b["plan"]["row_token"][r]
+        if t < 0:
+            continue
+        want = O.mx_fake_quant(a["A"][r:r + 1], 1) @ O.mx_fake_quant(w2[e], 0)
+        np.testing.assert_allclose(b["Y"][r], want[0], rtol=1e-13, atol=1e-15)
+    assert np.abs(b["Y"] - a["Y"]).max() > 0             # A and W2 are not on the grid
+    ga = O.layer_bwd(dout, x, wg, w1, w3, w2, a, staged=False)
+    gb = O.layer_bwd(dout, x, wg, w1, w3, w2, b, staged=False)
+    for n in ("dx", "dw1", "dw3", "dw2", "dS", "dlogits"):   # same H, same STE backward
+        np.testing.assert_allclose(gb[n], ga[n], rtol=1e-12, atol=1e-12)
