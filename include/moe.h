@@ -192,6 +192,49 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
                        void* H, void* Y_perm, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * MXFP8 expert FFN forward (the "MXFP8 low-precision switch" of the Olmo-core
+ * 3 news piece; FP8/MXFP8 support is the SonicMoE summary's future work).
+ * Format: OCP Microscaling (MX) v1.0 with E4M3 elements -- blocks of 32
+ * consecutive elements along each GEMM's contraction dimension share one E8M0
+ * scale 2^(code-127); shared exponent floor(log2 max|v|) - 8 (clamped to
+ * [-127, 127]), elements rounded to nearest-even and saturated to +-448.
+ * Scale arrays are 512-byte blocks [rows/128][K/128]; the scale of row r and
+ * 32-element K-block j is byte (r%32)*16 + ((r/32)%4)*4 + (j%4) of its block.
+ * The GEMMs run on the tcgen05 block-scaled tensor cores (kind::mxf8f6f4)
+ * with fp32 accumulation; H and Y are bf16 as in moe_expert_ffn_fwd, and
+ * moe_layer_bwd (bf16 weights, saved H) is the backward: the quantisers pass
+ * gradients straight through.
+ *
+ * moe_mxfp8_weight_sizes: sizes[4] out = bytes of W13q, W13s, W2q, W2s for
+ *   E experts (d and f multiples of 128, else MOE_ERR_UNSUPPORTED).
+ * moe_mxfp8_quantize_weights: w1, w3 [E,d,f] and w2 [E,f,d] bf16 ->
+ *   W13q [E, 2f, d] E4M3 (K = d contiguous; rows 128t..128t+63 are columns
+ *   64t..64t+63 of W1 and rows 128t+64..128t+127 the same columns of W3),
+ *   W13s its scales, W2q [E, d, f] E4M3 (K = f contiguous), W2s its scales.
+ *   Run it once per weight update; caller-owned device buffers of the sizes
+ *   above, 16-byte aligned.
+ * moe_expert_ffn_fwd_mxfp8: as moe_expert_ffn_fwd (bf16 x, same plan
+ *   arguments, H [cap,2f] and Y_perm [cap,d] bf16 out) with the quantised
+ *   weights; x rows are quantised while they are scattered and A in the
+ *   up-projection's epilogue.  ws: at least
+ *   moe_ffn_fwd_mxfp8_workspace_size() bytes; after the call it holds, each
+ *   piece starting at the next multiple of 256 bytes: Xq [capr, d] E4M3, its
+ *   scales, Aq [capr, f] E4M3, its scales (capr = cap rounded up to 128).
+ *   Needs an sm_100 device.
+ */
+int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes);
+int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
+                               int f, uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                               void* stream);
+size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
+int moe_expert_ffn_fwd_mxfp8(const void* x, const uint8_t* w13q, const uint8_t* w13s,
+                             const uint8_t* w2q, const uint8_t* w2s,
+                             const int32_t* row_token, const int32_t* offsets,
+                             const int32_t* slot_row, const int32_t* extra_row,
+                             int T, int d, int f, int E, int k,
+                             void* H, void* Y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_combine -- routing-weighted unpermute: O_t = sum over token t's rows of
  * row_gate[row] * Y_perm[row], summed in fp32 in a fixed order (kept slots in
  * slot order, then rows added by rounding in ascending expert id).

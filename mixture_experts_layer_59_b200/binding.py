@@ -27,6 +27,8 @@ EXPORTS = [
     "moe_expert_ffn_fwd", "moe_combine", "moe_layer_bwd_workspace_size", "moe_layer_bwd",
     "moe_check_status", "moe_profile_enable", "moe_profile_report", "moe_permute_noalloc",
     "moe_balance_loss_workspace_size", "moe_balance_loss",
+    "moe_mxfp8_weight_sizes", "moe_mxfp8_quantize_weights", "moe_ffn_fwd_mxfp8_workspace_size",
+    "moe_expert_ffn_fwd_mxfp8",
 ]
 
 _lib = None
@@ -56,6 +58,10 @@ _SIGS = {
     "moe_layer_bwd": (_i, [_vp] * 10 + [_i] + [_vp] * 6 + [_i] * 7 + [_vp] * 7 + [_vp, _sz, _vp]),
     "moe_balance_loss_workspace_size": (_sz, [_i, _i, _i]),
     "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_mxfp8_weight_sizes": (_i, [_i, _i, _i, ctypes.POINTER(_sz)]),
+    "moe_mxfp8_quantize_weights": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_ffn_fwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_expert_ffn_fwd_mxfp8": (_i, [_vp] * 9 + [_i] * 5 + [_vp, _vp, _vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
     "moe_profile_enable": (_i, [_i]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -190,6 +196,45 @@ def moe_expert_ffn_fwd(x, w1, w3, w2, plan, k, H=None, Y_perm=None, ws=None, str
                                     _p(plan["offsets"]), _p(plan["slot_row"]),
                                     _p(plan.get("extra_row")), T, d, f, E, k, dt, _p(H),
                                     _p(Y_perm), _p(ws), ws.numel(), _stream(stream)))
+    return H, Y_perm
+
+
+def moe_mxfp8_weight_sizes(E, d, f):
+    """Bytes of (W13q, W13s, W2q, W2s)."""
+    sz = (_sz * 4)()
+    _check(lib().moe_mxfp8_weight_sizes(E, d, f, sz))
+    return tuple(int(v) for v in sz)
+
+
+def moe_mxfp8_quantize_weights(w1, w3, w2, out=None, stream=None):
+    """MXFP8 copies of the expert weights: dict w13q, w13s, w2q, w2s (uint8)."""
+    E, d, f = w1.shape
+    o = dict(out) if out else {}
+    for name, n in zip(("w13q", "w13s", "w2q", "w2s"), moe_mxfp8_weight_sizes(E, d, f)):
+        o.setdefault(name, torch.empty(n, device=w1.device, dtype=torch.uint8))
+    _check(lib().moe_mxfp8_quantize_weights(_p(w1), _p(w3), _p(w2), E, d, f, _p(o["w13q"]),
+                                            _p(o["w13s"]), _p(o["w2q"]), _p(o["w2s"]),
+                                            _stream(stream)))
+    return o
+
+
+def moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k) -> int:
+    return lib().moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k)
+
+
+def moe_expert_ffn_fwd_mxfp8(x, wq, plan, k, E, f, H=None, Y_perm=None, ws=None, stream=None):
+    """MXFP8 forward of the expert FFN.  wq: dict from moe_mxfp8_quantize_weights."""
+    T, d = x.shape
+    cap = moe_row_capacity(T, E, k)
+    H = H if H is not None else torch.empty(cap, 2 * f, device=x.device, dtype=x.dtype)
+    Y_perm = Y_perm if Y_perm is not None else torch.empty(cap, d, device=x.device, dtype=x.dtype)
+    if ws is None:
+        ws = torch.empty(max(moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k), 1), device=x.device,
+                         dtype=torch.uint8)
+    _check(lib().moe_expert_ffn_fwd_mxfp8(
+        _p(x), _p(wq["w13q"]), _p(wq["w13s"]), _p(wq["w2q"]), _p(wq["w2s"]), _p(plan["row_token"]),
+        _p(plan["offsets"]), _p(plan["slot_row"]), _p(plan.get("extra_row")), T, d, f, E, k,
+        _p(H), _p(Y_perm), _p(ws), ws.numel(), _stream(stream)))
     return H, Y_perm
 
 

@@ -130,6 +130,19 @@ struct FwdWs {
 };
 
 template <class A>
+struct FwdMxWs {
+  uint8_t *xq = nullptr, *xs = nullptr, *actq = nullptr, *acts = nullptr;
+  void carve(A& a, int T, int d, int f, int E, int k) {
+    const size_t cap = (size_t)T * k + (size_t)E * 128;
+    const size_t capr = (cap + 127) / 128 * 128;   // scale blocks cover 128 rows
+    xq = a.template take<uint8_t>(capr * d);
+    xs = a.template take<uint8_t>(capr * d / 32);
+    actq = a.template take<uint8_t>(capr * f);
+    acts = a.template take<uint8_t>(capr * f / 32);
+  }
+};
+
+template <class A>
 struct BwdWs {
   void *dog = nullptr, *xg = nullptr, *dH = nullptr, *gact = nullptr, *dxp = nullptr;
   float *dap = nullptr, *ds = nullptr, *dl = nullptr, *dx_acc = nullptr, *dwg_part = nullptr;
@@ -289,6 +302,68 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
     return tc_ffn_fwd(p, w.xg, H, w.act, Y_perm, device_sm_count(), s);
   }
   return simt_ffn_fwd(p, H, w.act, Y_perm, s);
+}
+
+int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes) {
+  REQUIRE_PTR(sizes);
+  if (E < 0 || d <= 0 || f <= 0 || d % 128 || f % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "MXFP8 needs d and f positive multiples of 128");
+  const size_t n = (size_t)E * d * f;
+  sizes[0] = 2 * n;        // W13q
+  sizes[1] = 2 * n / 32;   // W13s
+  sizes[2] = n;            // W2q
+  sizes[3] = n / 32;       // W2s
+  return MOE_OK;
+}
+
+int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
+                               int f, uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                               void* stream) {
+  size_t sz[4];
+  if (int rc = moe_mxfp8_weight_sizes(E, d, f, sz)) return rc;
+  if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
+  REQUIRE_PTR(w13q); REQUIRE_PTR(w13s); REQUIRE_PTR(w2q); REQUIRE_PTR(w2s);
+  REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2);
+  REQUIRE_ALIGNED(w13q); REQUIRE_ALIGNED(w13s); REQUIRE_ALIGNED(w2q); REQUIRE_ALIGNED(w2s);
+  return launch_mx_quant_weights(w1, w3, w2, E, d, f, w13q, w13s, w2q, w2s, (cudaStream_t)stream);
+}
+
+size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k) {
+  if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0) return 0;
+  Sizer z;
+  FwdMxWs<Sizer> w;
+  w.carve(z, T, d, f, E, k);
+  return z.used;
+}
+
+int moe_expert_ffn_fwd_mxfp8(const void* x, const uint8_t* w13q, const uint8_t* w13s,
+                             const uint8_t* w2q, const uint8_t* w2s, const int32_t* row_token,
+                             const int32_t* offsets, const int32_t* slot_row,
+                             const int32_t* extra_row, int T, int d, int f, int E, int k, void* H,
+                             void* Y_perm, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_common(T, E, k, MOE_BF16)) return rc;
+  if (int rc = check_dims(d, f, MOE_BF16)) return rc;
+  if (!tc_available()) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 GEMMs need an sm_100 device");
+  REQUIRE_PTR(x); REQUIRE_PTR(w13q); REQUIRE_PTR(w13s); REQUIRE_PTR(w2q); REQUIRE_PTR(w2s);
+  REQUIRE_PTR(row_token); REQUIRE_PTR(offsets); REQUIRE_PTR(H); REQUIRE_PTR(Y_perm);
+  if (T > 0) REQUIRE_PTR(slot_row);
+  REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w13q); REQUIRE_ALIGNED(w13s); REQUIRE_ALIGNED(w2q);
+  REQUIRE_ALIGNED(w2s); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(Y_perm); REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k))
+    return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_ffn_fwd_mxfp8_workspace_size()");
+  Carve c(ws, ws_bytes);
+  FwdMxWs<Carve> w;
+  w.carve(c, T, d, f, E, k);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "mxfp8 workspace too small");
+  cudaStream_t s = (cudaStream_t)stream;
+  FfnPtrs p{x, nullptr, nullptr, nullptr, row_token, offsets, T, d, f, E,
+            (int)((size_t)T * k + (size_t)E * 128), MOE_BF16};
+  if (int rc = launch_mx_scatter_rows(x, slot_row, extra_row, row_token, offsets, T, d, E, k,
+                                      w.xq, w.xs, s))
+    return rc;
+  return tc_ffn_fwd_mx(p, w.xq, w.xs, w13q, w13s, w2q, w2s, H, w.actq, w.acts, Y_perm,
+                       device_sm_count(), s);
 }
 
 int moe_combine(const void* Y_perm, const float* row_gate, const int32_t* slot_row,

@@ -84,6 +84,9 @@ int simt_router_bwd_gemms(const void* x, const void* wg, const float* dl, const 
 bool tc_available();
 int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, int num_sms,
                cudaStream_t s);
+int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const uint8_t* w13q,
+                  const uint8_t* w13s, const uint8_t* w2q, const uint8_t* w2s, void* H,
+                  uint8_t* actq, uint8_t* acts, void* Y, int num_sms, cudaStream_t s);
 int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* row_gate,
                const void* H, void* dH, void* gact, float* ds_part, void* dXp, void* dw1,
                void* dw3, void* dw2, int num_sms, cudaStream_t s);
@@ -98,5 +101,13 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
                   void* dx, int num_sms, cudaStream_t s);
 
 int device_sm_count();
+
+// ---------------------------------------------------------------- MXFP8 (mx.cu, tc_gemm.cu)
+int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int E, int d, int f,
+                            uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                            cudaStream_t s);
+int launch_mx_scatter_rows(const void* x, const int32_t* slot_row, const int32_t* extra_row,
+                           const int32_t* row_token, const int32_t* offsets, int T, int d, int E,
+                           int k, uint8_t* q, uint8_t* sf, cudaStream_t s);
 
 }  // namespace moe

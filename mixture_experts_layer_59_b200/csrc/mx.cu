@@ -1,0 +1,160 @@
+// MXFP8 operand preparation for the block-scaled expert GEMMs (format and
+// scale layout: mx.cuh).
+//   weights  W1, W3 [E, d, f] -> W13q [E, 2f, d] (K = d contiguous; rows of
+//            128-row tile t: 64 columns t*64.. of W1, then the same of W3, so
+//            one tile yields matching H1 / H3 columns) and W2 [E, f, d] ->
+//            W2q [E, d, f] (K = f contiguous), blocks of 32 along K.
+//   rows     x [T, d] -> Xq [cap, d]: each token row quantised once (blocks
+//            of 32 along d) and written to all of its rows in the row space;
+//            padding rows get zero elements and zero scales.
+#include "common.cuh"
+#include "internal.h"
+#include "mx.cuh"
+
+namespace moe {
+
+// ============================================================== weights
+// One block per (128 K, 128 output rows, expert): the bf16 source tile goes
+// to shared memory as [k][n], then thread (n, j) quantises column n over the
+// 32 K-values 32j..32j+31 and writes 32 contiguous bytes of output row n.
+constexpr int WQ_THREADS = 512;
+
+template <bool W13>
+__global__ void __launch_bounds__(WQ_THREADS)
+k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __restrict__ wb,
+                   int K, int N, int Nout, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  __shared__ __align__(16) __nv_bfloat16 tile[128][128];
+  const int k0 = blockIdx.x * 128, t = blockIdx.y, e = blockIdx.z;
+  const int kchunks = K / 128;
+  // source tile: 128 K-rows x 128 output rows (16-byte vectors of 8 bf16)
+  for (int v = threadIdx.x; v < 128 * 16; v += WQ_THREADS) {
+    const int kk = v >> 4, c8 = (v & 15) * 8;
+    const __nv_bfloat16* src;
+    if (W13) {  // output rows 0..63 from W1 columns t*64.., 64..127 from W3
+      src = (c8 < 64 ? wa : wb) + ((size_t)e * K + k0 + kk) * N + t * 64 + (c8 & 63);
+    } else {
+      src = wa + ((size_t)e * K + k0 + kk) * N + t * 128 + c8;
+    }
+    *reinterpret_cast<uint4*>(&tile[kk][c8]) = __ldg(reinterpret_cast<const uint4*>(src));
+  }
+  __syncthreads();
+  const int n = threadIdx.x & 127, j = threadIdx.x >> 7;
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[32 * j + i][n]);
+  const int row = e * Nout + t * 128 + n;   // output row across experts (Nout % 128 == 0)
+  mx_store_block(v, q + (size_t)row * K + k0 + 32 * j,
+                 sf + mx_sf_offset(row, (k0 >> 5) + j, kchunks));
+}
+
+int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int E, int d, int f,
+                            uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                            cudaStream_t s) {
+  if (E == 0) return MOE_OK;
+  {
+    ProfScope _ps("mx_quant_weights", s);
+    k_mx_quant_weights<true><<<dim3(d / 128, (2 * f) / 128, E), WQ_THREADS, 0, s>>>(
+        (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w3, d, f, 2 * f, w13q, w13s);
+    k_mx_quant_weights<false><<<dim3(f / 128, d / 128, E), WQ_THREADS, 0, s>>>(
+        (const __nv_bfloat16*)w2, nullptr, f, d, d, w2q, w2s);
+  }
+  MOE_CHECK_LAUNCH("mx_quant_weights");
+  return MOE_OK;
+}
+
+// ============================================================== rows
+// Blocks [0, nbt) own tokens (one warp per token): lanes 4g..4g+3 hold the 32
+// elements of one block as four 16-byte vectors, share its maximum by
+// shuffles, and write 8 E4M3 bytes each to every row of the token; the first
+// lane of the group writes the scale.  The remaining blocks zero the padding
+// rows (elements and scales).
+__global__ void __launch_bounds__(256)
+k_mx_scatter_rows(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_row,
+                  const int32_t* __restrict__ extra_row, const int32_t* __restrict__ row_token,
+                  const int32_t* __restrict__ offsets, int T_, int d, int E, int k, int nbt,
+                  uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  __shared__ int s_extra[8][256];   // rows added by rounding, per warp (E <= 256)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nvec = d / 8, kchunks = d / 128;
+  if ((int)blockIdx.x < nbt) {
+    const int t = blockIdx.x * 8 + w;
+    if (t >= T_) return;  // whole warp
+    const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    int rk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
+    int n_extra = 0;
+    if (extra_row != nullptr) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int re = e0 + lane < E ? extra_row[(size_t)t * E + e0 + lane] : -1;
+        const unsigned bal = __ballot_sync(0xffffffffu, re >= 0);
+        if (re >= 0) s_extra[w][n_extra + __popc(bal & ((1u << lane) - 1u))] = re;
+        n_extra += __popc(bal);
+      }
+      __syncwarp();
+    }
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    for (int i0 = 0; i0 < nvec; i0 += 32) {
+      const int i = i0 + lane;
+      const bool valid = i < nvec;
+      float b[8];
+      float amax = 0.f;
+      if (valid) {
+        const uint4 u = __ldg(src + i);
+        const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          b[e] = __bfloat162float(h[e]);
+          amax = fmaxf(amax, fabsf(b[e]));
+        }
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      if (!valid) continue;
+      const uint32_t code = mx_scale_code(amax);
+      const float inv = mx_inv_scale(code);
+      uint2 pk;
+      pk.x = cvt_e4m3x2(b[0] * inv, b[1] * inv) | (cvt_e4m3x2(b[2] * inv, b[3] * inv) << 16);
+      pk.y = cvt_e4m3x2(b[4] * inv, b[5] * inv) | (cvt_e4m3x2(b[6] * inv, b[7] * inv) << 16);
+      const bool first = (lane & 3) == 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int r = rk[j];
+        if (r >= 0) {
+          *reinterpret_cast<uint2*>(q + (size_t)r * d + 8 * i) = pk;
+          if (first) sf[mx_sf_offset(r, i >> 2, kchunks)] = (uint8_t)code;
+        }
+      }
+      for (int j = 0; j < n_extra; ++j) {
+        const int r = s_extra[w][j];
+        *reinterpret_cast<uint2*>(q + (size_t)r * d + 8 * i) = pk;
+        if (first) sf[mx_sf_offset(r, i >> 2, kchunks)] = (uint8_t)code;
+      }
+    }
+  } else {
+    const int R = offsets[E];
+    const int nb = gridDim.x - nbt;
+    for (int r = (blockIdx.x - nbt) * 8 + w; r < R; r += nb * 8) {
+      if (row_token[r] >= 0) continue;
+      uint4* d4 = reinterpret_cast<uint4*>(q + (size_t)r * d);
+      for (int i = lane; i < d / 16; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
+      for (int kb = lane; kb < d / 32; kb += 32) sf[mx_sf_offset(r, kb, kchunks)] = 0;
+    }
+  }
+}
+
+int launch_mx_scatter_rows(const void* x, const int32_t* slot_row, const int32_t* extra_row,
+                           const int32_t* row_token, const int32_t* offsets, int T, int d, int E,
+                           int k, uint8_t* q, uint8_t* sf, cudaStream_t s) {
+  const int nbt = (T + 7) / 8;
+  const int blocks = nbt + device_sm_count() * 2;
+  {
+    ProfScope _ps("mx_scatter_rows", s);
+    k_mx_scatter_rows<<<blocks, 256, 0, s>>>((const __nv_bfloat16*)x, slot_row, extra_row,
+                                             row_token, offsets, T, d, E, k, nbt, q, sf);
+  }
+  MOE_CHECK_LAUNCH("mx_scatter_rows");
+  return MOE_OK;
+}
+
+}  // namespace moe

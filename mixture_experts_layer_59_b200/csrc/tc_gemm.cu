@@ -20,6 +20,11 @@
 //                                    bf16 hi part plus a bf16 lo remainder,
 //                                    accumulated in the same fp32 accumulator
 //   DXR   dx = (fp32 sum of the token's dX_perm rows) + dlogits W_gate^T
+//   UPQ   UP with MXFP8 operands (E4M3, one E8M0 scale per 32 along K):
+//         Xq [W13q], epilogue as UP but A leaves as MXFP8 (blocks along f)
+//   DOWNQ DOWN with MXFP8 operands: Aq W2q
+//         (kind::mxf8f6f4 block-scaled MMAs, K = 32 per instruction; the two
+//         512-byte scale blocks of each stage go shared -> TMEM by tcgen05.cp)
 // The grouped GEMM replaces the per-expert loop of the Beam article's
 // MoELayer (sec. 5.3); Olmo-core 3 names grouped GEMM for the same purpose;
 // dS = <dA', A> without a stored Y is the SonicMoE summary's sec. 1.
@@ -40,6 +45,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mx.cuh"
 #include "tcgen05.cuh"
 
 namespace moe {
@@ -47,8 +53,12 @@ namespace moe {
 using namespace tc;
 
 enum Kind : int {
-  K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8
+  K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8,
+  K_UPQ = 9, K_DOWNQ = 10
 };
+constexpr int NUM_KINDS = 11;
+constexpr int MX_SF_BYTES = 1024;      // MXFP8 stage: 512-byte A and B scale blocks
+constexpr int MX_SF_COL = 256;         // TMEM columns of the scale blocks (after 2 x 128 accumulators)
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
@@ -91,6 +101,12 @@ struct TcArgs {
   float* gate;               // RT: [T, k]
   float* dwg_part;           // DWG: [splits, d, E]
   const float* dx_acc;       // DXR: [T, d] fp32 sums of each token's dX_perm rows
+  // MXFP8 kinds: 512-byte scale blocks [rows/128][K/128] of A and [E][N/128][K/128] of B
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  int kchunks;               // K / 128
+  uint8_t* act_q;            // UPQ: A as E4M3 [cap, f]
+  uint8_t* act_s;            // UPQ: its scale blocks [cap/128][f/128]
 };
 
 template <int KIND> struct KT {
@@ -99,15 +115,20 @@ template <int KIND> struct KT {
   static constexpr bool B_MN = (KIND == K_UP || KIND == K_DOWN || VARLEN_K || KIND == K_RT ||
                                 KIND == K_DWG);
   static constexpr bool ROUTER = (KIND == K_RT || KIND == K_DWG || KIND == K_DXR);
+  static constexpr bool MX = (KIND == K_UPQ || KIND == K_DOWNQ);
 };
 
-template <int BN> struct Cfg {
+// A stage holds a 128 x 128-byte A tile and a BN x 128-byte B tile (64 bf16
+// or 128 E4M3 elements of K), plus the scale blocks for the MXFP8 kinds.
+template <int BN, bool MX = false> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int STAGE = A_BYTES + B_BYTES + (MX ? MX_SF_BYTES : 0);
+  static constexpr int STAGES = MX ? 5 : ((BN == 256) ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int OUT_BYTES = 8 * 2 * 2048;  // two 32 x 32 bf16 staging tiles per epilogue warp
   static constexpr int SMEM = STAGES * STAGE + OUT_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
+  static_assert(!MX || BN == 128, "MXFP8 kinds use 128-column tiles");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 struct TileInfo {
@@ -165,7 +186,7 @@ __device__ __forceinline__ bool tile_info(int t, const TcArgs& a, const int* s_o
     }
     ti.e = lo;
     ti.krow0 = 0;
-    ti.kb_count = a.K / BK;
+    ti.kb_count = KT<KIND>::MX ? a.kchunks : a.K / BK;
   }
   return true;
 }
@@ -241,7 +262,7 @@ __device__ __forceinline__ void stage_store(uint8_t* tiles, int& which, const fl
 
 template <int KIND, int BN>
 __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ TcArgs a) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, KT<KIND>::MX>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[C::STAGES];
   __shared__ __align__(8) uint64_t empty_bar[C::STAGES];
@@ -345,6 +366,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
 #pragma unroll
             for (int h = 0; h < BN / 64; ++h)
               tma_load_2d(sB + h * ATOM, mb, &full_bar[stage], 64 * h, r);
+          } else if constexpr (KT<KIND>::MX) {
+            // E4M3 tiles: 128 elements of K = 128 bytes; then the A and B
+            // scale blocks of this K chunk
+            tma_load_3d(sA, &a.mA, &full_bar[stage], kb * 128, ti.m0, 0);
+            tma_load_3d(sB, &a.mB0, &full_bar[stage], kb * 128, ti.n0, ti.e);
+            uint8_t* sSF = sB + C::B_BYTES;
+            bulk_load(sSF, a.sfa + ((size_t)(ti.m0 / BM) * a.kchunks + kb) * 512, 512,
+                      &full_bar[stage]);
+            bulk_load(sSF + 512,
+                      a.sfb + ((size_t)(ti.e * (a.N / BM) + ti.n0 / BM) * a.kchunks + kb) * 512,
+                      512, &full_bar[stage]);
           } else if constexpr (KIND == K_DXR) {
             const int nkb = ti.kb_count / 2;
             const int pass = kb >= nkb;
@@ -383,6 +415,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           fence_after_sync();
           const uint32_t sA = smem_u32(smem + stage * C::STAGE);
           const uint32_t sB = sA + A_BYTES;
+          if constexpr (KT<KIND>::MX) {
+            // scale blocks -> TMEM (in order with the MMAs below and with the
+            // previous stage's MMAs, which have read the old blocks)
+            const uint32_t sSF = sB + C::B_BYTES;
+            const uint32_t sfa = tmem_base + MX_SF_COL, sfb = tmem_base + MX_SF_COL + 4;
+            tmem_cp_32x128b_x4(sfa, sdesc_noswz(sSF, 16, 128));
+            tmem_cp_32x128b_x4(sfb, sdesc_noswz(sSF + 512, 16, 128));
+#pragma unroll
+            for (uint32_t ks = 0; ks < 4; ++ks) {   // K = 32 E4M3 (32 bytes) per MMA
+              umma_mxf8(d_tmem, sdesc_sw128(sA + ks * 32, 16, 1024),
+                        sdesc_sw128(sB + ks * 32, 16, 1024), idesc_mxf8(BM, BN, ks),
+                        sfa | (ks << 30), sfb | (ks << 30), (kb | ks) != 0);
+            }
+          } else {
 #pragma unroll
           for (int ks = 0; ks < BK / 16; ++ks) {
             const uint64_t ad = KT<KIND>::A_MN ? sdesc_sw128(sA + ks * 2048, ATOM, 1024)
@@ -390,6 +436,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             const uint64_t bd = KT<KIND>::B_MN ? sdesc_sw128(sB + ks * 2048, ATOM, 1024)
                                                : sdesc_sw128(sB + ks * 32, 16, 1024);
             umma_bf16(d_tmem, ad, bd, IDESC, (kb | ks) != 0);
+          }
           }
           umma_commit(&empty_bar[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
@@ -429,7 +476,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       uint32_t r[32];
       uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * 4096;
       const int row0 = ti.m0 + q * 32;           // first row of this warp's 32-row slab
-      if constexpr (KIND == K_UP) {
+      if constexpr (KIND == K_UP || KIND == K_UPQ) {
         const int f = a.f, nf = ti.ntile * (BN / 2);
         float h3[32];
         for (int c = half * (BN / 4); c < (half + 1) * (BN / 4); c += 32) {
@@ -448,9 +495,15 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             const float h1 = bf16_round(v[i]);
             v[i] = h1 * sigmoid_fast(h1) * bf16_round(h3[i]);
           }
-          stage_store(otile, obuf, v, &a.sO1, nf + c, row0, lane);        // A
+          if constexpr (KIND == K_UPQ) {
+            // A (bf16-rounded) as one MXFP8 block: this thread's 32 columns
+            mx_store_block(v, a.act_q + (size_t)row * f + nf + c,
+                           a.act_s + mx_sf_offset(row, (nf + c) / 32, f / 128));
+          } else {
+            stage_store(otile, obuf, v, &a.sO1, nf + c, row0, lane);      // A
+          }
         }
-      } else if constexpr (KIND == K_DOWN || KIND == K_DX) {
+      } else if constexpr (KIND == K_DOWN || KIND == K_DX || KIND == K_DOWNQ) {
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
@@ -691,6 +744,23 @@ static int make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t
   return MOE_OK;
 }
 
+// 8-bit [d2, d1, d0] (d0 innermost; d2 = 1 for a matrix) in boxes of box1 x
+// box0 bytes, 128-byte swizzle (E4M3 operand tiles).
+static int make_map_u8(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+                       uint32_t box0, uint32_t box1) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0, d0 * d1};
+  cuuint32_t box[3] = {box0, box1, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
 // Output map of the epilogue's TMA stores: 32 x 32 boxes, 64-byte swizzle.
 static int make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer) {
   return make_map_2d(m, ptr, inner, outer, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
@@ -714,13 +784,14 @@ static int make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1
 
 template <int KIND, int BN>
 static int launch(const TcArgs& a, int grid, cudaStream_t s) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, KT<KIND>::MX>;
   cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<KIND, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return cuda_fail(e, "tc gemm smem attribute");
-  static const char* kNames[9] = {"tc_up",   "tc_down",   "tc_dap",      "tc_dx",    "tc_dw2",
-                                  "tc_dw13", "tc_router", "tc_router_dw", "tc_dx_router"};
-  static_assert(KIND >= 0 && KIND < 9, "kind out of range");
+  static const char* kNames[NUM_KINDS] = {
+      "tc_up",   "tc_down",   "tc_dap",       "tc_dx",        "tc_dw2",   "tc_dw13",
+      "tc_router", "tc_router_dw", "tc_dx_router", "tc_up_mxfp8", "tc_down_mxfp8"};
+  static_assert(KIND >= 0 && KIND < NUM_KINDS, "kind out of range");
   {
     ProfScope _ps(kNames[KIND], s);
     k_tc_gemm<KIND, BN><<<grid, THREADS, C::SMEM, s>>>(a);
@@ -874,6 +945,43 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
     if ((rc = make_map_3d(&a.mB0, p.w2, d, f, E, 64, 64))) return rc;
     if ((rc = make_store_map(&a.sO0, Y, d, cap))) return rc;
     if ((rc = launch_bn<K_DOWN>(a, bn, num_sms, s))) return rc;
+  }
+  return MOE_OK;
+}
+
+// MXFP8 forward: H = Xq [W1q | W3q] (bf16 out), A -> E4M3 blocks along f in
+// the epilogue, Y = Aq W2q (bf16 out).  xq/xs: quantised rows; w13q/w13s and
+// w2q/w2s: quantised weights (layouts in mx.cu); actq/acts: A's workspace.
+int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const uint8_t* w13q,
+                  const uint8_t* w13s, const uint8_t* w2q, const uint8_t* w2s, void* H,
+                  uint8_t* actq, uint8_t* acts, void* Y, int num_sms, cudaStream_t s) {
+  const int d = p.d, f = p.f, E = p.E, cap = p.cap;
+  int rc;
+  {  // UPQ
+    TcArgs a = base_args(p);
+    a.N = 2 * f;
+    a.K = d;
+    a.kchunks = d / 128;
+    a.sfa = xs;
+    a.sfb = w13s;
+    a.act_q = actq;
+    a.act_s = acts;
+    if ((rc = make_map_u8(&a.mA, xq, d, cap, 1, 128, BM))) return rc;
+    if ((rc = make_map_u8(&a.mB0, w13q, d, 2 * f, E, 128, 128))) return rc;
+    if ((rc = make_store_map(&a.sO0, H, 2 * f, cap))) return rc;
+    if ((rc = launch<K_UPQ, 128>(a, num_sms, s))) return rc;
+  }
+  {  // DOWNQ
+    TcArgs a = base_args(p);
+    a.N = d;
+    a.K = f;
+    a.kchunks = f / 128;
+    a.sfa = acts;
+    a.sfb = w2s;
+    if ((rc = make_map_u8(&a.mA, actq, f, cap, 1, 128, BM))) return rc;
+    if ((rc = make_map_u8(&a.mB0, w2q, f, d, E, 128, 128))) return rc;
+    if ((rc = make_store_map(&a.sO0, Y, d, cap))) return rc;
+    if ((rc = launch<K_DOWNQ, 128>(a, num_sms, s))) return rc;
   }
   return MOE_OK;
 }

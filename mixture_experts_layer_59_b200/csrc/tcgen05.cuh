@@ -61,6 +61,16 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// Plain bulk copy global -> shared (no tensor map): `bytes` a multiple of 16,
+// both addresses 16-byte aligned; completes a transaction count on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Shared -> global tile store through a tensor map (bulk async group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
   asm volatile(
@@ -120,6 +130,31 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z), "r"(z), "r"(z), "r"(z));
 }
 
+// D[tmem] (+)= (A * scale_A) (B * scale_B), kind::mxf8f6f4 with one E8M0
+// scale per 32 K-elements (K = 32 per instruction): the scale of row m of A
+// is byte `sf_id` of TMEM column sfa + m/32, lane m%32 (and likewise for B),
+// the layout tcgen05.cp .32x128b.warpx4 writes.  The byte index rides in
+// bits 30-31 of the scale addresses and in the instruction descriptor.
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem));
+}
+
+// Copy 32 rows x 16 bytes of shared memory (descriptor `sdesc`) into TMEM at
+// `taddr`: row i lands in lane i as four consecutive 32-bit columns and is
+// broadcast to the other three lane quarters.  Ordered with this thread's
+// tcgen05.mma instructions.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread finish.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -161,6 +196,27 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// Shared-memory descriptor without swizzle (K-major core matrices of 8 rows
+// x 16 bytes): SBO = distance between 8-row core matrices, LBO = distance
+// between core matrices adjacent in K.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with E4M3 A/B (K-major), fp32 D
+// and E8M0 block scales:
+//   bits 4-5 B scale byte, 7-9 A format (0 = E4M3), 10-12 B format,
+//   17-22 N >> 3, 23 scale format (1 = E8M0), 24-28 M >> 4, 29-30 A scale byte.
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id) {
+  return (sf_id << 4) | ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24) |
+         (sf_id << 29);
 }
 
 // Instruction descriptor of kind::f16 with bf16 A/B and fp32 D:

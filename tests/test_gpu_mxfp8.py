@@ -1,0 +1,161 @@
+"""GPU parity of the MXFP8 expert forward against the oracle's MXFP8
+definition (OCP MX, E4M3 elements, E8M0 scale per 32 along K).
+
+Quantised codes and scales that both sides compute from the same bf16 inputs
+(weights, token rows) are compared bit for bit; A is quantised from each
+side's own SwiGLU output, so its codes are compared where they are unique and
+checked to be valid elsewhere; H, the combined output and the (straight-
+through) backward meet the bf16 float tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_59_b200 import binding as B
+from mixture_experts_layer_59_b200 import synth
+from oracle import moe_oracle as O
+
+from helpers import BF16_TOL, assert_close, compare_plan, f64, fp32_router_logits, i64
+
+pytestmark = pytest.mark.gpu
+
+
+def sf_offset(r, kb, kchunks):
+    """Byte offset of the scale of row r, 32-element K-block kb (the layout
+    documented with the MXFP8 entry points)."""
+    r, kb = np.asarray(r), np.asarray(kb)
+    return ((r >> 7) * kchunks + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3)
+
+
+def u8(t):
+    return t.detach().to("cpu").numpy().astype(np.uint8)
+
+
+def expected_rows(q, se):
+    """E4M3 codes of quantised rows (blocks along the last axis) and E8M0 codes."""
+    return O.e4m3_encode(q), (se + 127).astype(np.uint8)
+
+
+def test_mxfp8_weight_quantisation_bitexact():
+    E, d, f = 3, 256, 384
+    g = torch.Generator().manual_seed(40)
+    w1 = (torch.randn(E, d, f, generator=g) * 0.02)
+    w3 = (torch.randn(E, d, f, generator=g) * 0.02)
+    w2 = (torch.randn(E, f, d, generator=g) * 0.02)
+    w1[0, :32, 5] = 0.0                       # an all-zero block
+    w1[1, 32:64, 7] *= 1e4                    # a block with a large maximum
+    w3[2, :32, 9] = torch.tensor([1e-30] * 32)  # tiny values: scale at the E8M0 floor
+    w2[0, 64:96, 3] = 448.0 * 2.0 ** 10       # elements that scale to exactly 448
+    w1, w3, w2 = (w.to(torch.bfloat16) for w in (w1, w3, w2))
+    wq = B.moe_mxfp8_quantize_weights(w1.cuda(), w3.cuda(), w2.cuda())
+    torch.cuda.synchronize()
+    w13q = u8(wq["w13q"]).reshape(E, 2 * f, d)
+    w13s, w2s = u8(wq["w13s"]), u8(wq["w2s"])
+    w2q = u8(wq["w2q"]).reshape(E, d, f)
+    for e in range(E):
+        for src, half in ((w1, 0), (w3, 1)):
+            q, se = O.mx_quantize(f64(src[e]), 0)          # blocks along d, per column
+            codes, scodes = expected_rows(q.T, se.T)        # [f, d], [f, d/32]
+            for t in range(f // 64):
+                rows = e * 2 * f + 128 * t + 64 * half + np.arange(64)
+                cols = 64 * t + np.arange(64)
+                np.testing.assert_array_equal(w13q[e, rows - e * 2 * f], codes[cols])
+                kb = np.arange(d // 32)
+                off = sf_offset(rows[:, None], kb[None, :], d // 128)
+                np.testing.assert_array_equal(w13s[off], scodes[cols])
+        q, se = O.mx_quantize(f64(w2[e]), 0)                # blocks along f, per column of d
+        codes, scodes = expected_rows(q.T, se.T)            # [d, f], [d, f/32]
+        np.testing.assert_array_equal(w2q[e], codes)
+        rows = e * d + np.arange(d)
+        off = sf_offset(rows[:, None], np.arange(f // 32)[None, :], f // 128)
+        np.testing.assert_array_equal(w2s[off], scodes)
+    assert w13s[sf_offset(0 * 2 * f + 5, 0, d // 128)] == 0           # zero block -> code 0
+    assert u8(wq["w2q"]).reshape(E, d, f)[0, 3, 64:96].tolist() == [0x7E] * 32   # 448
+
+
+def _mx_layer(cfg, seed, round_mode):
+    inp = synth.make_inputs(cfg, seed=seed, device="cuda")
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    bias = torch.linspace(0.5, -0.5, cfg.E)
+    lg = fp32_router_logits(x, wg, bias)
+    logits, idx, gate = B.moe_route(x, wg, cfg.k, logits_override=torch.from_numpy(lg).cuda())
+    plan = B.moe_permute(idx, gate, logits, cfg.E, round_mode)
+    wq = B.moe_mxfp8_quantize_weights(w1, w3, w2)
+    ws = torch.empty(B.moe_ffn_fwd_mxfp8_workspace_size(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k),
+                     device="cuda", dtype=torch.uint8)
+    H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, cfg.k, cfg.E, cfg.f, ws=ws)
+    out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], cfg.T, cfg.E,
+                        cfg.k)
+    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H)
+    B.moe_check_status()
+    torch.cuda.synchronize()
+    fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), cfg.k, round_mode=round_mode,
+                      logits_override=lg.astype(np.float64), precision="mxfp8")
+    bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd)
+    return inp, plan, ws, H, out, g, fwd, bwd
+
+
+def _ws_pieces(ws, cfg):
+    cap = B.moe_row_capacity(cfg.T, cfg.E, cfg.k)
+    capr = (cap + 127) // 128 * 128
+    up = lambda n: (n + 255) // 256 * 256
+    sizes = [capr * cfg.d, capr * cfg.d // 32, capr * cfg.f, capr * cfg.f // 32]
+    raw, out, off = u8(ws), [], 0
+    for n in sizes:
+        out.append(raw[off:off + n])
+        off += up(n)
+    return out
+
+
+@pytest.mark.parametrize("round_mode", [0, 1])
+def test_mxfp8_forward_and_backward(round_mode):
+    cfg = synth.MoEConfig("test", 1000, 256, 256, 8, 2, std=0.05)
+    inp, plan, ws, H, out, g, fwd, bwd = _mx_layer(cfg, 41 + round_mode, round_mode)
+    oplan = fwd["plan"]
+    compare_plan(plan, oplan)
+    R = oplan["R"]
+    toks = oplan["row_token"][:R]
+    live = toks >= 0
+    xq, xs, aq, as_ = _ws_pieces(ws, cfg)
+    d, f = cfg.d, cfg.f
+    # quantised token rows: bit-exact codes and scales; padding rows zero
+    q, se = O.mx_quantize(f64(inp["x"]), 1)
+    codes, scodes = expected_rows(q, se)
+    rows = np.arange(R)
+    np.testing.assert_array_equal(xq.reshape(-1, d)[:R][live], codes[toks[live]])
+    assert not xq.reshape(-1, d)[:R][~live].any()
+    soff = sf_offset(rows[:, None], np.arange(d // 32)[None, :], d // 128)
+    np.testing.assert_array_equal(xs[soff][live], scodes[toks[live]])
+    assert not xs[soff][~live].any()
+    # H from the block-scaled up-projection
+    assert_close(f64(H)[:R][live], fwd["H"][:R][live], "H", BF16_TOL)
+    # A's codes: from each side's own SwiGLU output -- identical almost
+    # everywhere, elsewhere a neighbouring code of the same sign and scale
+    qa, sea = O.mx_quantize(fwd["A"][:R], 1)
+    acodes, ascodes = expected_rows(qa, sea)
+    got = aq.reshape(-1, f)[:R]
+    aoff = sf_offset(rows[:, None], np.arange(f // 32)[None, :], f // 128)
+    gs = as_[aoff]
+    same_scale = gs[live] == ascodes[live]
+    assert same_scale.mean() > 0.999
+    same = got[live] == acodes[live]
+    assert same.mean() > 0.999, same.mean()
+    mag = lambda c: (c.astype(np.int64) & 0x7F)
+    ok_blocks = np.repeat(same_scale, 32, axis=1)
+    diff = ~same & ok_blocks
+    assert np.all(np.abs(mag(got[live][diff]) - mag(acodes[live][diff])) <= 1)
+    # combined output and the straight-through backward
+    assert_close(out, fwd["out"], "out", BF16_TOL)
+    assert_close(f64(g["dS"])[:R][live], bwd["dS"][:R][live], "dS", BF16_TOL)
+    for n in ("dlogits", "dx", "dw_gate", "dw1", "dw3", "dw2"):
+        assert_close(g[n], bwd[n], n, BF16_TOL)
+
+
+def test_mxfp8_forward_differs_from_bf16_by_the_quantisation():
+    """The MXFP8 output is not the bf16 output: their gap is of the size the
+    format implies (a few E4M3 half-ulps), far above the parity tolerance."""
+    cfg = synth.MoEConfig("test", 512, 256, 256, 8, 2, std=0.05)
+    inp, plan, ws, H, out, g, fwd, bwd = _mx_layer(cfg, 43, 0)
+    ref_bf16 = O.layer_fwd(f64(inp["x"]), f64(inp["w_gate"]), f64(inp["w1"]), f64(inp["w3"]),
+                           f64(inp["w2"]), cfg.k, logits_override=fwd["logits"])["out"]
+    rel = np.abs(f64(out) - ref_bf16).sum() / np.abs(ref_bf16).sum()
+    assert 5e-3 < rel < 0.1, rel
