@@ -208,8 +208,8 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
  * moe_mxfp8_weight_sizes: sizes[4] out = bytes of W13q, W13s, W2q, W2s for
  *   E experts (d and f multiples of 128, else MOE_ERR_UNSUPPORTED).
  * moe_mxfp8_quantize_weights: w1, w3 [E,d,f] and w2 [E,f,d] bf16 ->
- *   W13q [E, 2f, d] E4M3 (K = d contiguous; rows 128t..128t+63 are columns
- *   64t..64t+63 of W1 and rows 128t+64..128t+127 the same columns of W3),
+ *   W13q [E, 2f, d] E4M3 (K = d contiguous; rows 256b..256b+127 are columns
+ *   128b..128b+127 of W1 and rows 256b+128..256b+255 the same columns of W3),
  *   W13s its scales, W2q [E, d, f] E4M3 (K = f contiguous), W2s its scales.
  *   Run it once per weight update; caller-owned device buffers of the sizes
  *   above, 16-byte aligned.

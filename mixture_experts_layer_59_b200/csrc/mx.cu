@@ -1,8 +1,9 @@
 // MXFP8 operand preparation for the block-scaled expert GEMMs (format and
 // scale layout: mx.cuh).
-//   weights  W1, W3 [E, d, f] -> W13q [E, 2f, d] (K = d contiguous; rows of
-//            128-row tile t: 64 columns t*64.. of W1, then the same of W3, so
-//            one tile yields matching H1 / H3 columns) and W2 [E, f, d] ->
+//   weights  W1, W3 [E, d, f] -> W13q [E, 2f, d] (K = d contiguous; rows
+//            256b..256b+127 are columns 128b.. of W1, rows 256b+128..256b+255
+//            the same columns of W3, so one 256-row GEMM tile yields
+//            matching H1 / H3 columns) and W2 [E, f, d] ->
 //            W2q [E, d, f] (K = f contiguous), blocks of 32 along K.
 //   rows     x [T, d] -> Xq [cap, d]: each token row quantised once (blocks
 //            of 32 along d) and written to all of its rows in the row space;
@@ -26,16 +27,22 @@ k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __
   __shared__ __align__(16) __nv_bfloat16 tile[128][128];
   const int k0 = blockIdx.x * 128, t = blockIdx.y, e = blockIdx.z;
   const int kchunks = K / 128;
-  // source tile: 128 K-rows x 128 output rows (16-byte vectors of 8 bf16)
-  for (int v = threadIdx.x; v < 128 * 16; v += WQ_THREADS) {
-    const int kk = v >> 4, c8 = (v & 15) * 8;
-    const __nv_bfloat16* src;
-    if (W13) {  // output rows 0..63 from W1 columns t*64.., 64..127 from W3
-      src = (c8 < 64 ? wa : wb) + ((size_t)e * K + k0 + kk) * N + t * 64 + (c8 & 63);
-    } else {
-      src = wa + ((size_t)e * K + k0 + kk) * N + t * 128 + c8;
-    }
-    *reinterpret_cast<uint4*>(&tile[kk][c8]) = __ldg(reinterpret_cast<const uint4*>(src));
+  // source tile: 128 K-rows x 128 output rows (16-byte vectors of 8 bf16);
+  // output tile t of W13q is W1 (t even) or W3 (t odd), columns 128 (t/2)..
+  const __nv_bfloat16* base = W13 ? ((t & 1) ? wb : wa) + (size_t)(t >> 1) * 128
+                                  : wa + (size_t)t * 128;
+  constexpr int PER = 128 * 16 / WQ_THREADS;
+  uint4 u[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {   // all loads in flight before the shared stores
+    const int v = threadIdx.x + i * WQ_THREADS;
+    u[i] = __ldg(reinterpret_cast<const uint4*>(base + ((size_t)e * K + k0 + (v >> 4)) * N +
+                                                (v & 15) * 8));
+  }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int v = threadIdx.x + i * WQ_THREADS;
+    *reinterpret_cast<uint4*>(&tile[v >> 4][(v & 15) * 8]) = u[i];
   }
   __syncthreads();
   const int n = threadIdx.x & 127, j = threadIdx.x >> 7;

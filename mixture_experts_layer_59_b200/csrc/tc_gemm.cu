@@ -21,7 +21,8 @@
 //                                    accumulated in the same fp32 accumulator
 //   DXR   dx = (fp32 sum of the token's dX_perm rows) + dlogits W_gate^T
 //   UPQ   UP with MXFP8 operands (E4M3, one E8M0 scale per 32 along K):
-//         Xq [W13q], epilogue as UP but A leaves as MXFP8 (blocks along f)
+//         Xq [W13q], epilogue as UP but A leaves as MXFP8 (blocks along f);
+//         256-column tiles (128 W1 + 128 W3 columns), one accumulator
 //   DOWNQ DOWN with MXFP8 operands: Aq W2q
 //         (kind::mxf8f6f4 block-scaled MMAs, K = 32 per instruction; the two
 //         512-byte scale blocks of each stage go shared -> TMEM by tcgen05.cp)
@@ -57,8 +58,7 @@ enum Kind : int {
   K_UPQ = 9, K_DOWNQ = 10
 };
 constexpr int NUM_KINDS = 11;
-constexpr int MX_SF_BYTES = 1024;      // MXFP8 stage: 512-byte A and B scale blocks
-constexpr int MX_SF_COL = 256;         // TMEM columns of the scale blocks (after 2 x 128 accumulators)
+constexpr int MX_SF_COL = 256;         // TMEM column of the scale blocks (after the accumulators)
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
@@ -119,15 +119,25 @@ template <int KIND> struct KT {
 };
 
 // A stage holds a 128 x 128-byte A tile and a BN x 128-byte B tile (64 bf16
-// or 128 E4M3 elements of K), plus the scale blocks for the MXFP8 kinds.
+// or 128 E4M3 elements of K), plus, for the MXFP8 kinds, one 512-byte scale
+// block of A and BN/128 of B (the stage is padded to a 1 KB multiple).
+// Accumulators are double-buffered in TMEM except for 256-column MXFP8 tiles,
+// whose scale blocks need the columns of the second buffer; those also keep
+// one 2 KB staging tile per epilogue warp instead of two, to fit 4 stages.
 template <int BN, bool MX = false> struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE = A_BYTES + B_BYTES + (MX ? MX_SF_BYTES : 0);
-  static constexpr int STAGES = MX ? 5 : ((BN == 256) ? 4 : (BN == 128 ? 6 : 8));
-  static constexpr int OUT_BYTES = 8 * 2 * 2048;  // two 32 x 32 bf16 staging tiles per epilogue warp
+  static constexpr int SF_TX = MX ? 512 * (1 + BN / 128) : 0;   // scale bytes copied per stage
+  static constexpr int SF_BYTES = (SF_TX + 1023) / 1024 * 1024;
+  static constexpr int STAGE = A_BYTES + B_BYTES + SF_BYTES;
+  static constexpr int TX = A_BYTES + B_BYTES + SF_TX;           // bytes a stage's copies deliver
+  static constexpr int STAGES = MX ? (BN == 256 ? 4 : 5) : ((BN == 256) ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int NACC = (MX && BN == 256) ? 1 : 2;
+  static constexpr int OUT_TILES = (MX && BN == 256) ? 1 : 2;    // 32 x 32 bf16 staging tiles per epilogue warp
+  static constexpr int OUT_BYTES = 8 * OUT_TILES * 2048;
   static constexpr int SMEM = STAGES * STAGE + OUT_BYTES;
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
-  static_assert(!MX || BN == 128, "MXFP8 kinds use 128-column tiles");
+  static_assert(!MX || NACC * BN == MX_SF_COL, "scale blocks follow the accumulators");
+  static_assert(STAGE % 1024 == 0, "stages must keep 1 KB alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -235,11 +245,15 @@ __device__ __forceinline__ void ld_bf16x32(const __nv_bfloat16* src, float* v) {
 // c ^ ((r >> 1) & 3)) and store it with one TMA tile store at (col, row0).
 // The tiles alternate; before a tile is rewritten, the store issued from it
 // two calls ago must have finished reading it.
+template <int NT = 2>
 __device__ __forceinline__ void stage_store(uint8_t* tiles, int& which, const float* v,
                                             const CUtensorMap* map, int col, int row0, int lane) {
   uint8_t* tile = tiles + which * 2048;
-  which ^= 1;
-  if (lane == 0) bulk_wait_read_1();
+  if (NT == 2) which ^= 1;
+  if (lane == 0) {
+    if (NT == 2) bulk_wait_read_1();
+    else bulk_wait_read_all();
+  }
   __syncwarp();
   uint8_t* rowp = tile + lane * 64;
   const int sw = (lane >> 1) & 3;
@@ -325,7 +339,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           if (!bounded_wait(&empty_bar[stage], phase ^ 1, &s_abort, a.status, 1)) goto producer_done;
           uint8_t* sA = smem + stage * C::STAGE;
           uint8_t* sB = sA + A_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], C::STAGE);
+          mbar_arrive_expect_tx(&full_bar[stage], C::TX);
           const int k0 = kb * BK;
           if constexpr (KIND == K_UP) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
@@ -374,9 +388,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             uint8_t* sSF = sB + C::B_BYTES;
             bulk_load(sSF, a.sfa + ((size_t)(ti.m0 / BM) * a.kchunks + kb) * 512, 512,
                       &full_bar[stage]);
-            bulk_load(sSF + 512,
-                      a.sfb + ((size_t)(ti.e * (a.N / BM) + ti.n0 / BM) * a.kchunks + kb) * 512,
-                      512, &full_bar[stage]);
+#pragma unroll
+            for (int b = 0; b < BN / 128; ++b)
+              bulk_load(sSF + 512 * (1 + b),
+                        a.sfb + ((size_t)(ti.e * (a.N / 128) + ti.n0 / 128 + b) * a.kchunks + kb) * 512,
+                        512, &full_bar[stage]);
           } else if constexpr (KIND == K_DXR) {
             const int nkb = ti.kb_count / 2;
             const int pass = kb >= nkb;
@@ -405,8 +421,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       int it = 0;
       TileInfo ti;
       for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = C::NACC == 1 ? 0 : (it & 1);
+        const uint32_t acc_phase = C::NACC == 1 ? (it & 1) : ((it >> 1) & 1);
         if (!bounded_wait(&tempty_bar[acc], acc_phase ^ 1, &s_abort, a.status, 2)) break;
         fence_after_sync();
         const uint32_t d_tmem = tmem_base + acc * BN;
@@ -421,7 +437,9 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             const uint32_t sSF = sB + C::B_BYTES;
             const uint32_t sfa = tmem_base + MX_SF_COL, sfb = tmem_base + MX_SF_COL + 4;
             tmem_cp_32x128b_x4(sfa, sdesc_noswz(sSF, 16, 128));
-            tmem_cp_32x128b_x4(sfb, sdesc_noswz(sSF + 512, 16, 128));
+#pragma unroll
+            for (int b = 0; b < BN / 128; ++b)      // B rows 128b.. -> columns sfb + 4b..
+              tmem_cp_32x128b_x4(sfb + 4 * b, sdesc_noswz(sSF + 512 * (1 + b), 16, 128));
 #pragma unroll
             for (uint32_t ks = 0; ks < 4; ++ks) {   // K = 32 E4M3 (32 bytes) per MMA
               umma_mxf8(d_tmem, sdesc_sw128(sA + ks * 32, 16, 1024),
@@ -455,8 +473,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
     int it = 0;
     TileInfo ti;
     for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = C::NACC == 1 ? 0 : (it & 1);
+      const uint32_t acc_phase = C::NACC == 1 ? (it & 1) : ((it >> 1) & 1);
       // DAP: the first chunk of H does not depend on the accumulator, so its
       // loads are issued before waiting for the main loop
       uint4 hn1[4], hn3[4];
@@ -474,9 +492,58 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       const int row = ti.m0 + rloc;
       float v[32];
       uint32_t r[32];
-      uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * 4096;
+      uint8_t* otile = smem + C::STAGES * C::STAGE + (warp - 2) * (C::OUT_TILES * 2048);
       const int row0 = ti.m0 + q * 32;           // first row of this warp's 32-row slab
-      if constexpr (KIND == K_UP || KIND == K_UPQ) {
+      bool released = false;  // accumulator handed back before the end of the epilogue
+      if constexpr (KT<KIND>::MX && C::NACC == 1) {
+        // one accumulator: copy this thread's 4 x 32 columns to registers and
+        // release it at once, so that the next tile's MMAs overlap the math
+        // and stores below
+        uint32_t ra[32], rb[32], rc[32], rd[32];
+        int col[4];
+        if constexpr (KIND == K_UPQ) {   // H1 cols half*64.., H3 cols 128 + half*64..
+          col[0] = half * 64; col[1] = half * 64 + 32; col[2] = 128 + half * 64; col[3] = 160 + half * 64;
+        } else {
+          col[0] = half * 128; col[1] = col[0] + 32; col[2] = col[0] + 64; col[3] = col[0] + 96;
+        }
+        tmem_ld32(tbase + col[0], ra);
+        tmem_ld32(tbase + col[1], rb);
+        tmem_ld32(tbase + col[2], rc);
+        tmem_ld32(tbase + col[3], rd);
+        tmem_ld_wait();
+        fence_before_sync();
+        mbar_arrive(&tempty_bar[acc]);
+        released = true;
+        if constexpr (KIND == K_UPQ) {
+          const int f = a.f, nf = ti.ntile * (BN / 2);
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t* r1 = j ? rb : ra;
+            const uint32_t* r3 = j ? rd : rc;
+            const int c = half * 64 + 32 * j;
+            float h3[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { v[i] = __uint_as_float(r1[i]); h3[i] = __uint_as_float(r3[i]); }
+            stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, nf + c, row0, lane);        // H1
+            stage_store<C::OUT_TILES>(otile, obuf, h3, &a.sO0, f + nf + c, row0, lane);   // H3
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float h1 = bf16_round(v[i]);
+              v[i] = h1 * sigmoid_fast(h1) * bf16_round(h3[i]);
+            }
+            mx_store_block(v, a.act_q + (size_t)row * f + nf + c,
+                           a.act_s + mx_sf_offset(row, (nf + c) / 32, f / 128));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t* rr = j == 0 ? ra : (j == 1 ? rb : (j == 2 ? rc : rd));
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(rr[i]);
+            stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + col[j], row0, lane);
+          }
+        }
+      } else if constexpr (KIND == K_UP || KIND == K_UPQ) {
         const int f = a.f, nf = ti.ntile * (BN / 2);
         float h3[32];
         for (int c = half * (BN / 4); c < (half + 1) * (BN / 4); c += 32) {
@@ -488,8 +555,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) h3[i] = __uint_as_float(r[i]);
-          stage_store(otile, obuf, v, &a.sO0, nf + c, row0, lane);        // H1
-          stage_store(otile, obuf, h3, &a.sO0, f + nf + c, row0, lane);   // H3
+          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, nf + c, row0, lane);        // H1
+          stage_store<C::OUT_TILES>(otile, obuf, h3, &a.sO0, f + nf + c, row0, lane);   // H3
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float h1 = bf16_round(v[i]);
@@ -500,7 +567,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             mx_store_block(v, a.act_q + (size_t)row * f + nf + c,
                            a.act_s + mx_sf_offset(row, (nf + c) / 32, f / 128));
           } else {
-            stage_store(otile, obuf, v, &a.sO1, nf + c, row0, lane);      // A
+            stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, nf + c, row0, lane);      // A
           }
         }
       } else if constexpr (KIND == K_DOWN || KIND == K_DX || KIND == K_DOWNQ) {
@@ -509,7 +576,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          stage_store(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);
+          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);
         }
       } else if constexpr (KIND == K_DAP) {
         const int f = a.f;
@@ -543,11 +610,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             da3[i] = da * sl;
             r[i] = __float_as_uint(g * av);                           // s * A
           }
-          stage_store(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
-          stage_store(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
+          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
+          stage_store<C::OUT_TILES>(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          stage_store(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);      // s * A
+          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);      // s * A
         }
         a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
       } else if constexpr (KIND == K_RT) {
@@ -654,7 +721,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             }
           }
           // rows at or beyond T are clipped by the tensor map
-          stage_store(otile, obuf, v, &a.sO0, col, row0, lane);
+          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, col, row0, lane);
         }
       } else {  // DW2 / DW13: output row m = row of dW_e (maps view dW as [E*M, N])
         const int orow0 = ti.e * a.M + row0;
@@ -670,15 +737,17 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           }
           const int col = ti.n0 + c;
           if constexpr (KIND == K_DW2) {
-            stage_store(otile, obuf, v, &a.sO0, col, orow0, lane);
+            stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, col, orow0, lane);
           } else {
-            if (col < a.f) stage_store(otile, obuf, v, &a.sO0, col, orow0, lane);
-            else stage_store(otile, obuf, v, &a.sO1, col - a.f, orow0, lane);
+            if (col < a.f) stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, col, orow0, lane);
+            else stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, col - a.f, orow0, lane);
           }
         }
       }
-      fence_before_sync();
-      mbar_arrive(&tempty_bar[acc]);
+      if (!released) {
+        fence_before_sync();
+        mbar_arrive(&tempty_bar[acc]);
+      }
     }
   }
 
@@ -967,9 +1036,9 @@ int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const 
     a.act_q = actq;
     a.act_s = acts;
     if ((rc = make_map_u8(&a.mA, xq, d, cap, 1, 128, BM))) return rc;
-    if ((rc = make_map_u8(&a.mB0, w13q, d, 2 * f, E, 128, 128))) return rc;
+    if ((rc = make_map_u8(&a.mB0, w13q, d, 2 * f, E, 128, 256))) return rc;
     if ((rc = make_store_map(&a.sO0, H, 2 * f, cap))) return rc;
-    if ((rc = launch<K_UPQ, 128>(a, num_sms, s))) return rc;
+    if ((rc = launch<K_UPQ, 256>(a, num_sms, s))) return rc;
   }
   {  // DOWNQ
     TcArgs a = base_args(p);
@@ -979,9 +1048,14 @@ int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const 
     a.sfa = acts;
     a.sfb = w2s;
     if ((rc = make_map_u8(&a.mA, actq, f, cap, 1, 128, BM))) return rc;
-    if ((rc = make_map_u8(&a.mB0, w2q, f, d, E, 128, 128))) return rc;
+    const int bn = pick_bn(d);
+    if ((rc = make_map_u8(&a.mB0, w2q, f, d, E, 128, bn))) return rc;
     if ((rc = make_store_map(&a.sO0, Y, d, cap))) return rc;
-    if ((rc = launch<K_DOWNQ, 128>(a, num_sms, s))) return rc;
+    if (bn == 256) {
+      if ((rc = launch<K_DOWNQ, 256>(a, num_sms, s))) return rc;
+    } else if ((rc = launch<K_DOWNQ, 128>(a, num_sms, s))) {
+      return rc;
+    }
   }
   return MOE_OK;
 }

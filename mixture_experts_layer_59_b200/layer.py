@@ -16,10 +16,13 @@ class MoELayerStep:
 
     def __init__(self, T, d, f, E, k, dtype=torch.bfloat16, device="cuda",
                  round_mode=B.MOE_ROUND_NONE, balance_lambda=None,
-                 gate_mode=B.MOE_GATE_TOPK_SOFTMAX, capacity_factor=None):
+                 gate_mode=B.MOE_GATE_TOPK_SOFTMAX, capacity_factor=None, precision="bf16"):
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         self.dtype, self.device, self.round_mode = dtype, device, round_mode
         self.gate_mode = gate_mode
+        if precision not in ("bf16", "mxfp8"):
+            raise ValueError("precision must be 'bf16' or 'mxfp8'")
+        self.precision = precision
         if round_mode == B.MOE_ROUND_CAPACITY:
             if capacity_factor is None:
                 raise ValueError("MOE_ROUND_CAPACITY needs capacity_factor")
@@ -40,6 +43,11 @@ class MoELayerStep:
         self.out = e(T, d, dt_=dtype)
         self.ws_perm = e(max(B.moe_permute_workspace_size(T, E, k, round_mode), 1), dt_=torch.uint8)
         self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
+        if precision == "mxfp8":
+            self.wq = {n: e(sz, dt_=torch.uint8) for n, sz in
+                       zip(("w13q", "w13s", "w2q", "w2s"), B.moe_mxfp8_weight_sizes(E, d, f))}
+            self.ws_mx = e(max(B.moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k), 1),
+                           dt_=torch.uint8)
         self.ws_bwd = e(max(B.moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
         self.balance_lambda = balance_lambda
         if balance_lambda is not None:
@@ -62,8 +70,14 @@ class MoELayerStep:
         if self.balance_lambda is not None:
             self.balance = B.moe_balance_loss(self.idx, self.gate, self.E, self.balance_lambda,
                                               ws=self.ws_bal, stream=stream)
-        B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan, self.k, self.H, self.Y, self.ws_fwd,
-                             stream=stream)
+        if self.precision == "mxfp8":
+            # weights change every optimizer step: quantise them in the step
+            B.moe_mxfp8_quantize_weights(w1, w3, w2, out=self.wq, stream=stream)
+            B.moe_expert_ffn_fwd_mxfp8(x, self.wq, self.plan, self.k, self.E, self.f, self.H,
+                                       self.Y, self.ws_mx, stream=stream)
+        else:
+            B.moe_expert_ffn_fwd(x, w1, w3, w2, self.plan, self.k, self.H, self.Y, self.ws_fwd,
+                                 stream=stream)
         B.moe_combine(self.Y, self.plan["row_gate"], self.plan["slot_row"],
                       self.plan["extra_row"], self.T, self.E, self.k, self.out, stream=stream)
         return self.out

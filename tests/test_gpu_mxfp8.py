@@ -55,9 +55,9 @@ def test_mxfp8_weight_quantisation_bitexact():
         for src, half in ((w1, 0), (w3, 1)):
             q, se = O.mx_quantize(f64(src[e]), 0)          # blocks along d, per column
             codes, scodes = expected_rows(q.T, se.T)        # [f, d], [f, d/32]
-            for t in range(f // 64):
-                rows = e * 2 * f + 128 * t + 64 * half + np.arange(64)
-                cols = 64 * t + np.arange(64)
+            for b in range(f // 128):
+                rows = e * 2 * f + 256 * b + 128 * half + np.arange(128)
+                cols = 128 * b + np.arange(128)
                 np.testing.assert_array_equal(w13q[e, rows - e * 2 * f], codes[cols])
                 kb = np.arange(d // 32)
                 off = sf_offset(rows[:, None], kb[None, :], d // 128)
@@ -159,3 +159,40 @@ def test_mxfp8_forward_differs_from_bf16_by_the_quantisation():
                            f64(inp["w2"]), cfg.k, logits_override=fwd["logits"])["out"]
     rel = np.abs(f64(out) - ref_bf16).sum() / np.abs(ref_bf16).sum()
     assert 5e-3 < rel < 0.1, rel
+
+
+@pytest.mark.parametrize("name,n_tok", [("coarse", 48), ("fine", 48)])
+def test_mxfp8_full_size_sampled_tokens(name, n_tok):
+    """Full workload sizes in the bench's launch configuration: out, dx,
+    dlogits and dS of sampled tokens against the oracle's MXFP8 layer (each
+    depends only on the token and its experts' weights)."""
+    from test_gpu_full_configs import DeviceExperts
+    cfg = synth.CONFIGS[name]
+    T, E, k = cfg.T, cfg.E, cfg.k
+    inp = synth.make_inputs(cfg, seed=0, device="cuda")
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    x64, wg64 = f64(x), f64(wg)
+    lg = fp32_router_logits(x64, wg64, inp["logit_bias"])
+    logits, idx, gate = B.moe_route(x, wg, k, logits_override=torch.from_numpy(lg).cuda())
+    plan = B.moe_permute(idx, gate, logits, E)
+    wq = B.moe_mxfp8_quantize_weights(w1, w3, w2)
+    H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, k, E, cfg.f)
+    out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)
+    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H)
+    B.moe_check_status()
+    torch.cuda.synchronize()
+    lg64 = lg.astype(np.float64)
+    _, oidx, ogate = O.route(None, None, k, logits_override=lg64)
+    oplan = O.exact_plan(oidx, ogate, E)
+    compare_plan(plan, oplan)
+    fwd = dict(logits=lg64, idx=oidx, gate=ogate, plan=oplan, precision="mxfp8")
+    rng = np.random.default_rng(7)
+    tokens = sorted(set([0, T - 1] + list(rng.choice(T, n_tok - 2, replace=False))))
+    s = O.sampled_tokens(tokens, f64(dout), x64, wg64, DeviceExperts(w1), DeviceExperts(w3),
+                         DeviceExperts(w2), fwd)
+    assert_close(f64(out)[tokens], np.stack([s["out"][t] for t in tokens]), "out", BF16_TOL)
+    assert_close(f64(g["dx"])[tokens], np.stack([s["dx"][t] for t in tokens]), "dx", BF16_TOL)
+    assert_close(f64(g["dlogits"])[tokens], np.stack([s["dlogits"][t] for t in tokens]),
+                 "dlogits", BF16_TOL)
+    rows = sorted(s["dS"])
+    assert_close(f64(g["dS"])[rows], np.array([s["dS"][r] for r in rows]), "dS", BF16_TOL)
