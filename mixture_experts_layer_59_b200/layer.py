@@ -82,6 +82,27 @@ class MoELayerStep:
                       self.plan["extra_row"], self.T, self.E, self.k, self.out, stream=stream)
         return self.out
 
+    def capture(self, x, w_gate, w1, w3, w2, dout, logits_override=None, logit_bias=None,
+                logit_noise=None):
+        """Record one forward + backward step into a CUDA graph and return it.
+
+        Every library call only enqueues kernels on the current stream (no host
+        synchronisation, no allocation), so the whole step can be captured;
+        ``graph.replay()`` then re-runs it on the current contents of the given
+        tensors and of this object's buffers.  One eager step first (on a side
+        stream) sets the kernels' shared-memory attributes outside capture."""
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            self.forward(x, w_gate, w1, w3, w2, logits_override, logit_bias, logit_noise=logit_noise)
+            self.backward(dout)
+        torch.cuda.current_stream().wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="thread_local"):
+            self.forward(x, w_gate, w1, w3, w2, logits_override, logit_bias, logit_noise=logit_noise)
+            self.backward(dout)
+        return graph
+
     def backward(self, dout, stream=None):
         x, w_gate, w1, w3, w2 = self._saved
         return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
