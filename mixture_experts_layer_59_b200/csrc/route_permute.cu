@@ -343,8 +343,11 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                int32_t* __restrict__ row_token, float* __restrict__ row_gate,
                int32_t* __restrict__ row_slot, int32_t* __restrict__ slot_row,
-               int32_t* __restrict__ extra_row) {
-  extern __shared__ uint32_t bm[];  // membership bitmap of the assigned tokens, T bits
+               int32_t* __restrict__ extra_row, int key_cache) {
+  // dynamic shared memory: membership bitmap of the assigned tokens (T bits),
+  // then, when key_cache != 0, every candidate's 64-bit key (computed once
+  // instead of once per radix pass)
+  extern __shared__ uint32_t bm[];
   __shared__ int s_off[257];
   __shared__ int s_hist[256];
   __shared__ int s_warp[33];
@@ -414,6 +417,13 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
   auto cand_key = [&](int t) -> uint64_t {
     return order_key((double)logits[(size_t)t * E + e] - lse[t]);
   };
+  uint64_t* kc = key_cache ? reinterpret_cast<uint64_t*>(bm + ((nwords + 1) & ~1)) : nullptr;
+  if (kc != nullptr && m > 0) {
+    for (int i = threadIdx.x; i < ncand; i += blockDim.x)
+      kc[i] = is_cand(i) ? cand_key(cand_token(i)) : 0;
+    __syncthreads();
+  }
+  auto key_of = [&](int i) -> uint64_t { return kc ? kc[i] : cand_key(cand_token(i)); };
 
   // radix select of the m-th largest key among the candidates
   uint64_t prefix = 0, pmask = 0;
@@ -422,20 +432,44 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
     for (int shift = 56; shift >= 0; shift -= 8) {
       for (int i = threadIdx.x; i < 256; i += blockDim.x) s_hist[i] = 0;
       __syncthreads();
-      for (int i = threadIdx.x; i < ncand; i += blockDim.x) {
-        if (!is_cand(i)) continue;
-        uint64_t u = cand_key(cand_token(i));
-        if ((u & pmask) == prefix) atomicAdd(&s_hist[(u >> shift) & 255], 1);
+      // histogram of the current digit: keys share few digits in the high
+      // passes, so lanes with equal digits add once per warp
+      for (int i0 = 0; i0 < ncand; i0 += blockDim.x) {
+        const int i = i0 + threadIdx.x;
+        int bin = -1;
+        if (i < ncand && is_cand(i)) {
+          const uint64_t u = key_of(i);
+          if ((u & pmask) == prefix) bin = (int)((u >> shift) & 255);
+        }
+        const unsigned grp = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(grp) - 1)
+          atomicAdd(&s_hist[bin], __popc(grp));
       }
       __syncthreads();
-      if (threadIdx.x == 0) {
-        int cum = 0, sel = 0;
-        for (int dg = 255; dg >= 0; --dg) {
-          if (cum + s_hist[dg] >= rem) { sel = dg; break; }
-          cum += s_hist[dg];
+      // digit of the rem-th largest key: lane l holds digits 255-8l .. 248-8l
+      if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int loc[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { loc[j] = s_hist[255 - (8 * lane + j)]; sum += loc[j]; }
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
         }
-        s_sel = sel;
-        s_rem = rem - cum;
+        int cum = inc - sum;   // keys with a larger digit than this lane's range
+        if (cum < rem && inc >= rem) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (cum + loc[j] >= rem) {
+              s_sel = 255 - (8 * lane + j);
+              s_rem = rem - cum;
+              break;
+            }
+            cum += loc[j];
+          }
+        }
       }
       __syncthreads();
       prefix |= (uint64_t)s_sel << shift;
@@ -458,7 +492,7 @@ k_round_select(const float* __restrict__ logits, const double* __restrict__ lse,
       cand = is_cand(i);
       assigned = drop ? 1 : !cand;
       if (cand && m > 0) {
-        u = cand_key(t);
+        u = key_of(i);
         eq = (u == thr);
         gt = (u > thr);
       }
@@ -518,8 +552,13 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
       if (e != cudaSuccess) return cuda_fail(e, "memset extra_row");
     }
   }
-  const size_t smem = (size_t)((T + 31) / 32 + 1) * sizeof(uint32_t);
+  size_t smem = (size_t)((T + 31) / 32 + 1) * sizeof(uint32_t);
   if (smem > 200 * 1024) return fail(MOE_ERR_UNSUPPORTED, "token rounding supports T <= 1.6M");
+  // candidate keys in shared memory when all T of them fit next to the bitmap
+  const size_t words = (size_t)(((T + 31) / 32 + 1) & ~1);
+  const size_t with_keys = words * sizeof(uint32_t) + (size_t)T * sizeof(uint64_t);
+  const int key_cache = with_keys <= 200 * 1024 ? 1 : 0;
+  if (key_cache) smem = with_keys;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(k_round_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -530,7 +569,7 @@ int launch_permute_round(const int32_t* idx, const float* gate, const float* log
     k_round_select<<<E, RS_THREADS, smem, s>>>(logits, w.lse, w.ex_counts, w.ex_offsets,
                                                w.ex_row_token, w.ex_row_gate, w.ex_row_slot, T, E,
                                                tile, capacity, counts, offsets, row_token, row_gate,
-                                               row_slot, slot_row, extra_row);
+                                               row_slot, slot_row, extra_row, key_cache);
   }
   MOE_CHECK_LAUNCH("round_select");
   return MOE_OK;
