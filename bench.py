@@ -97,6 +97,47 @@ def peak_ratio(kind):
     return 2.0 if kind.endswith("_mxfp8") else 1.0
 
 
+def gemm_bytes(kind, T, d, f, E, k):
+    """Algorithmic HBM bytes of one launch of each grouped GEMM: expert
+    weights once, row-space operands once, outputs once (bf16; E4M3 = 1 B)."""
+    R, w = T * k, E * d * f
+    b = {
+        "tc_up": 2 * w * 2 + R * d * 2 + R * 2 * f * 2 + R * f * 2,
+        "tc_down": w * 2 + R * f * 2 + R * d * 2,
+        "tc_dap": w * 2 + R * d * 2 + R * 2 * f * 2 + R * 2 * f * 2 + R * f * 2,
+        "tc_dx": 2 * w * 2 + R * 2 * f * 2 + R * d * 2,
+        "tc_dw2": w * 2 + R * f * 2 + R * d * 2,
+        "tc_dw13": 2 * w * 2 + R * d * 2 + R * 2 * f * 2,
+        "tc_up_mxfp8": 2 * w * 1.03125 + R * d * 1.03125 + R * 2 * f * 2 + R * f * 1.03125,
+        "tc_down_mxfp8": w * 1.03125 + R * f * 1.03125 + R * d * 2,
+    }
+    return b.get(kind)
+
+
+def hbm_bytes(kind, T, d, f, E, k, launches):
+    """Algorithmic HBM bytes per launch of the memory-bound kernels (None for
+    the latency-bound ones: permutation, router backward, reductions)."""
+    R = T * k
+    if kind == "tc_router":
+        return T * d * 2 + d * E * 2 + T * E * 4 + T * k * 8
+    if kind == "tc_router_dw":
+        return T * d * 2 + T * E * 4
+    if kind == "tc_dx_router":
+        return T * d * 4 + T * d * 2 + T * E * 4
+    if kind == "scatter_rows":
+        return T * d * 2 + R * d * 2
+    if kind == "mx_scatter_rows":
+        return T * d * 2 + R * d * 1.03125
+    if kind == "dx_fused":
+        return R * d * 2 + T * d * 2 + T * E * 4
+    if kind == "token_reduce":   # combine (bf16 out), plus the fp32 dX row sums when launched twice
+        per = [R * d * 2 + R * 4 + T * d * 2, R * d * 2 + T * d * 4]
+        return sum(per[:launches]) / launches
+    if kind == "mx_quant_weights":
+        return E * d * f * 2 * 3 + E * d * f * 3 * 1.03125
+    return None
+
+
 def step_flops(T, d, f, E, k, router=True):
     return 18.0 * T * k * d * f + 2.0 * T * k * f + (6.0 * T * d * E if router else 0.0)
 
@@ -372,9 +413,25 @@ def run_ours(args, cfg, rank, world, local_rank):
         # time the GEMMs would take at their dtype's peak, over the time they took
         ideal_s = sum(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) * v[0] / (bf16_peak * peak_ratio(n) * 1e12)
                       for n, v in gemm.items())
+        # roofline of the phase: each kernel at the slower of its math and its
+        # algorithmic HBM bytes, over the time the GEMMs took
+        bw = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+        roof_s = sum(max(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) / (bf16_peak * peak_ratio(n) * 1e12),
+                         gemm_bytes(n, cfg.T, cfg.d, cfg.f, cfg.E, cfg.k) / bw) * v[0]
+                     for n, v in gemm.items())
         gemm_summary = {"tflops": g_fl / (g_ms / 1e3) / 1e12,
                         "frac_of_peak": ideal_s / (g_ms / 1e3),
+                        "frac_roof": roof_s / (g_ms / 1e3),
                         "ms_per_step": g_ms / args.steps}
+    # memory-bound kernels: algorithmic bytes / live time vs the measured copy bandwidth
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    hbm_kernels = {}
+    for n, (nl, tot) in prof.items():
+        by = hbm_bytes(n, cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, max(nl // args.steps, 1))
+        if by:
+            us = 1e3 * tot / nl
+            hbm_kernels[n] = {"avg_us": us, "gb_per_launch": by / 1e9,
+                              "gbs": by / (us * 1e-6) / 1e9, "frac": by / (us * 1e-6) / 1e9 / hbm_peak}
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         n, times, threads = oracle_tokens_per_s(cfg, args.cpu_sample, args)
@@ -397,6 +454,7 @@ def run_ours(args, cfg, rank, world, local_rank):
                 "ms_per_step": e2e_total / len(e2e_ms) if e2e_ms else None},
         "clocks": clocks,
         "gpu_launches": launches,
+        "hbm_kernels": hbm_kernels,
         "kernels": kernels,
     }
     print(json.dumps(line), flush=True)
