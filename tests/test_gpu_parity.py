@@ -365,3 +365,42 @@ def test_layer_bf16_fused_dx_shapes(d, E, k, round_mode):
     if round_mode:
         assert fwd["plan"]["added"].any()
     compare_layer(g, fwd, bwd, BF16_TOL)
+
+
+# ------------------------------------------------------------------ degenerate shapes
+
+@pytest.mark.parametrize("T,E,k,round_mode", [
+    (300, 8, 1, 0),       # top-1 routing: every token has one row, gates are 1
+    (260, 4, 4, 0),       # k = E: every token goes to every expert
+    (260, 4, 4, 1),       # ... with token rounding (counts 260 -> 256: drops only)
+    (1, 8, 2, 0),         # a single token
+    (129, 16, 8, 1),      # one more token than a tile, maximal k
+])
+def test_layer_degenerate_routing_shapes(T, E, k, round_mode):
+    cfg = _cfg(T, 128, 128, E, k, std=0.08)
+    inp = synth.make_inputs(cfg, seed=T + E + k, device="cuda")
+    lg = fp32_router_logits(inp["x"], inp["w_gate"])
+    g = gpu_layer(inp, cfg.k, round_mode, lg)
+    fwd, bwd = oracle_layer(inp, cfg.k, round_mode, lg)
+    if k == 1:
+        assert np.all(fwd["gate"] == 1.0)
+    if k == E:
+        assert np.all(np.sort(fwd["idx"], 1) == np.arange(E))
+    compare_layer(g, fwd, bwd, BF16_TOL)
+
+
+@pytest.mark.parametrize("T,E,k", [(300, 8, 1), (1, 8, 2)])
+def test_mxfp8_degenerate_routing_shapes(T, E, k):
+    cfg = _cfg(T, 256, 256, E, k, std=0.05)
+    inp = synth.make_inputs(cfg, seed=7 * T + k, device="cuda")
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    lg = fp32_router_logits(x, wg)
+    logits, idx, gate = B.moe_route(x, wg, k, logits_override=torch.from_numpy(lg).cuda())
+    plan = B.moe_permute(idx, gate, logits, E)
+    wq = B.moe_mxfp8_quantize_weights(w1, w3, w2)
+    H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, k, E, cfg.f)
+    out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)
+    torch.cuda.synchronize()
+    fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), k,
+                      logits_override=lg.astype(np.float64), precision="mxfp8")
+    assert_close(out, fwd["out"], "out", BF16_TOL)
