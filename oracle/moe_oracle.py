@@ -406,13 +406,17 @@ def expert_rows_forward(xr, w1e, w3e, w2e, staged, precision="bf16"):
     return h1, h3, a, y
 
 
-def expert_rows_backward(dor, gr, h1, h3, w1e, w3e, w2e, staged):
+def expert_rows_backward(dor, gr, h1, h3, w1e, w3e, w2e, staged, precision="bf16"):
     """Backward of one expert's rows given dO rows ``dor`` and row weights ``gr``.
 
     dA' = dO W2^T                       (gradient of A before gate scaling)
     dS  = <dA', A>                      ([SonicMoE] sec. 1: no stored Y needed)
     dA  = g dA';  da3 = dA silu(h1);  da1 = dA h3 silu'(h1)
     g*A (operand of dW2), dX_perm = da1 W1^T + da3 W3^T.
+
+    precision "mxfp8": the dX_perm GEMM takes MXFP8 operands -- dH (after its
+    bf16 staging) and W1, W3, all in blocks along f; the other GEMMs keep the
+    unquantised operands.
     """
     dor = np.asarray(dor, np.float64)
     a = _stage(silu(h1) * h3, staged)
@@ -422,7 +426,11 @@ def expert_rows_backward(dor, gr, h1, h3, w1e, w3e, w2e, staged):
     da3 = _stage(da * silu(h1), staged)
     da1 = _stage(da * h3 * silu_grad(h1), staged)
     ga = _stage(gr[:, None] * a, staged)
-    dxp = _stage(da1 @ w1e.T + da3 @ w3e.T, staged)
+    if precision == "mxfp8":
+        dxp = _stage(mx_fake_quant(da1, 1) @ mx_fake_quant(w1e, 1).T
+                     + mx_fake_quant(da3, 1) @ mx_fake_quant(w3e, 1).T, staged)
+    else:
+        dxp = _stage(da1 @ w1e.T + da3 @ w3e.T, staged)
     return ds, da1, da3, ga, dxp
 
 
@@ -437,9 +445,10 @@ def _f64(a):
 def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True, precision="bf16"):
     """Forward (and, given dout, backward) quantities of the listed rows.
 
-    With precision "mxfp8" the forward GEMMs take MXFP8 operands; the backward
-    uses that forward's H and the unquantised x and weights (the quantisers
-    pass gradients straight through).
+    With precision "mxfp8" the forward GEMMs and the backward dX_perm GEMM
+    take MXFP8 operands; the backward uses that forward's H, and the gradients
+    pass the quantisers straight through (the other backward GEMMs use the
+    unquantised x, weights and staged intermediates).
 
     Rows are grouped by the expert that owns them; padding rows give zeros.
     w1, w3, w2 may be arrays or any object whose [e] gives expert e's matrix
@@ -466,7 +475,7 @@ def rows_compute(rows, plan, x, w1, w3, w2, dout=None, staged=True, precision="b
         if dout is not None:
             g = plan["row_gate"][rows[sel]]
             ds, da1, da3, ga, dxp = expert_rows_backward(
-                dout[toks], g, h1, h3, w1e, w3e, w2e, staged)
+                dout[toks], g, h1, h3, w1e, w3e, w2e, staged, precision)
             res["dS"][sel] = ds
             res["dH"][sel, :f], res["dH"][sel, f:] = da1, da3
             res["gA"][sel] = ga

@@ -692,5 +692,35 @@ def test_mxfp8_layer_equals_bf16_layer_on_the_mx_grid():
     assert np.abs(b["Y"] - a["Y"]).max() > 0             # A and W2 are not on the grid
     ga = O.layer_bwd(dout, x, wg, w1, w3, w2, a, staged=False)
     gb = O.layer_bwd(dout, x, wg, w1, w3, w2, b, staged=False)
-    for n in ("dx", "dw1", "dw3", "dw2", "dS", "dlogits"):   # same H, same STE backward
+    for n in ("dw1", "dw3", "dw2", "dS", "dlogits"):   # same H, straight-through backward
         np.testing.assert_allclose(gb[n], ga[n], rtol=1e-12, atol=1e-12)
+    # dX_perm takes MXFP8 dH and W1/W3 (blocks along f): exactly the dH rows
+    # of the unquantised backward, quantised, times the quantised weights
+    f = w1.shape[2]
+    for r in range(R):
+        e, t = O.row_expert(b["plan"], [r])[0], b["plan"]["row_token"][r]
+        if t < 0:
+            continue
+        dh = ga["dH"][r:r + 1]
+        want = (O.mx_fake_quant(dh[:, :f], 1) @ O.mx_fake_quant(w1[e], 1).T
+                + O.mx_fake_quant(dh[:, f:], 1) @ O.mx_fake_quant(w3[e], 1).T)
+        np.testing.assert_allclose(gb["dXp"][r], want[0], rtol=1e-12, atol=1e-14)
+
+
+
+def test_mx_fake_quant_matches_torch_float8_along_either_axis():
+    """The MXFP8 image of a matrix, blocks along rows or columns, against an
+    independent torch construction: per-block maximum, scale 2^(e-9) from
+    torch.frexp (max = m 2^e, m in [0.5, 1)), clamp to +-448 and torch's
+    float8_e4m3fn rounding."""
+    rng = np.random.default_rng(34)
+    a = rng.standard_normal((64, 96)) * np.exp(rng.uniform(-6, 6, (64, 1)))
+    for axis in (0, 1):
+        t = torch.from_numpy(np.moveaxis(a, axis, -1).copy())
+        blk = t.reshape(*t.shape[:-1], -1, 32)
+        amax = blk.abs().amax(-1, keepdim=True)
+        _, ex = torch.frexp(amax)
+        scale = torch.pow(2.0, (ex - 9).to(torch.float64))
+        q = (blk / scale).clamp(-448, 448).to(torch.float8_e4m3fn).to(torch.float64)
+        ref = np.moveaxis((q * scale).reshape(t.shape).numpy(), -1, axis)
+        np.testing.assert_array_equal(O.mx_fake_quant(a, axis), ref)
