@@ -49,7 +49,8 @@ def parse_args():
     ap.add_argument("--capacity-factor", type=float, default=1.0,
                     help="tokens per expert = ceil(factor * T * k / E) with --round 2")
     ap.add_argument("--precision", choices=["bf16", "mxfp8"], default="bf16",
-                    help="mxfp8: forward expert GEMMs on MXFP8 operands (weights quantised in the step)")
+                    help="mxfp8: forward expert GEMMs and the backward dX GEMM on MXFP8 operands "
+                         "(weights quantised in the step)")
     ap.add_argument("--noise-std", type=float, default=0.0,
                     help="noisy top-k gating: Gaussian routing noise of this std on the scores")
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1],
@@ -87,6 +88,7 @@ def gemm_flops(kind, T, d, f, k):
         "tc_dw13": 2.0 * rows * d * 2 * f,
         "tc_up_mxfp8": 2.0 * rows * d * 2 * f,
         "tc_down_mxfp8": 2.0 * rows * f * d,
+        "tc_dx_mxfp8": 2.0 * rows * 2 * f * d,
     }.get(kind)
 
 
@@ -110,6 +112,7 @@ def gemm_bytes(kind, T, d, f, E, k):
         "tc_dw13": 2 * w * 2 + R * d * 2 + R * 2 * f * 2,
         "tc_up_mxfp8": 2 * w * 1.03125 + R * d * 1.03125 + R * 2 * f * 2 + R * f * 1.03125,
         "tc_down_mxfp8": w * 1.03125 + R * f * 1.03125 + R * d * 2,
+        "tc_dx_mxfp8": 2 * w * 1.03125 + R * 2 * f * 1.03125 + R * d * 2,
     }
     return b.get(kind)
 
@@ -442,7 +445,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if args.precision == "bf16" else "mxfp8 fwd GEMMs + bf16",
+        "dtype": "bf16" if args.precision == "bf16" else "mxfp8 (fwd + dX GEMMs) + bf16",
         "data": "synthetic (seeded; random-init weights N(0,0.02^2), x,dO ~ N(0,1))",
         "config": workload_config(cfg, args),
         "tflops_per_gpu": step_flops(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k) / (ms_per_step / 1e3) / 1e12,

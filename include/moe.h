@@ -201,18 +201,22 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
  * Scale arrays are 512-byte blocks [rows/128][K/128]; the scale of row r and
  * 32-element K-block j is byte (r%32)*16 + ((r/32)%4)*4 + (j%4) of its block.
  * The GEMMs run on the tcgen05 block-scaled tensor cores (kind::mxf8f6f4)
- * with fp32 accumulation; H and Y are bf16 as in moe_expert_ffn_fwd, and
- * moe_layer_bwd (bf16 weights, saved H) is the backward: the quantisers pass
+ * with fp32 accumulation; H and Y are bf16 as in moe_expert_ffn_fwd.  The
+ * backward is moe_layer_bwd (all bf16) or moe_layer_bwd_mxfp8, whose dX GEMM
+ * takes MXFP8 dH and W1/W3 (blocks along f); either way the quantisers pass
  * gradients straight through.
  *
- * moe_mxfp8_weight_sizes: sizes[4] out = bytes of W13q, W13s, W2q, W2s for
- *   E experts (d and f multiples of 128, else MOE_ERR_UNSUPPORTED).
+ * moe_mxfp8_weight_sizes: sizes[8] out = bytes of W13q, W13s, W2q, W2s,
+ *   W1r, W1r scales, W3r, W3r scales for E experts (d and f multiples of 128,
+ *   else MOE_ERR_UNSUPPORTED).
  * moe_mxfp8_quantize_weights: w1, w3 [E,d,f] and w2 [E,f,d] bf16 ->
  *   W13q [E, 2f, d] E4M3 (K = d contiguous; rows 256b..256b+127 are columns
  *   128b..128b+127 of W1 and rows 256b+128..256b+255 the same columns of W3),
- *   W13s its scales, W2q [E, d, f] E4M3 (K = f contiguous), W2s its scales.
- *   Run it once per weight update; caller-owned device buffers of the sizes
- *   above, 16-byte aligned.
+ *   W13s its scales, W2q [E, d, f] E4M3 (K = f contiguous), W2s its scales,
+ *   and, when w1rq.. are not NULL (all four or none), W1r / W3r [E, d, f]
+ *   E4M3 in the weights' own layout with blocks along f, for
+ *   moe_layer_bwd_mxfp8.  Run it once per weight update; caller-owned device
+ *   buffers of the sizes above, 16-byte aligned.
  * moe_expert_ffn_fwd_mxfp8: as moe_expert_ffn_fwd (bf16 x, same plan
  *   arguments, H [cap,2f] and Y_perm [cap,d] bf16 out) with the quantised
  *   weights; x rows are quantised while they are scattered and A in the
@@ -225,8 +229,29 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
 int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes);
 int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
                                int f, uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                               uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
                                void* stream);
 size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
+/*
+ * moe_layer_bwd_mxfp8 -- moe_layer_bwd (bf16 only) whose dX_perm GEMM runs
+ * on MXFP8 operands: the dA' epilogue also writes dH in E4M3 with blocks
+ * along 2f, and W1r/W3r come from moe_mxfp8_quantize_weights.  The other
+ * backward GEMMs, the router gradient and every output are as in
+ * moe_layer_bwd.  ws: at least moe_layer_bwd_mxfp8_workspace_size() bytes.
+ */
+size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
+int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate,
+                        const void* w1, const void* w3, const void* w2,
+                        const uint8_t* w1rq, const uint8_t* w1rs,
+                        const uint8_t* w3rq, const uint8_t* w3rs,
+                        const int32_t* idx, const float* gate, const float* gate_grad,
+                        const float* logits, int gate_mode, const int32_t* offsets,
+                        const int32_t* row_token, const float* row_gate,
+                        const int32_t* slot_row, const int32_t* extra_row, const void* H,
+                        int T, int d, int f, int E, int k, int router_grad,
+                        void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2,
+                        float* dS, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
 int moe_expert_ffn_fwd_mxfp8(const void* x, const uint8_t* w13q, const uint8_t* w13s,
                              const uint8_t* w2q, const uint8_t* w2s,
                              const int32_t* row_token, const int32_t* offsets,

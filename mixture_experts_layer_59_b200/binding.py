@@ -28,7 +28,7 @@ EXPORTS = [
     "moe_check_status", "moe_profile_enable", "moe_profile_report", "moe_permute_noalloc",
     "moe_balance_loss_workspace_size", "moe_balance_loss",
     "moe_mxfp8_weight_sizes", "moe_mxfp8_quantize_weights", "moe_ffn_fwd_mxfp8_workspace_size",
-    "moe_expert_ffn_fwd_mxfp8",
+    "moe_expert_ffn_fwd_mxfp8", "moe_layer_bwd_mxfp8_workspace_size", "moe_layer_bwd_mxfp8",
 ]
 
 _lib = None
@@ -59,7 +59,9 @@ _SIGS = {
     "moe_balance_loss_workspace_size": (_sz, [_i, _i, _i]),
     "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_mxfp8_weight_sizes": (_i, [_i, _i, _i, ctypes.POINTER(_sz)]),
-    "moe_mxfp8_quantize_weights": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp]),
+    "moe_mxfp8_quantize_weights": (_i, [_vp, _vp, _vp, _i, _i, _i] + [_vp] * 9),
+    "moe_layer_bwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "moe_layer_bwd_mxfp8": (_i, [_vp] * 14 + [_i] + [_vp] * 6 + [_i] * 6 + [_vp] * 8 + [_sz, _vp]),
     "moe_ffn_fwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "moe_expert_ffn_fwd_mxfp8": (_i, [_vp] * 9 + [_i] * 5 + [_vp, _vp, _vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
@@ -199,21 +201,27 @@ def moe_expert_ffn_fwd(x, w1, w3, w2, plan, k, H=None, Y_perm=None, ws=None, str
     return H, Y_perm
 
 
+MX_WEIGHT_NAMES = ("w13q", "w13s", "w2q", "w2s", "w1rq", "w1rs", "w3rq", "w3rs")
+
+
 def moe_mxfp8_weight_sizes(E, d, f):
-    """Bytes of (W13q, W13s, W2q, W2s)."""
-    sz = (_sz * 4)()
+    """Bytes of (W13q, W13s, W2q, W2s, W1r, W1r scales, W3r, W3r scales)."""
+    sz = (_sz * 8)()
     _check(lib().moe_mxfp8_weight_sizes(E, d, f, sz))
     return tuple(int(v) for v in sz)
 
 
-def moe_mxfp8_quantize_weights(w1, w3, w2, out=None, stream=None):
-    """MXFP8 copies of the expert weights: dict w13q, w13s, w2q, w2s (uint8)."""
+def moe_mxfp8_quantize_weights(w1, w3, w2, out=None, stream=None, backward=True):
+    """MXFP8 copies of the expert weights: dict w13q, w13s, w2q, w2s and, with
+    ``backward``, w1rq, w1rs, w3rq, w3rs (for moe_layer_bwd_mxfp8); uint8."""
     E, d, f = w1.shape
     o = dict(out) if out else {}
-    for name, n in zip(("w13q", "w13s", "w2q", "w2s"), moe_mxfp8_weight_sizes(E, d, f)):
+    names = MX_WEIGHT_NAMES if backward else MX_WEIGHT_NAMES[:4]
+    for name, n in zip(names, moe_mxfp8_weight_sizes(E, d, f)):
         o.setdefault(name, torch.empty(n, device=w1.device, dtype=torch.uint8))
+    r = [_p(o.get(n)) if backward else None for n in MX_WEIGHT_NAMES[4:]]
     _check(lib().moe_mxfp8_quantize_weights(_p(w1), _p(w3), _p(w2), E, d, f, _p(o["w13q"]),
-                                            _p(o["w13s"]), _p(o["w2q"]), _p(o["w2s"]),
+                                            _p(o["w13s"]), _p(o["w2q"]), _p(o["w2s"]), *r,
                                             _stream(stream)))
     return o
 
@@ -276,6 +284,41 @@ def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=T
         _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(idx), _p(gate), _p(gate_grad),
         _p(logits), gate_mode, _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
         _p(plan.get("extra_row")), _p(H), T, d, f, E, k, dt, 1 if router_grad else 0,
+        _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
+        _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k) -> int:
+    return lib().moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k)
+
+
+def moe_layer_bwd_mxfp8(dout, x, w_gate, w1, w3, w2, wq, idx, gate, plan, H, router_grad=True,
+                        out=None, ws=None, stream=None, gate_grad=None, logits=None,
+                        gate_mode=MOE_GATE_TOPK_SOFTMAX):
+    """moe_layer_bwd with the dX GEMM on MXFP8 operands.  wq: dict from
+    moe_mxfp8_quantize_weights (backward=True)."""
+    T, d = x.shape
+    E, _, f = w1.shape
+    k = idx.shape[1]
+    cap = moe_row_capacity(T, E, k)
+    dev = x.device
+    o = dict(out) if out else {}
+    o.setdefault("dx", torch.empty(T, d, device=dev, dtype=x.dtype))
+    o.setdefault("dw_gate", torch.empty(d, E, device=dev, dtype=torch.float32))
+    o.setdefault("dw1", torch.empty_like(w1))
+    o.setdefault("dw3", torch.empty_like(w3))
+    o.setdefault("dw2", torch.empty_like(w2))
+    o.setdefault("dS", torch.empty(cap, device=dev, dtype=torch.float32))
+    o.setdefault("dlogits", torch.empty(T, E, device=dev, dtype=torch.float32))
+    if ws is None:
+        ws = torch.empty(max(moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k), 1), device=dev,
+                         dtype=torch.uint8)
+    _check(lib().moe_layer_bwd_mxfp8(
+        _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(wq["w1rq"]), _p(wq["w1rs"]),
+        _p(wq["w3rq"]), _p(wq["w3rs"]), _p(idx), _p(gate), _p(gate_grad), _p(logits), gate_mode,
+        _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
+        _p(plan.get("extra_row")), _p(H), T, d, f, E, k, 1 if router_grad else 0,
         _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
         _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
     return o

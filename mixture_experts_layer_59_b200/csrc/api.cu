@@ -313,20 +313,32 @@ int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes) {
   sizes[1] = 2 * n / 32;   // W13s
   sizes[2] = n;            // W2q
   sizes[3] = n / 32;       // W2s
+  sizes[4] = n;            // W1r (backward dX GEMM)
+  sizes[5] = n / 32;
+  sizes[6] = n;            // W3r
+  sizes[7] = n / 32;
   return MOE_OK;
 }
 
 int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
                                int f, uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                               uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
                                void* stream) {
-  size_t sz[4];
+  size_t sz[8];
   if (int rc = moe_mxfp8_weight_sizes(E, d, f, sz)) return rc;
   if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
   REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
   REQUIRE_PTR(w13q); REQUIRE_PTR(w13s); REQUIRE_PTR(w2q); REQUIRE_PTR(w2s);
   REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2);
   REQUIRE_ALIGNED(w13q); REQUIRE_ALIGNED(w13s); REQUIRE_ALIGNED(w2q); REQUIRE_ALIGNED(w2s);
-  return launch_mx_quant_weights(w1, w3, w2, E, d, f, w13q, w13s, w2q, w2s, (cudaStream_t)stream);
+  const bool bwd = w1rq != nullptr;
+  if (bwd != (w1rs != nullptr) || bwd != (w3rq != nullptr) || bwd != (w3rs != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "w1rq, w1rs, w3rq, w3rs must be all set or all NULL");
+  if (bwd) {
+    REQUIRE_ALIGNED(w1rq); REQUIRE_ALIGNED(w1rs); REQUIRE_ALIGNED(w3rq); REQUIRE_ALIGNED(w3rs);
+  }
+  return launch_mx_quant_weights(w1, w3, w2, E, d, f, w13q, w13s, w2q, w2s, w1rq, w1rs, w3rq,
+                                 w3rs, (cudaStream_t)stream);
 }
 
 size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k) {
@@ -386,14 +398,14 @@ size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype
   return z.used;
 }
 
-int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
+static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, const void* w1,
                   const void* w3, const void* w2, const int32_t* idx, const float* gate,
                   const float* gate_grad, const float* logits, int gate_mode,
                   const int32_t* offsets, const int32_t* row_token, const float* row_gate,
                   const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
                   int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
                   void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
-                  size_t ws_bytes, void* stream) {
+                  size_t ws_bytes, void* stream, const uint8_t* const* mxw) {
   if (int rc = check_common(T, E, k, dtype)) return rc;
   if (int rc = check_dims(d, f, dtype)) return rc;
   REQUIRE_PTR(dout); REQUIRE_PTR(x); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
@@ -407,11 +419,19 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   REQUIRE_ALIGNED(dout); REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3);
   REQUIRE_ALIGNED(w2); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(dx); REQUIRE_ALIGNED(dw1);
   REQUIRE_ALIGNED(dw3); REQUIRE_ALIGNED(dw2); REQUIRE_ALIGNED(ws);
-  if (ws_bytes < moe_layer_bwd_workspace_size(T, d, f, E, k, dtype))
-    return fail(MOE_ERR_WORKSPACE, "bwd workspace smaller than moe_layer_bwd_workspace_size()");
+  const size_t need = mxw ? moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k)
+                         : moe_layer_bwd_workspace_size(T, d, f, E, k, dtype);
+  if (ws_bytes < need)
+    return fail(MOE_ERR_WORKSPACE, "bwd workspace smaller than the matching *_workspace_size()");
   Carve c(ws, ws_bytes);
   BwdWs<Carve> w;
   w.carve(c, T, d, f, E, k, dtype);
+  MxBwd mx{};
+  if (mxw) {  // dH in MXFP8 for the dX GEMM, after the bf16 workspace
+    const size_t capr = ((size_t)T * k + (size_t)E * 128 + 127) / 128 * 128;
+    mx = MxBwd{mxw[0], mxw[1], mxw[2], mxw[3], c.take<uint8_t>(capr * 2 * f),
+               c.take<uint8_t>(capr * 2 * f / 32)};
+  }
   if (!c.ok) return fail(MOE_ERR_WORKSPACE, "bwd workspace too small");
   cudaStream_t s = (cudaStream_t)stream;
   FfnPtrs p{x, w1, w3, w2, row_token, offsets, T, d, f, E, (int)((size_t)T * k + (size_t)E * 128), dtype};
@@ -424,7 +444,7 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
                                   w.xg, s)))
       return rc;
     if ((rc = tc_ffn_bwd(p, w.dog, w.xg, row_gate, H, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2,
-                         device_sm_count(), s)))
+                         device_sm_count(), s, mxw ? &mx : nullptr)))
       return rc;
   } else {
     if ((rc = simt_ffn_bwd(p, dout, row_gate, H, w.dap, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2, s)))
@@ -463,6 +483,50 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
   if (e != cudaSuccess) return cuda_fail(e, "memset dw_gate");
   return launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false, false,
                              dx, s);
+}
+
+int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
+                  const void* w3, const void* w2, const int32_t* idx, const float* gate,
+                  const float* gate_grad, const float* logits, int gate_mode,
+                  const int32_t* offsets, const int32_t* row_token, const float* row_gate,
+                  const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
+                  int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
+                  void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
+                  size_t ws_bytes, void* stream) {
+  return layer_bwd_impl(dout, x, w_gate, w1, w3, w2, idx, gate, gate_grad, logits, gate_mode,
+                        offsets, row_token, row_gate, slot_row, extra_row, H, T, d, f, E, k, dtype,
+                        router_grad, dx, dw_gate, dw1, dw3, dw2, dS, dlogits, ws, ws_bytes, stream,
+                        nullptr);
+}
+
+size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k) {
+  if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0) return 0;
+  Sizer z;
+  BwdWs<Sizer> w;
+  w.carve(z, T, d, f, E, k, MOE_BF16);
+  const size_t capr = ((size_t)T * k + (size_t)E * 128 + 127) / 128 * 128;
+  z.take<uint8_t>(capr * 2 * f);
+  z.take<uint8_t>(capr * 2 * f / 32);
+  return z.used;
+}
+
+int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate, const void* w1,
+                        const void* w3, const void* w2, const uint8_t* w1rq, const uint8_t* w1rs,
+                        const uint8_t* w3rq, const uint8_t* w3rs, const int32_t* idx,
+                        const float* gate, const float* gate_grad, const float* logits,
+                        int gate_mode, const int32_t* offsets, const int32_t* row_token,
+                        const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
+                        const void* H, int T, int d, int f, int E, int k, int router_grad,
+                        void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2, float* dS,
+                        float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE_PTR(w1rq); REQUIRE_PTR(w1rs); REQUIRE_PTR(w3rq); REQUIRE_PTR(w3rs);
+  REQUIRE_ALIGNED(w1rq); REQUIRE_ALIGNED(w1rs); REQUIRE_ALIGNED(w3rq); REQUIRE_ALIGNED(w3rs);
+  if (!tc_available()) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 GEMMs need an sm_100 device");
+  const uint8_t* mxw[4] = {w1rq, w1rs, w3rq, w3rs};
+  return layer_bwd_impl(dout, x, w_gate, w1, w3, w2, idx, gate, gate_grad, logits, gate_mode,
+                        offsets, row_token, row_gate, slot_row, extra_row, H, T, d, f, E, k,
+                        MOE_BF16, router_grad, dx, dw_gate, dw1, dw3, dw2, dS, dlogits, ws,
+                        ws_bytes, stream, mxw);
 }
 
 int moe_profile_enable(int on) {

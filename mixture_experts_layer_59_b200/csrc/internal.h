@@ -87,9 +87,14 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
 int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const uint8_t* w13q,
                   const uint8_t* w13s, const uint8_t* w2q, const uint8_t* w2s, void* H,
                   uint8_t* actq, uint8_t* acts, void* Y, int num_sms, cudaStream_t s);
+// MXFP8 operands of the backward dX GEMM (null: bf16 dX GEMM).
+struct MxBwd {
+  const uint8_t *w1rq, *w1rs, *w3rq, *w3rs;   // W1, W3 [E, d, f] quantised along f
+  uint8_t *dhq, *dhs;                          // dH [cap, 2f] quantised along 2f (DAP writes it)
+};
 int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* row_gate,
                const void* H, void* dH, void* gact, float* ds_part, void* dXp, void* dw1,
-               void* dw3, void* dw2, int num_sms, cudaStream_t s);
+               void* dw3, void* dw2, int num_sms, cudaStream_t s, const MxBwd* mx = nullptr);
 int tc_num_dS_parts(int f);
 bool tc_router_ok(int E);
 int tc_dwg_splits(int T, int d, int* chunk);
@@ -105,6 +110,7 @@ int device_sm_count();
 // ---------------------------------------------------------------- MXFP8 (mx.cu, tc_gemm.cu)
 int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int E, int d, int f,
                             uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                            uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
                             cudaStream_t s);
 int launch_mx_scatter_rows(const void* x, const int32_t* slot_row, const int32_t* extra_row,
                            const int32_t* row_token, const int32_t* offsets, int T, int d, int E,

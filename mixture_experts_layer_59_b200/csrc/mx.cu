@@ -4,7 +4,9 @@
 //            256b..256b+127 are columns 128b.. of W1, rows 256b+128..256b+255
 //            the same columns of W3, so one 256-row GEMM tile yields
 //            matching H1 / H3 columns) and W2 [E, f, d] ->
-//            W2q [E, d, f] (K = f contiguous), blocks of 32 along K.
+//            W2q [E, d, f] (K = f contiguous), blocks of 32 along K; for the
+//            backward dX GEMM also W1r, W3r [E, d, f] (the weights' own
+//            layout, blocks of 32 along f), from the same loaded tiles.
 //   rows     x [T, d] -> Xq [cap, d]: each token row quantised once (blocks
 //            of 32 along d) and written to all of its rows in the row space;
 //            padding rows get zero elements and zero scales.
@@ -23,8 +25,12 @@ constexpr int WQ_THREADS = 512;
 template <bool W13>
 __global__ void __launch_bounds__(WQ_THREADS)
 k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __restrict__ wb,
-                   int K, int N, int Nout, uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
-  __shared__ __align__(16) __nv_bfloat16 tile[128][128];
+                   int K, int N, int Nout, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                   uint8_t* __restrict__ qa_r, uint8_t* __restrict__ sfa_r,
+                   uint8_t* __restrict__ qb_r, uint8_t* __restrict__ sfb_r) {
+  // rows padded by 16 bytes: the row-wise pass reads 16-byte vectors of
+  // consecutive rows without bank conflicts
+  __shared__ __align__(16) __nv_bfloat16 tile[128][136];
   const int k0 = blockIdx.x * 128, t = blockIdx.y, e = blockIdx.z;
   const int kchunks = K / 128;
   // source tile: 128 K-rows x 128 output rows (16-byte vectors of 8 bf16);
@@ -52,18 +58,37 @@ k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __
   const int row = e * Nout + t * 128 + n;   // output row across experts (Nout % 128 == 0)
   mx_store_block(v, q + (size_t)row * K + k0 + 32 * j,
                  sf + mx_sf_offset(row, (k0 >> 5) + j, kchunks));
+  if (W13 && qa_r != nullptr) {
+    // row-wise: source row k0 + kk of W1 (t even) or W3 (t odd), 32 columns
+    // starting at 128 (t/2) + 32 jb, in the weight's own [E, d, f] layout
+    const int kk = threadIdx.x & 127, jb = threadIdx.x >> 7;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 u = *reinterpret_cast<const uint4*>(&tile[kk][32 * jb + 8 * i]);
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v[8 * i + c] = __bfloat162float(h[c]);
+    }
+    const int srow = e * K + k0 + kk;         // row of [E*d, f]
+    const int col = (t >> 1) * 128 + 32 * jb;
+    uint8_t* qr = (t & 1) ? qb_r : qa_r;
+    uint8_t* sr = (t & 1) ? sfb_r : sfa_r;
+    mx_store_block(v, qr + (size_t)srow * N + col, sr + mx_sf_offset(srow, col >> 5, N / 128));
+  }
 }
 
 int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int E, int d, int f,
                             uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
+                            uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
                             cudaStream_t s) {
   if (E == 0) return MOE_OK;
   {
     ProfScope _ps("mx_quant_weights", s);
     k_mx_quant_weights<true><<<dim3(d / 128, (2 * f) / 128, E), WQ_THREADS, 0, s>>>(
-        (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w3, d, f, 2 * f, w13q, w13s);
+        (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w3, d, f, 2 * f, w13q, w13s, w1rq, w1rs,
+        w3rq, w3rs);
     k_mx_quant_weights<false><<<dim3(f / 128, d / 128, E), WQ_THREADS, 0, s>>>(
-        (const __nv_bfloat16*)w2, nullptr, f, d, d, w2q, w2s);
+        (const __nv_bfloat16*)w2, nullptr, f, d, d, w2q, w2s, nullptr, nullptr, nullptr, nullptr);
   }
   MOE_CHECK_LAUNCH("mx_quant_weights");
   return MOE_OK;

@@ -24,6 +24,9 @@
 //         Xq [W13q], epilogue as UP but A leaves as MXFP8 (blocks along f);
 //         256-column tiles (128 W1 + 128 W3 columns), one accumulator
 //   DOWNQ DOWN with MXFP8 operands: Aq W2q
+//   DXQ   DX with MXFP8 operands: dHq [W1r | W3r]^T (dH quantised along 2f by
+//         DAPQ, the weights along f in their own layout)
+//   DAPQ  DAP whose epilogue also writes dH as MXFP8 for DXQ
 //         (kind::mxf8f6f4 block-scaled MMAs, K = 32 per instruction; the two
 //         512-byte scale blocks of each stage go shared -> TMEM by tcgen05.cp)
 // The grouped GEMM replaces the per-expert loop of the Beam article's
@@ -55,9 +58,9 @@ using namespace tc;
 
 enum Kind : int {
   K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8,
-  K_UPQ = 9, K_DOWNQ = 10
+  K_UPQ = 9, K_DOWNQ = 10, K_DXQ = 11, K_DAPQ = 12
 };
-constexpr int NUM_KINDS = 11;
+constexpr int NUM_KINDS = 13;
 constexpr int MX_SF_COL = 256;         // TMEM column of the scale blocks (after the accumulators)
 
 constexpr int BM = 128;
@@ -107,6 +110,10 @@ struct TcArgs {
   int kchunks;               // K / 128
   uint8_t* act_q;            // UPQ: A as E4M3 [cap, f]
   uint8_t* act_s;            // UPQ: its scale blocks [cap/128][f/128]
+  uint8_t* dh_q;             // DAP (MXFP8 backward): dH as E4M3 [cap, 2f], or null
+  uint8_t* dh_s;             // its scale blocks [cap/128][2f/128]
+  const uint8_t* sfb1;       // DXQ: scale blocks of W3r (sfb: of W1r)
+  int kh;                    // DXQ: K chunks per weight half (f / 128)
 };
 
 template <int KIND> struct KT {
@@ -115,7 +122,7 @@ template <int KIND> struct KT {
   static constexpr bool B_MN = (KIND == K_UP || KIND == K_DOWN || VARLEN_K || KIND == K_RT ||
                                 KIND == K_DWG);
   static constexpr bool ROUTER = (KIND == K_RT || KIND == K_DWG || KIND == K_DXR);
-  static constexpr bool MX = (KIND == K_UPQ || KIND == K_DOWNQ);
+  static constexpr bool MX = (KIND == K_UPQ || KIND == K_DOWNQ || KIND == K_DXQ);
 };
 
 // A stage holds a 128 x 128-byte A tile and a BN x 128-byte B tile (64 bf16
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
     fence_mbar_init();
     prefetch_tmap(&a.mA);
     prefetch_tmap(&a.mB0);
-    if (KIND == K_UP || KIND == K_DX || KIND == K_DWG) prefetch_tmap(&a.mB1);
+    if (KIND == K_UP || KIND == K_DX || KIND == K_DWG || KIND == K_DXQ) prefetch_tmap(&a.mB1);
     if (KIND == K_DXR) prefetch_tmap(&a.mA1);
   }
   if (warp == 1) {
@@ -354,7 +361,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
 #pragma unroll
             for (int h = 0; h < BN / 64; ++h)
               tma_load_3d(sB + h * ATOM, &a.mB0, &full_bar[stage], ti.n0 + 64 * h, k0, ti.e);
-          } else if constexpr (KIND == K_DAP) {
+          } else if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
             tma_load_3d(sB, &a.mB0, &full_bar[stage], k0, ti.n0, ti.e);
           } else if constexpr (KIND == K_DX) {
@@ -383,15 +390,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           } else if constexpr (KT<KIND>::MX) {
             // E4M3 tiles: 128 elements of K = 128 bytes; then the A and B
             // scale blocks of this K chunk
+            // DXQ: K chunks [0, kh) come from W1r, [kh, 2kh) from W3r
+            const bool hi = KIND == K_DXQ && kb >= a.kh;
+            const int kk = hi ? kb - a.kh : kb;
+            const int kcs = KIND == K_DXQ ? a.kh : a.kchunks;
             tma_load_3d(sA, &a.mA, &full_bar[stage], kb * 128, ti.m0, 0);
-            tma_load_3d(sB, &a.mB0, &full_bar[stage], kb * 128, ti.n0, ti.e);
+            tma_load_3d(sB, hi ? &a.mB1 : &a.mB0, &full_bar[stage], kk * 128, ti.n0, ti.e);
             uint8_t* sSF = sB + C::B_BYTES;
             bulk_load(sSF, a.sfa + ((size_t)(ti.m0 / BM) * a.kchunks + kb) * 512, 512,
                       &full_bar[stage]);
+            const uint8_t* sfb = hi ? a.sfb1 : a.sfb;
 #pragma unroll
             for (int b = 0; b < BN / 128; ++b)
               bulk_load(sSF + 512 * (1 + b),
-                        a.sfb + ((size_t)(ti.e * (a.N / 128) + ti.n0 / 128 + b) * a.kchunks + kb) * 512,
+                        sfb + ((size_t)(ti.e * (a.N / 128) + ti.n0 / 128 + b) * kcs + kk) * 512,
                         512, &full_bar[stage]);
           } else if constexpr (KIND == K_DXR) {
             const int nkb = ti.kb_count / 2;
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       // loads are issued before waiting for the main loop
       uint4 hn1[4], hn3[4];
       const __nv_bfloat16* hrow = nullptr;
-      if constexpr (KIND == K_DAP) {
+      if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
         hrow = a.hin + (size_t)(ti.m0 + rloc) * 2 * a.f;
         const uint4* s1 = reinterpret_cast<const uint4*>(hrow + ti.n0 + half * (BN / 2));
         const uint4* s3 = reinterpret_cast<const uint4*>(hrow + a.f + ti.n0 + half * (BN / 2));
@@ -570,7 +582,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, nf + c, row0, lane);      // A
           }
         }
-      } else if constexpr (KIND == K_DOWN || KIND == K_DX || KIND == K_DOWNQ) {
+      } else if constexpr (KIND == K_DOWN || KIND == K_DX || KIND == K_DOWNQ || KIND == K_DXQ) {
         for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
           tmem_ld32(tbase + c, r);
           tmem_ld_wait();
@@ -578,7 +590,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);
         }
-      } else if constexpr (KIND == K_DAP) {
+      } else if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
         const int f = a.f;
         const float g = a.row_gate[row];
         float ds = 0.f;
@@ -612,6 +624,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           }
           stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
           stage_store<C::OUT_TILES>(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
+          if constexpr (KIND == K_DAPQ) {  // MXFP8 backward: dH blocks along 2f for the dX GEMM
+            const int kc = (2 * f) / 128;
+            mx_store_block(v, a.dh_q + (size_t)row * 2 * f + ti.n0 + c,
+                           a.dh_s + mx_sf_offset(row, (ti.n0 + c) / 32, kc));
+            mx_store_block(da3, a.dh_q + (size_t)row * 2 * f + f + ti.n0 + c,
+                           a.dh_s + mx_sf_offset(row, (f + ti.n0 + c) / 32, kc));
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);      // s * A
@@ -859,7 +878,8 @@ static int launch(const TcArgs& a, int grid, cudaStream_t s) {
   if (e != cudaSuccess) return cuda_fail(e, "tc gemm smem attribute");
   static const char* kNames[NUM_KINDS] = {
       "tc_up",   "tc_down",   "tc_dap",       "tc_dx",        "tc_dw2",   "tc_dw13",
-      "tc_router", "tc_router_dw", "tc_dx_router", "tc_up_mxfp8", "tc_down_mxfp8"};
+      "tc_router", "tc_router_dw", "tc_dx_router", "tc_up_mxfp8", "tc_down_mxfp8", "tc_dx_mxfp8",
+      "tc_dap"};
   static_assert(KIND >= 0 && KIND < NUM_KINDS, "kind out of range");
   {
     ProfScope _ps(kNames[KIND], s);
@@ -1062,7 +1082,7 @@ int tc_ffn_fwd_mx(const FfnPtrs& p, const uint8_t* xq, const uint8_t* xs, const 
 
 int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* row_gate,
                const void* H, void* dH, void* gact, float* ds_part, void* dXp, void* dw1,
-               void* dw3, void* dw2, int num_sms, cudaStream_t s) {
+               void* dw3, void* dw2, int num_sms, cudaStream_t s, const MxBwd* mx) {
   const int d = p.d, f = p.f, E = p.E, cap = p.cap;
   int rc;
   {  // DAP: dA' = dOg W2^T with the SwiGLU-backward epilogue
@@ -1077,11 +1097,38 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if ((rc = make_store_map(&a.sO0, dH, 2 * f, cap))) return rc;
     if ((rc = make_store_map(&a.sO1, gact, f, cap))) return rc;
     a.ds_part = ds_part;
+    if (mx != nullptr) {
+      a.dh_q = mx->dhq;
+      a.dh_s = mx->dhs;
+    }
     a.nparts = 2 * (f / bn);
     if (a.nparts != tc_num_dS_parts(f)) return fail(MOE_ERR_UNSUPPORTED, "dS partition mismatch");
-    if ((rc = launch_bn<K_DAP>(a, bn, num_sms, s))) return rc;
+    if (mx != nullptr) {
+      if ((rc = launch_bn<K_DAPQ>(a, bn, num_sms, s))) return rc;
+    } else if ((rc = launch_bn<K_DAP>(a, bn, num_sms, s))) {
+      return rc;
+    }
   }
-  {  // DX: dXp = dH [W1 | W3]^T
+  if (mx != nullptr) {  // DXQ: dXp = dHq [W1r | W3r]^T on the block-scaled tensor cores
+    TcArgs a = base_args(p);
+    a.N = d;
+    a.K = 2 * f;
+    a.kchunks = (2 * f) / 128;
+    a.kh = f / 128;
+    a.sfa = mx->dhs;
+    a.sfb = mx->w1rs;
+    a.sfb1 = mx->w3rs;
+    const int bn = pick_bn(d);
+    if ((rc = make_map_u8(&a.mA, mx->dhq, 2 * f, cap, 1, 128, BM))) return rc;
+    if ((rc = make_map_u8(&a.mB0, mx->w1rq, f, d, E, 128, bn))) return rc;
+    if ((rc = make_map_u8(&a.mB1, mx->w3rq, f, d, E, 128, bn))) return rc;
+    if ((rc = make_store_map(&a.sO0, dXp, d, cap))) return rc;
+    if (bn == 256) {
+      if ((rc = launch<K_DXQ, 256>(a, num_sms, s))) return rc;
+    } else if ((rc = launch<K_DXQ, 128>(a, num_sms, s))) {
+      return rc;
+    }
+  } else {  // DX: dXp = dH [W1 | W3]^T
     TcArgs a = base_args(p);
     a.N = d;
     a.K = 2 * f;

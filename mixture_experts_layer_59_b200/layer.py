@@ -42,13 +42,18 @@ class MoELayerStep:
         self.H, self.Y = e(cap, 2 * f, dt_=dtype), e(cap, d, dt_=dtype)
         self.out = e(T, d, dt_=dtype)
         self.ws_perm = e(max(B.moe_permute_workspace_size(T, E, k, round_mode), 1), dt_=torch.uint8)
-        self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
         if precision == "mxfp8":
             self.wq = {n: e(sz, dt_=torch.uint8) for n, sz in
-                       zip(("w13q", "w13s", "w2q", "w2s"), B.moe_mxfp8_weight_sizes(E, d, f))}
+                       zip(B.MX_WEIGHT_NAMES, B.moe_mxfp8_weight_sizes(E, d, f))}
             self.ws_mx = e(max(B.moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k), 1),
                            dt_=torch.uint8)
-        self.ws_bwd = e(max(B.moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1), dt_=torch.uint8)
+            self.ws_bwd = e(max(B.moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k), 1),
+                            dt_=torch.uint8)
+        else:
+            self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1),
+                            dt_=torch.uint8)
+            self.ws_bwd = e(max(B.moe_layer_bwd_workspace_size(T, d, f, E, k, dt), 1),
+                            dt_=torch.uint8)
         self.balance_lambda = balance_lambda
         if balance_lambda is not None:
             self.ws_bal = e(max(B.lib().moe_balance_loss_workspace_size(T, E, k), 1), dt_=torch.uint8)
@@ -105,8 +110,14 @@ class MoELayerStep:
 
     def backward(self, dout, stream=None):
         x, w_gate, w1, w3, w2 = self._saved
+        gate_grad = self.balance["dgate"] if self.balance else None
+        if self.precision == "mxfp8":   # dX GEMM on MXFP8 operands
+            return B.moe_layer_bwd_mxfp8(dout, x, w_gate, w1, w3, w2, self.wq, self.idx,
+                                         self.gate, self.plan, self.H, self.router_grad,
+                                         out=self.grads, ws=self.ws_bwd, stream=stream,
+                                         gate_grad=gate_grad, logits=self.logits,
+                                         gate_mode=self.gate_mode)
         return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
                                self.H, self.router_grad, out=self.grads, ws=self.ws_bwd,
-                               stream=stream,
-                               gate_grad=self.balance["dgate"] if self.balance else None,
-                               logits=self.logits, gate_mode=self.gate_mode)
+                               stream=stream, gate_grad=gate_grad, logits=self.logits,
+                               gate_mode=self.gate_mode)

@@ -68,6 +68,14 @@ def test_mxfp8_weight_quantisation_bitexact():
         rows = e * d + np.arange(d)
         off = sf_offset(rows[:, None], np.arange(f // 32)[None, :], f // 128)
         np.testing.assert_array_equal(w2s[off], scodes)
+        # W1r / W3r: the weights' own [d, f] layout, blocks along f
+        for src, qn, sn in ((w1, "w1rq", "w1rs"), (w3, "w3rq", "w3rs")):
+            q, se = O.mx_quantize(f64(src[e]), 1)
+            codes, scodes = expected_rows(q, se)            # [d, f], [d, f/32]
+            np.testing.assert_array_equal(u8(wq[qn]).reshape(E, d, f)[e], codes)
+            rows = e * d + np.arange(d)
+            off = sf_offset(rows[:, None], np.arange(f // 32)[None, :], f // 128)
+            np.testing.assert_array_equal(u8(wq[sn])[off], scodes)
     assert w13s[sf_offset(0 * 2 * f + 5, 0, d // 128)] == 0           # zero block -> code 0
     assert u8(wq["w2q"]).reshape(E, d, f)[0, 3, 64:96].tolist() == [0x7E] * 32   # 448
 
@@ -85,7 +93,7 @@ def _mx_layer(cfg, seed, round_mode):
     H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, cfg.k, cfg.E, cfg.f, ws=ws)
     out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], cfg.T, cfg.E,
                         cfg.k)
-    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H)
+    g = B.moe_layer_bwd_mxfp8(dout, x, wg, w1, w3, w2, wq, idx, gate, plan, H)
     B.moe_check_status()
     torch.cuda.synchronize()
     fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), cfg.k, round_mode=round_mode,
@@ -143,7 +151,7 @@ def test_mxfp8_forward_and_backward(round_mode):
     ok_blocks = np.repeat(same_scale, 32, axis=1)
     diff = ~same & ok_blocks
     assert np.all(np.abs(mag(got[live][diff]) - mag(acodes[live][diff])) <= 1)
-    # combined output and the straight-through backward
+    # combined output and the backward (dX GEMM on MXFP8 operands)
     assert_close(out, fwd["out"], "out", BF16_TOL)
     assert_close(f64(g["dS"])[:R][live], bwd["dS"][:R][live], "dS", BF16_TOL)
     for n in ("dlogits", "dx", "dw_gate", "dw1", "dw3", "dw2"):
@@ -178,7 +186,7 @@ def test_mxfp8_full_size_sampled_tokens(name, n_tok):
     wq = B.moe_mxfp8_quantize_weights(w1, w3, w2)
     H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, k, E, cfg.f)
     out = B.moe_combine(Y, plan["row_gate"], plan["slot_row"], plan["extra_row"], T, E, k)
-    g = B.moe_layer_bwd(dout, x, wg, w1, w3, w2, idx, gate, plan, H)
+    g = B.moe_layer_bwd_mxfp8(dout, x, wg, w1, w3, w2, wq, idx, gate, plan, H)
     B.moe_check_status()
     torch.cuda.synchronize()
     lg64 = lg.astype(np.float64)
