@@ -143,3 +143,27 @@ def test_balance_loss_rejects_empty_batch_and_small_workspace():
     f = ctypes.c_void_p(256)
     assert lib.moe_balance_loss(f, f, 0, 8, 2, 0.1, f, f, None, f, 1 << 20, None) == -1
     assert lib.moe_balance_loss(f, f, 100, 8, 2, 0.1, f, f, None, f, 4, None) == -5
+
+
+def test_mxfp8_entry_points_check_their_arguments():
+    lib = B.lib()
+    f = ctypes.c_void_p(256)
+    sizes = (ctypes.c_size_t * 8)()
+    assert lib.moe_mxfp8_weight_sizes(8, 2048, 1024, sizes) == 0
+    n = 8 * 2048 * 1024
+    assert list(sizes) == [2 * n, 2 * n // 32, n, n // 32, n, n // 32, n, n // 32]
+    assert lib.moe_mxfp8_weight_sizes(8, 2000, 1024, sizes) == -2       # d % 128 != 0
+    # the four backward outputs are all given or all NULL
+    rc = lib.moe_mxfp8_quantize_weights(f, f, f, 8, 256, 256, f, f, f, f, f, None, f, f, None)
+    assert rc == -1 and b"all set or all NULL" in lib.moe_last_error()
+    # forward: workspace too small is refused before any launch
+    rc = lib.moe_expert_ffn_fwd_mxfp8(f, f, f, f, f, f, f, f, None, 16, 256, 256, 8, 2, f, f, f,
+                                      16, None)
+    assert rc == -5
+    assert B.moe_ffn_fwd_mxfp8_workspace_size(16, 256, 256, 8, 2) > 0
+    # backward: the quantised weights are required
+    args = [f, f, f, f, f, f, None, f, f, f, f, f, None, None, 0, f, f, f, f, None, f, 16, 256,
+            256, 8, 2, 1, f, f, f, f, f, None, None, f, 1 << 40, None]
+    assert lib.moe_layer_bwd_mxfp8(*args) == -1 and b"w1rq" in lib.moe_last_error()
+    assert (B.moe_layer_bwd_mxfp8_workspace_size(16, 256, 256, 8, 2)
+            > B.moe_layer_bwd_workspace_size(16, 256, 256, 8, 2, B.MOE_BF16))
