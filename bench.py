@@ -141,6 +141,17 @@ def hbm_bytes(kind, T, d, f, E, k, launches):
     return None
 
 
+def activation_bytes(cfg, R):
+    """Bytes one layer keeps for its backward (H [R, 2f] bf16, logits, top-k
+    ids and gates, the row maps), against what storing the gathered x rows,
+    A and Y as well would add (the dS = <dA', A> backward needs none of them)."""
+    T, d, f, E, k = cfg.T, cfg.d, cfg.f, cfg.E, cfg.k
+    cap = T * k + E * 128
+    saved = R * 2 * f * 2 + T * E * 4 + T * k * 8 + cap * 12 + T * k * 4 + (E + 1) * 4
+    return {"saved": saved, "H": R * 2 * f * 2,
+            "if_x_perm_A_Y_were_kept": saved + R * d * 2 + R * f * 2 + R * d * 2}
+
+
 def step_flops(T, d, f, E, k, router=True):
     return 18.0 * T * k * d * f + 2.0 * T * k * f + (6.0 * T * d * E if router else 0.0)
 
@@ -492,6 +503,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "clocks": clocks,
         "gpu_launches": launches,
         "hbm_kernels": hbm_kernels,
+        "activation_bytes": activation_bytes(cfg, int(step.plan["offsets"][-1])),
         "kernels": kernels,
     }
     print(json.dumps(line), flush=True)
