@@ -27,7 +27,7 @@ Sources (cited by page title and section):
              distributed training" -- challenge 1, solution 1: load-balance
              loss L = lambda * CV(mean over the batch of G_i)^2.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * top-k then softmax over the k selected logits (sec. 5.3 / example 1); ties
     in the logits go to the lowest expert id.
   * experts are SwiGLU: A = silu(x W1) * (x W3), Y = A W2.
