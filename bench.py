@@ -117,6 +117,39 @@ def gemm_bytes(kind, T, d, f, E, k):
     return b.get(kind)
 
 
+# Per routed row: (FLOPs, row-space bytes), and weight matrices read per expert,
+# for each grouped GEMM (bf16 = 2 B, E4M3 + scales = 1.03125 B).
+def gemm_unit(kind, d, f):
+    q = 1.03125
+    return {
+        "tc_up": (4.0 * d * f, d * 2 + 2 * f * 2 + f * 2, 2 * 2),
+        "tc_down": (2.0 * d * f, f * 2 + d * 2, 1 * 2),
+        "tc_dap": (2.0 * d * f + 2 * f, d * 2 + 2 * f * 2 + 2 * f * 2 + f * 2, 1 * 2),
+        "tc_dx": (4.0 * d * f, 2 * f * 2 + d * 2, 2 * 2),
+        "tc_dw2": (2.0 * d * f, f * 2 + d * 2, 1 * 2),
+        "tc_dw13": (4.0 * d * f, d * 2 + 2 * f * 2, 2 * 2),
+        "tc_up_mxfp8": (4.0 * d * f, d * q + 2 * f * 2 + f * q, 2 * q),
+        "tc_down_mxfp8": (2.0 * d * f, f * q + d * 2, 1 * q),
+        "tc_dx_mxfp8": (4.0 * d * f, 2 * f * q + d * 2, 2 * q),
+    }.get(kind)
+
+
+def frac_roof_per_expert(gemm, rows_e, d, f, peak_tf, bw, steps):
+    """SURVEY-style roofline of the grouped-GEMM phase: per expert the slower of
+    its math and its bytes (its weights plus its rows), summed over experts and
+    launches, over the time the GEMMs took."""
+    ideal = 0.0
+    for n, (nl, tot_ms) in gemm.items():
+        u = gemm_unit(n, d, f)
+        if u is None:
+            continue
+        fl_row, by_row, wmats = u
+        p = peak_tf * peak_ratio(n) * 1e12
+        per_launch = sum(max(r * fl_row / p, (wmats * d * f + r * by_row) / bw) for r in rows_e)
+        ideal += per_launch * nl
+    return ideal / (sum(v[1] for v in gemm.values()) / 1e3)
+
+
 def hbm_bytes(kind, T, d, f, E, k, launches):
     """Algorithmic HBM bytes per launch of the memory-bound kernels (None for
     the latency-bound ones: permutation, router backward, reductions)."""
@@ -466,9 +499,19 @@ def run_ours(args, cfg, rank, world, local_rank):
         roof_s = sum(max(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) / (bf16_peak * peak_ratio(n) * 1e12),
                          gemm_bytes(n, cfg.T, cfg.d, cfg.f, cfg.E, cfg.k) / bw) * v[0]
                      for n, v in gemm.items())
+        # live rows per expert of the last plan (read after the timed region)
+        import numpy as np
+        counts = step.plan["counts"].cpu().numpy().astype(float)
+        if args.round == 1:
+            seg = step.plan["offsets"].cpu().numpy()
+            counts = (seg[1:] - seg[:-1]).astype(float)       # rounded counts are tile multiples
+        elif args.round == 2:
+            counts = np.minimum(counts, step.capacity)
         gemm_summary = {"tflops": g_fl / (g_ms / 1e3) / 1e12,
                         "frac_of_peak": ideal_s / (g_ms / 1e3),
                         "frac_roof": roof_s / (g_ms / 1e3),
+                        "frac_roof_per_expert": frac_roof_per_expert(
+                            gemm, counts, cfg.d, cfg.f, bf16_peak, bw, args.steps),
                         "ms_per_step": g_ms / args.steps}
     # memory-bound kernels: algorithmic bytes / live time vs the measured copy bandwidth
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
