@@ -145,7 +145,11 @@ def frac_roof_per_expert(gemm, rows_e, d, f, peak_tf, bw, steps):
             continue
         fl_row, by_row, wmats = u
         p = peak_tf * peak_ratio(n) * 1e12
-        per_launch = sum(max(r * fl_row / p, (wmats * d * f + r * by_row) / bw) for r in rows_e)
+        # an expert without rows reads no weights; the weight-gradient GEMMs
+        # still write its (zero) gradient
+        writes_all = n in ("tc_dw2", "tc_dw13")
+        per_launch = sum(max(r * fl_row / p, (wmats * d * f + r * by_row) / bw)
+                         for r in rows_e if r > 0 or writes_all)
         ideal += per_launch * nl
     return ideal / (sum(v[1] for v in gemm.values()) / 1e3)
 
