@@ -60,6 +60,7 @@ def parse_args():
     ap.add_argument("--ref-sample", type=int, default=256, help="tokens per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None, help="override T (profiling runs)")
+    ap.add_argument("--experts", type=int, default=None, help="override E (profiling runs)")
     ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer written between steps")
     ap.add_argument("--balance-loss", type=float, default=None,
                     help="add the load-balance loss (this lambda) and its gradient to every step")
@@ -565,6 +566,8 @@ def main():
         cfg = cfg.with_(routing=args.routing)
     if args.tokens:
         cfg = cfg.with_(T=args.tokens)
+    if args.experts:
+        cfg = cfg.with_(E=args.experts)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

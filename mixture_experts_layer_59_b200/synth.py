@@ -16,7 +16,11 @@ Workloads (all seeded, no datasets, no trained weights):
 Routing variants: ``learned`` (logits = x.W_gate), ``uniform`` (logits drawn
 i.i.d. U(0,1), the random-routing system benchmark), ``gauss`` (i.i.d. N(0,1)
 logits) and ``zipf`` (learned logits plus a per-expert bias -s*ln(rank_e),
-rank_e a seeded permutation of 1..E, which makes expert loads Zipf-skewed).
+rank_e a seeded permutation of 1..E, which makes expert loads Zipf-skewed)
+and ``balanced`` (token t scores experts (t*k + j) mod E, j < k, above all
+others, so every expert receives exactly T*k/E rows when E divides T*k: a
+load-balanced router, used to time the grouped GEMMs at a fixed row count
+per expert).
 """
 from __future__ import annotations
 
@@ -37,7 +41,7 @@ class MoEConfig:
     dtype: str = "bf16"          # "bf16" or "f32"
     init: str = "fixed"          # "fixed": N(0, std^2) everywhere; "fan_in": N(0, 1/fan_in)
     std: float = 0.02
-    routing: str = "learned"     # learned | uniform | gauss | zipf
+    routing: str = "learned"     # learned | uniform | gauss | zipf | balanced
     zipf_s: float = 1.1
 
     def with_(self, **kw) -> "MoEConfig":
@@ -108,6 +112,12 @@ def make_inputs(cfg: MoEConfig, seed: int = 0, device="cpu") -> dict:
         g = _gen(seed, "zipf_rank", "cpu")
         rank = torch.randperm(E, generator=g).to(torch.float64) + 1.0
         out["logit_bias"] = (-cfg.zipf_s * torch.log(rank)).to(torch.float32).to(device)
+    elif cfg.routing == "balanced":
+        t = torch.arange(T, device=device)
+        lo = torch.zeros((T, E), device=device, dtype=torch.float32)
+        for j in range(cfg.k):
+            lo[t, (t * cfg.k + j) % E] = 2.0 - 1e-3 * j
+        out["logits_override"] = lo
     elif cfg.routing != "learned":
         raise ValueError(f"unknown routing variant {cfg.routing!r}")
     return out

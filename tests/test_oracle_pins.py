@@ -724,3 +724,18 @@ def test_mx_fake_quant_matches_torch_float8_along_either_axis():
         q = (blk / scale).clamp(-448, 448).to(torch.float8_e4m3fn).to(torch.float64)
         ref = np.moveaxis((q * scale).reshape(t.shape).numpy(), -1, axis)
         np.testing.assert_array_equal(O.mx_fake_quant(a, axis), ref)
+
+
+def test_balanced_routing_gives_equal_expert_loads():
+    """The `balanced` synthetic router sends exactly T*k/E rows to every
+    expert (each token's k experts distinct), so grouped-GEMM timings at a
+    fixed row count per expert can use it."""
+    from mixture_experts_layer_59_b200 import synth
+    for T, E, k in ((512, 16, 8), (96, 8, 4), (64, 64, 1)):
+        cfg = synth.CONFIGS["coarse"].with_(T=T, d=64, f=64, E=E, k=k, routing="balanced")
+        inp = synth.make_inputs(cfg, seed=0)
+        _, idx, gate = O.route(None, None, k, logits_override=inp["logits_override"].numpy())
+        assert all(len(set(r)) == k for r in idx.tolist())
+        counts = np.bincount(idx.ravel(), minlength=E)
+        assert (counts == T * k // E).all()
+        np.testing.assert_allclose(gate.sum(axis=1), 1.0, rtol=0, atol=1e-12)
