@@ -136,7 +136,7 @@ def gemm_unit(kind, d, f):
 
 
 def frac_roof_per_expert(gemm, rows_e, d, f, peak_tf, bw, steps):
-    """SURVEY-style roofline of the grouped-GEMM phase: per expert the slower of
+    """Per-expert roofline of the grouped-GEMM phase: per expert the slower of
     its math and its bytes (its weights plus its rows), summed over experts and
     launches, over the time the GEMMs took."""
     ideal = 0.0
