@@ -41,6 +41,32 @@ def test_route_learned_logits_and_topk():
     np.testing.assert_allclose(f64(gate), g_ref, rtol=1e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("T,d,E,k,gate_mode,extras", [
+    (1000, 2048, 8, 4, 0, False), (4109, 2048, 8, 2, 1, True), (333, 256, 4, 2, 0, True),
+    (77, 512, 5, 5, 1, False), (31, 1024, 8, 8, 0, True), (1, 768, 2, 1, 0, False)])
+def test_route_small_e_learned(T, d, E, k, gate_mode, extras):
+    """Learned routing with few experts (the tensor-core router at E = 8, the
+    generic logits + top-k kernels otherwise), bias, noise and both gate
+    modes, ragged T.  Logits against the oracle's fp64 product of the same
+    bf16 inputs; choice and gates against the oracle fed the GPU's own
+    logits."""
+    cfg = _cfg(T, d, 64, E, k, std=0.05)
+    inp = synth.make_inputs(cfg, seed=17 + T, device="cuda")
+    bias = torch.linspace(-0.2, 0.3, E, device="cuda") if extras else None
+    noise = synth.logit_noise(T, E, 0.3, seed=T, device="cuda") if extras else None
+    logits, idx, gate = B.moe_route(inp["x"], inp["w_gate"], k, logit_bias=bias,
+                                    logit_noise=noise, gate_mode=gate_mode)
+    torch.cuda.synchronize()
+    ref_l, _, _ = O.route(f64(inp["x"]), f64(inp["w_gate"]), k,
+                          logit_bias=None if bias is None else f64(bias),
+                          logit_noise=None if noise is None else f64(noise))
+    scale = np.abs(ref_l).max()
+    np.testing.assert_allclose(f64(logits), ref_l, atol=1e-5 * scale, rtol=0)
+    _, ridx, rgate = O.route(None, None, k, logits_override=f64(logits), gate_mode=gate_mode)
+    np.testing.assert_array_equal(i64(idx), ridx)
+    np.testing.assert_allclose(f64(gate), rgate, rtol=2e-6, atol=1e-7)
+
+
 @pytest.mark.parametrize("E,k", [(8, 2), (64, 8), (256, 8), (5, 5), (33, 3)])
 def test_route_override_ties_bitexact(E, k):
     T = 777
