@@ -130,41 +130,91 @@ __global__ void k_perm_count(const int32_t* __restrict__ idx, int T, int E, int 
 }
 
 // Single block: per-expert running sums over blocks, padded exclusive scan
-// over experts, padding rows.
-__global__ void k_perm_scan(const int32_t* __restrict__ blockcnt, int nb, int E, int tile,
-                            int32_t* __restrict__ blockbase, int32_t* __restrict__ counts,
-                            int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
-                            float* __restrict__ row_gate, int32_t* __restrict__ row_slot) {
+// over experts, padding rows.  With few experts warp w scans the block
+// counts of experts w, w + 32, ... (lanes over blocks, shuffle scans); with
+// many, a thread per expert walks the blocks (reads coalesced over experts).
+// Warp 0 then scans the tile-padded totals over experts.
+__device__ __forceinline__ int warp_incl_scan(int v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(512)
+k_perm_scan(const int32_t* __restrict__ blockcnt, int nb, int E, int tile,
+            int32_t* __restrict__ blockbase, int32_t* __restrict__ counts,
+            int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+            float* __restrict__ row_gate, int32_t* __restrict__ row_slot) {
   __shared__ int s_cnt[256];
   __shared__ int s_off[257];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int b = 0; b < nb; ++b) {
-      blockbase[(size_t)b * E + e] = run;
-      run += blockcnt[(size_t)b * E + e];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // blockbase = running count within the expert (the segment offset is added below)
+  if (E <= 16) {   // few experts: lanes over blocks, shuffle scans
+    for (int e = warp; e < E; e += nw) {
+      int base = 0;
+      for (int b0 = 0; b0 < nb; b0 += 32) {
+        const int b = b0 + lane;
+        const int c = b < nb ? blockcnt[(size_t)b * E + e] : 0;
+        const int incl = warp_incl_scan(c, lane);
+        if (b < nb) blockbase[(size_t)b * E + e] = base + incl - c;
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) {
+        s_cnt[e] = base;
+        counts[e] = base;
+      }
     }
-    s_cnt[e] = run;
-    counts[e] = run;
+  } else {         // many experts: a thread per expert, coalesced over experts
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int run = 0, b = 0;
+      for (; b + 8 <= nb; b += 8) {
+        int c[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[j] = blockcnt[(size_t)(b + j) * E + e];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          blockbase[(size_t)(b + j) * E + e] = run;
+          run += c[j];
+        }
+      }
+      for (; b < nb; ++b) {
+        const int c = blockcnt[(size_t)b * E + e];
+        blockbase[(size_t)b * E + e] = run;
+        run += c;
+      }
+      s_cnt[e] = run;
+      counts[e] = run;
+    }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int acc = 0;
-    for (int e = 0; e < E; ++e) {
-      s_off[e] = acc;
-      acc += (s_cnt[e] + tile - 1) / tile * tile;
+  if (warp == 0) {
+    int run = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int p = e < E ? (s_cnt[e] + tile - 1) / tile * tile : 0;
+      const int incl = warp_incl_scan(p, lane);
+      if (e < E) s_off[e] = run + incl - p;
+      run += __shfl_sync(0xffffffffu, incl, 31);
     }
-    s_off[E] = acc;
+    if (lane == 0) s_off[E] = run;
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = s_off[e];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int o = s_off[e];
-    for (int b = 0; b < nb; ++b) blockbase[(size_t)b * E + e] += o;
+  if (E <= 16) {
+    for (int e = warp; e < E; e += nw) {
+      const int o = s_off[e];
+      for (int b = lane; b < nb; b += 32) blockbase[(size_t)b * E + e] += o;
+    }
+  } else {
+    for (int i = threadIdx.x; i < nb * E; i += blockDim.x) blockbase[i] += s_off[i % E];
   }
-  // padding rows of every segment
-  for (int e = 0; e < E; ++e) {
-    int lo = s_off[e] + s_cnt[e], hi = s_off[e + 1];
-    for (int r = lo + threadIdx.x; r < hi; r += blockDim.x) {
+  // padding rows of every segment (fewer than `tile` per expert): a warp per expert
+  for (int e = warp; e < E; e += nw) {
+    const int lo = s_off[e] + s_cnt[e], hi = s_off[e + 1];
+    for (int r = lo + lane; r < hi; r += 32) {
       row_token[r] = -1;
       row_gate[r] = 0.f;
       row_slot[r] = -1;
@@ -260,8 +310,8 @@ int launch_permute_exact(const int32_t* idx, const float* gate, int T, int E, in
   }
   {
     ProfScope _ps("perm_scan", s);
-    k_perm_scan<<<1, 256, 0, s>>>(w.blockcnt, nb, E, tile, w.blockbase, counts, offsets, row_token,
-                                  row_gate, row_slot);
+    k_perm_scan<<<1, 512, 0, s>>>(w.blockcnt, nb, E, tile, w.blockbase, counts, offsets,
+                                   row_token, row_gate, row_slot);
   }
   MOE_CHECK_LAUNCH("perm_scan");
   if (nb > 0) {

@@ -516,6 +516,7 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
       const int r = slot_row[(size_t)t * k + lane];
       if (r >= 0) {
         float ds = 0.f;
+#pragma unroll 4
         for (int p = 0; p < nparts; ++p) ds += ds_part[(size_t)r * nparts + p];
         if (dS_out) dS_out[r] = ds;
         const float v = row_gate[r] * ds;
@@ -528,6 +529,7 @@ __global__ void k_router_bwd(const float* __restrict__ ds_part, int nparts,
         const int r = extra_row[(size_t)t * E + e];
         if (r >= 0) {
           float ds = 0.f;
+#pragma unroll 4
           for (int p = 0; p < nparts; ++p) ds += ds_part[(size_t)r * nparts + p];
           if (dS_out) dS_out[r] = ds;
           const float v = row_gate[r] * ds;
