@@ -1,0 +1,120 @@
+"""Host logic of bench.py (no GPU): the FLOP and byte model behind its
+roofline fields, checked against the per-config totals printed in the scope
+table (fwd + bwd FLOPs = 18 k d f T + 2 k f T + 6 d E T) and against the
+closed forms each model is built from."""
+import math
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+BF16_KINDS = ["tc_up", "tc_down", "tc_dap", "tc_dx", "tc_dw2", "tc_dw13"]
+MX_KINDS = ["tc_up_mxfp8", "tc_down_mxfp8", "tc_dx_mxfp8"]
+
+# (T, d, f, E, k) and the printed fwd+bwd TFLOP of each bf16 workload
+WORKLOADS = {
+    "coarse": ((16384, 2048, 1024, 8, 4), 2.48),
+    "pool": ((16384, 2048, 1024, 128, 4), 2.50),
+    "fine": ((32768, 1536, 256, 64, 8), 1.88),
+    "sparse": ((8192, 7168, 2048, 256, 8), 17.4),
+}
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_step_flops_match_the_printed_totals(name):
+    (T, d, f, E, k), tflop = WORKLOADS[name]
+    # the totals are printed to three significant figures
+    assert bench.step_flops(T, d, f, E, k) / 1e12 == pytest.approx(tflop, rel=5e-3)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_grouped_gemm_flops_add_up_to_the_layer_without_router(name):
+    (T, d, f, E, k), _ = WORKLOADS[name]
+    total = sum(bench.gemm_flops(n, T, d, f, k) for n in BF16_KINDS)
+    assert total == pytest.approx(bench.step_flops(T, d, f, E, k, router=False), rel=1e-12)
+    # forward: up + down = 6 d f per row; backward twice that plus the dS dot products
+    R = T * k
+    fwd = bench.gemm_flops("tc_up", T, d, f, k) + bench.gemm_flops("tc_down", T, d, f, k)
+    assert fwd == 6.0 * d * f * R
+    assert total - fwd == 12.0 * d * f * R + 2.0 * f * R
+
+
+@pytest.mark.parametrize("kind", BF16_KINDS + MX_KINDS)
+def test_per_row_model_agrees_with_per_launch_model(kind):
+    T, d, f, E, k = 4096, 1536, 512, 16, 4
+    R = T * k
+    fl_row, by_row, wmats = bench.gemm_unit(kind, d, f)
+    assert bench.gemm_flops(kind, T, d, f, k) == pytest.approx(R * fl_row, rel=1e-12)
+    assert bench.gemm_bytes(kind, T, d, f, E, k) == pytest.approx(
+        R * by_row + wmats * E * d * f, rel=1e-12)
+
+
+def test_mxfp8_kinds_do_the_bf16_math_at_twice_the_peak():
+    T, d, f, k = 1024, 2048, 1024, 4
+    for mx, bf in zip(MX_KINDS, ["tc_up", "tc_down", "tc_dx"]):
+        assert bench.gemm_flops(mx, T, d, f, k) == bench.gemm_flops(bf, T, d, f, k)
+        assert bench.peak_ratio(mx) == 2.0 and bench.peak_ratio(bf) == 1.0
+        # E4M3 operands with one scale byte per 32 elements: 33/32 bytes each
+        assert bench.gemm_bytes(mx, T, d, f, 8, k) < bench.gemm_bytes(bf, T, d, f, 8, k)
+
+
+def test_memory_bound_kernel_bytes_coarse():
+    T, d, f, E, k = 16384, 2048, 1024, 8, 4
+    R = T * k
+    # row scatter: each x row read once and written to its k rows
+    assert bench.hbm_bytes("scatter_rows", T, d, f, E, k, 3) == 67108864 + 268435456
+    # combine: the R gathered rows (and their weights) read, T rows written
+    assert bench.hbm_bytes("token_reduce", T, d, f, E, k, 1) == R * d * 2 + R * 4 + T * d * 2
+    # two launches: the bf16 combine and the fp32 row sums of dX_perm, averaged
+    two = bench.hbm_bytes("token_reduce", T, d, f, E, k, 2)
+    assert two == ((R * d * 2 + R * 4 + T * d * 2) + (R * d * 2 + T * d * 4)) / 2
+    # router: x once, W_gate once, logits and the (idx, gate) pairs written
+    assert bench.hbm_bytes("tc_router", T, d, f, E, k, 1) == T * d * 2 + d * E * 2 + T * E * 4 + T * k * 8
+    # latency-bound kernels carry no byte model
+    for n in ("perm_scan", "perm_count", "perm_scatter", "router_bwd", "dwg_reduce"):
+        assert bench.hbm_bytes(n, T, d, f, E, k, 1) is None
+
+
+def test_per_expert_roofline_closed_forms():
+    d, f = 1024, 512
+    peak_tf, bw = 1000.0, 5e12
+    p = peak_tf * 1e12
+    fl_row, by_row, wmats = bench.gemm_unit("tc_up", d, f)
+    # one launch of 1 ms; a single expert with many rows is math-bound
+    rows = [100000]
+    frac = bench.frac_roof_per_expert({"tc_up": (1, 1.0)}, rows, d, f, peak_tf, bw, 1)
+    assert frac == pytest.approx(rows[0] * fl_row / p / 1e-3, rel=1e-12)
+    # a single row is weight-bound: the expert's weights plus the row's bytes
+    frac = bench.frac_roof_per_expert({"tc_up": (1, 1.0)}, [1], d, f, peak_tf, bw, 1)
+    assert frac == pytest.approx((wmats * d * f + by_row) / bw / 1e-3, rel=1e-12)
+    # an expert without rows costs nothing in the forward GEMMs ...
+    a = bench.frac_roof_per_expert({"tc_up": (1, 1.0)}, [64, 0, 0], d, f, peak_tf, bw, 1)
+    b = bench.frac_roof_per_expert({"tc_up": (1, 1.0)}, [64], d, f, peak_tf, bw, 1)
+    assert a == pytest.approx(b, rel=1e-12)
+    # ... but the weight-gradient GEMMs still write its (zero) gradient
+    wmats2 = bench.gemm_unit("tc_dw2", d, f)[2]
+    a = bench.frac_roof_per_expert({"tc_dw2": (1, 1.0)}, [64, 0], d, f, peak_tf, bw, 1)
+    b = bench.frac_roof_per_expert({"tc_dw2": (1, 1.0)}, [64], d, f, peak_tf, bw, 1)
+    assert a - b == pytest.approx(wmats2 * d * f / bw / 1e-3, rel=1e-9)
+
+
+def test_activation_bytes_keep_h_but_not_y_or_a():
+    from mixture_experts_layer_59_b200 import synth
+    cfg = synth.CONFIGS["coarse"]
+    R = cfg.T * cfg.k
+    a = bench.activation_bytes(cfg, R)
+    assert a["H"] == R * 2 * cfg.f * 2
+    # storing the gathered x rows, A and Y as well would add R (2d + 2f + 2d) bytes
+    assert a["if_x_perm_A_Y_were_kept"] - a["saved"] == R * (cfg.d * 2 + cfg.f * 2 + cfg.d * 2)
+
+
+def test_capacity_rounds_up():
+    from mixture_experts_layer_59_b200 import binding as B
+    assert B.capacity_from_factor(16384, 8, 4, 1.0) == 8192
+    assert B.capacity_from_factor(1000, 8, 2, 1.25) == math.ceil(1.25 * 1000 * 2 / 8)
+    assert B.capacity_from_factor(10, 3, 1, 1.0) == 4
