@@ -329,6 +329,24 @@ def run_reference(args, cfg, rank, world):
     return 0
 
 
+def max_over_ranks(value, world, device="cpu"):
+    """The largest value over all ranks: the slowest replica sets the job's
+    time.  One all-reduce (MAX) on the default process group when world > 1."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens, steps, total_ms):
+    """Whole-job throughput: tokens every replica processed over the
+    slowest replica's time."""
+    return world * tokens * steps / (total_ms / 1e3)
+
+
 def workload_config(cfg, args):
     return {"workload": cfg.name, "T": cfg.T, "d_model": cfg.d, "d_ff": cfg.f, "E": cfg.E,
             "k": cfg.k, "routing": cfg.routing, "token_rounding": args.round == 1,
@@ -397,13 +415,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     clocks = sampler.stop(t0, t1)
     prof = B.moe_profile_report()
     B.moe_check_status()
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
     ms_per_step = total_ms / args.steps
-    value = world * cfg.T * args.steps / (total_ms / 1e3)
+    value = job_tokens_per_s(world, cfg.T, args.steps, total_ms)
 
     # ---- end to end through the public API with host buffers: every step
     # uploads its own inputs (x, dO) from pinned host memory and reads its
@@ -459,12 +473,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     if args.e2e_steps > 0:
         pipeline(3)                                     # warm-up
         e2e_ms = [pipeline(args.e2e_steps) / args.e2e_steps] * args.e2e_steps
-    e2e_total = sum(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e_value = world * cfg.T * len(e2e_ms) / (e2e_total / 1e3) if e2e_ms else None
+    e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
+    e2e_value = job_tokens_per_s(world, cfg.T, len(e2e_ms), e2e_total) if e2e_ms else None
     h2d = x.numel() * x.element_size() + dout.numel() * dout.element_size()
     d2h = step.out.numel() * step.out.element_size() * 2
 
