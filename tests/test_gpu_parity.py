@@ -85,7 +85,11 @@ def test_route_override_ties_bitexact(E, k):
 # ------------------------------------------------------------------ permutation
 
 @pytest.mark.parametrize("T,E,k", [(1, 8, 2), (255, 8, 2), (1000, 16, 4), (4097, 64, 8),
-                                   (3000, 256, 8), (300, 4, 4)])
+                                   (3000, 256, 8), (300, 4, 4),
+                                   # the block-count scan: several 32-block chunks with a
+                                   # ragged tail (few experts), a thread per expert with
+                                   # and without a tail of blocks (many experts)
+                                   (20000, 8, 4), (70000, 2, 2), (16384, 17, 3), (9000, 32, 8)])
 def test_permute_exact_bitexact(T, E, k):
     g = torch.Generator().manual_seed(T + E)
     lo = torch.randn(T, E, generator=g)
@@ -98,7 +102,8 @@ def test_permute_exact_bitexact(T, E, k):
 
 
 @pytest.mark.parametrize("T,E,k,skew", [(1000, 8, 2, 0.0), (1000, 8, 2, 1.5), (5000, 16, 4, 1.1),
-                                        (8192, 64, 8, 1.1), (3000, 256, 8, 1.1), (200, 8, 2, 0.0)])
+                                        (8192, 64, 8, 1.1), (3000, 256, 8, 1.1), (200, 8, 2, 0.0),
+                                        (20000, 8, 4, 1.1)])
 def test_permute_rounded_bitexact(T, E, k, skew):
     g = torch.Generator().manual_seed(7 * T + E)
     lo = torch.randn(T, E, generator=g)
