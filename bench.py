@@ -190,6 +190,21 @@ def activation_bytes(cfg, R):
             "if_x_perm_A_Y_were_kept": saved + R * d * 2 + R * f * 2 + R * d * 2}
 
 
+def routing_stats(counts, offsets, row_token, row_slot, slot_row):
+    """Load and row-space statistics of one permutation plan (host arrays):
+    the busiest expert's load over the mean (before rounding or dropping),
+    rows of the padded row space, rows holding a token, padding rows, slots
+    dropped (by rounding or the capacity) and rows added by rounding."""
+    import numpy as np
+    counts = np.asarray(counts, np.float64)
+    R = int(offsets[-1])
+    live = np.asarray(row_token[:R]) >= 0
+    return {"max_over_mean_load": float(counts.max() / counts.mean()) if counts.mean() > 0 else None,
+            "rows": R, "live_rows": int(live.sum()), "padding_rows": int(R - live.sum()),
+            "dropped_slots": int((np.asarray(slot_row) < 0).sum()),
+            "added_rows": int((live & (np.asarray(row_slot[:R]) < 0)).sum())}
+
+
 def step_flops(T, d, f, E, k, router=True):
     return 18.0 * T * k * d * f + 2.0 * T * k * f + (6.0 * T * d * E if router else 0.0)
 
@@ -562,6 +577,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "gpu_launches": launches,
         "hbm_kernels": hbm_kernels,
         "activation_bytes": activation_bytes(cfg, int(step.plan["offsets"][-1])),
+        "routing_stats": routing_stats(*(step.plan[n].cpu().numpy() for n in
+                                         ("counts", "offsets", "row_token", "row_slot", "slot_row"))),
         "kernels": kernels,
     }
     print(json.dumps(line), flush=True)

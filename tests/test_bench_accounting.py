@@ -118,3 +118,31 @@ def test_capacity_rounds_up():
     assert B.capacity_from_factor(16384, 8, 4, 1.0) == 8192
     assert B.capacity_from_factor(1000, 8, 2, 1.25) == math.ceil(1.25 * 1000 * 2 / 8)
     assert B.capacity_from_factor(10, 3, 1, 1.0) == 4
+
+
+@pytest.mark.parametrize("round_mode", [0, 1, 2])
+def test_routing_stats_against_the_oracle_plan(round_mode):
+    """Counting from the row maps agrees with the oracle's own bookkeeping of
+    dropped and added pairs."""
+    import numpy as np
+    import torch
+    from oracle import moe_oracle as O
+    T, E, k = 3000, 16, 4
+    g = torch.Generator().manual_seed(3)
+    lo = torch.randn(T, E, generator=g).double()
+    lo = lo + (-1.1 * torch.log(torch.randperm(E, generator=g).double() + 1))[None, :]
+    _, idx, gate = O.route(None, None, k, logits_override=lo.numpy())
+    cap = int(math.ceil(1.0 * T * k / E))
+    plan = O.make_plan(idx, gate, lo.numpy(), E, round_mode=round_mode,
+                       capacity=cap if round_mode == 2 else None)
+    st = bench.routing_stats(plan["counts"], plan["offsets"], plan["row_token"],
+                             plan["row_slot"], plan["slot_row"])
+    counts = np.bincount(idx.ravel(), minlength=E)
+    assert st["max_over_mean_load"] == pytest.approx(counts.max() / counts.mean())
+    dropped = int(plan["dropped"].sum()) if round_mode else 0
+    added = int(plan["added"].sum()) if round_mode == 1 else 0
+    assert st["dropped_slots"] == dropped and st["added_rows"] == added
+    assert st["live_rows"] == T * k - dropped + added
+    assert st["rows"] == plan["R"] and st["padding_rows"] == plan["R"] - st["live_rows"]
+    if round_mode == 1:
+        assert st["padding_rows"] == 0          # rounded segments are whole tiles
