@@ -435,3 +435,29 @@ def test_mxfp8_degenerate_routing_shapes(T, E, k):
     fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), k,
                       logits_override=lg.astype(np.float64), precision="mxfp8")
     assert_close(out, fwd["out"], "out", BF16_TOL)
+
+
+def test_device_check_reports_and_clears():
+    """Failure detection without a GPU fault: expert ids out of range are
+    flagged by the permutation kernels (device status word, code 0x120) and
+    skipped; moe_check_status reports the flag once, then it is clear, and the
+    valid slots are still placed."""
+    T, E, k = 500, 8, 2
+    g = torch.Generator().manual_seed(41)
+    lo = torch.randn(T, E, generator=g)
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo.cuda(), T=T, E=E)
+    torch.cuda.synchronize()
+    bad = idx.clone()
+    bad[3, 0] = E          # one past the last expert
+    bad[77, 1] = -3
+    plan = B.moe_permute(bad, gate, logits, E, B.MOE_ROUND_NONE)
+    with pytest.raises(B.MoEError) as ei:
+        B.moe_check_status()
+    assert ei.value.code == -4 and "0x120" in str(ei.value)
+    B.moe_check_status()   # cleared by the read
+    slot_row = i64(plan["slot_row"]).reshape(T, k)
+    assert slot_row[3, 0] == -1 and slot_row[77, 1] == -1
+    valid = i64(bad) >= 0
+    valid &= i64(bad) < E
+    assert (slot_row[valid] >= 0).all()
+    assert int(i64(plan["counts"]).sum()) == int(valid.sum())
