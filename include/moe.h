@@ -27,6 +27,8 @@
  *     allocated and owned by the caller, row-major and contiguous.  The
  *     library allocates no device memory; scratch comes from a caller
  *     workspace whose size the matching *_workspace_size() call returns.
+ *     The one exception is moe_permute_noalloc, whose scratch is a static
+ *     512 KiB device array that every device loading the library keeps.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
  *     enqueue kernels on it; none synchronises or copies routing metadata to
  *     the host, so the row count R lives on the device only (offsets[E]).
@@ -35,8 +37,10 @@
  *   - Return value: MOE_OK or a negative MOE_ERR_* code; moe_last_error()
  *     gives a message.  Arguments are checked on the host before any launch;
  *     a failed check launches nothing.  Device-side waits are bounded: if one
- *     expires the kernel records MOE_ERR_DEVICE_TIMEOUT in a device flag,
- *     returns, and moe_check_status() reports it.
+ *     expires the kernel records a code in a device status word and returns,
+ *     and moe_check_status() reports it as MOE_ERR_DEVICE_TIMEOUT.  Device-side
+ *     data checks (an expert id out of range) skip the bad item and record a
+ *     code that moe_check_status() reports as MOE_ERR_DEVICE_CHECK.
  *   - Shapes: 1 <= k <= 8, k <= E <= 256, T >= 0.  The bf16 path needs
  *     d % 128 == 0 and f % 128 == 0; the f32 path d % 64 == 0 and f % 64 == 0.
  *   - Row space: expert e owns rows [offsets[e], offsets[e+1]); each segment
@@ -60,6 +64,7 @@ extern "C" {
 #define MOE_ERR_CUDA (-3)
 #define MOE_ERR_DEVICE_TIMEOUT (-4)
 #define MOE_ERR_WORKSPACE (-5)
+#define MOE_ERR_DEVICE_CHECK (-6)
 
 #define MOE_F32 0
 #define MOE_BF16 1
@@ -329,11 +334,28 @@ int moe_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k,
                      void* stream);
 
 /*
- * moe_check_status -- synchronises `stream`, then returns MOE_OK, a CUDA
- * error (MOE_ERR_CUDA) or MOE_ERR_DEVICE_TIMEOUT if a bounded device wait
- * expired since the last check (the flag is cleared by this call).
+ * moe_check_status -- synchronises `stream`, then reads and clears the
+ * device status word of the current device.  Returns MOE_OK, MOE_ERR_CUDA
+ * (a CUDA error), MOE_ERR_DEVICE_TIMEOUT if a bounded device wait expired
+ * since the last check (codes 0x2nn: the kernel gave up, drained its copies,
+ * freed its TMEM and returned; its outputs are undefined), or
+ * MOE_ERR_DEVICE_CHECK if a kernel met invalid data and skipped it (0x120:
+ * an expert id outside [0, E); 0x1ff: shared memory not 1 KB aligned).  The
+ * code is in moe_last_error()'s message.
  */
 int moe_check_status(void* stream);
+
+/*
+ * moe_debug_expire_next_wait -- test hook for the bounded device waits (the
+ * pages have no counterpart).  The next tensor-core GEMM launch of the
+ * library (on any stream of this process) runs with its TMA producer issuing
+ * no copies and every bounded wait limited to wait_ns nanoseconds, so that
+ * the MMA issuer's wait for a full stage expires with nothing in flight; the
+ * hook then resets itself.  That launch's outputs are undefined and
+ * moe_check_status() afterwards returns MOE_ERR_DEVICE_TIMEOUT.  wait_ns <= 0
+ * cancels a pending request.  Returns MOE_OK.
+ */
+int moe_debug_expire_next_wait(long long wait_ns);
 
 /*
  * Measurement hook (the pages have no counterpart; it serves the benchmark).

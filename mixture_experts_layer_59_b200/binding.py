@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_F32, MOE_BF16 = 0, 1
 MOE_ROUND_NONE, MOE_ROUND_NEAREST, MOE_ROUND_CAPACITY = 0, 1, 2
 MOE_GATE_TOPK_SOFTMAX, MOE_GATE_SOFTMAX_TOPK = 0, 1
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, -1, -2, -3
+MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_WORKSPACE, MOE_ERR_DEVICE_CHECK = -4, -5, -6
 TILE = 128
 
 EXPORTS = [
@@ -29,6 +31,7 @@ EXPORTS = [
     "moe_balance_loss_workspace_size", "moe_balance_loss",
     "moe_mxfp8_weight_sizes", "moe_mxfp8_quantize_weights", "moe_ffn_fwd_mxfp8_workspace_size",
     "moe_expert_ffn_fwd_mxfp8", "moe_layer_bwd_mxfp8_workspace_size", "moe_layer_bwd_mxfp8",
+    "moe_debug_expire_next_wait",
 ]
 
 _lib = None
@@ -68,6 +71,7 @@ _SIGS = {
     "moe_profile_enable": (_i, [_i]),
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_profile_report": (_i, [ctypes.c_char_p, _sz]),
+    "moe_debug_expire_next_wait": (_i, [ctypes.c_longlong]),
 }
 
 

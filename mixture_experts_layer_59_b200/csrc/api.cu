@@ -1,4 +1,5 @@
 // extern "C" entry points: argument checks, workspace layout, kernel order.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -25,16 +26,30 @@ int cuda_fail(cudaError_t e, const char* what) {
 
 __device__ int g_moe_status = 0;
 
+// The host-side name of a __device__ variable is only a stand-in: its device
+// address is looked up once per device (with that device current) and kept
+// in an atomic slot, so concurrent host threads may race to fill it safely.
 int* status_ptr() {
-  static int* cache[64] = {nullptr};
+  static std::atomic<int*> cache[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (cache[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_moe_status) == cudaSuccess) cache[dev] = static_cast<int*>(p);
+  int* p = cache[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_moe_status) == cudaSuccess) {
+      p = static_cast<int*>(q);
+      cache[dev].store(p, std::memory_order_release);
+    }
   }
-  return cache[dev];
+  return p;
+}
+
+static std::atomic<long long> g_debug_expire{0};
+
+long long take_debug_expire() {
+  if (g_debug_expire.load(std::memory_order_relaxed) == 0) return 0;
+  return g_debug_expire.exchange(0);
 }
 
 // ------------------------------------------------------------ profiling hook
@@ -76,16 +91,17 @@ ProfScope::~ProfScope() {
 }
 
 int device_sm_count() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64];
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
-  if (cache[dev] == 0) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 1;
+    n = n > 0 ? n : 1;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // ------------------------------------------------------------ checks
@@ -589,11 +605,21 @@ int moe_check_status(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "read status flag");
   if (flag != 0) {
     int zero = 0;
-    cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int));
+    e = cudaMemcpyToSymbol(g_moe_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status flag");
     char buf[96];
-    snprintf(buf, sizeof(buf), "device-side check failed (code 0x%x)", flag);
-    return fail(MOE_ERR_DEVICE_TIMEOUT, buf);
+    if (flag & 0x200) {
+      snprintf(buf, sizeof(buf), "a bounded device wait expired (code 0x%x)", flag);
+      return fail(MOE_ERR_DEVICE_TIMEOUT, buf);
+    }
+    snprintf(buf, sizeof(buf), "device-side data check failed (code 0x%x)", flag);
+    return fail(MOE_ERR_DEVICE_CHECK, buf);
   }
+  return MOE_OK;
+}
+
+int moe_debug_expire_next_wait(long long wait_ns) {
+  g_debug_expire.store(wait_ns > 0 ? wait_ns : 0);
   return MOE_OK;
 }
 

@@ -107,6 +107,10 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
 
 int device_sm_count();
 
+// Test hook of the bounded device waits: the wait limit (ns) requested for
+// the next tensor-core GEMM launch, or 0; taking it clears the request.
+long long take_debug_expire();
+
 // ---------------------------------------------------------------- MXFP8 (mx.cu, tc_gemm.cu)
 int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int E, int d, int f,
                             uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,

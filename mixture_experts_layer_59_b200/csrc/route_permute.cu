@@ -5,6 +5,8 @@
 // expert-contiguous rows: Trinity example 2-3, Olmo-core 3 ("row-wise EP puts
 // data straight into expert input buffers", routing kept on the GPU).
 // Token rounding: SonicMoE summary sec. 3.
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -654,19 +656,23 @@ static __device__ __align__(256) int32_t g_permute_scratch[NOALLOC_WORDS];
 // Device address of g_permute_scratch on the current device.  The host-side
 // name of a __device__ array is only a stand-in, so the address is looked up
 // once per device (with that device current) and cached.
+// The cache slots are atomic, so host threads that make their first calls
+// at the same time may both look the address up; they store the same value.
 static int permute_scratch_address(int32_t** out) {
-  static int32_t* cache[64] = {nullptr};
+  static std::atomic<int32_t*> cache[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
-  if (cache[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_permute_scratch);
+  int32_t* p = cache[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    void* q = nullptr;
+    e = cudaGetSymbolAddress(&q, g_permute_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(permute scratch)");
-    cache[dev] = static_cast<int32_t*>(p);
+    p = static_cast<int32_t*>(q);
+    cache[dev].store(p, std::memory_order_release);
   }
-  *out = cache[dev];
+  *out = p;
   return MOE_OK;
 }
 

@@ -114,6 +114,10 @@ struct TcArgs {
   uint8_t* dh_s;             // its scale blocks [cap/128][2f/128]
   const uint8_t* sfb1;       // DXQ: scale blocks of W3r (sfb: of W1r)
   int kh;                    // DXQ: K chunks per weight half (f / 128)
+  // bounded waits give up after wait_ns; dbg_no_load (test hook) makes the
+  // producer issue no copies so that the consumers' waits expire
+  uint64_t wait_ns;
+  int dbg_no_load;
 };
 
 template <int KIND> struct KT {
@@ -209,14 +213,14 @@ __device__ __forceinline__ bool tile_info(int t, const TcArgs& a, const int* s_o
 }
 
 __device__ __forceinline__ bool bounded_wait(uint64_t* bar, uint32_t parity, volatile int* s_abort,
-                                             int* status, int code) {
+                                             int* status, int code, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (*s_abort) return false;
-      if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *s_abort = 1;
         record_status(status, 0x200 | code);
         return false;
@@ -297,7 +301,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // 128-byte swizzled tiles need a 1024-byte aligned base: refuse to run otherwise
   if (smem_u32(smem_raw) & 1023u) {
-    if (threadIdx.x == 0) record_status(a.status, 0x2ff);
+    if (threadIdx.x == 0) record_status(a.status, 0x1ff);
     return;
   }
 
@@ -337,13 +341,13 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !a.dbg_no_load) {
       int stage = 0;
       uint32_t phase = 0;
       TileInfo ti;
       for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x) {
         for (int kb = 0; kb < ti.kb_count; ++kb) {
-          if (!bounded_wait(&empty_bar[stage], phase ^ 1, &s_abort, a.status, 1)) goto producer_done;
+          if (!bounded_wait(&empty_bar[stage], phase ^ 1, &s_abort, a.status, 1, a.wait_ns)) goto producer_done;
           uint8_t* sA = smem + stage * C::STAGE;
           uint8_t* sB = sA + A_BYTES;
           mbar_arrive_expect_tx(&full_bar[stage], C::TX);
@@ -435,11 +439,11 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       for (int t = blockIdx.x; tile_info<KIND, BN>(t, a, s_off, total, ti); t += gridDim.x, ++it) {
         const int acc = C::NACC == 1 ? 0 : (it & 1);
         const uint32_t acc_phase = C::NACC == 1 ? (it & 1) : ((it >> 1) & 1);
-        if (!bounded_wait(&tempty_bar[acc], acc_phase ^ 1, &s_abort, a.status, 2)) break;
+        if (!bounded_wait(&tempty_bar[acc], acc_phase ^ 1, &s_abort, a.status, 2, a.wait_ns)) break;
         fence_after_sync();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < ti.kb_count; ++kb) {
-          if (!bounded_wait(&full_bar[stage], phase, &s_abort, a.status, 3)) goto mma_done;
+          if (!bounded_wait(&full_bar[stage], phase, &s_abort, a.status, 3, a.wait_ns)) goto mma_done;
           fence_after_sync();
           const uint32_t sA = smem_u32(smem + stage * C::STAGE);
           const uint32_t sB = sA + A_BYTES;
@@ -498,7 +502,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
 #pragma unroll
         for (int q = 0; q < 4; ++q) { hn1[q] = s1[q]; hn3[q] = s3[q]; }
       }
-      if (!bounded_wait(&tfull_bar[acc], acc_phase, &s_abort, a.status, 4)) break;
+      if (!bounded_wait(&tfull_bar[acc], acc_phase, &s_abort, a.status, 4, a.wait_ns)) break;
       fence_after_sync();
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
       const int row = ti.m0 + rloc;
@@ -871,8 +875,15 @@ static int make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1
 }
 
 template <int KIND, int BN>
-static int launch(const TcArgs& a, int grid, cudaStream_t s) {
+static int launch(const TcArgs& args, int grid, cudaStream_t s) {
   using C = Cfg<BN, KT<KIND>::MX>;
+  TcArgs a = args;
+  a.wait_ns = WAIT_LIMIT_NS;
+  a.dbg_no_load = 0;
+  if (const long long dbg = take_debug_expire(); dbg > 0) {
+    a.wait_ns = (uint64_t)dbg;
+    a.dbg_no_load = 1;
+  }
   cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<KIND, BN>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return cuda_fail(e, "tc gemm smem attribute");

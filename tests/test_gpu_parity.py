@@ -453,7 +453,7 @@ def test_device_check_reports_and_clears():
     plan = B.moe_permute(bad, gate, logits, E, B.MOE_ROUND_NONE)
     with pytest.raises(B.MoEError) as ei:
         B.moe_check_status()
-    assert ei.value.code == -4 and "0x120" in str(ei.value)
+    assert ei.value.code == B.MOE_ERR_DEVICE_CHECK and "0x120" in str(ei.value)
     B.moe_check_status()   # cleared by the read
     slot_row = i64(plan["slot_row"]).reshape(T, k)
     assert slot_row[3, 0] == -1 and slot_row[77, 1] == -1
@@ -461,3 +461,38 @@ def test_device_check_reports_and_clears():
     valid &= i64(bad) < E
     assert (slot_row[valid] >= 0).all()
     assert int(i64(plan["counts"]).sum()) == int(valid.sum())
+
+
+def test_bounded_wait_expires_then_next_call_is_clean():
+    """Failure detection of the bounded device waits, without a GPU fault: the
+    test hook makes the next tensor-core GEMM's producer issue no copies, so
+    the MMA issuer's wait for a full stage runs out (5 ms limit) with nothing
+    in flight; the kernel records a 0x2nn code, frees its TMEM and returns.
+    moe_check_status reports MOE_ERR_DEVICE_TIMEOUT once, and the same call
+    repeated afterwards gives bit-identical results to a clean run."""
+    T, d, f, E, k = 512, 256, 256, 8, 2
+    g = torch.Generator().manual_seed(43)
+    x = (torch.randn(T, d, generator=g)).to(torch.bfloat16).cuda()
+    w1, w3 = ((0.05 * torch.randn(E, d, f, generator=g)).to(torch.bfloat16).cuda() for _ in range(2))
+    w2 = (0.05 * torch.randn(E, f, d, generator=g)).to(torch.bfloat16).cuda()
+    lo = torch.randn(T, E, generator=g).cuda()
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=T, E=E)
+    plan = B.moe_permute(idx, gate, logits, E)
+    H0, Y0 = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
+    B.moe_check_status()
+    assert B.lib().moe_debug_expire_next_wait(5_000_000) == 0
+    B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
+    with pytest.raises(B.MoEError) as ei:
+        B.moe_check_status()
+    assert ei.value.code == B.MOE_ERR_DEVICE_TIMEOUT and "0x20" in str(ei.value)
+    B.moe_check_status()   # cleared by the read
+    H1, Y1 = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
+    B.moe_check_status()
+    R = int(plan["offsets"][-1].item())
+    assert torch.equal(H1[:R], H0[:R]) and torch.equal(Y1[:R], Y0[:R])
+    # a cancelled request leaves the next launch alone
+    assert B.lib().moe_debug_expire_next_wait(5_000_000) == 0
+    assert B.lib().moe_debug_expire_next_wait(0) == 0
+    H2, _ = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
+    B.moe_check_status()
+    assert torch.equal(H2[:R], H0[:R])
