@@ -313,6 +313,98 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate,
                   float* dS, float* dlogits, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Expert parallelism across G ranks (one GPU each): rank g owns experts
+ * g*El .. g*El+El-1 (El = E/G) and keeps their weights resident; the
+ * permuted rows travel to the experts instead ("Olmo-core 3" news piece:
+ * experts stay on their GPU and data is routed to them, row-wise expert
+ * parallelism places rows straight into the experts' input buffers; "From
+ * 501B to 23B: what is Beam doing", sec. 4.2: tokens reach the GPU holding
+ * their expert through an all-to-all exchange).  The token side (route,
+ * permute, combine, router gradient, dx) runs where the tokens are; the
+ * expert side (grouped GEMMs, dS, expert weight gradients) where the
+ * experts are.  The calls below are those pieces; the exchange itself is
+ * the caller's (NCCL send/recv of whole 128-aligned segments).
+ *
+ * moe_gather_rows -- dst[r] = src[row_token[r]] for every row r < offsets[E]
+ *   of a plan from moe_permute (padding rows zero): the row gather that
+ *   moe_expert_ffn_fwd and moe_layer_bwd run internally.  src [T,width],
+ *   dst [cap,width] (dtype); width a multiple of 8.  The segments of rank
+ *   g's experts, rows offsets[g*El] .. offsets[g*El+El], are what this rank
+ *   sends to rank g.
+ */
+int moe_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets,
+                    const int32_t* slot_row, const int32_t* extra_row, int T, int width, int E,
+                    int k, int dtype, void* dst, void* stream);
+
+/*
+ * moe_ep_dispatch_counts -- seg_rows[e] = offsets[e+1] - offsets[e] [E]: the
+ *   rows this rank sends for expert e (to the rank owning e), a multiple of
+ *   128.  Exchanged between ranks, they become the receivers' recv_rows.
+ * moe_ep_receive_plan -- placement of received segments on a rank owning El
+ *   experts.  recv_rows [G, El]: rows source s sends for local expert j.
+ *   local_offsets [El+1] out: local expert j owns rows local_offsets[j] ..
+ *   local_offsets[j+1] (sources in rank order; local_offsets[El] = rows
+ *   received).  recv_row [G, El] out: first local row of the segment from
+ *   (s, j).  A count that is negative or not a multiple of 128 is treated as
+ *   0 and recorded as a device data check (code 0x130, MOE_ERR_DEVICE_CHECK
+ *   from moe_check_status).  El <= 256.
+ */
+int moe_ep_dispatch_counts(const int32_t* offsets, int E, int32_t* seg_rows, void* stream);
+int moe_ep_receive_plan(const int32_t* recv_rows, int G, int El, int32_t* local_offsets,
+                        int32_t* recv_row, void* stream);
+
+/*
+ * moe_expert_rows_fwd -- the expert side of moe_expert_ffn_fwd on rows that
+ *   are already in expert-contiguous order: H = [xg W1_e | xg W3_e], A =
+ *   silu(H1) * H3, Y = A W2_e for the rows of each expert e < E, segments
+ *   offsets[e] .. offsets[e+1] (multiples of 128; offsets[E] <= rows; rows
+ *   of zeros give zeros).  xg [rows,d], w1, w3 [E,d,f], w2 [E,f,d], H
+ *   [rows,2f] out, Y [rows,d] out; bf16 only (sm_100 tensor cores); rows a
+ *   positive multiple of 128.  ws: at least
+ *   moe_expert_rows_fwd_workspace_size() bytes.
+ */
+size_t moe_expert_rows_fwd_workspace_size(int rows, int f, int dtype);
+int moe_expert_rows_fwd(const void* xg, const void* w1, const void* w3, const void* w2,
+                        const int32_t* offsets, int rows, int d, int f, int E, int dtype, void* H,
+                        void* Y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_rows_bwd -- the expert side of moe_layer_bwd on the same rows:
+ *   dA' = dog W2_e^T, dS = <dA', A> (A recomputed from H; "SonicMoE"
+ *   summary, sec. 1), dA = row_gate * dA', SwiGLU backward -> dH,
+ *   dX_rows = dH [W1_e | W3_e]^T, dW2_e = (row_gate A)^T dog,
+ *   [dW1_e | dW3_e] = xg^T dH, every output written (experts without rows
+ *   get zero gradients).  dog [rows,d] (gathered dO rows), xg [rows,d], H
+ *   [rows,2f] (from moe_expert_rows_fwd), row_gate [rows] fp32 (the rows'
+ *   weights, moe_permute's row_gate carried with the rows); dX_rows
+ *   [rows,d] out; dS [rows] fp32 out (rows below offsets[E]); dw1, dw3
+ *   [E,d,f], dw2 [E,f,d] out.  bf16 only; ws: at least
+ *   moe_expert_rows_bwd_workspace_size() bytes.
+ */
+size_t moe_expert_rows_bwd_workspace_size(int rows, int d, int f, int dtype);
+int moe_expert_rows_bwd(const void* dog, const void* xg, const float* row_gate, const void* H,
+                        const void* w1, const void* w3, const void* w2, const int32_t* offsets,
+                        int rows, int d, int f, int E, int dtype, void* dX_rows, float* dS,
+                        void* dw1, void* dw3, void* dw2, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * moe_token_bwd -- the token side of moe_layer_bwd: from each row's dX_rows
+ *   and dS in this rank's own row space (returned by the experts' ranks),
+ *   dlogits (as in moe_layer_bwd), dW_gate = x^T dlogits over this rank's
+ *   tokens (data-parallel ranks add theirs), dx = unpermute-sum of dX_rows +
+ *   dlogits W_gate^T.  Arguments as in moe_layer_bwd; dX_rows [cap,d]
+ *   (dtype), dS [cap] fp32.  ws: at least moe_token_bwd_workspace_size().
+ */
+size_t moe_token_bwd_workspace_size(int T, int d, int E, int k, int dtype);
+int moe_token_bwd(const void* dX_rows, const float* dS, const void* x, const void* w_gate,
+                  const int32_t* idx, const float* gate, const float* gate_grad,
+                  const float* logits, int gate_mode, const float* row_gate,
+                  const int32_t* slot_row, const int32_t* extra_row, int T, int d, int E, int k,
+                  int dtype, int router_grad, void* dx, float* dw_gate, float* dlogits, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/*
  * moe_balance_loss -- load-balance loss and routing statistics.
  * ["Breaking the hundred-billion-parameter barrier: how MoE reshapes
  * distributed training", challenge 1, solution 1]: L = lambda * CV(m)^2 with

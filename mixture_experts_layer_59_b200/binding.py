@@ -31,7 +31,10 @@ EXPORTS = [
     "moe_balance_loss_workspace_size", "moe_balance_loss",
     "moe_mxfp8_weight_sizes", "moe_mxfp8_quantize_weights", "moe_ffn_fwd_mxfp8_workspace_size",
     "moe_expert_ffn_fwd_mxfp8", "moe_layer_bwd_mxfp8_workspace_size", "moe_layer_bwd_mxfp8",
-    "moe_debug_expire_next_wait",
+    "moe_debug_expire_next_wait", "moe_gather_rows", "moe_ep_dispatch_counts",
+    "moe_ep_receive_plan", "moe_expert_rows_fwd_workspace_size", "moe_expert_rows_fwd",
+    "moe_expert_rows_bwd_workspace_size", "moe_expert_rows_bwd", "moe_token_bwd_workspace_size",
+    "moe_token_bwd",
 ]
 
 _lib = None
@@ -72,6 +75,15 @@ _SIGS = {
     "moe_permute_noalloc": (_i, [_vp, _vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_profile_report": (_i, [ctypes.c_char_p, _sz]),
     "moe_debug_expire_next_wait": (_i, [ctypes.c_longlong]),
+    "moe_gather_rows": (_i, [_vp] * 5 + [_i] * 5 + [_vp, _vp]),
+    "moe_ep_dispatch_counts": (_i, [_vp, _i, _vp, _vp]),
+    "moe_ep_receive_plan": (_i, [_vp, _i, _i, _vp, _vp, _vp]),
+    "moe_expert_rows_fwd_workspace_size": (_sz, [_i, _i, _i]),
+    "moe_expert_rows_fwd": (_i, [_vp] * 5 + [_i] * 5 + [_vp] * 3 + [_sz, _vp]),
+    "moe_expert_rows_bwd_workspace_size": (_sz, [_i] * 4),
+    "moe_expert_rows_bwd": (_i, [_vp] * 8 + [_i] * 5 + [_vp] * 6 + [_sz, _vp]),
+    "moe_token_bwd_workspace_size": (_sz, [_i] * 5),
+    "moe_token_bwd": (_i, [_vp] * 8 + [_i] + [_vp] * 3 + [_i] * 6 + [_vp] * 4 + [_sz, _vp]),
 }
 
 
@@ -382,3 +394,96 @@ def moe_balance_loss(idx, gate, E, lam, dgate=True, ws=None, stream=None):
     _check(lib().moe_balance_loss(_p(idx), _p(gate), T, E, k, float(lam), _p(stats), _p(imp),
                                   _p(dg), _p(ws), ws.numel(), _stream(stream)))
     return dict(stats=stats, importance=imp, dgate=dg)
+
+
+# ------------------------------------------------------------------ expert parallelism
+def moe_gather_rows(src, plan, k, out=None, stream=None):
+    """Rows of a plan gathered from token-major ``src`` [T, width]; padding rows zero."""
+    T, width = src.shape
+    E = plan["offsets"].numel() - 1
+    cap = moe_row_capacity(T, E, k)
+    out = out if out is not None else torch.empty(cap, width, device=src.device, dtype=src.dtype)
+    _check(lib().moe_gather_rows(_p(src), _p(plan["row_token"]), _p(plan["offsets"]),
+                                 _p(plan["slot_row"]), _p(plan.get("extra_row")), T, width, E, k,
+                                 dtype_code(src.dtype), _p(out), _stream(stream)))
+    return out
+
+
+def moe_ep_dispatch_counts(offsets, out=None, stream=None):
+    """Rows of each expert's segment [E] (int32, device)."""
+    E = offsets.numel() - 1
+    out = out if out is not None else torch.empty(E, device=offsets.device, dtype=torch.int32)
+    _check(lib().moe_ep_dispatch_counts(_p(offsets), E, _p(out), _stream(stream)))
+    return out
+
+
+def moe_ep_receive_plan(recv_rows, stream=None):
+    """recv_rows [G, El] int32 -> (local_offsets [El+1], recv_row [G, El])."""
+    G, El = recv_rows.shape
+    lo = torch.empty(El + 1, device=recv_rows.device, dtype=torch.int32)
+    rr = torch.empty(G, El, device=recv_rows.device, dtype=torch.int32)
+    _check(lib().moe_ep_receive_plan(_p(recv_rows), G, El, _p(lo), _p(rr), _stream(stream)))
+    return lo, rr
+
+
+def moe_expert_rows_fwd(xg, w1, w3, w2, offsets, H=None, Y=None, ws=None, stream=None):
+    """Grouped SwiGLU FFN on expert-contiguous rows: H [rows, 2f], Y [rows, d]."""
+    rows, d = xg.shape
+    E, _, f = w1.shape
+    dt = dtype_code(xg.dtype)
+    H = H if H is not None else torch.empty(rows, 2 * f, device=xg.device, dtype=xg.dtype)
+    Y = Y if Y is not None else torch.empty(rows, d, device=xg.device, dtype=xg.dtype)
+    if ws is None:
+        ws = torch.empty(max(lib().moe_expert_rows_fwd_workspace_size(rows, f, dt), 1),
+                         device=xg.device, dtype=torch.uint8)
+    _check(lib().moe_expert_rows_fwd(_p(xg), _p(w1), _p(w3), _p(w2), _p(offsets), rows, d, f, E,
+                                     dt, _p(H), _p(Y), _p(ws), ws.numel(), _stream(stream)))
+    return H, Y
+
+
+def moe_expert_rows_bwd(dog, xg, row_gate, H, w1, w3, w2, offsets, out=None, ws=None,
+                        stream=None):
+    """Expert side of the backward on expert-contiguous rows.  Returns dict
+    dX_rows [rows, d], dS [rows] f32, dw1, dw3 [E, d, f], dw2 [E, f, d]."""
+    rows, d = xg.shape
+    E, _, f = w1.shape
+    dt = dtype_code(xg.dtype)
+    dev = xg.device
+    o = dict(out) if out else {}
+    o.setdefault("dX_rows", torch.empty(rows, d, device=dev, dtype=xg.dtype))
+    o.setdefault("dS", torch.empty(rows, device=dev, dtype=torch.float32))
+    o.setdefault("dw1", torch.empty(E, d, f, device=dev, dtype=xg.dtype))
+    o.setdefault("dw3", torch.empty(E, d, f, device=dev, dtype=xg.dtype))
+    o.setdefault("dw2", torch.empty(E, f, d, device=dev, dtype=xg.dtype))
+    if ws is None:
+        ws = torch.empty(max(lib().moe_expert_rows_bwd_workspace_size(rows, d, f, dt), 1),
+                         device=dev, dtype=torch.uint8)
+    _check(lib().moe_expert_rows_bwd(_p(dog), _p(xg), _p(row_gate), _p(H), _p(w1), _p(w3),
+                                     _p(w2), _p(offsets), rows, d, f, E, dt, _p(o["dX_rows"]),
+                                     _p(o["dS"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]),
+                                     _p(ws), ws.numel(), _stream(stream)))
+    return o
+
+
+def moe_token_bwd(dX_rows, dS, x, w_gate, idx, gate, plan, router_grad=True, gate_grad=None,
+                  logits=None, gate_mode=MOE_GATE_TOPK_SOFTMAX, out=None, ws=None, stream=None):
+    """Token side of the backward.  Returns dict dx [T, d], dw_gate [d, E] f32,
+    dlogits [T, E] f32."""
+    T, d = x.shape
+    k = idx.shape[1]
+    E = plan["offsets"].numel() - 1
+    dt = dtype_code(x.dtype)
+    dev = x.device
+    o = dict(out) if out else {}
+    o.setdefault("dx", torch.empty(T, d, device=dev, dtype=x.dtype))
+    o.setdefault("dw_gate", torch.empty(d, E, device=dev, dtype=torch.float32))
+    o.setdefault("dlogits", torch.empty(T, E, device=dev, dtype=torch.float32))
+    if ws is None:
+        ws = torch.empty(max(lib().moe_token_bwd_workspace_size(T, d, E, k, dt), 1), device=dev,
+                         dtype=torch.uint8)
+    _check(lib().moe_token_bwd(_p(dX_rows), _p(dS), _p(x), _p(w_gate), _p(idx), _p(gate),
+                               _p(gate_grad), _p(logits), gate_mode, _p(plan["row_gate"]),
+                               _p(plan["slot_row"]), _p(plan.get("extra_row")), T, d, E, k, dt,
+                               1 if router_grad else 0, _p(o["dx"]), _p(o["dw_gate"]),
+                               _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
+    return o

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 
-SOURCES = ["api.cu", "mx.cu", "route_permute.cu", "rowops.cu", "simt.cu", "tc_gemm.cu"]
+SOURCES = ["api.cu", "ep.cu", "mx.cu", "route_permute.cu", "rowops.cu", "simt.cu", "tc_gemm.cu"]
 HEADERS = ["common.cuh", "internal.h", "mx.cuh", "tcgen05.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

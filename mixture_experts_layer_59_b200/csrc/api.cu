@@ -191,6 +191,30 @@ struct BwdWs {
   }
 };
 
+// Workspace of the token side of the backward (router gradient and dx).
+struct TokenWs {
+  float *dl, *dx_acc;
+  void *dl_hi, *dl_lo;
+  float* dwg_part;
+};
+
+template <class A>
+struct TokenBwdWs {
+  TokenWs w{};
+  void carve(A& a, int T, int d, int E, int dtype) {
+    const bool tc = dtype == MOE_BF16 && tc_available();
+    w.dl = a.template take<float>((size_t)T * E + 1);
+    w.dx_acc = a.template take<float>((size_t)T * d + 1);
+    if (tc && tc_router_ok(E)) {
+      int chunk = 0;
+      const int splits = tc_dwg_splits(T, d, &chunk);
+      w.dl_hi = a.template take<uint16_t>((size_t)T * E + 8);
+      w.dl_lo = a.template take<uint16_t>((size_t)T * E + 8);
+      w.dwg_part = a.template take<float>((size_t)splits * d * E);
+    }
+  }
+};
+
 }  // namespace moe
 
 using namespace moe;
@@ -414,6 +438,52 @@ size_t moe_layer_bwd_workspace_size(int T, int d, int f, int E, int k, int dtype
   return z.used;
 }
 
+// Token side of the backward, from the expert side's per-row results:
+// dlogits from dS (partials summed in a fixed order), dW_gate = x^T dlogits,
+// dx = unpermute-sum of dX_perm + dlogits W_gate^T.
+static int token_bwd_impl(const void* dxp, const float* ds_part, int nparts, const void* x,
+                          const void* w_gate, const int32_t* idx, const float* gate,
+                          const float* gate_grad, const float* logits, int gate_mode,
+                          const float* row_gate, const int32_t* slot_row,
+                          const int32_t* extra_row, int T, int d, int E, int k, int dtype,
+                          int router_grad, void* dx, float* dw_gate, float* dS, float* dlogits,
+                          const TokenWs& w, cudaStream_t s) {
+  int rc;
+  float* dl = dlogits ? dlogits : w.dl;
+  const bool tc_router = router_grad && w.dl_hi != nullptr;
+  if ((rc = launch_router_bwd(ds_part, nparts, idx, gate, row_gate, slot_row, extra_row,
+                              gate_grad, logits, gate_mode, T, E, k, dl, dS,
+                              tc_router ? w.dl_hi : nullptr,
+                              tc_router ? w.dl_lo : nullptr, s)))
+    return rc;
+  if (tc_router) {
+    // dW_gate on the tensor cores (split-K, hi/lo dlogits); dx = unpermute-sum
+    // of dX_perm + dl W_gate^T: one CUDA-core pass when W_gate fits in shared
+    // memory, otherwise fp32 row sums + the tensor-core router term
+    if (dx_fused_ok(d, E)) {
+      if ((rc = tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate,
+                              nullptr, nullptr, device_sm_count(), s)))
+        return rc;
+      return launch_dx_fused(dxp, slot_row, extra_row, dl, w_gate, T, d, E, k, dx, s);
+    }
+    if ((rc = launch_token_reduce(dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
+                                  true, w.dx_acc, s)))
+      return rc;
+    return tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate, w.dx_acc,
+                         dx, device_sm_count(), s);
+  }
+  if (router_grad) {
+    if ((rc = launch_token_reduce(dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
+                                  true, w.dx_acc, s)))
+      return rc;
+    return simt_router_bwd_gemms(x, w_gate, dl, w.dx_acc, T, d, E, dtype, dw_gate, dx, s);
+  }
+  cudaError_t e = cudaMemsetAsync(dw_gate, 0, (size_t)d * E * sizeof(float), s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset dw_gate");
+  return launch_token_reduce(dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false, false,
+                             dx, s);
+}
+
 static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, const void* w1,
                   const void* w3, const void* w2, const int32_t* idx, const float* gate,
                   const float* gate_grad, const float* logits, int gate_mode,
@@ -466,39 +536,9 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
     if ((rc = simt_ffn_bwd(p, dout, row_gate, H, w.dap, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2, s)))
       return rc;
   }
-  float* dl = dlogits ? dlogits : w.dl;
-  const bool tc_router = router_grad && w.dl_hi != nullptr;
-  if ((rc = launch_router_bwd(w.ds, w.nparts, idx, gate, row_gate, slot_row, extra_row,
-                              gate_grad, logits, gate_mode, T, E, k, dl, dS,
-                              tc_router ? w.dl_hi : nullptr,
-                              tc_router ? w.dl_lo : nullptr, s)))
-    return rc;
-  if (tc_router) {
-    // dW_gate on the tensor cores (split-K, hi/lo dlogits); dx = unpermute-sum
-    // of dX_perm + dl W_gate^T: one CUDA-core pass when W_gate fits in shared
-    // memory, otherwise fp32 row sums + the tensor-core router term
-    if (dx_fused_ok(d, E)) {
-      if ((rc = tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate,
-                              nullptr, nullptr, device_sm_count(), s)))
-        return rc;
-      return launch_dx_fused(w.dxp, slot_row, extra_row, dl, w_gate, T, d, E, k, dx, s);
-    }
-    if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
-                                  true, w.dx_acc, s)))
-      return rc;
-    return tc_router_bwd(x, w_gate, w.dl_hi, w.dl_lo, T, d, E, k, w.dwg_part, dw_gate, w.dx_acc,
-                         dx, device_sm_count(), s);
-  }
-  if (router_grad) {
-    if ((rc = launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false,
-                                  true, w.dx_acc, s)))
-      return rc;
-    return simt_router_bwd_gemms(x, w_gate, dl, w.dx_acc, T, d, E, dtype, dw_gate, dx, s);
-  }
-  cudaError_t e = cudaMemsetAsync(dw_gate, 0, (size_t)d * E * sizeof(float), s);
-  if (e != cudaSuccess) return cuda_fail(e, "memset dw_gate");
-  return launch_token_reduce(w.dxp, row_gate, slot_row, extra_row, T, d, E, k, dtype, false, false,
-                             dx, s);
+  return token_bwd_impl(w.dxp, w.ds, w.nparts, x, w_gate, idx, gate, gate_grad, logits, gate_mode,
+                        row_gate, slot_row, extra_row, T, d, E, k, dtype, router_grad, dx, dw_gate,
+                        dS, dlogits, TokenWs{w.dl, w.dx_acc, w.dl_hi, w.dl_lo, w.dwg_part}, s);
 }
 
 int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const void* w1,
@@ -543,6 +583,144 @@ int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate, con
                         offsets, row_token, row_gate, slot_row, extra_row, H, T, d, f, E, k,
                         MOE_BF16, router_grad, dx, dw_gate, dw1, dw3, dw2, dS, dlogits, ws,
                         ws_bytes, stream, mxw);
+}
+
+// ------------------------------------------------------------ row-space pieces
+// (expert parallelism: the token side and the expert side of the layer run on
+// different ranks, with the permuted rows exchanged in between)
+
+int moe_gather_rows(const void* src, const int32_t* row_token, const int32_t* offsets,
+                    const int32_t* slot_row, const int32_t* extra_row, int T, int width, int E,
+                    int k, int dtype, void* dst, void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (width <= 0 || width % 8) return fail(MOE_ERR_UNSUPPORTED, "width must be a positive multiple of 8");
+  REQUIRE_PTR(row_token); REQUIRE_PTR(offsets); REQUIRE_PTR(dst);
+  if (T > 0) { REQUIRE_PTR(src); REQUIRE_PTR(slot_row); }
+  REQUIRE_ALIGNED(src); REQUIRE_ALIGNED(dst);
+  return launch_scatter_rows(src, slot_row, extra_row, row_token, offsets, T, width, E, k, dtype,
+                             dst, (cudaStream_t)stream);
+}
+
+static int check_rows_args(int rows, int d, int f, int E, int dtype) {
+  if (dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "the row-space entry points take bf16");
+  if (!tc_available()) return fail(MOE_ERR_UNSUPPORTED, "the row-space entry points need an sm_100 device");
+  if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  if (rows < 128 || rows % 128) return fail(MOE_ERR_UNSUPPORTED, "rows must be a positive multiple of 128");
+  return check_dims(d, f, dtype);
+}
+
+size_t moe_expert_rows_fwd_workspace_size(int rows, int f, int dtype) {
+  if (rows < 0 || f <= 0) return 0;
+  Sizer z;
+  z.take<char>((size_t)rows * f * esize(dtype));
+  return z.used;
+}
+
+int moe_expert_rows_fwd(const void* xg, const void* w1, const void* w3, const void* w2,
+                        const int32_t* offsets, int rows, int d, int f, int E, int dtype, void* H,
+                        void* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_rows_args(rows, d, f, E, dtype)) return rc;
+  REQUIRE_PTR(xg); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2); REQUIRE_PTR(offsets);
+  REQUIRE_PTR(H); REQUIRE_PTR(Y);
+  REQUIRE_ALIGNED(xg); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2);
+  REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(Y); REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_expert_rows_fwd_workspace_size(rows, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_expert_rows_fwd_workspace_size()");
+  Carve c(ws, ws_bytes);
+  void* act = c.take<char>((size_t)rows * f * esize(dtype));
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  FfnPtrs p{nullptr, w1, w3, w2, nullptr, offsets, 0, d, f, E, rows, dtype};
+  return tc_ffn_fwd(p, xg, H, act, Y, device_sm_count(), (cudaStream_t)stream);
+}
+
+size_t moe_expert_rows_bwd_workspace_size(int rows, int d, int f, int dtype) {
+  if (rows < 0 || d <= 0 || f <= 0) return 0;
+  const size_t es = esize(dtype);
+  Sizer z;
+  z.take<char>((size_t)rows * 2 * f * es);                  // dH
+  z.take<char>((size_t)rows * f * es);                      // s * A
+  z.take<float>((size_t)rows * tc_num_dS_parts(f));         // dS partials
+  return z.used;
+}
+
+int moe_expert_rows_bwd(const void* dog, const void* xg, const float* row_gate, const void* H,
+                        const void* w1, const void* w3, const void* w2, const int32_t* offsets,
+                        int rows, int d, int f, int E, int dtype, void* dX_rows, float* dS,
+                        void* dw1, void* dw3, void* dw2, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (int rc = check_rows_args(rows, d, f, E, dtype)) return rc;
+  REQUIRE_PTR(dog); REQUIRE_PTR(xg); REQUIRE_PTR(row_gate); REQUIRE_PTR(H); REQUIRE_PTR(w1);
+  REQUIRE_PTR(w3); REQUIRE_PTR(w2); REQUIRE_PTR(offsets); REQUIRE_PTR(dX_rows); REQUIRE_PTR(dS);
+  REQUIRE_PTR(dw1); REQUIRE_PTR(dw3); REQUIRE_PTR(dw2);
+  REQUIRE_ALIGNED(dog); REQUIRE_ALIGNED(xg); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(w1);
+  REQUIRE_ALIGNED(w3); REQUIRE_ALIGNED(w2); REQUIRE_ALIGNED(dX_rows); REQUIRE_ALIGNED(dw1);
+  REQUIRE_ALIGNED(dw3); REQUIRE_ALIGNED(dw2); REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_expert_rows_bwd_workspace_size(rows, d, f, dtype))
+    return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_expert_rows_bwd_workspace_size()");
+  const size_t es = esize(dtype);
+  const int nparts = tc_num_dS_parts(f);
+  Carve c(ws, ws_bytes);
+  void* dH = c.take<char>((size_t)rows * 2 * f * es);
+  void* gact = c.take<char>((size_t)rows * f * es);
+  float* ds_part = c.take<float>((size_t)rows * nparts);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = (cudaStream_t)stream;
+  FfnPtrs p{nullptr, w1, w3, w2, nullptr, offsets, 0, d, f, E, rows, dtype};
+  if (int rc = tc_ffn_bwd(p, dog, xg, row_gate, H, dH, gact, ds_part, dX_rows, dw1, dw3, dw2,
+                          device_sm_count(), s))
+    return rc;
+  return launch_ds_rows(ds_part, nparts, offsets, E, rows, dS, s);
+}
+
+size_t moe_token_bwd_workspace_size(int T, int d, int E, int k, int dtype) {
+  (void)k;
+  if (T < 0 || d <= 0 || E <= 0) return 0;
+  Sizer z;
+  TokenBwdWs<Sizer> w;
+  w.carve(z, T, d, E, dtype);
+  return z.used;
+}
+
+int moe_token_bwd(const void* dX_rows, const float* dS, const void* x, const void* w_gate,
+                  const int32_t* idx, const float* gate, const float* gate_grad,
+                  const float* logits, int gate_mode, const float* row_gate,
+                  const int32_t* slot_row, const int32_t* extra_row, int T, int d, int E, int k,
+                  int dtype, int router_grad, void* dx, float* dw_gate, float* dlogits, void* ws,
+                  size_t ws_bytes, void* stream) {
+  if (int rc = check_common(T, E, k, dtype)) return rc;
+  if (d <= 0 || d % 8) return fail(MOE_ERR_UNSUPPORTED, "d must be a positive multiple of 8");
+  if (gate_mode != MOE_GATE_TOPK_SOFTMAX && gate_mode != MOE_GATE_SOFTMAX_TOPK)
+    return fail(MOE_ERR_INVALID_ARG, "gate_mode must be MOE_GATE_TOPK_SOFTMAX or MOE_GATE_SOFTMAX_TOPK");
+  REQUIRE_PTR(dX_rows); REQUIRE_PTR(dS); REQUIRE_PTR(x); REQUIRE_PTR(idx); REQUIRE_PTR(gate);
+  REQUIRE_PTR(row_gate); REQUIRE_PTR(slot_row); REQUIRE_PTR(dx); REQUIRE_PTR(dw_gate);
+  if (router_grad) REQUIRE_PTR(w_gate);
+  if (gate_mode == MOE_GATE_SOFTMAX_TOPK) REQUIRE_PTR(logits);
+  REQUIRE_ALIGNED(dX_rows); REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w_gate); REQUIRE_ALIGNED(dx);
+  REQUIRE_ALIGNED(ws);
+  if (ws_bytes < moe_token_bwd_workspace_size(T, d, E, k, dtype))
+    return fail(MOE_ERR_WORKSPACE, "workspace smaller than moe_token_bwd_workspace_size()");
+  if (T == 0) return MOE_OK;
+  Carve c(ws, ws_bytes);
+  TokenBwdWs<Carve> w;
+  w.carve(c, T, d, E, dtype);
+  if (!c.ok) return fail(MOE_ERR_WORKSPACE, "workspace too small");
+  return token_bwd_impl(dX_rows, dS, 1, x, w_gate, idx, gate, gate_grad, logits, gate_mode,
+                        row_gate, slot_row, extra_row, T, d, E, k, dtype, router_grad, dx, dw_gate,
+                        nullptr, dlogits, w.w, (cudaStream_t)stream);
+}
+
+int moe_ep_dispatch_counts(const int32_t* offsets, int E, int32_t* seg_rows, void* stream) {
+  if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  REQUIRE_PTR(offsets); REQUIRE_PTR(seg_rows);
+  return launch_ep_dispatch_counts(offsets, E, seg_rows, (cudaStream_t)stream);
+}
+
+int moe_ep_receive_plan(const int32_t* recv_rows, int G, int El, int32_t* local_offsets,
+                        int32_t* recv_row, void* stream) {
+  if (G < 1) return fail(MOE_ERR_INVALID_ARG, "G must be >= 1");
+  if (El < 1 || El > 256) return fail(MOE_ERR_UNSUPPORTED, "El must be in [1, 256]");
+  REQUIRE_PTR(recv_rows); REQUIRE_PTR(local_offsets); REQUIRE_PTR(recv_row);
+  return launch_ep_receive_plan(recv_rows, G, El, local_offsets, recv_row, (cudaStream_t)stream);
 }
 
 int moe_profile_enable(int on) {

@@ -107,6 +107,14 @@ int tc_router_bwd(const void* x, const void* wg, const void* dl_hi, const void* 
 
 int device_sm_count();
 
+// ---------------------------------------------------------------- expert parallelism (ep.cu)
+int launch_ep_dispatch_counts(const int32_t* offsets, int E, int32_t* seg_rows, cudaStream_t s);
+int launch_ep_receive_plan(const int32_t* recv_rows, int G, int El, int32_t* local_offsets,
+                           int32_t* recv_row, cudaStream_t s);
+// dS[r] = sum over p of ds_part[r, p] (fixed order) for r < offsets[E].
+int launch_ds_rows(const float* ds_part, int nparts, const int32_t* offsets, int E, int rows,
+                   float* dS, cudaStream_t s);
+
 // Test hook of the bounded device waits: the wait limit (ns) requested for
 // the next tensor-core GEMM launch, or 0; taking it clears the request.
 long long take_debug_expire();
