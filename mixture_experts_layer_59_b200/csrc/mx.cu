@@ -18,12 +18,39 @@ namespace moe {
 
 // ============================================================== weights
 // One block per (128 K, 128 output rows, expert): the bf16 source tile goes
-// to shared memory as [k][n], then thread (n, j) quantises column n over the
-// 32 K-values 32j..32j+31 and writes 32 contiguous bytes of output row n.
-constexpr int WQ_THREADS = 512;
+// to shared memory as [k][n] (all of the block's loads in flight before the
+// first store); then thread (p, j) quantises the two adjacent output rows
+// 2p, 2p+1 over the 32 K-values 32j..32j+31, reading both with one 32-bit
+// shared load per K-value, and writes 32 contiguous bytes of each row.
+// 256-thread blocks of at most 80 registers keep three blocks (96 KB of
+// loads) in flight per SM.
+constexpr int WQ_THREADS = 256;
+
+// Quantise 32 bf16 values held as the low (hi = false) or high halves of
+// packed pairs as one MXFP8 block (same arithmetic as mx_store_block, whose
+// bf16 rounding is exact here).
+__device__ __forceinline__ void mx_store_block_packed(const uint32_t* pk, bool hi, uint8_t* dst,
+                                                      uint8_t* sf) {
+  auto val = [&](int i) -> float {
+    return __uint_as_float(hi ? (pk[i] & 0xffff0000u) : (pk[i] << 16));
+  };
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(val(i)));
+  const uint32_t code = mx_scale_code(amax);
+  const float inv = mx_inv_scale(code);
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    w[i] = cvt_e4m3x2(val(4 * i) * inv, val(4 * i + 1) * inv) |
+           (cvt_e4m3x2(val(4 * i + 2) * inv, val(4 * i + 3) * inv) << 16);
+  reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  *sf = (uint8_t)code;
+}
 
 template <bool W13>
-__global__ void __launch_bounds__(WQ_THREADS)
+__global__ void __launch_bounds__(WQ_THREADS, 3)
 k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __restrict__ wb,
                    int K, int N, int Nout, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                    uint8_t* __restrict__ qa_r, uint8_t* __restrict__ sfa_r,
@@ -51,29 +78,42 @@ k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __
     *reinterpret_cast<uint4*>(&tile[v >> 4][(v & 15) * 8]) = u[i];
   }
   __syncthreads();
-  const int n = threadIdx.x & 127, j = threadIdx.x >> 7;
-  float v[32];
+  {
+    const int p = threadIdx.x & 63, j = threadIdx.x >> 6;
+    uint32_t pk[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(tile[32 * j + i][n]);
-  const int row = e * Nout + t * 128 + n;   // output row across experts (Nout % 128 == 0)
-  mx_store_block(v, q + (size_t)row * K + k0 + 32 * j,
-                 sf + mx_sf_offset(row, (k0 >> 5) + j, kchunks));
+    for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(&tile[32 * j + i][2 * p]);
+    const int row = e * Nout + t * 128 + 2 * p;   // output row across experts (Nout % 128 == 0)
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      mx_store_block_packed(pk, h == 1, q + (size_t)(row + h) * K + k0 + 32 * j,
+                            sf + mx_sf_offset(row + h, (k0 >> 5) + j, kchunks));
+  }
   if (W13 && qa_r != nullptr) {
     // row-wise: source row k0 + kk of W1 (t even) or W3 (t odd), 32 columns
     // starting at 128 (t/2) + 32 jb, in the weight's own [E, d, f] layout
-    const int kk = threadIdx.x & 127, jb = threadIdx.x >> 7;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 u = *reinterpret_cast<const uint4*>(&tile[kk][32 * jb + 8 * i]);
-      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) v[8 * i + c] = __bfloat162float(h[c]);
-    }
-    const int srow = e * K + k0 + kk;         // row of [E*d, f]
-    const int col = (t >> 1) * 128 + 32 * jb;
     uint8_t* qr = (t & 1) ? qb_r : qa_r;
     uint8_t* sr = (t & 1) ? sfb_r : sfa_r;
-    mx_store_block(v, qr + (size_t)srow * N + col, sr + mx_sf_offset(srow, col >> 5, N / 128));
+#pragma unroll
+    for (int it = 0; it < 512 / WQ_THREADS; ++it) {
+      const int item = threadIdx.x + it * WQ_THREADS;
+      const int kk = item & 127, jb = item >> 7;
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(&tile[kk][32 * jb + 8 * i]);
+        pk[4 * i] = w4.x; pk[4 * i + 1] = w4.y; pk[4 * i + 2] = w4.z; pk[4 * i + 3] = w4.w;
+      }
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        v[2 * i] = __uint_as_float(pk[i] << 16);
+        v[2 * i + 1] = __uint_as_float(pk[i] & 0xffff0000u);
+      }
+      const int srow = e * K + k0 + kk;         // row of [E*d, f]
+      const int col = (t >> 1) * 128 + 32 * jb;
+      mx_store_block(v, qr + (size_t)srow * N + col, sr + mx_sf_offset(srow, col >> 5, N / 128));
+    }
   }
 }
 
