@@ -544,6 +544,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         fl = gemm_flops(dom, cfg.T, cfg.d, cfg.f, cfg.k)
         roof = gemm_roofline(dom, fl, avg_s, peaks, peak_src)
         roof["traffic"] = traffic_for(dom, cfg.name)
+        # long runs settle under the power cap at a lower clock than the burst
+        # peak's: the burst peak scaled by the run's median over maximum SM clock
+        if clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+            scale = min(1.0, clocks["sm_mhz"] / clocks["sm_max_mhz"])
+            roof["frac_at_run_clock"] = roof["achieved"] / (roof["peak"] * scale)
         bf16_peak, bf16_sust = tensor_peaks(peaks, "bf16")
         g_fl = sum(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) * v[0] for n, v in gemm.items())
         g_ms = sum(v[1] for v in gemm.values())
