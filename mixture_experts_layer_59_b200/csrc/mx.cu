@@ -17,14 +17,18 @@
 namespace moe {
 
 // ============================================================== weights
-// One block per (128 K, 128 output rows, expert): the bf16 source tile goes
-// to shared memory as [k][n] (all of the block's loads in flight before the
-// first store); then thread (p, j) quantises the two adjacent output rows
-// 2p, 2p+1 over the 32 K-values 32j..32j+31, reading both with one 32-bit
-// shared load per K-value, and writes 32 contiguous bytes of each row.
-// 256-thread blocks of at most 80 registers keep three blocks (96 KB of
-// loads) in flight per SM.
+// One block per (32 K-rows, up to 512 columns, source matrix, expert) of a
+// weight [E, K, N] (N contiguous): the 32 rows' 1 KB runs arrive with all of
+// the block's loads in flight (8 per thread), so DRAM sees long contiguous
+// runs.  Thread p then quantises the two columns 2p, 2p+1 over these 32
+// K-values -- one MXFP8 block each, both read with one 32-bit shared load per
+// K-value -- and writes the 32 bytes into each column's output row (blocks
+// along K).  For the backward copies (blocks along N) the same tile gives
+// each of its 32 rows ncols / 32 blocks.
 constexpr int WQ_THREADS = 256;
+constexpr int WQ_ROWS = 32;          // one MXFP8 block along K
+constexpr int WQ_COLS = 512;
+constexpr int WQ_LD = WQ_COLS + 8;   // shared row stride (bf16): 16 bytes of padding
 
 // Quantise 32 bf16 values held as the low (hi = false) or high halves of
 // packed pairs as one MXFP8 block (same arithmetic as mx_store_block, whose
@@ -49,69 +53,72 @@ __device__ __forceinline__ void mx_store_block_packed(const uint32_t* pk, bool h
   *sf = (uint8_t)code;
 }
 
+// W13 = true: sources W1 (blockIdx.z even) and W3 (odd) [E, d, f] -> W13q
+// [E, 2f, d] (column n of W1 is row 256 (n/128) + n%128, of W3 that row +
+// 128) and, when qa_r is set, W1r / W3r [E, d, f] with blocks along f.
+// W13 = false: source W2 [E, f, d] -> W2q [E, d, f] (column n is row n).
 template <bool W13>
 __global__ void __launch_bounds__(WQ_THREADS, 3)
 k_mx_quant_weights(const __nv_bfloat16* __restrict__ wa, const __nv_bfloat16* __restrict__ wb,
-                   int K, int N, int Nout, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
+                   int K, int N, uint8_t* __restrict__ q, uint8_t* __restrict__ sf,
                    uint8_t* __restrict__ qa_r, uint8_t* __restrict__ sfa_r,
                    uint8_t* __restrict__ qb_r, uint8_t* __restrict__ sfb_r) {
-  // rows padded by 16 bytes: the row-wise pass reads 16-byte vectors of
-  // consecutive rows without bank conflicts
-  __shared__ __align__(16) __nv_bfloat16 tile[128][136];
-  const int k0 = blockIdx.x * 128, t = blockIdx.y, e = blockIdx.z;
-  const int kchunks = K / 128;
-  // source tile: 128 K-rows x 128 output rows (16-byte vectors of 8 bf16);
-  // output tile t of W13q is W1 (t even) or W3 (t odd), columns 128 (t/2)..
-  const __nv_bfloat16* base = W13 ? ((t & 1) ? wb : wa) + (size_t)(t >> 1) * 128
-                                  : wa + (size_t)t * 128;
-  constexpr int PER = 128 * 16 / WQ_THREADS;
+  __shared__ __align__(16) __nv_bfloat16 tile[WQ_ROWS][WQ_LD];
+  const int k0 = blockIdx.x * WQ_ROWS, c0 = blockIdx.y * WQ_COLS;
+  const int which = W13 ? (blockIdx.z & 1) : 0;
+  const int e = W13 ? (blockIdx.z >> 1) : blockIdx.z;
+  const int ncols = min(WQ_COLS, N - c0);             // a multiple of 128
+  const __nv_bfloat16* src = (which ? wb : wa) + ((size_t)e * K + k0) * N + c0;
+  constexpr int VPR = WQ_COLS / 8;                     // 16-byte vectors per tile row
+  constexpr int PER = WQ_ROWS * VPR / WQ_THREADS;
   uint4 u[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {   // all loads in flight before the shared stores
     const int v = threadIdx.x + i * WQ_THREADS;
-    u[i] = __ldg(reinterpret_cast<const uint4*>(base + ((size_t)e * K + k0 + (v >> 4)) * N +
-                                                (v & 15) * 8));
+    const int r = v / VPR, c = (v % VPR) * 8;
+    if (c < ncols) u[i] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)r * N + c));
   }
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int v = threadIdx.x + i * WQ_THREADS;
-    *reinterpret_cast<uint4*>(&tile[v >> 4][(v & 15) * 8]) = u[i];
+    const int r = v / VPR, c = (v % VPR) * 8;
+    if (c < ncols) *reinterpret_cast<uint4*>(&tile[r][c]) = u[i];
   }
   __syncthreads();
-  {
-    const int p = threadIdx.x & 63, j = threadIdx.x >> 6;
+  const int kchunks = K / 128;
+  if (2 * (int)threadIdx.x < ncols) {
+    const int p = threadIdx.x;
     uint32_t pk[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(&tile[32 * j + i][2 * p]);
-    const int row = e * Nout + t * 128 + 2 * p;   // output row across experts (Nout % 128 == 0)
+    for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(&tile[i][2 * p]);
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-      mx_store_block_packed(pk, h == 1, q + (size_t)(row + h) * K + k0 + 32 * j,
-                            sf + mx_sf_offset(row + h, (k0 >> 5) + j, kchunks));
+    for (int h = 0; h < 2; ++h) {
+      const int n = c0 + 2 * p + h;                    // source column
+      const int row = W13 ? e * 2 * N + 256 * (n >> 7) + 128 * which + (n & 127) : e * N + n;
+      mx_store_block_packed(pk, h == 1, q + (size_t)row * K + k0,
+                            sf + mx_sf_offset(row, k0 >> 5, kchunks));
+    }
   }
   if (W13 && qa_r != nullptr) {
-    // row-wise: source row k0 + kk of W1 (t even) or W3 (t odd), 32 columns
-    // starting at 128 (t/2) + 32 jb, in the weight's own [E, d, f] layout
-    uint8_t* qr = (t & 1) ? qb_r : qa_r;
-    uint8_t* sr = (t & 1) ? sfb_r : sfa_r;
-#pragma unroll
-    for (int it = 0; it < 512 / WQ_THREADS; ++it) {
-      const int item = threadIdx.x + it * WQ_THREADS;
-      const int kk = item & 127, jb = item >> 7;
+    uint8_t* qr = which ? qb_r : qa_r;
+    uint8_t* sr = which ? sfb_r : sfa_r;
+    const int nb = ncols / 32;                         // blocks along N per tile row
+    for (int item = threadIdx.x; item < WQ_ROWS * nb; item += WQ_THREADS) {
+      const int i = item / nb, b = item % nb;
       uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 w4 = *reinterpret_cast<const uint4*>(&tile[kk][32 * jb + 8 * i]);
-        pk[4 * i] = w4.x; pk[4 * i + 1] = w4.y; pk[4 * i + 2] = w4.z; pk[4 * i + 3] = w4.w;
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(&tile[i][32 * b + 8 * j]);
+        pk[4 * j] = w4.x; pk[4 * j + 1] = w4.y; pk[4 * j + 2] = w4.z; pk[4 * j + 3] = w4.w;
       }
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        v[2 * i] = __uint_as_float(pk[i] << 16);
-        v[2 * i + 1] = __uint_as_float(pk[i] & 0xffff0000u);
+      for (int j = 0; j < 16; ++j) {
+        v[2 * j] = __uint_as_float(pk[j] << 16);
+        v[2 * j + 1] = __uint_as_float(pk[j] & 0xffff0000u);
       }
-      const int srow = e * K + k0 + kk;         // row of [E*d, f]
-      const int col = (t >> 1) * 128 + 32 * jb;
+      const int srow = e * K + k0 + i;                 // row of [E*d, f]
+      const int col = c0 + 32 * b;
       mx_store_block(v, qr + (size_t)srow * N + col, sr + mx_sf_offset(srow, col >> 5, N / 128));
     }
   }
@@ -124,11 +131,12 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
   if (E == 0) return MOE_OK;
   {
     ProfScope _ps("mx_quant_weights", s);
-    k_mx_quant_weights<true><<<dim3(d / 128, (2 * f) / 128, E), WQ_THREADS, 0, s>>>(
-        (const __nv_bfloat16*)w1, (const __nv_bfloat16*)w3, d, f, 2 * f, w13q, w13s, w1rq, w1rs,
-        w3rq, w3rs);
-    k_mx_quant_weights<false><<<dim3(f / 128, d / 128, E), WQ_THREADS, 0, s>>>(
-        (const __nv_bfloat16*)w2, nullptr, f, d, d, w2q, w2s, nullptr, nullptr, nullptr, nullptr);
+    k_mx_quant_weights<true><<<dim3(d / WQ_ROWS, (f + WQ_COLS - 1) / WQ_COLS, 2 * E), WQ_THREADS,
+                               0, s>>>((const __nv_bfloat16*)w1, (const __nv_bfloat16*)w3, d, f,
+                                       w13q, w13s, w1rq, w1rs, w3rq, w3rs);
+    k_mx_quant_weights<false><<<dim3(f / WQ_ROWS, (d + WQ_COLS - 1) / WQ_COLS, E), WQ_THREADS,
+                                0, s>>>((const __nv_bfloat16*)w2, nullptr, f, d, w2q, w2s, nullptr,
+                                        nullptr, nullptr, nullptr);
   }
   MOE_CHECK_LAUNCH("mx_quant_weights");
   return MOE_OK;
