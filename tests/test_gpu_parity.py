@@ -496,3 +496,31 @@ def test_bounded_wait_expires_then_next_call_is_clean():
     H2, _ = B.moe_expert_ffn_fwd(x, w1, w3, w2, plan, k)
     B.moe_check_status()
     assert torch.equal(H2[:R], H0[:R])
+
+
+@pytest.mark.parametrize("T,d,E,k,round_mode", [(1000, 2048, 8, 4, B.MOE_ROUND_NONE),
+                                               (777, 7168, 16, 2, B.MOE_ROUND_NEAREST),
+                                               (130, 128, 4, 1, B.MOE_ROUND_NONE),
+                                               (0, 256, 8, 2, B.MOE_ROUND_NONE)])
+def test_gather_rows_bit_exact_with_padding_zeroed(T, d, E, k, round_mode):
+    """moe_gather_rows (the row gather behind every grouped GEMM): row r of
+    the row space is row row_token[r] of the token-major source, bit for bit,
+    including rows added by token rounding; padding rows are zeros, and rows
+    at or beyond offsets[E] are left untouched."""
+    g = torch.Generator().manual_seed(T + d)
+    x = torch.randn(max(T, 1), d, generator=g).to(torch.bfloat16)[:T].cuda()
+    lo = torch.randn(T, E, generator=g).cuda()
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=T, E=E)
+    plan = B.moe_permute(idx, gate, logits, E, round_mode)
+    cap = B.moe_row_capacity(T, E, k)
+    out = torch.full((cap, d), 7.0, dtype=torch.bfloat16, device="cuda")   # sentinel
+    B.moe_gather_rows(x, plan, k, out=out)
+    torch.cuda.synchronize()
+    B.moe_check_status()
+    R = int(plan["offsets"][-1])
+    tok = plan["row_token"][:R].long()
+    live = tok >= 0
+    want = torch.zeros(R, d, dtype=torch.bfloat16, device="cuda")
+    want[live] = x[tok[live]]
+    assert torch.equal(out[:R], want)
+    assert bool((out[R:] == 7.0).all())
