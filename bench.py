@@ -66,6 +66,9 @@ def parse_args():
     ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer written between steps")
     ap.add_argument("--balance-loss", type=float, default=None,
                     help="add the load-balance loss (this lambda) and its gradient to every step")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism: each rank keeps E/N experts and its own T tokens; "
+                         "rows travel to the experts' ranks (NCCL send/recv)")
     return ap.parse_args()
 
 
@@ -630,6 +633,75 @@ def run_ours(args, cfg, rank, world, local_rank):
     return 0
 
 
+def run_ep(args, cfg, rank, world, local_rank):
+    """Expert-parallel step (ExpertParallelMoE over torch.distributed): every
+    rank routes its own T tokens, owns E / world experts, and exchanges the
+    permuted rows with the experts' ranks.  Timed like the main arm: CUDA
+    events around each step (the exchange's host synchronisation included),
+    L2 flushed between steps, max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_layer_59_b200 import binding as B
+    from mixture_experts_layer_59_b200 import synth
+    from mixture_experts_layer_59_b200.ep import ExpertParallelMoE, TorchDistExchange
+
+    dev = torch.device("cuda", local_rank)
+    inp = synth.make_inputs(cfg, seed=rank, device=dev)
+    wts = synth.make_inputs(cfg, seed=0, device=dev)     # the same weights on every rank
+    El = cfg.E // world
+    sl = slice(rank * El, (rank + 1) * El)
+    w1, w3, w2 = (wts[n][sl].contiguous() for n in ("w1", "w3", "w2"))
+    wg = wts["w_gate"]
+    x, dout, lo = inp["x"], inp["dout"], inp["logits_override"]
+    layer = ExpertParallelMoE(TorchDistExchange(), cfg.E, cfg.k)
+    flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
+
+    def one_step():
+        layer.forward(x, wg, w1, w3, w2, logits_override=lo)
+        layer.backward(dout)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    B.moe_check_status()
+    torch.cuda.synchronize()
+    dist.barrier()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record()
+        one_step()
+        ends[i].record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    dist.barrier()
+    clocks = sampler.stop(t0, t1)
+    B.moe_check_status()
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": job_tokens_per_s(world, cfg.T, args.steps, total_ms),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; random-init weights N(0,0.02^2), x,dO ~ N(0,1))",
+        "config": dict(workload_config(cfg, args), parallelism=f"ep{world}",
+                       experts_per_rank=El),
+        "local_rows_rank0": layer.routing["local_rows"],
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     from mixture_experts_layer_59_b200 import synth
@@ -645,16 +717,30 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, cfg, rank, world)
-    if world > 1:
+    pg = world > 1 or args.ep
+    if pg:
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
+        if world == 1:   # a one-rank group for the expert-parallel arm
+            import socket
+            with socket.socket() as sk:
+                sk.bind(("127.0.0.1", 0))
+                port = sk.getsockname()[1]
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(port))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local_rank))
     try:
+        if args.ep:
+            if cfg.E % world:
+                raise SystemExit(f"--ep needs E ({cfg.E}) divisible by the number of GPUs ({world})")
+            return run_ep(args, cfg, rank, world, local_rank)
         return run_ours(args, cfg, rank, world, local_rank)
     finally:
-        if world > 1:
+        if pg:
             import torch.distributed as dist
             dist.destroy_process_group()
 

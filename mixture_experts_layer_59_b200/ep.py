@@ -244,14 +244,23 @@ class ExpertParallelMoE:
         offsets_h, seg_h, recv_rows_h, recv_row_h, loc_h = (tab[cut[i]:cut[i + 1]]
                                                              for i in range(len(n)))
         sends, recvs = self._blocks(offsets_h, seg_h, recv_rows_h, recv_row_h)
-        rows = max(128, loc_h[El])
-        xg_loc = torch.empty(rows, d, device=x.device, dtype=x.dtype)
-        gate_loc = torch.zeros(rows, device=x.device, dtype=plan["row_gate"].dtype)
-        self.ex.move(xg, xg_loc, sends, recvs)
-        self.ex.move(plan["row_gate"], gate_loc, sends, recvs)
+        # one rank: the received layout is the row space itself, so the rows stay put
+        self.alone = G == 1
+        if self.alone:
+            rows = max(128, xg.shape[0] // 128 * 128)     # >= offsets[E], a multiple of 128
+            xg_loc, gate_loc = xg[:rows], plan["row_gate"][:rows]
+        else:
+            rows = max(128, loc_h[El])
+            xg_loc = torch.empty(rows, d, device=x.device, dtype=x.dtype)
+            gate_loc = torch.zeros(rows, device=x.device, dtype=plan["row_gate"].dtype)
+            self.ex.move(xg, xg_loc, sends, recvs)
+            self.ex.move(plan["row_gate"], gate_loc, sends, recvs)
         H_loc, Y_loc = ops.expert_rows_fwd(xg_loc, w1, w3, w2, local_offsets)
-        y_perm = torch.empty_like(xg)
-        self.ex.move(Y_loc, y_perm, recvs, sends)          # back to the tokens' ranks
+        if self.alone:
+            y_perm = Y_loc
+        else:
+            y_perm = torch.empty_like(xg)
+            self.ex.move(Y_loc, y_perm, recvs, sends)      # back to the tokens' ranks
         out = ops.combine(y_perm, plan, T, E, k)
         self._saved = dict(x=x, w_gate=w_gate, w=(w1, w3, w2), logits=logits, idx=idx, gate=gate,
                            plan=plan, xg_loc=xg_loc, gate_loc=gate_loc, H_loc=H_loc,
@@ -265,15 +274,21 @@ class ExpertParallelMoE:
         s, ops, k = self._saved, self.ops, self.k
         T, d = dout.shape
         dog = ops.gather_rows(dout, s["plan"], k)
-        dog_loc = torch.empty(s["rows"], d, device=dout.device, dtype=dout.dtype)
-        self.ex.move(dog, dog_loc, s["sends"], s["recvs"])
+        if self.alone:
+            dog_loc = dog[:s["rows"]]
+        else:
+            dog_loc = torch.empty(s["rows"], d, device=dout.device, dtype=dout.dtype)
+            self.ex.move(dog, dog_loc, s["sends"], s["recvs"])
         w1, w3, w2 = s["w"]
         g = ops.expert_rows_bwd(dog_loc, s["xg_loc"], s["gate_loc"], s["H_loc"], w1, w3, w2,
                                 s["local_offsets"])
-        dx_rows = torch.empty_like(dog)
-        dS = torch.zeros(s["cap"], device=dout.device, dtype=g["dS"].dtype)
-        self.ex.move(g["dX_rows"], dx_rows, s["recvs"], s["sends"])
-        self.ex.move(g["dS"], dS, s["recvs"], s["sends"])
+        if self.alone:
+            dx_rows, dS = g["dX_rows"], g["dS"]
+        else:
+            dx_rows = torch.empty_like(dog)
+            dS = torch.zeros(s["cap"], device=dout.device, dtype=g["dS"].dtype)
+            self.ex.move(g["dX_rows"], dx_rows, s["recvs"], s["sends"])
+            self.ex.move(g["dS"], dS, s["recvs"], s["sends"])
         t = ops.token_bwd(dx_rows, dS, s["x"], s["w_gate"], s["idx"], s["gate"], s["plan"],
                           s["router_grad"])
         dw_gate = self.ex.all_reduce_sum(t["dw_gate"])
