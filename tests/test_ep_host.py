@@ -126,3 +126,39 @@ def test_ep_two_gloo_ranks_match_the_one_device_layer(tmp_path):
     for r in res:
         r["local_rows"] = int(r["local_rows"])
     _check(res, 2, s["T"], s["d"], s["f"], s["E"], s["k"], 5)
+
+
+def test_ep_rank_with_no_rows_gets_zero_expert_gradients():
+    """Routing that sends every token to the first rank's experts: the other
+    rank receives no rows, its grouped GEMMs see empty segments, and its
+    expert gradients come back zero; the layer still matches the oracle."""
+    import torch
+    from mixture_experts_layer_59_b200.ep import ExpertParallelMoE
+    G, T, d, f, E, k = 2, 64, 64, 32, 4, 2
+    x, dout, wg, w1, w3, w2 = EO.make_problem(G, T, d, f, E, k, 9)
+    lo = np.full((G * T, E), -5.0)
+    lo[:, 0], lo[:, 1] = 1.0, 0.5               # experts 0 and 1 live on rank 0
+    lo += 1e-3 * np.random.default_rng(9).standard_normal(lo.shape)
+    El = E // G
+    t = torch.from_numpy
+
+    def fn(r, ex):
+        sl, el = slice(r * T, (r + 1) * T), slice(r * El, (r + 1) * El)
+        layer = ExpertParallelMoE(ex, E, k, ops=EO.OracleOps())
+        out = layer.forward(t(x[sl]), t(wg), t(w1[el]), t(w3[el]), t(w2[el]),
+                            logits_override=t(lo[sl]))
+        g = layer.backward(t(dout[sl]))
+        return dict(out=out.numpy(), dx=g["dx"].numpy(), dw1=g["dw1"].numpy(),
+                    dw2=g["dw2"].numpy(), local_rows=layer.routing["local_rows"])
+
+    res = LocalGroup(G, timeout=60).run(fn)
+    from oracle import moe_oracle as O
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k, logits_override=lo, staged=False)
+    bwd = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False, router_grad_on=False)
+    assert res[1]["local_rows"] == 0
+    assert not res[1]["dw1"].any() and not res[1]["dw2"].any()
+    for r in range(G):
+        sl, el = slice(r * T, (r + 1) * T), slice(r * El, (r + 1) * El)
+        np.testing.assert_allclose(res[r]["out"], fwd["out"][sl], rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(res[r]["dx"], bwd["dx"][sl], rtol=1e-9, atol=1e-11)
+        np.testing.assert_allclose(res[r]["dw1"], bwd["dw1"][el], rtol=1e-9, atol=1e-11)

@@ -143,3 +143,42 @@ def test_ep_receive_plan_matches_brute_force_and_flags_bad_counts():
     off = plan["offsets"].cpu().numpy()
     np.testing.assert_array_equal(seg.cpu().numpy(), off[1:] - off[:-1])
     B.moe_check_status()
+
+
+def test_ep_emulated_rank_without_rows():
+    """Every token routed to the first rank's experts: the second rank runs
+    its grouped GEMMs on an empty row space (offsets all zero) and returns
+    zero expert gradients; both ranks match the oracle."""
+    G, T, d, f, E, k = 2, 256, 256, 256, 8, 2
+    El = E // G
+    x, dout, wg, w1, w3, w2, _ = _problem(G, T, d, f, E, k, 31)
+    g = torch.Generator().manual_seed(31)
+    lo = torch.full((G * T, E), -5.0) + 1e-3 * torch.randn(G * T, E, generator=g)
+    lo[:, :El] += 6.0 + torch.rand(G * T, El, generator=g)     # experts 0..El-1: rank 0
+    B.lib()
+    dev = [t.cuda() for t in (x, dout, wg, w1, w3, w2, lo)]
+
+    def rank_fn(r, ex):
+        xc, dc, wgc, w1c, w3c, w2c, loc = dev
+        sl, el = slice(r * T, (r + 1) * T), slice(r * El, (r + 1) * El)
+        layer = EP.ExpertParallelMoE(ex, E, k)
+        out = layer.forward(xc[sl].contiguous(), wgc, w1c[el].contiguous(), w3c[el].contiguous(),
+                            w2c[el].contiguous(), logits_override=loc[sl].contiguous())
+        gr = layer.backward(dc[sl].contiguous())
+        torch.cuda.synchronize()
+        return dict(out=out.clone(), rows=layer.routing["local_rows"],
+                    **{n: gr[n].clone() for n in ("dx", "dw1", "dw3", "dw2")})
+
+    res = EP.LocalGroup(G, timeout=120).run(rank_fn)
+    B.moe_check_status()
+    assert res[1]["rows"] == 0
+    for n in ("dw1", "dw3", "dw2"):
+        assert not bool(res[1][n].any()), n
+    fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), k, logits_override=f64(lo))
+    bwd = O.layer_bwd(f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd,
+                      router_grad_on=False)
+    for r in range(G):
+        sl, el = slice(r * T, (r + 1) * T), slice(r * El, (r + 1) * El)
+        assert_close(res[r]["out"], fwd["out"][sl], f"out rank {r}", BF16_TOL)
+        assert_close(res[r]["dx"], bwd["dx"][sl], f"dx rank {r}", BF16_TOL)
+    assert_close(res[0]["dw1"], bwd["dw1"][:El], "dw1 rank 0", BF16_TOL)
