@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1],
                     help="0 = softmax over the top-k logits, 1 = softmax over all E then top-k")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--e2e-chunks", type=int, default=2,
+                    help="row chunks per copied tensor in the e2e pipeline (one copy stream each)")
     ap.add_argument("--cpu-sample", type=int, default=2048, help="tokens of the cpu_baseline sample")
     ap.add_argument("--cpu-sample-1core", type=int, default=512,
                     help="tokens of the one-core oracle timing (0: skip)")
@@ -482,9 +484,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     # ---- end to end through the public API with host buffers: every step
     # uploads its own inputs (x, dO) from pinned host memory and reads its
     # results (out, dx) back.  As in a training loop with a prefetching loader,
-    # the copies of neighbouring steps run on two copy streams while this
-    # step's kernels run; two layer objects alternate so that no buffer is
-    # rewritten while a copy still reads it.  (No L2 flush here: each step's
+    # the copies of neighbouring steps run on copy streams while this step's
+    # kernels run; two layer objects alternate so that no buffer is rewritten
+    # while a copy still reads it.  (No L2 flush here: each step's
     # inputs arrive by copy.)
     step2 = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round,
                          balance_lambda=args.balance_loss, gate_mode=args.gate_mode,
@@ -497,37 +499,63 @@ def run_ours(args, cfg, rank, world, local_rank):
     dx_h = [torch.empty_like(step.grads["dx"], device="cpu").pin_memory() for _ in range(2)]
     x_d = [torch.empty_like(x) for _ in range(2)]
     d_d = [torch.empty_like(dout) for _ in range(2)]
-    up_s, comp_s, down_s = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    # the copies are split into row chunks, one copy stream per chunk and
+    # direction (x and dO up, out and dx down), so that they spread over the
+    # copy engines
+    nch = max(1, args.e2e_chunks)
+
+    def chunks(t):
+        return list(t.chunk(nch, dim=0))
+
+    up_s = [torch.cuda.Stream() for _ in range(2 * nch)]
+    down_s = [torch.cuda.Stream() for _ in range(2 * nch)]
+    comp_s = torch.cuda.Stream()
+    up_pairs = [list(zip(chunks(x_d[b]) + chunks(d_d[b]), chunks(x_h) + chunks(d_h)))
+                for b in range(2)]
+    down_pairs = [list(zip(chunks(out_h[b]) + chunks(dx_h[b]),
+                           chunks(objs[b].out) + chunks(objs[b].grads["dx"]))) for b in range(2)]
 
     def pipeline(n):
         done, down = [None] * n, [None] * n
         start = torch.cuda.Event(enable_timing=True)
-        start.record(up_s)
+        start.record(up_s[0])
+        for s_ in up_s[1:]:
+            s_.wait_event(start)
         for i in range(n):
             b = i % 2
-            with torch.cuda.stream(up_s):
-                if i >= 2:
-                    up_s.wait_event(done[i - 2])        # step i-2 finished with x_d[b], d_d[b]
-                x_d[b].copy_(x_h, non_blocking=True)
-                d_d[b].copy_(d_h, non_blocking=True)
-                up = torch.cuda.Event()
-                up.record(up_s)
+            ups = []
+            for s_, (dst, src) in zip(up_s, up_pairs[b]):
+                with torch.cuda.stream(s_):
+                    if i >= 2:
+                        s_.wait_event(done[i - 2])      # step i-2 finished with this buffer
+                    dst.copy_(src, non_blocking=True)
+                    ev = torch.cuda.Event()
+                    ev.record(s_)
+                    ups.append(ev)
             with torch.cuda.stream(comp_s):
-                comp_s.wait_event(up)
+                for ev in ups:
+                    comp_s.wait_event(ev)
                 if i >= 2:
-                    comp_s.wait_event(down[i - 2])      # step i-2's results are read back
+                    for ev in down[i - 2]:              # step i-2's results are read back
+                        comp_s.wait_event(ev)
                 objs[b].forward(x_d[b], wg, w1, w3, w2, lo, lb, logit_noise=noise)
                 objs[b].backward(d_d[b])
                 done[i] = torch.cuda.Event()
                 done[i].record(comp_s)
-            with torch.cuda.stream(down_s):
-                down_s.wait_event(done[i])
-                out_h[b].copy_(objs[b].out, non_blocking=True)
-                dx_h[b].copy_(objs[b].grads["dx"], non_blocking=True)
-                down[i] = torch.cuda.Event(enable_timing=True)
-                down[i].record(down_s)
+            down[i] = []
+            for s_, (dst, src) in zip(down_s, down_pairs[b]):
+                with torch.cuda.stream(s_):
+                    s_.wait_event(done[i])
+                    dst.copy_(src, non_blocking=True)
+                    ev = torch.cuda.Event(enable_timing=True)
+                    ev.record(s_)
+                    down[i].append(ev)
+        end = torch.cuda.Event(enable_timing=True)
+        for ev in down[n - 1][1:]:
+            down_s[0].wait_event(ev)
+        end.record(down_s[0])
         torch.cuda.synchronize()
-        return start.elapsed_time(down[n - 1])
+        return start.elapsed_time(end)
 
     e2e_ms = []
     if args.e2e_steps > 0:
@@ -631,7 +659,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_total / len(e2e_ms) if e2e_ms else None,
-                "pipelined": "upload of step i+1 and read-back of step i-1 overlap step i's kernels"},
+                "pipelined": "upload of step i+1 and read-back of step i-1 overlap step i's kernels; "
+                             f"{nch} row chunk(s) per tensor, one copy stream per chunk and direction"},
         "clocks": clocks,
         "gpu_launches": launches,
         "hbm_kernels": hbm_kernels,
