@@ -354,17 +354,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           const int k0 = kb * BK;
           if constexpr (KIND == K_UP) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
-            const int nf = ti.ntile * (BN / 2);
-#pragma unroll
-            for (int h = 0; h < BN / 128; ++h) {
-              tma_load_3d(sB + h * ATOM, &a.mB0, &full_bar[stage], nf + 64 * h, k0, ti.e);
-              tma_load_3d(sB + (BN / 128 + h) * ATOM, &a.mB1, &full_bar[stage], nf + 64 * h, k0, ti.e);
-            }
+            const int nf = ti.ntile * (BN / 2);   // BN / 128 atoms of W1, then of W3
+            tma_load_4d(sB, &a.mB0, &full_bar[stage], 0, k0, nf / 64, ti.e);
+            tma_load_4d(sB + (BN / 128) * ATOM, &a.mB1, &full_bar[stage], 0, k0, nf / 64, ti.e);
           } else if constexpr (KIND == K_DOWN) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
-#pragma unroll
-            for (int h = 0; h < BN / 64; ++h)
-              tma_load_3d(sB + h * ATOM, &a.mB0, &full_bar[stage], ti.n0 + 64 * h, k0, ti.e);
+            tma_load_4d(sB, &a.mB0, &full_bar[stage], 0, k0, ti.n0 / 64, ti.e);   // BN / 64 atoms
           } else if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
             tma_load_3d(sB, &a.mB0, &full_bar[stage], k0, ti.n0, ti.e);
@@ -417,11 +412,8 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             tma_load_2d(sB, &a.mB0, &full_bar[stage], kk, ti.n0);
           } else {  // varlen-K: A and B are row-space activations, MN-major
             const int r = ti.krow0 + k0;
-            tma_load_2d(sA, &a.mA, &full_bar[stage], ti.m0, r);
-            tma_load_2d(sA + ATOM, &a.mA, &full_bar[stage], ti.m0 + 64, r);
-#pragma unroll
-            for (int h = 0; h < BN / 64; ++h)
-              tma_load_2d(sB + h * ATOM, &a.mB0, &full_bar[stage], ti.n0 + 64 * h, r);
+            tma_load_4d(sA, &a.mA, &full_bar[stage], 0, r, ti.m0 / 64, 0);    // 2 atoms
+            tma_load_4d(sB, &a.mB0, &full_bar[stage], 0, r, ti.n0 / 64, 0);   // BN / 64 atoms
           }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
@@ -857,6 +849,27 @@ static int make_store_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint6
   return make_map_2d(m, ptr, inner, outer, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// bf16 [batch, outer, inner] (inner contiguous, a multiple of 64) as the
+// 4-d view [batch][inner / 64][outer][64]: one box brings `atoms` adjacent
+// 64-column blocks of BK rows, stored block after block (BK x 128 bytes
+// each, 128-byte swizzle) -- the shared-memory layout of an MN-major
+// operand -- so a stage's operand takes one copy instead of one per block.
+static int make_map_atoms(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer,
+                          uint64_t batch, uint32_t atoms) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (inner % 64 != 0) return fail(MOE_ERR_INVALID_ARG, "operand width not a multiple of 64");
+  cuuint64_t dims[4] = {64, outer, inner / 64, batch};
+  cuuint64_t strides[3] = {inner * 2, 128, inner * outer * 2};
+  cuuint32_t box[4] = {64, (cuuint32_t)BK, atoms, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (atoms) failed: " + std::to_string((int)r));
+  return MOE_OK;
+}
+
 // bf16 [d2, d1, d0] (d0 innermost) viewed in boxes of box1 x box0.
 static int make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
                        uint32_t box0, uint32_t box1) {
@@ -1029,8 +1042,8 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
     a.N = 2 * f;
     a.K = d;
     if ((rc = make_map_2d(&a.mA, xg, d, cap, 64, BM))) return rc;
-    if ((rc = make_map_3d(&a.mB0, p.w1, f, d, E, 64, 64))) return rc;
-    if ((rc = make_map_3d(&a.mB1, p.w3, f, d, E, 64, 64))) return rc;
+    if ((rc = make_map_atoms(&a.mB0, p.w1, f, d, E, 256 / 128))) return rc;
+    if ((rc = make_map_atoms(&a.mB1, p.w3, f, d, E, 256 / 128))) return rc;
     if ((rc = make_store_map(&a.sO0, H, 2 * f, cap))) return rc;
     if ((rc = make_store_map(&a.sO1, act, f, cap))) return rc;
     if ((rc = launch<K_UP, 256>(a, num_sms, s))) return rc;
@@ -1041,7 +1054,7 @@ int tc_ffn_fwd(const FfnPtrs& p, const void* xg, void* H, void* act, void* Y, in
     a.K = f;
     const int bn = pick_bn(d);
     if ((rc = make_map_2d(&a.mA, act, f, cap, 64, BM))) return rc;
-    if ((rc = make_map_3d(&a.mB0, p.w2, d, f, E, 64, 64))) return rc;
+    if ((rc = make_map_atoms(&a.mB0, p.w2, d, f, E, bn / 64))) return rc;
     if ((rc = make_store_map(&a.sO0, Y, d, cap))) return rc;
     if ((rc = launch_bn<K_DOWN>(a, bn, num_sms, s))) return rc;
   }
@@ -1154,8 +1167,8 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     a.M = f;
     a.N = d;
     const int bn = pick_bn(d);
-    if ((rc = make_map_2d(&a.mA, gact, f, cap, 64, 64))) return rc;
-    if ((rc = make_map_2d(&a.mB0, dog, d, cap, 64, 64))) return rc;
+    if ((rc = make_map_atoms(&a.mA, gact, f, cap, 1, BM / 64))) return rc;
+    if ((rc = make_map_atoms(&a.mB0, dog, d, cap, 1, bn / 64))) return rc;
     if ((rc = make_store_map(&a.sO0, dw2, d, (uint64_t)E * f))) return rc;
     if ((rc = launch_bn<K_DW2>(a, bn, num_sms, s))) return rc;
   }
@@ -1164,8 +1177,8 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     a.M = d;
     a.N = 2 * f;
     const int bn = pick_bn(2 * f);
-    if ((rc = make_map_2d(&a.mA, xg, d, cap, 64, 64))) return rc;
-    if ((rc = make_map_2d(&a.mB0, dH, 2 * f, cap, 64, 64))) return rc;
+    if ((rc = make_map_atoms(&a.mA, xg, d, cap, 1, BM / 64))) return rc;
+    if ((rc = make_map_atoms(&a.mB0, dH, 2 * f, cap, 1, bn / 64))) return rc;
     if ((rc = make_store_map(&a.sO0, dw1, f, (uint64_t)E * d))) return rc;
     if ((rc = make_store_map(&a.sO1, dw3, f, (uint64_t)E * d))) return rc;
     if ((rc = launch_bn<K_DW13>(a, bn, num_sms, s))) return rc;
