@@ -143,11 +143,11 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
 }
 
 // ============================================================== rows
-// Blocks [0, nbt) own tokens (one warp per token): lanes 4g..4g+3 hold the 32
-// elements of one block as four 16-byte vectors, share its maximum by
+// The last nbt blocks own tokens (one warp per token): lanes 4g..4g+3 hold
+// the 32 elements of one block as four 16-byte vectors, share its maximum by
 // shuffles, and write 8 E4M3 bytes each to every row of the token; the first
-// lane of the group writes the scale.  The remaining blocks zero the padding
-// rows (elements and scales).
+// lane of the group writes the scale.  The first blocks of the grid zero the
+// padding rows (elements and scales) beside them.
 __global__ void __launch_bounds__(256)
 k_mx_scatter_rows(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_row,
                   const int32_t* __restrict__ extra_row, const int32_t* __restrict__ row_token,
@@ -156,8 +156,9 @@ k_mx_scatter_rows(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict
   __shared__ int s_extra[8][256];   // rows added by rounding, per warp (E <= 256)
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nvec = d / 8, kchunks = d / 128;
-  if ((int)blockIdx.x < nbt) {
-    const int t = blockIdx.x * 8 + w;
+  const int nzb = gridDim.x - nbt;        // the first nzb blocks zero the padding rows
+  if ((int)blockIdx.x >= nzb) {
+    const int t = (blockIdx.x - nzb) * 8 + w;
     if (t >= T_) return;  // whole warp
     const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
     int rk[8];
@@ -212,13 +213,17 @@ k_mx_scatter_rows(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict
       }
     }
   } else {
+    // a warp tests 32 rows at once and zeroes the padding rows among them
     const int R = offsets[E];
-    const int nb = gridDim.x - nbt;
-    for (int r = (blockIdx.x - nbt) * 8 + w; r < R; r += nb * 8) {
-      if (row_token[r] >= 0) continue;
-      uint4* d4 = reinterpret_cast<uint4*>(q + (size_t)r * d);
-      for (int i = lane; i < d / 16; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
-      for (int kb = lane; kb < d / 32; kb += 32) sf[mx_sf_offset(r, kb, kchunks)] = 0;
+    for (int r0 = (blockIdx.x * 8 + w) * 32; r0 < R; r0 += nzb * 8 * 32) {
+      unsigned bal = __ballot_sync(0xffffffffu, r0 + lane < R && row_token[r0 + lane] < 0);
+      while (bal) {
+        const int r = r0 + __ffs(bal) - 1;
+        bal &= bal - 1;
+        uint4* d4 = reinterpret_cast<uint4*>(q + (size_t)r * d);
+        for (int i = lane; i < d / 16; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
+        for (int kb = lane; kb < d / 32; kb += 32) sf[mx_sf_offset(r, kb, kchunks)] = 0;
+      }
     }
   }
 }

@@ -33,9 +33,10 @@ template <> struct Vec<float> {
 // ============================================================== scatter rows
 // dst[row, :] = src[t, :] for every row of token t (its kept slots, then the
 // rows added by token rounding); rows that hold no pair (padding, token -1)
-// are zeroed.  Blocks [0, nbt) own tokens, one warp per token, so each source
-// row is read once and written to its k rows with coalesced 16-byte stores;
-// the remaining blocks zero the padding rows.
+// are zeroed.  The last nbt blocks own tokens, one warp per token, so each
+// source row is read once and written to its k rows with coalesced 16-byte
+// stores; the first blocks of the grid zero the padding rows (first, so that
+// this runs beside the token blocks instead of after them).
 template <class T>
 __global__ void __launch_bounds__(256)
 k_scatter_rows(const T* __restrict__ src, const int32_t* __restrict__ slot_row,
@@ -44,8 +45,9 @@ k_scatter_rows(const T* __restrict__ src, const int32_t* __restrict__ slot_row,
                T* __restrict__ dst) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int nvec = width / Vec<T>::N;
-  if ((int)blockIdx.x < nbt) {
-    const int t = blockIdx.x * 8 + w;
+  const int nzb = gridDim.x - nbt;        // the first nzb blocks zero the padding rows
+  if ((int)blockIdx.x >= nzb) {
+    const int t = (blockIdx.x - nzb) * 8 + w;
     if (t >= T_) return;
     const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
     int rk[8];
@@ -72,12 +74,105 @@ k_scatter_rows(const T* __restrict__ src, const int32_t* __restrict__ slot_row,
       }
     }
   } else {
+    // a warp tests 32 rows at once and zeroes the padding rows among them
     const int R = offsets[E];
-    const int nb = gridDim.x - nbt;
-    for (int r = (blockIdx.x - nbt) * 8 + w; r < R; r += nb * 8) {
-      if (row_token[r] >= 0) continue;
-      uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)r * width);
-      for (int i = lane; i < nvec; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
+    for (int r0 = (blockIdx.x * 8 + w) * 32; r0 < R; r0 += nzb * 8 * 32) {
+      const int r = r0 + lane;
+      unsigned bal = __ballot_sync(0xffffffffu, r < R && row_token[r] < 0);
+      while (bal) {
+        const int b = __ffs(bal) - 1;
+        bal &= bal - 1;
+        uint4* d4 = reinterpret_cast<uint4*>(dst + (size_t)(r0 + b) * width);
+        for (int i = lane; i < nvec; i += 32) d4[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+}
+
+// 32-byte global accesses (sm_100 256-bit loads and stores).
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint4& a, uint4& b) {
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+               : "l"(p));
+}
+__device__ __forceinline__ void st_v8(void* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y),
+               "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+// The same scatter for rows of a multiple of 32 bytes (32-byte aligned): a
+// warp loads a whole 32 * SR_UNITS-unit slice of its token's row (SR_UNITS
+// 32-byte loads per lane in flight) and then writes that slice to each of
+// the token's rows in turn, so each destination row is written as one
+// contiguous burst.  Rows of up to 32 * SR_UNITS * 32 bytes take one pass.
+// The padding rows are zeroed by the first blocks of the grid, so that this
+// work runs beside the token blocks instead of after them.
+constexpr int SR_UNITS = 4;
+
+__global__ void __launch_bounds__(256)
+k_scatter_rows_wide(const uint8_t* __restrict__ src, const int32_t* __restrict__ slot_row,
+                    const int32_t* __restrict__ extra_row, const int32_t* __restrict__ row_token,
+                    const int32_t* __restrict__ offsets, int T_, int nunit, int E, int k, int nbt,
+                    uint8_t* __restrict__ dst) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const size_t rb = (size_t)nunit * 32;   // bytes per row
+  const int nzb = gridDim.x - nbt;        // the first nzb blocks zero the padding rows
+  if ((int)blockIdx.x >= nzb) {
+    const int t = (blockIdx.x - nzb) * 8 + w;
+    if (t >= T_) return;
+    const int mine = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    int rk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) rk[j] = __shfl_sync(0xffffffffu, mine, j);
+    const uint8_t* s = src + (size_t)t * rb;
+    for (int u0 = 0; u0 < nunit; u0 += 32 * SR_UNITS) {
+      uint4 va[SR_UNITS], vb[SR_UNITS];
+#pragma unroll
+      for (int q = 0; q < SR_UNITS; ++q) {
+        const int u = u0 + q * 32 + lane;
+        if (u < nunit) ld_nc_v8(s + (size_t)u * 32, va[q], vb[q]);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (rk[j] < 0) continue;
+        uint8_t* d = dst + (size_t)rk[j] * rb;
+#pragma unroll
+        for (int q = 0; q < SR_UNITS; ++q) {
+          const int u = u0 + q * 32 + lane;
+          if (u < nunit) st_v8(d + (size_t)u * 32, va[q], vb[q]);
+        }
+      }
+      if (extra_row != nullptr) {
+        for (int e0 = 0; e0 < E; e0 += 32) {
+          const int re = e0 + lane < E ? extra_row[(size_t)t * E + e0 + lane] : -1;
+          unsigned bal = __ballot_sync(0xffffffffu, re >= 0);
+          while (bal) {
+            const int b = __ffs(bal) - 1;
+            bal &= bal - 1;
+            uint8_t* d = dst + (size_t)__shfl_sync(0xffffffffu, re, b) * rb;
+#pragma unroll
+            for (int q = 0; q < SR_UNITS; ++q) {
+              const int u = u0 + q * 32 + lane;
+              if (u < nunit) st_v8(d + (size_t)u * 32, va[q], vb[q]);
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // a warp tests 32 rows at once and zeroes the padding rows among them
+    const int R = offsets[E];
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    for (int r0 = (blockIdx.x * 8 + w) * 32; r0 < R; r0 += nzb * 8 * 32) {
+      const int r = r0 + lane;
+      unsigned bal = __ballot_sync(0xffffffffu, r < R && row_token[r] < 0);
+      while (bal) {
+        const int b = __ffs(bal) - 1;
+        bal &= bal - 1;
+        uint8_t* d = dst + (size_t)(r0 + b) * rb;
+        for (int u = lane; u < nunit; u += 32) st_v8(d + (size_t)u * 32, z, z);
+      }
     }
   }
 }
@@ -87,7 +182,13 @@ int launch_scatter_rows(const void* src, const int32_t* slot_row, const int32_t*
                         int k, int dtype, void* dst, cudaStream_t s) {
   const int nbt = (T + 7) / 8;
   const int blocks = nbt + device_sm_count() * 2;
-  if (dtype == MOE_BF16) {
+  const size_t row_bytes = (size_t)width * (dtype == MOE_BF16 ? 2 : 4);
+  if (row_bytes % 32 == 0 && (uintptr_t)src % 32 == 0 && (uintptr_t)dst % 32 == 0) {
+    ProfScope _ps("scatter_rows", s);
+    k_scatter_rows_wide<<<blocks, 256, 0, s>>>((const uint8_t*)src, slot_row, extra_row, row_token,
+                                               offsets, T, (int)(row_bytes / 32), E, k, nbt,
+                                               (uint8_t*)dst);
+  } else if (dtype == MOE_BF16) {
     ProfScope _ps("scatter_rows", s);
     k_scatter_rows<__nv_bfloat16><<<blocks, 256, 0, s>>>(
         (const __nv_bfloat16*)src, slot_row, extra_row, row_token, offsets, T, width, E, k, nbt,
