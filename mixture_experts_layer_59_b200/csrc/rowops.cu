@@ -434,13 +434,97 @@ k_token_reduce(const T* __restrict__ src, const float* __restrict__ row_gate,
   }
 }
 
+// The same reduction for bf16 rows of a multiple of 16 elements (32-byte
+// aligned) when a token has at most 4 kept slots: a lane owns 16 consecutive
+// columns per pass and loads them from each row with one 32-byte load, so a
+// 4 KB row takes half the passes (each a round trip to memory) of 16-byte
+// loads.  Rows are summed in the same order as above (bit-identical).
+template <class OutT>
+__global__ void __launch_bounds__(TR_WARPS * 32)
+k_token_reduce_w32(const __nv_bfloat16* __restrict__ src, const float* __restrict__ row_gate,
+                   const int32_t* __restrict__ slot_row, const int32_t* __restrict__ extra_row,
+                   int T_, int width, int E, int k, bool weighted, OutT* __restrict__ out) {
+  constexpr int RB = 4;   // rows whose loads are in flight together
+  __shared__ int s_rows[TR_WARPS][8 + 256];
+  __shared__ float s_wts[TR_WARPS][8 + 256];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int* rows = s_rows[w];
+  float* wts = s_wts[w];
+  const int nu = width / 16;   // 32-byte units per row
+  for (int t = blockIdx.x * TR_WARPS + w; t < T_; t += gridDim.x * TR_WARPS) {
+    const int rs = lane < k ? slot_row[(size_t)t * k + lane] : -1;
+    unsigned bal = __ballot_sync(0xffffffffu, rs >= 0);
+    int n = __popc(bal);
+    if (rs >= 0) rows[__popc(bal & ((1u << lane) - 1u))] = rs;
+    if (extra_row != nullptr) {
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int re = (e0 + lane < E) ? extra_row[(size_t)t * E + e0 + lane] : -1;
+        bal = __ballot_sync(0xffffffffu, re >= 0);
+        if (re >= 0) rows[n + __popc(bal & ((1u << lane) - 1u))] = re;
+        n += __popc(bal);
+      }
+    }
+    __syncwarp();
+    if (weighted)
+      for (int j = lane; j < n; j += 32) wts[j] = row_gate[rows[j]];
+    __syncwarp();
+    for (int u = lane; u < nu; u += 32) {
+      float acc[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc[q] = 0.f;
+      for (int j0 = 0; j0 < n; j0 += RB) {
+        Vec<__nv_bfloat16> va[RB], vb[RB];
+#pragma unroll
+        for (int j = 0; j < RB; ++j)
+          if (j0 + j < n) ld_nc_v8(src + (size_t)rows[j0 + j] * width + 16 * u, va[j].v, vb[j].v);
+#pragma unroll
+        for (int j = 0; j < RB; ++j) {
+          if (j0 + j < n) {
+            const float wt = weighted ? wts[j0 + j] : 1.0f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(wt, va[j].get(q), acc[q]);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[8 + q] = fmaf(wt, vb[j].get(q), acc[8 + q]);
+          }
+        }
+      }
+      OutT* o = out + (size_t)t * width + 16 * u;
+      if constexpr (sizeof(OutT) == 2) {
+        Vec<__nv_bfloat16> ra, rb;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) { ra.set(q, acc[q]); rb.set(q, acc[8 + q]); }
+        st_v8(o, ra.v, rb.v);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; q += 8)
+          st_v8(o + q, make_uint4(__float_as_uint(acc[q]), __float_as_uint(acc[q + 1]),
+                                  __float_as_uint(acc[q + 2]), __float_as_uint(acc[q + 3])),
+                make_uint4(__float_as_uint(acc[q + 4]), __float_as_uint(acc[q + 5]),
+                           __float_as_uint(acc[q + 6]), __float_as_uint(acc[q + 7])));
+      }
+    }
+    __syncwarp();
+  }
+}
+
 int launch_token_reduce(const void* src, const float* row_gate, const int32_t* slot_row,
                         const int32_t* extra_row, int T, int width, int E, int k, int dtype,
                         bool weighted, bool out_f32, void* out, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int blocks = (T + TR_WARPS - 1) / TR_WARPS;
   if (blocks > device_sm_count() * 32) blocks = device_sm_count() * 32;
-  if (dtype == MOE_BF16) {
+  if (dtype == MOE_BF16 && k <= 4 && width % 16 == 0 && (uintptr_t)src % 32 == 0 &&
+      (uintptr_t)out % 32 == 0) {
+    ProfScope _ps("token_reduce", s);
+    if (out_f32)
+      k_token_reduce_w32<float><<<blocks, TR_WARPS * 32, 0, s>>>(
+          (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
+          (float*)out);
+    else
+      k_token_reduce_w32<__nv_bfloat16><<<blocks, TR_WARPS * 32, 0, s>>>(
+          (const __nv_bfloat16*)src, row_gate, slot_row, extra_row, T, width, E, k, weighted,
+          (__nv_bfloat16*)out);
+  } else if (dtype == MOE_BF16) {
     if (out_f32) {
       ProfScope _ps("token_reduce", s);
       k_token_reduce<__nv_bfloat16, float><<<blocks, TR_WARPS * 32, 0, s>>>(
