@@ -294,22 +294,32 @@ class ClockSampler:
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
 
-    def stop(self, t0, t1):
+    def stop(self, t0=None, t1=None):
+        """End sampling; with a window, return its summary (see window())."""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return self.window(t0, t1) if t0 is not None else None
+
+    def window(self, t0, t1, pad=0.0, fallback=True):
+        """Median SM clock, maximum clock and throttle reasons of the samples
+        taken in [t0, t1] (widened by pad seconds); all samples if none fall
+        inside and fallback is set, else sm_mhz None."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
         rows = []
         for ts, ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 10:
                 continue
             rows.append((ts, parts))
-        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.15] or rows
+        inside = [r for r in rows if t0 - 0.05 - pad <= r[0] <= t1 + 0.15 + pad]
+        if not inside and fallback:
+            inside = rows
         sm = [float(p[2]) for _, p in inside if p[2].replace(".", "").isdigit()]
         smax = [float(p[3]) for _, p in inside if p[3].replace(".", "").isdigit()]
         names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
@@ -462,20 +472,25 @@ def run_ours(args, cfg, rank, world, local_rank):
     torch.cuda.synchronize()
     t1 = time.time()
     barrier()
-    clocks = sampler.stop(t0, t1)
     B.moe_check_status()
     total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world, dev)
     # per-kernel live times from a separate profiled pass (the profiling events
     # between kernels would otherwise sit inside the timed steps, and they
     # serialise the dependent launches that overlap a kernel's start with the
-    # previous kernel's end)
+    # previous kernel's end); the clock sampler keeps running through it, so
+    # that the per-kernel rates are set against the clock they ran at
     n_prof = min(args.steps, 20)
     B.moe_profile_enable(True)
+    t2 = time.time()
     for i in range(n_prof):
         flush.zero_()
         one_step()
     torch.cuda.synchronize()
+    t3 = time.time()
     B.moe_profile_enable(False)
+    sampler.stop()
+    clocks = sampler.window(t0, t1)
+    prof_clocks = sampler.window(t2, t3, pad=0.1, fallback=False)
     prof = B.moe_profile_report()
     B.moe_check_status()
     ms_per_step = total_ms / args.steps
@@ -587,9 +602,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         roof = gemm_roofline(dom, fl, avg_s, peaks, peak_src)
         roof["traffic"] = traffic_for(dom, cfg.name)
         # long runs settle under the power cap at a lower clock than the burst
-        # peak's: the burst peak scaled by the run's median over maximum SM clock
-        if clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
-            scale = min(1.0, clocks["sm_mhz"] / clocks["sm_max_mhz"])
+        # peak's: the burst peak scaled by the median over the maximum SM clock
+        # of the samples taken while the per-kernel times were measured
+        roof["clock_of_kernel_times"] = prof_clocks
+        if prof_clocks.get("sm_mhz") and prof_clocks.get("sm_max_mhz"):
+            scale = min(1.0, prof_clocks["sm_mhz"] / prof_clocks["sm_max_mhz"])
             roof["frac_at_run_clock"] = roof["achieved"] / (roof["peak"] * scale)
         bf16_peak, bf16_sust = tensor_peaks(peaks, "bf16")
         g_fl = sum(gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k) * v[0] for n, v in gemm.items())
