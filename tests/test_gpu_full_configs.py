@@ -80,6 +80,23 @@ def test_full_size_layer(name, routing, round_mode, n_tok, gate_mode, cf):
         ref_idx = O.route(None, None, k, logits_override=logits32.astype(np.float64))[1]
         np.testing.assert_array_equal(np.sort(i64(idx_g)[clear], 1), np.sort(ref_idx[clear], 1))
         np.testing.assert_array_equal(i64(idx_g)[ordered], ref_idx[ordered])
+        # top-k flips against the fp64 logits: tokens whose chosen expert set
+        # differs.  Every flip must sit at a near-tie (the k-th and (k+1)-th
+        # fp64 logits within the router's rounding); the count is reported.
+        l64 = x64 @ wg64 + (f64(inp["logit_bias"])[None, :] if inp["logit_bias"] is not None
+                            else 0.0)
+        set64 = np.sort(O.route(None, None, k, logits_override=l64)[1], 1)
+        flip = np.any(np.sort(i64(idx_g), 1) != set64, axis=1)
+        s64 = -np.sort(-l64, axis=1)
+        margin = s64[:, k - 1] - s64[:, k]
+        mag = np.maximum(np.abs(s64[:, k - 1]), np.abs(s64[:, k]))
+        assert np.all(margin[flip] <= 1e-4 * scale), margin[flip].max()
+        near = margin <= 1e-5 * mag
+        print(f"\ntop-k flips [{name}/{routing}/gate{gate_mode}]: {int(flip.sum())} of {T} tokens "
+              f"differ from the fp64 top-k set; {int((flip & near).sum())} of them, and "
+              f"{int(near.sum())} tokens in all, have a k-th margin <= 1e-5 |l|; largest flip "
+              f"margin {float(margin[flip].max()) if flip.any() else 0.0:.3g} (logit scale "
+              f"{scale:.3g})")
         # gates: the oracle's gate rule applied to the GPU's own logits and choice
         g_ref = O.route(None, None, k, logits_override=lg, gate_mode=gate_mode)[2]
         same = np.all(i64(idx_g) == O.route(None, None, k, logits_override=lg)[1], axis=1)

@@ -498,11 +498,17 @@ def test_bounded_wait_expires_then_next_call_is_clean():
     assert torch.equal(H2[:R], H0[:R])
 
 
-@pytest.mark.parametrize("T,d,E,k,round_mode", [(1000, 2048, 8, 4, B.MOE_ROUND_NONE),
-                                               (777, 7168, 16, 2, B.MOE_ROUND_NEAREST),
-                                               (130, 128, 4, 1, B.MOE_ROUND_NONE),
-                                               (0, 256, 8, 2, B.MOE_ROUND_NONE)])
-def test_gather_rows_bit_exact_with_padding_zeroed(T, d, E, k, round_mode):
+@pytest.mark.parametrize("T,d,E,k,round_mode,shift", [(1000, 2048, 8, 4, B.MOE_ROUND_NONE, 0),
+                                                     (777, 7168, 16, 2, B.MOE_ROUND_NEAREST, 0),
+                                                     (130, 128, 4, 1, B.MOE_ROUND_NONE, 0),
+                                                     (0, 256, 8, 2, B.MOE_ROUND_NONE, 0),
+                                                     # rows that are not 32-byte multiples, and
+                                                     # a destination 16 but not 32 bytes aligned:
+                                                     # the 16-byte kernel
+                                                     (300, 8, 8, 2, B.MOE_ROUND_NONE, 0),
+                                                     (257, 24, 4, 3, B.MOE_ROUND_NEAREST, 0),
+                                                     (500, 256, 8, 4, B.MOE_ROUND_NONE, 8)])
+def test_gather_rows_bit_exact_with_padding_zeroed(T, d, E, k, round_mode, shift):
     """moe_gather_rows (the row gather behind every grouped GEMM): row r of
     the row space is row row_token[r] of the token-major source, bit for bit,
     including rows added by token rounding; padding rows are zeros, and rows
@@ -513,7 +519,10 @@ def test_gather_rows_bit_exact_with_padding_zeroed(T, d, E, k, round_mode):
     logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=T, E=E)
     plan = B.moe_permute(idx, gate, logits, E, round_mode)
     cap = B.moe_row_capacity(T, E, k)
-    out = torch.full((cap, d), 7.0, dtype=torch.bfloat16, device="cuda")   # sentinel
+    # sentinel-filled destination, starting `shift` elements into its buffer
+    flat = torch.full((shift + cap * d,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = flat[shift:].view(cap, d)
+    assert out.data_ptr() % 16 == 0
     B.moe_gather_rows(x, plan, k, out=out)
     torch.cuda.synchronize()
     B.moe_check_status()
