@@ -541,13 +541,31 @@ def layer_fwd(x, w_gate, w1, w3, w2, k, tile=TILE, round_mode=0,
                 A=res["A"], Y=res["Y"], out=out, precision=precision)
 
 
+def _segment(live_vals, live, width):
+    """An expert's segment of the row space as a dense [rows, width] matrix:
+    the live rows' values in row order, zeros in the padding rows."""
+    out = np.zeros((len(live), width))
+    out[live] = live_vals
+    return out
+
+
+def mx_wgrad(a_seg, b_seg):
+    """Weight gradient of one expert on MXFP8 operands: a^T b with both
+    operands quantised along the token axis -- the contraction dimension of
+    this GEMM -- in blocks of 32 consecutive rows of the expert's segment of
+    the row space (padding rows are zero rows of the segment)."""
+    return mx_fake_quant(a_seg, 0).T @ mx_fake_quant(b_seg, 0)
+
+
 def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True,
-              extra_dlogits=None):
+              extra_dlogits=None, mx_wgrad_on=False):
     """Full backward from the saved set {x, logits, idx, gate, plan, H}.
 
     dW2_e = sum_rows (g A)^T dO,  [dW1|dW3]_e = sum_rows x^T dH,
     dx_t = sum over the rows of t of dX_perm + dlogits_t W_gate^T,
     dW_gate = x^T dlogits.  Returns dx, dw_gate, dw1, dw3, dw2, dS [R], dlogits.
+    mx_wgrad_on: the weight-gradient GEMMs take MXFP8 operands (mx_wgrad) over
+    each expert's whole segment, padding rows included.
     """
     dout, x, w_gate, w1, w3, w2 = map(_f64, (dout, x, w_gate, w1, w3, w2))
     plan = fwd["plan"]
@@ -562,6 +580,12 @@ def layer_bwd(dout, x, w_gate, w1, w3, w2, fwd, staged=True, router_grad_on=True
         toks = plan["row_token"][lo:hi]
         live = toks >= 0
         r = np.arange(lo, hi)[live]
+        if mx_wgrad_on:
+            seg = lambda rows_val, width: _segment(rows_val, live, width)
+            dw2[e] = mx_wgrad(seg(res["gA"][r], f), seg(dout[toks[live]], d))
+            dw13 = mx_wgrad(seg(x[toks[live]], d), seg(res["dH"][r], 2 * f))
+            dw1[e], dw3[e] = dw13[:, :f], dw13[:, f:]
+            continue
         dw2[e] = res["gA"][r].T @ dout[toks[live]]
         dw1[e] = x[toks[live]].T @ res["dH"][r, :f]
         dw3[e] = x[toks[live]].T @ res["dH"][r, f:]

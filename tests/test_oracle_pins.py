@@ -708,6 +708,51 @@ def test_mxfp8_layer_equals_bf16_layer_on_the_mx_grid():
 
 
 
+def test_mx_wgrad_blocks_run_along_tokens_within_the_segment():
+    """MXFP8 weight gradient: operands quantised in blocks of 32 consecutive
+    token rows.  Column 0 of a holds 2^10 in row 31 and 2^-10 in the other
+    rows of that block: the block's scale is 2^(10-8), so 2^-10 / 2^2 = 2^-12
+    falls below half the smallest E4M3 subnormal (2^-9) and rounds to zero.
+    Rows 32..63 form their own block (scale 2^(-10-8)) and keep 2^-10 exactly.
+    With b = ones the gradient is then 2^10 + 32 * 2^-10 in closed form,
+    against 2^10 + 63 * 2^-10 unquantised.  Column 1 of a is 3 everywhere
+    (exact in E4M3 at any shared scale): 64 * 3."""
+    a = np.full((64, 2), 2.0 ** -10)
+    a[31, 0] = 2.0 ** 10
+    a[:, 1] = 3.0
+    b = np.ones((64, 1))
+    got = O.mx_wgrad(a, b)
+    assert got.shape == (2, 1)
+    assert got[0, 0] == 2.0 ** 10 + 32 * 2.0 ** -10
+    assert got[1, 0] == 64 * 3.0
+    assert (a.T @ b)[0, 0] == 2.0 ** 10 + 63 * 2.0 ** -10
+    # the segment helper puts live rows where they sit, zeros in padding rows
+    live = np.array([True, False, True, True])
+    seg = O._segment(np.array([[1.0], [2.0], [3.0]]), live, 1)
+    np.testing.assert_array_equal(seg[:, 0], [1.0, 0.0, 2.0, 3.0])
+
+
+def test_layer_bwd_mx_wgrad_close_to_the_unquantised_gradient():
+    """The MXFP8 weight gradients differ from the straight-through (bf16)
+    ones by the format's rounding: relative error of a few E4M3 half-ulps
+    (2^-4) in aggregate, never zero, and nothing else in the backward moves."""
+    T, d, f, E, k = 96, 64, 32, 4, 2
+    rng = np.random.default_rng(35)
+    x = rng.standard_normal((T, d))
+    wg = 0.3 * rng.standard_normal((d, E))
+    w1, w3 = 0.2 * rng.standard_normal((E, d, f)), 0.2 * rng.standard_normal((E, d, f))
+    w2 = 0.2 * rng.standard_normal((E, f, d))
+    dout = rng.standard_normal((T, d))
+    fwd = O.layer_fwd(x, wg, w1, w3, w2, k, tile=32, staged=False)
+    ref = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False)
+    mx = O.layer_bwd(dout, x, wg, w1, w3, w2, fwd, staged=False, mx_wgrad_on=True)
+    for n in ("dw1", "dw3", "dw2"):
+        rel = np.abs(mx[n] - ref[n]).sum() / np.abs(ref[n]).sum()
+        assert 1e-4 < rel < 2 ** -4, (n, rel)
+    for n in ("dx", "dw_gate", "dlogits", "dS"):
+        np.testing.assert_array_equal(mx[n], ref[n])
+
+
 def test_mx_fake_quant_matches_torch_float8_along_either_axis():
     """The MXFP8 image of a matrix, blocks along rows or columns, against an
     independent torch construction: per-block maximum, scale 2^(e-9) from
