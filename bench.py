@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--precision", choices=["bf16", "mxfp8"], default="bf16",
                     help="mxfp8: forward expert GEMMs and the backward dX GEMM on MXFP8 operands "
                          "(weights quantised in the step)")
+    ap.add_argument("--mx-wgrad", action="store_true",
+                    help="with --precision mxfp8: the weight-gradient GEMMs on MXFP8 operands too "
+                         "(x, dO, s*A, dH quantised along tokens)")
     ap.add_argument("--noise-std", type=float, default=0.0,
                     help="noisy top-k gating: Gaussian routing noise of this std on the scores")
     ap.add_argument("--gate-mode", type=int, default=0, choices=[0, 1],
@@ -127,6 +130,8 @@ def gemm_flops(kind, T, d, f, k):
         "tc_up_mxfp8": 2.0 * rows * d * 2 * f,
         "tc_down_mxfp8": 2.0 * rows * f * d,
         "tc_dx_mxfp8": 2.0 * rows * 2 * f * d,
+        "tc_dw2_mxfp8": 2.0 * rows * f * d,
+        "tc_dw13_mxfp8": 2.0 * rows * d * 2 * f,
     }.get(kind)
 
 
@@ -151,6 +156,8 @@ def gemm_bytes(kind, T, d, f, E, k):
         "tc_up_mxfp8": 2 * w * 1.03125 + R * d * 1.03125 + R * 2 * f * 2 + R * f * 1.03125,
         "tc_down_mxfp8": w * 1.03125 + R * f * 1.03125 + R * d * 2,
         "tc_dx_mxfp8": 2 * w * 1.03125 + R * 2 * f * 1.03125 + R * d * 2,
+        "tc_dw2_mxfp8": w * 2 + R * f * 1.03125 + R * d * 1.03125,
+        "tc_dw13_mxfp8": 2 * w * 2 + R * d * 1.03125 + R * 2 * f * 1.03125,
     }
     return b.get(kind)
 
@@ -169,6 +176,8 @@ def gemm_unit(kind, d, f):
         "tc_up_mxfp8": (4.0 * d * f, d * q + 2 * f * 2 + f * q, 2 * q),
         "tc_down_mxfp8": (2.0 * d * f, f * q + d * 2, 1 * q),
         "tc_dx_mxfp8": (4.0 * d * f, 2 * f * q + d * 2, 2 * q),
+        "tc_dw2_mxfp8": (2.0 * d * f, f * q + d * q, 1 * 2),
+        "tc_dw13_mxfp8": (4.0 * d * f, d * q + 2 * f * q, 2 * 2),
     }.get(kind)
 
 
@@ -416,6 +425,7 @@ def workload_config(cfg, args):
             "gate": "softmax_then_topk" if args.gate_mode else "topk_then_softmax",
             "routing_noise_std": args.noise_std or None,
             "precision": args.precision,
+            "mxfp8_weight_gradients": bool(args.mx_wgrad and args.precision == "mxfp8"),
             "balance_loss_lambda": args.balance_loss,
             "l2": f"flushed between timed steps ({args.flush_mb} MiB write)", "replicas": args.gpus}
 
@@ -434,7 +444,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     inp = synth.make_inputs(cfg, seed=rank, device=dev)
     step = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round,
                         balance_lambda=args.balance_loss, gate_mode=args.gate_mode,
-                        precision=args.precision,
+                        precision=args.precision, mx_wgrad=args.mx_wgrad,
                         capacity_factor=args.capacity_factor if args.round == 2 else None)
     flush = torch.empty(max(args.flush_mb, 1) << 20, dtype=torch.uint8, device=dev)
     x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
@@ -505,7 +515,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     # inputs arrive by copy.)
     step2 = MoELayerStep(cfg.T, cfg.d, cfg.f, cfg.E, cfg.k, cfg.torch_dtype, dev, args.round,
                          balance_lambda=args.balance_loss, gate_mode=args.gate_mode,
-                         precision=args.precision,
+                         precision=args.precision, mx_wgrad=args.mx_wgrad,
                          capacity_factor=args.capacity_factor if args.round == 2 else None)
     objs = (step, step2)
     x_h = x.cpu().pin_memory()

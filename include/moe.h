@@ -238,13 +238,36 @@ int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, i
                                void* stream);
 size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
 /*
+ * moe_mxfp8_quantize_tokens -- a row-space matrix quantised along its rows
+ * (the token axis), as the MXFP8 weight-gradient GEMMs of
+ * moe_layer_bwd_mxfp8 take it.  Row r is src row r of a bf16 [rows, n]
+ * matrix, or, when gather_row is not NULL, token row gather_row[r] of a
+ * token-major bf16 [T, n] matrix (-1: a zero row).  Rows below offsets[E]
+ * (the plan's rows; segments are multiples of 128) are quantised in blocks
+ * of 32 consecutive rows: q [n, capr] E4M3 (column c of the source is row c
+ * of q, rows contiguous) and sf its E8M0 scales in the layout above with n
+ * as the row (MN) dimension and capr / 128 K chunks.  Bytes of q and sf for
+ * rows at or above offsets[E] are left untouched.  n and capr: multiples of
+ * 128 (capr >= offsets[E]); src and q 16-byte aligned; device buffers owned
+ * by the caller.  Needs no sm_100 features beyond the CUDA cores.
+ */
+int moe_mxfp8_quantize_tokens(const void* src, const int32_t* gather_row, const int32_t* offsets,
+                              int E, int n, int capr, uint8_t* q, uint8_t* sf, void* stream);
+/*
  * moe_layer_bwd_mxfp8 -- moe_layer_bwd (bf16 only) whose dX_perm GEMM runs
  * on MXFP8 operands: the dA' epilogue also writes dH in E4M3 with blocks
- * along 2f, and W1r/W3r come from moe_mxfp8_quantize_weights.  The other
- * backward GEMMs, the router gradient and every output are as in
- * moe_layer_bwd.  ws: at least moe_layer_bwd_mxfp8_workspace_size() bytes.
+ * along 2f, and W1r/W3r come from moe_mxfp8_quantize_weights.
+ * wgrad_mxfp8 = 1 also runs the weight-gradient GEMMs (dW2 = (s*A)^T dO,
+ * [dW1 | dW3] = x^T dH per expert) on MXFP8 operands: x, dO, s*A and dH are
+ * quantised along the tokens -- the contraction dimension of these GEMMs --
+ * in blocks of 32 consecutive rows of each expert's segment of the row space
+ * (padding rows count as zero rows); d and 2f must then be multiples of 256
+ * (else MOE_ERR_UNSUPPORTED).  wgrad_mxfp8 = 0 keeps them bf16.  dA' and the
+ * router gradient are as in moe_layer_bwd; the quantisers pass gradients
+ * straight through.  ws: at least
+ * moe_layer_bwd_mxfp8_workspace_size(..., wgrad_mxfp8) bytes.
  */
-size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
+size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k, int wgrad_mxfp8);
 int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate,
                         const void* w1, const void* w3, const void* w2,
                         const uint8_t* w1rq, const uint8_t* w1rs,
@@ -253,7 +276,7 @@ int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate,
                         const float* logits, int gate_mode, const int32_t* offsets,
                         const int32_t* row_token, const float* row_gate,
                         const int32_t* slot_row, const int32_t* extra_row, const void* H,
-                        int T, int d, int f, int E, int k, int router_grad,
+                        int T, int d, int f, int E, int k, int router_grad, int wgrad_mxfp8,
                         void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2,
                         float* dS, float* dlogits, void* ws, size_t ws_bytes, void* stream);
 

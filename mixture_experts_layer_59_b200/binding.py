@@ -30,6 +30,7 @@ EXPORTS = [
     "moe_check_status", "moe_profile_enable", "moe_profile_report", "moe_permute_noalloc",
     "moe_balance_loss_workspace_size", "moe_balance_loss",
     "moe_mxfp8_weight_sizes", "moe_mxfp8_quantize_weights", "moe_ffn_fwd_mxfp8_workspace_size",
+    "moe_mxfp8_quantize_tokens",
     "moe_expert_ffn_fwd_mxfp8", "moe_layer_bwd_mxfp8_workspace_size", "moe_layer_bwd_mxfp8",
     "moe_debug_expire_next_wait", "moe_gather_rows", "moe_ep_dispatch_counts",
     "moe_ep_receive_plan", "moe_expert_rows_fwd_workspace_size", "moe_expert_rows_fwd",
@@ -66,8 +67,9 @@ _SIGS = {
     "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_mxfp8_weight_sizes": (_i, [_i, _i, _i, ctypes.POINTER(_sz)]),
     "moe_mxfp8_quantize_weights": (_i, [_vp, _vp, _vp, _i, _i, _i] + [_vp] * 9),
-    "moe_layer_bwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
-    "moe_layer_bwd_mxfp8": (_i, [_vp] * 14 + [_i] + [_vp] * 6 + [_i] * 6 + [_vp] * 8 + [_sz, _vp]),
+    "moe_mxfp8_quantize_tokens": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_layer_bwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "moe_layer_bwd_mxfp8": (_i, [_vp] * 14 + [_i] + [_vp] * 6 + [_i] * 7 + [_vp] * 8 + [_sz, _vp]),
     "moe_ffn_fwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "moe_expert_ffn_fwd_mxfp8": (_i, [_vp] * 9 + [_i] * 5 + [_vp, _vp, _vp, _sz, _vp]),
     "moe_check_status": (_i, [_vp]),
@@ -227,6 +229,18 @@ def moe_mxfp8_weight_sizes(E, d, f):
     return tuple(int(v) for v in sz)
 
 
+def moe_mxfp8_quantize_tokens(src, offsets, capr, gather_row=None, stream=None):
+    """Row-space matrix quantised along its rows (blocks of 32 rows): returns
+    (q [n, capr] uint8 E4M3, sf uint8 scales) for the rows below offsets[E]."""
+    n = src.shape[1]
+    E = offsets.numel() - 1
+    q = torch.zeros(n, capr, device=src.device, dtype=torch.uint8)
+    sf = torch.zeros(n * capr // 32, device=src.device, dtype=torch.uint8)
+    _check(lib().moe_mxfp8_quantize_tokens(_p(src), _p(gather_row), _p(offsets), E, n, capr,
+                                           _p(q), _p(sf), _stream(stream)))
+    return q, sf
+
+
 def moe_mxfp8_quantize_weights(w1, w3, w2, out=None, stream=None, backward=True):
     """MXFP8 copies of the expert weights: dict w13q, w13s, w2q, w2s and, with
     ``backward``, w1rq, w1rs, w3rq, w3rs (for moe_layer_bwd_mxfp8); uint8."""
@@ -305,15 +319,16 @@ def moe_layer_bwd(dout, x, w_gate, w1, w3, w2, idx, gate, plan, H, router_grad=T
     return o
 
 
-def moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k) -> int:
-    return lib().moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k)
+def moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k, wgrad=False) -> int:
+    return lib().moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k, 1 if wgrad else 0)
 
 
 def moe_layer_bwd_mxfp8(dout, x, w_gate, w1, w3, w2, wq, idx, gate, plan, H, router_grad=True,
                         out=None, ws=None, stream=None, gate_grad=None, logits=None,
-                        gate_mode=MOE_GATE_TOPK_SOFTMAX):
-    """moe_layer_bwd with the dX GEMM on MXFP8 operands.  wq: dict from
-    moe_mxfp8_quantize_weights (backward=True)."""
+                        gate_mode=MOE_GATE_TOPK_SOFTMAX, wgrad=False):
+    """moe_layer_bwd with the dX GEMM on MXFP8 operands, and with wgrad the
+    weight-gradient GEMMs too.  wq: dict from moe_mxfp8_quantize_weights
+    (backward=True)."""
     T, d = x.shape
     E, _, f = w1.shape
     k = idx.shape[1]
@@ -328,13 +343,14 @@ def moe_layer_bwd_mxfp8(dout, x, w_gate, w1, w3, w2, wq, idx, gate, plan, H, rou
     o.setdefault("dS", torch.empty(cap, device=dev, dtype=torch.float32))
     o.setdefault("dlogits", torch.empty(T, E, device=dev, dtype=torch.float32))
     if ws is None:
-        ws = torch.empty(max(moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k), 1), device=dev,
-                         dtype=torch.uint8)
+        ws = torch.empty(max(moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k, wgrad), 1),
+                         device=dev, dtype=torch.uint8)
     _check(lib().moe_layer_bwd_mxfp8(
         _p(dout), _p(x), _p(w_gate), _p(w1), _p(w3), _p(w2), _p(wq["w1rq"]), _p(wq["w1rs"]),
         _p(wq["w3rq"]), _p(wq["w3rs"]), _p(idx), _p(gate), _p(gate_grad), _p(logits), gate_mode,
         _p(plan["offsets"]), _p(plan["row_token"]), _p(plan["row_gate"]), _p(plan["slot_row"]),
         _p(plan.get("extra_row")), _p(H), T, d, f, E, k, 1 if router_grad else 0,
+        1 if wgrad else 0,
         _p(o["dx"]), _p(o["dw_gate"]), _p(o["dw1"]), _p(o["dw3"]), _p(o["dw2"]), _p(o["dS"]),
         _p(o["dlogits"]), _p(ws), ws.numel(), _stream(stream)))
     return o

@@ -360,6 +360,16 @@ int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes) {
   return MOE_OK;
 }
 
+int moe_mxfp8_quantize_tokens(const void* src, const int32_t* gather_row, const int32_t* offsets,
+                              int E, int n, int capr, uint8_t* q, uint8_t* sf, void* stream) {
+  if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  if (n <= 0 || n % 128 || capr <= 0 || capr % 128)
+    return fail(MOE_ERR_UNSUPPORTED, "n and capr must be positive multiples of 128");
+  REQUIRE_PTR(src); REQUIRE_PTR(offsets); REQUIRE_PTR(q); REQUIRE_PTR(sf);
+  REQUIRE_ALIGNED(src); REQUIRE_ALIGNED(q);
+  return launch_mx_quant_cols(src, gather_row, offsets, E, n, capr, q, sf, (cudaStream_t)stream);
+}
+
 int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
                                int f, uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
                                uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
@@ -491,7 +501,7 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
                   const int32_t* slot_row, const int32_t* extra_row, const void* H, int T, int d,
                   int f, int E, int k, int dtype, int router_grad, void* dx, float* dw_gate,
                   void* dw1, void* dw3, void* dw2, float* dS, float* dlogits, void* ws,
-                  size_t ws_bytes, void* stream, const uint8_t* const* mxw) {
+                  size_t ws_bytes, void* stream, const uint8_t* const* mxw, int mx_wgrad = 0) {
   if (int rc = check_common(T, E, k, dtype)) return rc;
   if (int rc = check_dims(d, f, dtype)) return rc;
   REQUIRE_PTR(dout); REQUIRE_PTR(x); REQUIRE_PTR(w1); REQUIRE_PTR(w3); REQUIRE_PTR(w2);
@@ -505,7 +515,7 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
   REQUIRE_ALIGNED(dout); REQUIRE_ALIGNED(x); REQUIRE_ALIGNED(w1); REQUIRE_ALIGNED(w3);
   REQUIRE_ALIGNED(w2); REQUIRE_ALIGNED(H); REQUIRE_ALIGNED(dx); REQUIRE_ALIGNED(dw1);
   REQUIRE_ALIGNED(dw3); REQUIRE_ALIGNED(dw2); REQUIRE_ALIGNED(ws);
-  const size_t need = mxw ? moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k)
+  const size_t need = mxw ? moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k, mx_wgrad)
                          : moe_layer_bwd_workspace_size(T, d, f, E, k, dtype);
   if (ws_bytes < need)
     return fail(MOE_ERR_WORKSPACE, "bwd workspace smaller than the matching *_workspace_size()");
@@ -517,6 +527,20 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
     const size_t capr = ((size_t)T * k + (size_t)E * 128 + 127) / 128 * 128;
     mx = MxBwd{mxw[0], mxw[1], mxw[2], mxw[3], c.take<uint8_t>(capr * 2 * f),
                c.take<uint8_t>(capr * 2 * f / 32)};
+    if (mx_wgrad) {   // x, dO, s*A, dH quantised along the rows for the dW GEMMs
+      mx.wgrad = 1;
+      mx.capr = (int)capr;
+      mx.x = x;
+      mx.row_token = row_token;
+      mx.xq = c.take<uint8_t>(capr * d);
+      mx.xs = c.take<uint8_t>(capr * d / 32);
+      mx.oq = c.take<uint8_t>(capr * d);
+      mx.os = c.take<uint8_t>(capr * d / 32);
+      mx.aq = c.take<uint8_t>(capr * f);
+      mx.as = c.take<uint8_t>(capr * f / 32);
+      mx.hq = c.take<uint8_t>(capr * 2 * f);
+      mx.hs = c.take<uint8_t>(capr * 2 * f / 32);
+    }
   }
   if (!c.ok) return fail(MOE_ERR_WORKSPACE, "bwd workspace too small");
   cudaStream_t s = (cudaStream_t)stream;
@@ -526,7 +550,8 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
     if ((rc = launch_scatter_rows(dout, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
                                   w.dog, s)))
       return rc;
-    if ((rc = launch_scatter_rows(x, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
+    if (!mx.wgrad &&   // (MXFP8 weight gradients quantise x straight from the token rows)
+        (rc = launch_scatter_rows(x, slot_row, extra_row, row_token, offsets, T, d, E, k, dtype,
                                   w.xg, s)))
       return rc;
     if ((rc = tc_ffn_bwd(p, w.dog, w.xg, row_gate, H, w.dH, w.gact, w.ds, w.dxp, dw1, dw3, dw2,
@@ -555,7 +580,7 @@ int moe_layer_bwd(const void* dout, const void* x, const void* w_gate, const voi
                         nullptr);
 }
 
-size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k) {
+size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k, int wgrad_mxfp8) {
   if (T < 0 || d <= 0 || f <= 0 || E <= 0 || k <= 0) return 0;
   Sizer z;
   BwdWs<Sizer> w;
@@ -563,6 +588,12 @@ size_t moe_layer_bwd_mxfp8_workspace_size(int T, int d, int f, int E, int k) {
   const size_t capr = ((size_t)T * k + (size_t)E * 128 + 127) / 128 * 128;
   z.take<uint8_t>(capr * 2 * f);
   z.take<uint8_t>(capr * 2 * f / 32);
+  if (wgrad_mxfp8) {
+    for (size_t n : {(size_t)d, (size_t)d, (size_t)f, (size_t)2 * f}) {
+      z.take<uint8_t>(capr * n);
+      z.take<uint8_t>(capr * n / 32);
+    }
+  }
   return z.used;
 }
 
@@ -573,16 +604,20 @@ int moe_layer_bwd_mxfp8(const void* dout, const void* x, const void* w_gate, con
                         int gate_mode, const int32_t* offsets, const int32_t* row_token,
                         const float* row_gate, const int32_t* slot_row, const int32_t* extra_row,
                         const void* H, int T, int d, int f, int E, int k, int router_grad,
-                        void* dx, float* dw_gate, void* dw1, void* dw3, void* dw2, float* dS,
-                        float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+                        int wgrad_mxfp8, void* dx, float* dw_gate, void* dw1, void* dw3,
+                        void* dw2, float* dS, float* dlogits, void* ws, size_t ws_bytes,
+                        void* stream) {
   REQUIRE_PTR(w1rq); REQUIRE_PTR(w1rs); REQUIRE_PTR(w3rq); REQUIRE_PTR(w3rs);
+  if (wgrad_mxfp8 != 0 && wgrad_mxfp8 != 1) return fail(MOE_ERR_INVALID_ARG, "wgrad_mxfp8 must be 0 or 1");
+  if (wgrad_mxfp8 && (d % 256 || (2 * f) % 256))
+    return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weight gradients need d and 2f multiples of 256");
   REQUIRE_ALIGNED(w1rq); REQUIRE_ALIGNED(w1rs); REQUIRE_ALIGNED(w3rq); REQUIRE_ALIGNED(w3rs);
   if (!tc_available()) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 GEMMs need an sm_100 device");
   const uint8_t* mxw[4] = {w1rq, w1rs, w3rq, w3rs};
   return layer_bwd_impl(dout, x, w_gate, w1, w3, w2, idx, gate, gate_grad, logits, gate_mode,
                         offsets, row_token, row_gate, slot_row, extra_row, H, T, d, f, E, k,
                         MOE_BF16, router_grad, dx, dw_gate, dw1, dw3, dw2, dS, dlogits, ws,
-                        ws_bytes, stream, mxw);
+                        ws_bytes, stream, mxw, wgrad_mxfp8);
 }
 
 // ------------------------------------------------------------ row-space pieces

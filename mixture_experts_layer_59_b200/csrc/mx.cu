@@ -142,6 +142,86 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
   return MOE_OK;
 }
 
+// ============================================================== along tokens
+// Row-space matrix [rows, n] bf16 -> Q [n, capr] E4M3 with blocks of 32
+// along the rows (the contraction dimension of the weight-gradient GEMMs),
+// scales in the layout of mx.cuh with n as the MN dimension and the rows as
+// K (capr / 128 K chunks).  Row r of the source is src row r, or, with
+// gather_row, token row gather_row[r] of a token-major source (-1: a zero
+// row).  One block per (128 rows, 256 columns): the tile arrives in two
+// rounds of loads (8 per thread in flight), then thread p quantises columns
+// 2p', 2p'+1 over 64 rows -- two MXFP8 blocks each, every value pair read
+// with one 32-bit shared load -- and writes 64 bytes of each column's output
+// row; the two threads of a column pair write its 128-byte line, and the
+// column's four scale bytes of this 128-row chunk sit side by side.
+// Only rows below offsets[E] are read or written.
+constexpr int QC_ROWS = 128, QC_COLS = 256, QC_LD = QC_COLS + 8;
+
+__global__ void __launch_bounds__(WQ_THREADS, 2)
+k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict__ gather_row,
+                const int32_t* __restrict__ offsets, int E, int n, int capr,
+                uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+  extern __shared__ __align__(16) uint8_t qc_smem[];
+  __nv_bfloat16 (*tile)[QC_LD] = reinterpret_cast<__nv_bfloat16 (*)[QC_LD]>(qc_smem);
+  const int r0 = blockIdx.x * QC_ROWS, c0 = blockIdx.y * QC_COLS;
+  if (r0 >= offsets[E]) return;                        // whole block (segments are 128-aligned)
+  const int ncols = min(QC_COLS, n - c0);             // a multiple of 128
+  constexpr int VPR = QC_COLS / 8;                     // 16-byte vectors per tile row
+  constexpr int PER = QC_ROWS * VPR / WQ_THREADS / 2;  // per thread and round
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint4 u[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int v = threadIdx.x + (half * PER + i) * WQ_THREADS;
+      const int r = v / VPR, c = (v % VPR) * 8;
+      const int sr = gather_row != nullptr ? gather_row[r0 + r] : r0 + r;
+      u[i] = make_uint4(0, 0, 0, 0);
+      if (c < ncols && sr >= 0) u[i] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)sr * n + c0 + c));
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int v = threadIdx.x + (half * PER + i) * WQ_THREADS;
+      const int r = v / VPR, c = (v % VPR) * 8;
+      if (c < ncols) *reinterpret_cast<uint4*>(&tile[r][c]) = u[i];
+    }
+  }
+  __syncthreads();
+  const int p = threadIdx.x & (QC_COLS / 2 - 1);       // column pair
+  const int rh = threadIdx.x / (QC_COLS / 2);          // rows 64 rh .. 64 rh + 63
+  if (2 * p >= ncols) return;
+  const int kchunks = capr / 128;
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {                        // the two 32-row blocks of this thread
+    const int rb = 64 * rh + 32 * b;
+    uint32_t pk[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(&tile[rb + i][2 * p]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = c0 + 2 * p + h;
+      mx_store_block_packed(pk, h == 1, q + (size_t)col * capr + r0 + rb,
+                            sf + mx_sf_offset(col, (r0 + rb) >> 5, kchunks));
+    }
+  }
+}
+
+int launch_mx_quant_cols(const void* src, const int32_t* gather_row, const int32_t* offsets,
+                         int E, int n, int capr, uint8_t* q, uint8_t* sf, cudaStream_t s) {
+  if (n % 128 || capr % 128) return fail(MOE_ERR_UNSUPPORTED, "token-axis MXFP8 needs n and rows in multiples of 128");
+  dim3 grid(capr / QC_ROWS, (n + QC_COLS - 1) / QC_COLS);
+  const int smem = QC_ROWS * QC_LD * 2;
+  cudaError_t e = cudaFuncSetAttribute(k_mx_quant_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e, "mx_quant_cols smem attribute");
+  {
+    ProfScope _ps("mx_quant_cols", s);
+    k_mx_quant_cols<<<grid, WQ_THREADS, smem, s>>>((const __nv_bfloat16*)src, gather_row, offsets, E,
+                                                   n, capr, q, sf);
+  }
+  MOE_CHECK_LAUNCH("mx_quant_cols");
+  return MOE_OK;
+}
+
 // ============================================================== rows
 // The last nbt blocks own tokens (one warp per token): lanes 4g..4g+3 hold
 // the 32 elements of one block as four 16-byte vectors, share its maximum by

@@ -58,9 +58,9 @@ using namespace tc;
 
 enum Kind : int {
   K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8,
-  K_UPQ = 9, K_DOWNQ = 10, K_DXQ = 11, K_DAPQ = 12
+  K_UPQ = 9, K_DOWNQ = 10, K_DXQ = 11, K_DAPQ = 12, K_DW2Q = 13, K_DW13Q = 14
 };
-constexpr int NUM_KINDS = 13;
+constexpr int NUM_KINDS = 15;
 constexpr int MX_SF_COL = 256;         // TMEM column of the scale blocks (after the accumulators)
 
 constexpr int BM = 128;
@@ -121,12 +121,14 @@ struct TcArgs {
 };
 
 template <int KIND> struct KT {
-  static constexpr bool VARLEN_K = (KIND == K_DW2 || KIND == K_DW13);
+  static constexpr bool VARLEN_K = (KIND == K_DW2 || KIND == K_DW13 || KIND == K_DW2Q ||
+                                    KIND == K_DW13Q);
   static constexpr bool A_MN = VARLEN_K || KIND == K_DWG;
   static constexpr bool B_MN = (KIND == K_UP || KIND == K_DOWN || VARLEN_K || KIND == K_RT ||
                                 KIND == K_DWG);
   static constexpr bool ROUTER = (KIND == K_RT || KIND == K_DWG || KIND == K_DXR);
-  static constexpr bool MX = (KIND == K_UPQ || KIND == K_DOWNQ || KIND == K_DXQ);
+  static constexpr bool MX = (KIND == K_UPQ || KIND == K_DOWNQ || KIND == K_DXQ ||
+                              KIND == K_DW2Q || KIND == K_DW13Q);
 };
 
 // A stage holds a 128 x 128-byte A tile and a BN x 128-byte B tile (64 bf16
@@ -194,7 +196,8 @@ __device__ __forceinline__ bool tile_info(int t, const TcArgs& a, const int* s_o
     ti.ntile = rem % ntiles;
     ti.n0 = ti.ntile * BN;
     ti.krow0 = s_off[ti.e];
-    ti.kb_count = (s_off[ti.e + 1] - s_off[ti.e]) / BK;
+    // k-blocks of BK bf16 rows, or 128-row K chunks of E4M3
+    ti.kb_count = (s_off[ti.e + 1] - s_off[ti.e]) / (KT<KIND>::MX ? 128 : BK);
   } else {
     const int mt = t / ntiles;
     ti.ntile = t - mt * ntiles;
@@ -386,6 +389,20 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
 #pragma unroll
             for (int h = 0; h < BN / 64; ++h)
               tma_load_2d(sB + h * ATOM, mb, &full_bar[stage], 64 * h, r);
+          } else if constexpr (KT<KIND>::MX && KT<KIND>::VARLEN_K) {
+            // weight gradients on MXFP8 operands: A [M, capr] and B [N, capr]
+            // E4M3 with blocks along the rows of the row space (K); this
+            // expert's K chunks start at row krow0 (a multiple of 128)
+            const int kc = ti.krow0 / 128 + kb;
+            tma_load_3d(sA, &a.mA, &full_bar[stage], kc * 128, ti.m0, 0);
+            tma_load_3d(sB, &a.mB0, &full_bar[stage], kc * 128, ti.n0, 0);
+            uint8_t* sSF = sB + C::B_BYTES;
+            bulk_load(sSF, a.sfa + ((size_t)(ti.m0 / BM) * a.kchunks + kc) * 512, 512,
+                      &full_bar[stage]);
+#pragma unroll
+            for (int b = 0; b < BN / 128; ++b)
+              bulk_load(sSF + 512 * (1 + b), a.sfb + ((size_t)(ti.n0 / 128 + b) * a.kchunks + kc) * 512,
+                        512, &full_bar[stage]);
           } else if constexpr (KT<KIND>::MX) {
             // E4M3 tiles: 128 elements of K = 128 bytes; then the A and B
             // scale blocks of this K chunk
@@ -541,6 +558,22 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             }
             mx_store_block(v, a.act_q + (size_t)row * f + nf + c,
                            a.act_s + mx_sf_offset(row, (nf + c) / 32, f / 128));
+          }
+        } else if constexpr (KT<KIND>::VARLEN_K) {
+          // dW rows e*M + m; an expert without rows ran no MMA: zeros
+          const int orow0 = ti.e * a.M + row0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t* rr = j == 0 ? ra : (j == 1 ? rb : (j == 2 ? rc : rd));
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = ti.kb_count > 0 ? __uint_as_float(rr[i]) : 0.f;
+            const int cc = ti.n0 + col[j];
+            if constexpr (KIND == K_DW2Q) {
+              stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, cc, orow0, lane);
+            } else {
+              if (cc < a.f) stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, cc, orow0, lane);
+              else stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, cc - a.f, orow0, lane);
+            }
           }
         } else {
 #pragma unroll
@@ -902,7 +935,7 @@ static int launch(const TcArgs& args, int grid, cudaStream_t s) {
   static const char* kNames[NUM_KINDS] = {
       "tc_up",   "tc_down",   "tc_dap",       "tc_dx",        "tc_dw2",   "tc_dw13",
       "tc_router", "tc_router_dw", "tc_dx_router", "tc_up_mxfp8", "tc_down_mxfp8", "tc_dx_mxfp8",
-      "tc_dap"};
+      "tc_dap", "tc_dw2_mxfp8", "tc_dw13_mxfp8"};
   static_assert(KIND >= 0 && KIND < NUM_KINDS, "kind out of range");
   {
     ProfScope _ps(kNames[KIND], s);
@@ -1161,6 +1194,45 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if ((rc = make_map_3d(&a.mB1, p.w3, f, d, E, 64, bn))) return rc;
     if ((rc = make_store_map(&a.sO0, dXp, d, cap))) return rc;
     if ((rc = launch_bn<K_DX>(a, bn, num_sms, s))) return rc;
+  }
+  if (mx != nullptr && mx->wgrad) {
+    // dW2_e = (sA)^T dOg and [dW1 | dW3]_e = Xg^T dH on MXFP8 operands
+    // quantised along the rows of each expert's segment
+    const int capr = mx->capr;
+    if (d % 256 || (2 * f) % 256)
+      return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weight gradients need d and 2f multiples of 256");
+    if ((rc = launch_mx_quant_cols(mx->x, mx->row_token, p.offsets, E, d, capr, mx->xq, mx->xs, s)))
+      return rc;
+    if ((rc = launch_mx_quant_cols(dog, nullptr, p.offsets, E, d, capr, mx->oq, mx->os, s))) return rc;
+    if ((rc = launch_mx_quant_cols(gact, nullptr, p.offsets, E, f, capr, mx->aq, mx->as, s))) return rc;
+    if ((rc = launch_mx_quant_cols(dH, nullptr, p.offsets, E, 2 * f, capr, mx->hq, mx->hs, s)))
+      return rc;
+    {
+      TcArgs a = base_args(p);
+      a.M = f;
+      a.N = d;
+      a.kchunks = capr / 128;
+      a.sfa = mx->as;
+      a.sfb = mx->os;
+      if ((rc = make_map_u8(&a.mA, mx->aq, capr, f, 1, 128, BM))) return rc;
+      if ((rc = make_map_u8(&a.mB0, mx->oq, capr, d, 1, 128, 256))) return rc;
+      if ((rc = make_store_map(&a.sO0, dw2, d, (uint64_t)E * f))) return rc;
+      if ((rc = launch<K_DW2Q, 256>(a, num_sms, s))) return rc;
+    }
+    {
+      TcArgs a = base_args(p);
+      a.M = d;
+      a.N = 2 * f;
+      a.kchunks = capr / 128;
+      a.sfa = mx->xs;
+      a.sfb = mx->hs;
+      if ((rc = make_map_u8(&a.mA, mx->xq, capr, d, 1, 128, BM))) return rc;
+      if ((rc = make_map_u8(&a.mB0, mx->hq, capr, 2 * f, 1, 128, 256))) return rc;
+      if ((rc = make_store_map(&a.sO0, dw1, f, (uint64_t)E * d))) return rc;
+      if ((rc = make_store_map(&a.sO1, dw3, f, (uint64_t)E * d))) return rc;
+      if ((rc = launch<K_DW13Q, 256>(a, num_sms, s))) return rc;
+    }
+    return MOE_OK;
   }
   {  // DW2: dW2_e = (sA)^T dOg
     TcArgs a = base_args(p);

@@ -16,13 +16,15 @@ class MoELayerStep:
 
     def __init__(self, T, d, f, E, k, dtype=torch.bfloat16, device="cuda",
                  round_mode=B.MOE_ROUND_NONE, balance_lambda=None,
-                 gate_mode=B.MOE_GATE_TOPK_SOFTMAX, capacity_factor=None, precision="bf16"):
+                 gate_mode=B.MOE_GATE_TOPK_SOFTMAX, capacity_factor=None, precision="bf16",
+                 mx_wgrad=False):
         self.T, self.d, self.f, self.E, self.k = T, d, f, E, k
         self.dtype, self.device, self.round_mode = dtype, device, round_mode
         self.gate_mode = gate_mode
         if precision not in ("bf16", "mxfp8"):
             raise ValueError("precision must be 'bf16' or 'mxfp8'")
         self.precision = precision
+        self.mx_wgrad = bool(mx_wgrad) and precision == "mxfp8"
         if round_mode == B.MOE_ROUND_CAPACITY:
             if capacity_factor is None:
                 raise ValueError("MOE_ROUND_CAPACITY needs capacity_factor")
@@ -47,7 +49,8 @@ class MoELayerStep:
                        zip(B.MX_WEIGHT_NAMES, B.moe_mxfp8_weight_sizes(E, d, f))}
             self.ws_mx = e(max(B.moe_ffn_fwd_mxfp8_workspace_size(T, d, f, E, k), 1),
                            dt_=torch.uint8)
-            self.ws_bwd = e(max(B.moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k), 1),
+            self.ws_bwd = e(max(B.moe_layer_bwd_mxfp8_workspace_size(T, d, f, E, k,
+                                                                     self.mx_wgrad), 1),
                             dt_=torch.uint8)
         else:
             self.ws_fwd = e(max(B.moe_ffn_fwd_workspace_size(T, d, f, E, k, dt), 1),
@@ -111,12 +114,12 @@ class MoELayerStep:
     def backward(self, dout, stream=None):
         x, w_gate, w1, w3, w2 = self._saved
         gate_grad = self.balance["dgate"] if self.balance else None
-        if self.precision == "mxfp8":   # dX GEMM on MXFP8 operands
+        if self.precision == "mxfp8":   # dX (and with mx_wgrad the dW) GEMMs on MXFP8 operands
             return B.moe_layer_bwd_mxfp8(dout, x, w_gate, w1, w3, w2, self.wq, self.idx,
                                          self.gate, self.plan, self.H, self.router_grad,
                                          out=self.grads, ws=self.ws_bwd, stream=stream,
                                          gate_grad=gate_grad, logits=self.logits,
-                                         gate_mode=self.gate_mode)
+                                         gate_mode=self.gate_mode, wgrad=self.mx_wgrad)
         return B.moe_layer_bwd(dout, x, w_gate, w1, w3, w2, self.idx, self.gate, self.plan,
                                self.H, self.router_grad, out=self.grads, ws=self.ws_bwd,
                                stream=stream, gate_grad=gate_grad, logits=self.logits,

@@ -163,7 +163,15 @@ def test_mxfp8_entry_points_check_their_arguments():
     assert B.moe_ffn_fwd_mxfp8_workspace_size(16, 256, 256, 8, 2) > 0
     # backward: the quantised weights are required
     args = [f, f, f, f, f, f, None, f, f, f, f, f, None, None, 0, f, f, f, f, None, f, 16, 256,
-            256, 8, 2, 1, f, f, f, f, f, None, None, f, 1 << 40, None]
+            256, 8, 2, 1, 0, f, f, f, f, f, None, None, f, 1 << 40, None]
     assert lib.moe_layer_bwd_mxfp8(*args) == -1 and b"w1rq" in lib.moe_last_error()
     assert (B.moe_layer_bwd_mxfp8_workspace_size(16, 256, 256, 8, 2)
             > B.moe_layer_bwd_workspace_size(16, 256, 256, 8, 2, B.MOE_BF16))
+    # MXFP8 weight gradients: four more quantised row-space operands
+    assert (B.moe_layer_bwd_mxfp8_workspace_size(16, 256, 256, 8, 2, wgrad=True)
+            > B.moe_layer_bwd_mxfp8_workspace_size(16, 256, 256, 8, 2))
+    args[6:10] = [f, f, f, f]
+    args[27] = 2
+    assert lib.moe_layer_bwd_mxfp8(*args) == -1 and b"wgrad_mxfp8" in lib.moe_last_error()
+    args[27], args[22] = 1, 384          # d not a multiple of 256
+    assert lib.moe_layer_bwd_mxfp8(*args) == -2 and b"256" in lib.moe_last_error()

@@ -204,3 +204,92 @@ def test_mxfp8_full_size_sampled_tokens(name, n_tok):
                  "dlogits", BF16_TOL)
     rows = sorted(s["dS"])
     assert_close(f64(g["dS"])[rows], np.array([s["dS"][r] for r in rows]), "dS", BF16_TOL)
+
+
+# ---------------------------------------------------------------- weight gradients on MXFP8
+def _row_space(plan, width, g, gather_src=None):
+    """A row-space bf16 matrix [cap, width] with zero padding rows, or None
+    when gather_src (token rows) is given; the oracle's fp64 image [R, width]."""
+    R = int(plan["offsets"][-1])
+    tok = i64(plan["row_token"])[:R]
+    if gather_src is not None:
+        m = np.zeros((R, width))
+        m[tok >= 0] = f64(gather_src)[tok[tok >= 0]]
+        return None, m
+    cap = plan["row_token"].numel()
+    src = (torch.randn(cap, width, generator=g) * torch.exp(torch.randn(cap, 1, generator=g))
+           ).to(torch.bfloat16)
+    src[torch.from_numpy(np.concatenate([tok < 0, np.ones(cap - R, bool)]))] = 0
+    return src.cuda(), f64(src)[:R]
+
+
+@pytest.mark.parametrize("round_mode,gather", [(0, False), (1, False), (0, True), (1, True)])
+def test_mxfp8_token_quantisation_bitexact(round_mode, gather):
+    """moe_mxfp8_quantize_tokens: codes and scales of a row-space matrix
+    quantised along its rows (blocks of 32 rows), bit for bit against the
+    oracle's quantiser along axis 0; with gather_row, the rows come from
+    token rows (padding rows zero)."""
+    T, n, E, k = 700, 384, 8, 2
+    g = torch.Generator().manual_seed(50 + round_mode + 2 * gather)
+    lo = torch.randn(T, E, generator=g).cuda()
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=T, E=E)
+    plan = B.moe_permute(idx, gate, logits, E, round_mode)
+    R = int(plan["offsets"][-1])
+    capr = (B.moe_row_capacity(T, E, k) + 127) // 128 * 128
+    if gather:
+        x = (torch.randn(T, n, generator=g) * 3).to(torch.bfloat16).cuda()
+        _, m = _row_space(plan, n, g, gather_src=x)
+        q, sf = B.moe_mxfp8_quantize_tokens(x, plan["offsets"], capr, gather_row=plan["row_token"])
+    else:
+        src, m = _row_space(plan, n, g)
+        q, sf = B.moe_mxfp8_quantize_tokens(src, plan["offsets"], capr)
+    torch.cuda.synchronize()
+    B.moe_check_status()
+    oq, se = O.mx_quantize(m, 0)                         # [R, n], [R/32, n]
+    codes, scodes = expected_rows(oq, se)
+    np.testing.assert_array_equal(u8(q)[:, :R], codes.T)
+    assert not u8(q)[:, R:].any()                        # rows past the plan untouched (zeros)
+    kb = np.arange(R // 32)
+    off = sf_offset(np.arange(n)[:, None], kb[None, :], capr // 128)
+    np.testing.assert_array_equal(u8(sf)[off], scodes.T)
+
+
+@pytest.mark.parametrize("round_mode", [0, 1])
+def test_mxfp8_weight_gradients(round_mode):
+    """Weight-gradient GEMMs on MXFP8 operands (wgrad=True) against the
+    oracle's definition (operands quantised along tokens within each expert's
+    segment); an expert without rows gets zero gradients; everything else in
+    the backward is bit-identical to the bf16-wgrad run; and the MXFP8
+    gradients differ from the bf16 ones by the size the format implies."""
+    cfg = synth.MoEConfig("test", 900, 256, 256, 8, 2, std=0.05)
+    inp = synth.make_inputs(cfg, seed=60 + round_mode, device="cuda")
+    x, wg, w1, w3, w2, dout = (inp[n] for n in ("x", "w_gate", "w1", "w3", "w2", "dout"))
+    bias = torch.linspace(0.5, -0.5, cfg.E)
+    bias[5] = -1e4                                        # expert 5 receives no token
+    lg = fp32_router_logits(x, wg, bias)
+    logits, idx, gate = B.moe_route(x, wg, cfg.k, logits_override=torch.from_numpy(lg).cuda())
+    plan = B.moe_permute(idx, gate, logits, cfg.E, round_mode)
+    wq = B.moe_mxfp8_quantize_weights(w1, w3, w2)
+    H, Y = B.moe_expert_ffn_fwd_mxfp8(x, wq, plan, cfg.k, cfg.E, cfg.f)
+    g0 = B.moe_layer_bwd_mxfp8(dout, x, wg, w1, w3, w2, wq, idx, gate, plan, H)
+    g1 = B.moe_layer_bwd_mxfp8(dout, x, wg, w1, w3, w2, wq, idx, gate, plan, H, wgrad=True)
+    torch.cuda.synchronize()
+    B.moe_check_status()
+    assert int(plan["counts"][5]) == 0
+    R = int(plan["offsets"][-1])
+    for n in ("dx", "dw_gate", "dlogits"):
+        assert torch.equal(g0[n], g1[n]), n
+    live = plan["row_token"][:R] >= 0                   # (dS is written for live rows)
+    assert torch.equal(g0["dS"][:R][live], g1["dS"][:R][live])
+    for n in ("dw1", "dw3", "dw2"):
+        assert not bool(g1[n][5].any()), n
+    fwd = O.layer_fwd(f64(x), f64(wg), f64(w1), f64(w3), f64(w2), cfg.k, round_mode=round_mode,
+                      logits_override=lg.astype(np.float64), precision="mxfp8")
+    args = (f64(dout), f64(x), f64(wg), f64(w1), f64(w3), f64(w2), fwd)
+    ref_mx = O.layer_bwd(*args, mx_wgrad_on=True)
+    ref_bf = O.layer_bwd(*args)
+    for n in ("dw1", "dw3", "dw2"):
+        assert_close(g1[n], ref_mx[n], n, BF16_TOL)
+        gap = np.abs(f64(g1[n]) - ref_bf[n]).sum() / np.abs(ref_bf[n]).sum()
+        err = np.abs(f64(g1[n]) - ref_mx[n]).sum() / np.abs(ref_mx[n]).sum()
+        assert gap > 5 * err and gap > 2e-3, (n, gap, err)
