@@ -148,69 +148,84 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
 // scales in the layout of mx.cuh with n as the MN dimension and the rows as
 // K (capr / 128 K chunks).  Row r of the source is src row r, or, with
 // gather_row, token row gather_row[r] of a token-major source (-1: a zero
-// row).  One block per (128 rows, 256 columns): the tile arrives in two
-// rounds of loads (8 per thread in flight), then thread p quantises columns
-// 2p', 2p'+1 over 64 rows -- two MXFP8 blocks each, every value pair read
-// with one 32-bit shared load -- and writes 64 bytes of each column's output
-// row; the two threads of a column pair write its 128-byte line, and the
-// column's four scale bytes of this 128-row chunk sit side by side.
-// Only rows below offsets[E] are read or written.
-constexpr int QC_ROWS = 128, QC_COLS = 256, QC_LD = QC_COLS + 8;
+// row).  Each block owns a 256-column strip and walks its 64-row tiles
+// (grid-stride), double-buffered: the next tile's 16-byte cp.async copies
+// are in flight while thread p quantises column pair p' = p mod 128 over the
+// 32 rows 32 (p / 128).. of the current one (two MXFP8 blocks, each value
+// pair one 32-bit shared load) and writes 32 bytes of each column's output
+// row.  Only rows below offsets[E] are read or written.
+constexpr int QC_ROWS = 64, QC_COLS = 256, QC_LD = QC_COLS + 8;
+constexpr int QC_TILE = QC_ROWS * QC_LD;               // bf16 elements per buffer
 
-__global__ void __launch_bounds__(WQ_THREADS, 2)
+__device__ __forceinline__ void qc_load_tile(__nv_bfloat16* buf, const __nv_bfloat16* src,
+                                             const int32_t* gather_row, int n, int r0, int c0,
+                                             int ncols) {
+  constexpr int VPR = QC_COLS / 8;
+#pragma unroll
+  for (int i = 0; i < QC_ROWS * VPR / WQ_THREADS; ++i) {
+    const int v = threadIdx.x + i * WQ_THREADS;
+    const int r = v / VPR, c = (v % VPR) * 8;
+    if (c >= ncols) continue;
+    const int sr = gather_row != nullptr ? gather_row[r0 + r] : r0 + r;
+    const __nv_bfloat16* g = src + (size_t)(sr >= 0 ? sr : 0) * n + c0 + c;
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(buf + r * QC_LD + c);
+    const int bytes = sr >= 0 ? 16 : 0;                // 0: zero fill
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(g), "r"(bytes)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(WQ_THREADS, 3)
 k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict__ gather_row,
                 const int32_t* __restrict__ offsets, int E, int n, int capr,
                 uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
   extern __shared__ __align__(16) uint8_t qc_smem[];
-  __nv_bfloat16 (*tile)[QC_LD] = reinterpret_cast<__nv_bfloat16 (*)[QC_LD]>(qc_smem);
-  const int r0 = blockIdx.x * QC_ROWS, c0 = blockIdx.y * QC_COLS;
-  if (r0 >= offsets[E]) return;                        // whole block (segments are 128-aligned)
+  __nv_bfloat16* bufs = reinterpret_cast<__nv_bfloat16*>(qc_smem);
+  const int R = offsets[E];
+  const int c0 = blockIdx.y * QC_COLS;
   const int ncols = min(QC_COLS, n - c0);             // a multiple of 128
-  constexpr int VPR = QC_COLS / 8;                     // 16-byte vectors per tile row
-  constexpr int PER = QC_ROWS * VPR / WQ_THREADS / 2;  // per thread and round
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint4 u[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int v = threadIdx.x + (half * PER + i) * WQ_THREADS;
-      const int r = v / VPR, c = (v % VPR) * 8;
-      const int sr = gather_row != nullptr ? gather_row[r0 + r] : r0 + r;
-      u[i] = make_uint4(0, 0, 0, 0);
-      if (c < ncols && sr >= 0) u[i] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)sr * n + c0 + c));
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int v = threadIdx.x + (half * PER + i) * WQ_THREADS;
-      const int r = v / VPR, c = (v % VPR) * 8;
-      if (c < ncols) *reinterpret_cast<uint4*>(&tile[r][c]) = u[i];
-    }
-  }
-  __syncthreads();
+  const int ntiles = R / QC_ROWS;                      // R is a multiple of 128
   const int p = threadIdx.x & (QC_COLS / 2 - 1);       // column pair
-  const int rh = threadIdx.x / (QC_COLS / 2);          // rows 64 rh .. 64 rh + 63
-  if (2 * p >= ncols) return;
+  const int rb = 32 * (threadIdx.x / (QC_COLS / 2));   // this thread's 32 rows of a tile
   const int kchunks = capr / 128;
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {                        // the two 32-row blocks of this thread
-    const int rb = 64 * rh + 32 * b;
-    uint32_t pk[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(&tile[rb + i][2 * p]);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int col = c0 + 2 * p + h;
-      mx_store_block_packed(pk, h == 1, q + (size_t)col * capr + r0 + rb,
-                            sf + mx_sf_offset(col, (r0 + rb) >> 5, kchunks));
+  int t = blockIdx.x;
+  if (t < ntiles) qc_load_tile(bufs, src, gather_row, n, t * QC_ROWS, c0, ncols);
+  for (int it = 0; t < ntiles; ++it, t += gridDim.x) {
+    const int tn = t + gridDim.x;
+    __nv_bfloat16* cur = bufs + (it & 1) * QC_TILE;
+    if (tn < ntiles) {
+      qc_load_tile(bufs + ((it + 1) & 1) * QC_TILE, src, gather_row, n, tn * QC_ROWS, c0, ncols);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
+    __syncthreads();
+    if (2 * p < ncols) {
+      const int r0 = t * QC_ROWS + rb;
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) pk[i] = *reinterpret_cast<const uint32_t*>(cur + (rb + i) * QC_LD + 2 * p);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int col = c0 + 2 * p + h;
+        mx_store_block_packed(pk, h == 1, q + (size_t)col * capr + r0,
+                              sf + mx_sf_offset(col, r0 >> 5, kchunks));
+      }
+    }
+    __syncthreads();                                   // the buffer is refilled next iteration
   }
 }
 
 int launch_mx_quant_cols(const void* src, const int32_t* gather_row, const int32_t* offsets,
                          int E, int n, int capr, uint8_t* q, uint8_t* sf, cudaStream_t s) {
   if (n % 128 || capr % 128) return fail(MOE_ERR_UNSUPPORTED, "token-axis MXFP8 needs n and rows in multiples of 128");
-  dim3 grid(capr / QC_ROWS, (n + QC_COLS - 1) / QC_COLS);
-  const int smem = QC_ROWS * QC_LD * 2;
+  const int strips = (n + QC_COLS - 1) / QC_COLS;
+  int per = device_sm_count() * 3 / strips;            // resident blocks over the column strips
+  if (per < 1) per = 1;
+  if (per > capr / QC_ROWS) per = capr / QC_ROWS;
+  dim3 grid(per, strips);
+  const int smem = 2 * QC_TILE * 2;
   cudaError_t e = cudaFuncSetAttribute(k_mx_quant_cols, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e, "mx_quant_cols smem attribute");
   {
