@@ -248,11 +248,14 @@ size_t moe_ffn_fwd_mxfp8_workspace_size(int T, int d, int f, int E, int k);
  * of q, rows contiguous) and sf its E8M0 scales in the layout above with n
  * as the row (MN) dimension and capr / 128 K chunks.  Bytes of q and sf for
  * rows at or above offsets[E] are left untouched.  n and capr: multiples of
- * 128 (capr >= offsets[E]); src and q 16-byte aligned; device buffers owned
- * by the caller.  Needs no sm_100 features beyond the CUDA cores.
+ * 128 (capr >= offsets[E]); src has src_rows rows; src and q 16-byte
+ * aligned; device buffers owned by the caller.  A plan past capr, or a
+ * source row at or past src_rows, is a device data check (code 0x140 from
+ * moe_check_status; the plan is skipped, the row read as zeros).
  */
-int moe_mxfp8_quantize_tokens(const void* src, const int32_t* gather_row, const int32_t* offsets,
-                              int E, int n, int capr, uint8_t* q, uint8_t* sf, void* stream);
+int moe_mxfp8_quantize_tokens(const void* src, int src_rows, const int32_t* gather_row,
+                              const int32_t* offsets, int E, int n, int capr, uint8_t* q,
+                              uint8_t* sf, void* stream);
 /*
  * moe_layer_bwd_mxfp8 -- moe_layer_bwd (bf16 only) whose dX_perm GEMM runs
  * on MXFP8 operands: the dA' epilogue also writes dH in E4M3 with blocks
@@ -455,7 +458,9 @@ int moe_balance_loss(const int32_t* idx, const float* gate, int T, int E, int k,
  * since the last check (codes 0x2nn: the kernel gave up, drained its copies,
  * freed its TMEM and returned; its outputs are undefined), or
  * MOE_ERR_DEVICE_CHECK if a kernel met invalid data and skipped it (0x120:
- * an expert id outside [0, E); 0x1ff: shared memory not 1 KB aligned).  The
+ * an expert id outside [0, E); 0x130: an expert-parallel row count that is
+ * not a 128-multiple; 0x140: a row-space plan or source row outside the
+ * token-axis quantiser's buffers; 0x1ff: shared memory not 1 KB aligned).  The
  * code is in moe_last_error()'s message.
  */
 int moe_check_status(void* stream);

@@ -67,7 +67,7 @@ _SIGS = {
     "moe_balance_loss": (_i, [_vp, _vp, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_mxfp8_weight_sizes": (_i, [_i, _i, _i, ctypes.POINTER(_sz)]),
     "moe_mxfp8_quantize_weights": (_i, [_vp, _vp, _vp, _i, _i, _i] + [_vp] * 9),
-    "moe_mxfp8_quantize_tokens": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_mxfp8_quantize_tokens": (_i, [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
     "moe_layer_bwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moe_layer_bwd_mxfp8": (_i, [_vp] * 14 + [_i] + [_vp] * 6 + [_i] * 7 + [_vp] * 8 + [_sz, _vp]),
     "moe_ffn_fwd_mxfp8_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -236,8 +236,8 @@ def moe_mxfp8_quantize_tokens(src, offsets, capr, gather_row=None, stream=None):
     E = offsets.numel() - 1
     q = torch.zeros(n, capr, device=src.device, dtype=torch.uint8)
     sf = torch.zeros(n * capr // 32, device=src.device, dtype=torch.uint8)
-    _check(lib().moe_mxfp8_quantize_tokens(_p(src), _p(gather_row), _p(offsets), E, n, capr,
-                                           _p(q), _p(sf), _stream(stream)))
+    _check(lib().moe_mxfp8_quantize_tokens(_p(src), src.shape[0], _p(gather_row), _p(offsets), E,
+                                           n, capr, _p(q), _p(sf), _stream(stream)))
     return q, sf
 
 

@@ -360,14 +360,17 @@ int moe_mxfp8_weight_sizes(int E, int d, int f, size_t* sizes) {
   return MOE_OK;
 }
 
-int moe_mxfp8_quantize_tokens(const void* src, const int32_t* gather_row, const int32_t* offsets,
-                              int E, int n, int capr, uint8_t* q, uint8_t* sf, void* stream) {
+int moe_mxfp8_quantize_tokens(const void* src, int src_rows, const int32_t* gather_row,
+                              const int32_t* offsets, int E, int n, int capr, uint8_t* q,
+                              uint8_t* sf, void* stream) {
   if (E < 1 || E > 256) return fail(MOE_ERR_UNSUPPORTED, "E must be in [1, 256]");
+  if (src_rows < 0) return fail(MOE_ERR_INVALID_ARG, "src_rows must be >= 0");
   if (n <= 0 || n % 128 || capr <= 0 || capr % 128)
     return fail(MOE_ERR_UNSUPPORTED, "n and capr must be positive multiples of 128");
   REQUIRE_PTR(src); REQUIRE_PTR(offsets); REQUIRE_PTR(q); REQUIRE_PTR(sf);
   REQUIRE_ALIGNED(src); REQUIRE_ALIGNED(q);
-  return launch_mx_quant_cols(src, gather_row, offsets, E, n, capr, q, sf, (cudaStream_t)stream);
+  return launch_mx_quant_cols(src, src_rows, gather_row, offsets, E, n, capr, q, sf,
+                              (cudaStream_t)stream);
 }
 
 int moe_mxfp8_quantize_weights(const void* w1, const void* w3, const void* w2, int E, int d,
@@ -530,6 +533,7 @@ static int layer_bwd_impl(const void* dout, const void* x, const void* w_gate, c
     if (mx_wgrad) {   // x, dO, s*A, dH quantised along the rows for the dW GEMMs
       mx.wgrad = 1;
       mx.capr = (int)capr;
+      mx.T = T;
       mx.x = x;
       mx.row_token = row_token;
       mx.xq = c.take<uint8_t>(capr * d);

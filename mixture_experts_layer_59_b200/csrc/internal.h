@@ -94,7 +94,7 @@ struct MxBwd {
   // weight gradients on MXFP8 operands (wgrad = 1): x, dO, s*A and dH
   // quantised along the rows, [n, capr] E4M3 + scales; x is gathered from
   // the token rows through row_token
-  int wgrad, capr;
+  int wgrad, capr, T;
   const void* x;
   const int32_t* row_token;
   uint8_t *xq, *xs, *oq, *os, *aq, *as, *hq, *hs;
@@ -131,8 +131,9 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
                             uint8_t* w13q, uint8_t* w13s, uint8_t* w2q, uint8_t* w2s,
                             uint8_t* w1rq, uint8_t* w1rs, uint8_t* w3rq, uint8_t* w3rs,
                             cudaStream_t s);
-int launch_mx_quant_cols(const void* src, const int32_t* gather_row, const int32_t* offsets,
-                         int E, int n, int capr, uint8_t* q, uint8_t* sf, cudaStream_t s);
+int launch_mx_quant_cols(const void* src, int src_rows, const int32_t* gather_row,
+                         const int32_t* offsets, int E, int n, int capr, uint8_t* q, uint8_t* sf,
+                         cudaStream_t s);
 int launch_mx_scatter_rows(const void* x, const int32_t* slot_row, const int32_t* extra_row,
                            const int32_t* row_token, const int32_t* offsets, int T, int d, int E,
                            int k, uint8_t* q, uint8_t* sf, cudaStream_t s);

@@ -153,20 +153,26 @@ int launch_mx_quant_weights(const void* w1, const void* w3, const void* w2, int 
 // are in flight while thread p quantises column pair p' = p mod 128 over the
 // 32 rows 32 (p / 128).. of the current one (two MXFP8 blocks, each value
 // pair one 32-bit shared load) and writes 32 bytes of each column's output
-// row.  Only rows below offsets[E] are read or written.
+// row.  Only rows below offsets[E] are read or written.  A plan larger than
+// capr, or a source row at or past src_rows, is recorded as device data
+// check 0x140 (the plan is skipped, the row read as zeros).
 constexpr int QC_ROWS = 64, QC_COLS = 256, QC_LD = QC_COLS + 8;
 constexpr int QC_TILE = QC_ROWS * QC_LD;               // bf16 elements per buffer
 
 __device__ __forceinline__ void qc_load_tile(__nv_bfloat16* buf, const __nv_bfloat16* src,
-                                             const int32_t* gather_row, int n, int r0, int c0,
-                                             int ncols) {
+                                             const int32_t* gather_row, int src_rows, int n,
+                                             int r0, int c0, int ncols, int* status) {
   constexpr int VPR = QC_COLS / 8;
 #pragma unroll
   for (int i = 0; i < QC_ROWS * VPR / WQ_THREADS; ++i) {
     const int v = threadIdx.x + i * WQ_THREADS;
     const int r = v / VPR, c = (v % VPR) * 8;
     if (c >= ncols) continue;
-    const int sr = gather_row != nullptr ? gather_row[r0 + r] : r0 + r;
+    int sr = gather_row != nullptr ? gather_row[r0 + r] : r0 + r;
+    if (sr >= src_rows) {   // a row the source does not have: flag it, read a zero row
+      record_status(status, 0x140);
+      sr = -1;
+    }
     const __nv_bfloat16* g = src + (size_t)(sr >= 0 ? sr : 0) * n + c0 + c;
     const uint32_t d = (uint32_t)__cvta_generic_to_shared(buf + r * QC_LD + c);
     const int bytes = sr >= 0 ? 16 : 0;                // 0: zero fill
@@ -177,12 +183,16 @@ __device__ __forceinline__ void qc_load_tile(__nv_bfloat16* buf, const __nv_bflo
 }
 
 __global__ void __launch_bounds__(WQ_THREADS, 3)
-k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict__ gather_row,
-                const int32_t* __restrict__ offsets, int E, int n, int capr,
-                uint8_t* __restrict__ q, uint8_t* __restrict__ sf) {
+k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, int src_rows,
+                const int32_t* __restrict__ gather_row, const int32_t* __restrict__ offsets, int E,
+                int n, int capr, uint8_t* __restrict__ q, uint8_t* __restrict__ sf, int* status) {
   extern __shared__ __align__(16) uint8_t qc_smem[];
   __nv_bfloat16* bufs = reinterpret_cast<__nv_bfloat16*>(qc_smem);
-  const int R = offsets[E];
+  int R = offsets[E];
+  if (R > capr || R < 0 || R % 128) {   // a plan that does not fit the output: flag it, do nothing
+    if (threadIdx.x == 0) record_status(status, 0x140);
+    return;
+  }
   const int c0 = blockIdx.y * QC_COLS;
   const int ncols = min(QC_COLS, n - c0);             // a multiple of 128
   const int ntiles = R / QC_ROWS;                      // R is a multiple of 128
@@ -190,12 +200,13 @@ k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict
   const int rb = 32 * (threadIdx.x / (QC_COLS / 2));   // this thread's 32 rows of a tile
   const int kchunks = capr / 128;
   int t = blockIdx.x;
-  if (t < ntiles) qc_load_tile(bufs, src, gather_row, n, t * QC_ROWS, c0, ncols);
+  if (t < ntiles) qc_load_tile(bufs, src, gather_row, src_rows, n, t * QC_ROWS, c0, ncols, status);
   for (int it = 0; t < ntiles; ++it, t += gridDim.x) {
     const int tn = t + gridDim.x;
     __nv_bfloat16* cur = bufs + (it & 1) * QC_TILE;
     if (tn < ntiles) {
-      qc_load_tile(bufs + ((it + 1) & 1) * QC_TILE, src, gather_row, n, tn * QC_ROWS, c0, ncols);
+      qc_load_tile(bufs + ((it + 1) & 1) * QC_TILE, src, gather_row, src_rows, n, tn * QC_ROWS,
+                   c0, ncols, status);
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
       asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -217,8 +228,9 @@ k_mx_quant_cols(const __nv_bfloat16* __restrict__ src, const int32_t* __restrict
   }
 }
 
-int launch_mx_quant_cols(const void* src, const int32_t* gather_row, const int32_t* offsets,
-                         int E, int n, int capr, uint8_t* q, uint8_t* sf, cudaStream_t s) {
+int launch_mx_quant_cols(const void* src, int src_rows, const int32_t* gather_row,
+                         const int32_t* offsets, int E, int n, int capr, uint8_t* q, uint8_t* sf,
+                         cudaStream_t s) {
   if (n % 128 || capr % 128) return fail(MOE_ERR_UNSUPPORTED, "token-axis MXFP8 needs n and rows in multiples of 128");
   const int strips = (n + QC_COLS - 1) / QC_COLS;
   int per = device_sm_count() * 3 / strips;            // resident blocks over the column strips
@@ -230,8 +242,8 @@ int launch_mx_quant_cols(const void* src, const int32_t* gather_row, const int32
   if (e != cudaSuccess) return cuda_fail(e, "mx_quant_cols smem attribute");
   {
     ProfScope _ps("mx_quant_cols", s);
-    k_mx_quant_cols<<<grid, WQ_THREADS, smem, s>>>((const __nv_bfloat16*)src, gather_row, offsets, E,
-                                                   n, capr, q, sf);
+    k_mx_quant_cols<<<grid, WQ_THREADS, smem, s>>>((const __nv_bfloat16*)src, src_rows, gather_row,
+                                                   offsets, E, n, capr, q, sf, status_ptr());
   }
   MOE_CHECK_LAUNCH("mx_quant_cols");
   return MOE_OK;

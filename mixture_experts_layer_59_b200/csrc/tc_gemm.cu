@@ -1201,11 +1201,11 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     const int capr = mx->capr;
     if (d % 256 || (2 * f) % 256)
       return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weight gradients need d and 2f multiples of 256");
-    if ((rc = launch_mx_quant_cols(mx->x, mx->row_token, p.offsets, E, d, capr, mx->xq, mx->xs, s)))
+    if ((rc = launch_mx_quant_cols(mx->x, mx->T, mx->row_token, p.offsets, E, d, capr, mx->xq, mx->xs, s)))
       return rc;
-    if ((rc = launch_mx_quant_cols(dog, nullptr, p.offsets, E, d, capr, mx->oq, mx->os, s))) return rc;
-    if ((rc = launch_mx_quant_cols(gact, nullptr, p.offsets, E, f, capr, mx->aq, mx->as, s))) return rc;
-    if ((rc = launch_mx_quant_cols(dH, nullptr, p.offsets, E, 2 * f, capr, mx->hq, mx->hs, s)))
+    if ((rc = launch_mx_quant_cols(dog, cap, nullptr, p.offsets, E, d, capr, mx->oq, mx->os, s))) return rc;
+    if ((rc = launch_mx_quant_cols(gact, cap, nullptr, p.offsets, E, f, capr, mx->aq, mx->as, s))) return rc;
+    if ((rc = launch_mx_quant_cols(dH, cap, nullptr, p.offsets, E, 2 * f, capr, mx->hq, mx->hs, s)))
       return rc;
     {
       TcArgs a = base_args(p);

@@ -293,3 +293,35 @@ def test_mxfp8_weight_gradients(round_mode):
         gap = np.abs(f64(g1[n]) - ref_bf[n]).sum() / np.abs(ref_bf[n]).sum()
         err = np.abs(f64(g1[n]) - ref_mx[n]).sum() / np.abs(ref_mx[n]).sum()
         assert gap > 5 * err and gap > 2e-3, (n, gap, err)
+
+
+def test_mxfp8_token_quantisation_flags_rows_outside_its_buffers():
+    """The quantiser's own checks: a gather row past the source (read as a
+    zero row) and a plan longer than the output (skipped) are reported as
+    device data check 0x140 and write nothing outside the buffers."""
+    T, n, E, k = 300, 256, 4, 2
+    g = torch.Generator().manual_seed(70)
+    lo = torch.randn(T, E, generator=g).cuda()
+    logits, idx, gate = B.moe_route(None, None, k, logits_override=lo, T=T, E=E)
+    plan = B.moe_permute(idx, gate, logits, E)
+    R = int(plan["offsets"][-1])
+    capr = (B.moe_row_capacity(T, E, k) + 127) // 128 * 128
+    x = torch.randn(T, n, generator=g).to(torch.bfloat16).cuda()
+    bad = plan["row_token"].clone()
+    r_bad = int(torch.nonzero(bad[:R] >= 0)[3])
+    bad[r_bad] = T + 5
+    q, sf = B.moe_mxfp8_quantize_tokens(x, plan["offsets"], capr, gather_row=bad)
+    with pytest.raises(B.MoEError) as ei:
+        B.moe_check_status()
+    assert ei.value.code == B.MOE_ERR_DEVICE_CHECK and "0x140" in str(ei.value)
+    good = bad.clone()
+    good[r_bad] = -1                                      # what the kernel read instead
+    q2, sf2 = B.moe_mxfp8_quantize_tokens(x, plan["offsets"], capr, gather_row=good)
+    B.moe_check_status()
+    assert torch.equal(q, q2) and torch.equal(sf, sf2)
+    # a plan longer than the output rows: skipped, flagged
+    q3, sf3 = B.moe_mxfp8_quantize_tokens(x, plan["offsets"], 128, gather_row=plan["row_token"])
+    with pytest.raises(B.MoEError) as ei:
+        B.moe_check_status()
+    assert "0x140" in str(ei.value)
+    assert not bool(q3.any()) and not bool(sf3.any())
