@@ -58,9 +58,9 @@ using namespace tc;
 
 enum Kind : int {
   K_UP = 0, K_DOWN = 1, K_DAP = 2, K_DX = 3, K_DW2 = 4, K_DW13 = 5, K_RT = 6, K_DWG = 7, K_DXR = 8,
-  K_UPQ = 9, K_DOWNQ = 10, K_DXQ = 11, K_DAPQ = 12, K_DW2Q = 13, K_DW13Q = 14
+  K_UPQ = 9, K_DOWNQ = 10, K_DXQ = 11, K_DAPQ = 12, K_DW2Q = 13, K_DW13Q = 14, K_DAPQW = 15
 };
-constexpr int NUM_KINDS = 15;
+constexpr int NUM_KINDS = 16;
 constexpr int MX_SF_COL = 256;         // TMEM column of the scale blocks (after the accumulators)
 
 constexpr int BM = 128;
@@ -112,6 +112,13 @@ struct TcArgs {
   uint8_t* act_s;            // UPQ: its scale blocks [cap/128][f/128]
   uint8_t* dh_q;             // DAP (MXFP8 backward): dH as E4M3 [cap, 2f], or null
   uint8_t* dh_s;             // its scale blocks [cap/128][2f/128]
+  // DAPQ with MXFP8 weight gradients: dH and s*A quantised along the rows
+  // ([2f, capr] and [f, capr] E4M3 + scales) instead of written in bf16
+  uint8_t* dht_q;
+  uint8_t* dht_s;
+  uint8_t* gat_q;
+  uint8_t* gat_s;
+  int capr;
   const uint8_t* sfb1;       // DXQ: scale blocks of W3r (sfb: of W1r)
   int kh;                    // DXQ: K chunks per weight half (f / 128)
   // bounded waits give up after wait_ns; dbg_no_load (test hook) makes the
@@ -288,6 +295,46 @@ __device__ __forceinline__ void stage_store(uint8_t* tiles, int& which, const fl
   }
 }
 
+// A warp's 32 x 32 chunk (lane = row row0 + lane, v = its 32 columns col0..)
+// quantised along the rows: each column is one MXFP8 block of 32 rows (the
+// bf16 values, as stored).  The chunk goes through shared memory as bf16
+// pairs (lane l writes its row, 16 words; lane c then reads column c, one
+// 16-bit value per row, once for the maximum and once for the codes; rows
+// 17 words apart, so neither side collides in a bank).  Lane c owns its
+// column: the block maximum, scale and the 32 codes, written to row col0 + c
+// of q [n, capr] and sf.
+__device__ __forceinline__ void colq_store(const float* v, uint32_t* tbuf, uint8_t* q, uint8_t* sf,
+                                           int col0, int row0, int capr, int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+    uint32_t u;
+    memcpy(&u, &h, 4);
+    tbuf[lane * 17 + j] = u;
+  }
+  __syncwarp();
+  // column values read twice (maximum, then codes) rather than held in registers
+  auto val = [&](int i) {
+    const uint32_t u = tbuf[i * 17 + (lane >> 1)];
+    return __uint_as_float((lane & 1) ? (u & 0xffff0000u) : (u << 16));
+  };
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(val(i)));
+  const uint32_t code = mx_scale_code(amax);
+  const float inv = mx_inv_scale(code);
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    w[i] = cvt_e4m3x2(val(4 * i) * inv, val(4 * i + 1) * inv) |
+           (cvt_e4m3x2(val(4 * i + 2) * inv, val(4 * i + 3) * inv) << 16);
+  __syncwarp();
+  uint4* dst = reinterpret_cast<uint4*>(q + (size_t)(col0 + lane) * capr + row0);
+  dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  sf[mx_sf_offset(col0 + lane, row0 >> 5, capr / 128)] = (uint8_t)code;
+}
+
 template <int KIND, int BN>
 __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ TcArgs a) {
   using C = Cfg<BN, KT<KIND>::MX>;
@@ -363,7 +410,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           } else if constexpr (KIND == K_DOWN) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
             tma_load_4d(sB, &a.mB0, &full_bar[stage], 0, k0, ti.n0 / 64, ti.e);   // BN / 64 atoms
-          } else if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
+          } else if constexpr (KIND == K_DAP || KIND == K_DAPQ || KIND == K_DAPQW) {
             tma_load_2d(sA, &a.mA, &full_bar[stage], k0, ti.m0);
             tma_load_3d(sB, &a.mB0, &full_bar[stage], k0, ti.n0, ti.e);
           } else if constexpr (KIND == K_DX) {
@@ -504,7 +551,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
       // loads are issued before waiting for the main loop
       uint4 hn1[4], hn3[4];
       const __nv_bfloat16* hrow = nullptr;
-      if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
+      if constexpr (KIND == K_DAP || KIND == K_DAPQ || KIND == K_DAPQW) {
         hrow = a.hin + (size_t)(ti.m0 + rloc) * 2 * a.f;
         const uint4* s1 = reinterpret_cast<const uint4*>(hrow + ti.n0 + half * (BN / 2));
         const uint4* s3 = reinterpret_cast<const uint4*>(hrow + a.f + ti.n0 + half * (BN / 2));
@@ -619,7 +666,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
           stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);
         }
-      } else if constexpr (KIND == K_DAP || KIND == K_DAPQ) {
+      } else if constexpr (KIND == K_DAP || KIND == K_DAPQ || KIND == K_DAPQW) {
         const int f = a.f;
         const float g = a.row_gate[row];
         float ds = 0.f;
@@ -651,18 +698,29 @@ __global__ void __launch_bounds__(THREADS, 1) k_tc_gemm(const __grid_constant__ 
             da3[i] = da * sl;
             r[i] = __float_as_uint(g * av);                           // s * A
           }
-          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
-          stage_store<C::OUT_TILES>(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
-          if constexpr (KIND == K_DAPQ) {  // MXFP8 backward: dH blocks along 2f for the dX GEMM
+          // MXFP8 weight gradients: dH and s*A leave quantised along the rows
+          // instead of in bf16 (the staging tiles hold the transposes)
+          constexpr bool colq = KIND == K_DAPQW;
+          uint32_t* tbuf = reinterpret_cast<uint32_t*>(otile);
+          if constexpr (!colq) {
+            stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO0, ti.n0 + c, row0, lane);       // dH1
+            stage_store<C::OUT_TILES>(otile, obuf, da3, &a.sO0, f + ti.n0 + c, row0, lane); // dH3
+          }
+          if constexpr (KIND == K_DAPQ || KIND == K_DAPQW) {  // MXFP8 backward: dH blocks along 2f for the dX GEMM
             const int kc = (2 * f) / 128;
             mx_store_block(v, a.dh_q + (size_t)row * 2 * f + ti.n0 + c,
                            a.dh_s + mx_sf_offset(row, (ti.n0 + c) / 32, kc));
             mx_store_block(da3, a.dh_q + (size_t)row * 2 * f + f + ti.n0 + c,
                            a.dh_s + mx_sf_offset(row, (f + ti.n0 + c) / 32, kc));
+            if constexpr (colq) {
+              colq_store(v, tbuf, a.dht_q, a.dht_s, ti.n0 + c, row0, a.capr, lane);
+              colq_store(da3, tbuf, a.dht_q, a.dht_s, f + ti.n0 + c, row0, a.capr, lane);
+            }
           }
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-          stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);      // s * A
+          if constexpr (colq) colq_store(v, tbuf, a.gat_q, a.gat_s, ti.n0 + c, row0, a.capr, lane);   // s * A
+          else stage_store<C::OUT_TILES>(otile, obuf, v, &a.sO1, ti.n0 + c, row0, lane);   // s * A
         }
         a.ds_part[(size_t)row * a.nparts + 2 * ti.ntile + half] = ds;
       } else if constexpr (KIND == K_RT) {
@@ -935,7 +993,7 @@ static int launch(const TcArgs& args, int grid, cudaStream_t s) {
   static const char* kNames[NUM_KINDS] = {
       "tc_up",   "tc_down",   "tc_dap",       "tc_dx",        "tc_dw2",   "tc_dw13",
       "tc_router", "tc_router_dw", "tc_dx_router", "tc_up_mxfp8", "tc_down_mxfp8", "tc_dx_mxfp8",
-      "tc_dap", "tc_dw2_mxfp8", "tc_dw13_mxfp8"};
+      "tc_dap", "tc_dw2_mxfp8", "tc_dw13_mxfp8", "tc_dap"};
   static_assert(KIND >= 0 && KIND < NUM_KINDS, "kind out of range");
   {
     ProfScope _ps(kNames[KIND], s);
@@ -1156,11 +1214,22 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if (mx != nullptr) {
       a.dh_q = mx->dhq;
       a.dh_s = mx->dhs;
+      if (mx->wgrad) {   // dH and s*A straight to the rows-quantised operands of the dW GEMMs
+        a.dht_q = mx->hq;
+        a.dht_s = mx->hs;
+        a.gat_q = mx->aq;
+        a.gat_s = mx->as;
+        a.capr = mx->capr;
+      }
     }
     a.nparts = 2 * (f / bn);
     if (a.nparts != tc_num_dS_parts(f)) return fail(MOE_ERR_UNSUPPORTED, "dS partition mismatch");
     if (mx != nullptr) {
-      if ((rc = launch_bn<K_DAPQ>(a, bn, num_sms, s))) return rc;
+      if (mx->wgrad) {
+        if ((rc = launch_bn<K_DAPQW>(a, bn, num_sms, s))) return rc;
+      } else if ((rc = launch_bn<K_DAPQ>(a, bn, num_sms, s))) {
+        return rc;
+      }
     } else if ((rc = launch_bn<K_DAP>(a, bn, num_sms, s))) {
       return rc;
     }
@@ -1204,9 +1273,7 @@ int tc_ffn_bwd(const FfnPtrs& p, const void* dog, const void* xg, const float* r
     if ((rc = launch_mx_quant_cols(mx->x, mx->T, mx->row_token, p.offsets, E, d, capr, mx->xq, mx->xs, s)))
       return rc;
     if ((rc = launch_mx_quant_cols(dog, cap, nullptr, p.offsets, E, d, capr, mx->oq, mx->os, s))) return rc;
-    if ((rc = launch_mx_quant_cols(gact, cap, nullptr, p.offsets, E, f, capr, mx->aq, mx->as, s))) return rc;
-    if ((rc = launch_mx_quant_cols(dH, cap, nullptr, p.offsets, E, 2 * f, capr, mx->hq, mx->hs, s)))
-      return rc;
+    // (dH and s*A: quantised along the rows by the dA' epilogue)
     {
       TcArgs a = base_args(p);
       a.M = f;
