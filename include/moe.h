@@ -208,7 +208,8 @@ int moe_expert_ffn_fwd(const void* x, const void* w1, const void* w3, const void
  * The GEMMs run on the tcgen05 block-scaled tensor cores (kind::mxf8f6f4)
  * with fp32 accumulation; H and Y are bf16 as in moe_expert_ffn_fwd.  The
  * backward is moe_layer_bwd (all bf16) or moe_layer_bwd_mxfp8, whose dX GEMM
- * takes MXFP8 dH and W1/W3 (blocks along f); either way the quantisers pass
+ * takes MXFP8 dH and W1/W3 (blocks along f), and optionally its weight-
+ * gradient GEMMs MXFP8 operands along tokens; either way the quantisers pass
  * gradients straight through.
  *
  * moe_mxfp8_weight_sizes: sizes[8] out = bytes of W13q, W13s, W2q, W2s,
