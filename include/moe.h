@@ -484,8 +484,9 @@ int moe_debug_expire_next_wait(long long wait_ns);
  * bracketed by two CUDA events recorded on the kernel's own stream.
  * moe_profile_enable(0) stops recording.
  * moe_profile_report: waits for the recorded events, then writes one line
- * "<kernel> <launches> <total_ms>" per kernel name into buf (NUL-terminated)
- * and forgets the records.  Returns MOE_ERR_INVALID_ARG if buf is too small.
+ * "<kernel> <launches> <total_ms> <median_ms>" per kernel name into buf
+ * (NUL-terminated; median_ms is the median single-launch time) and forgets
+ * the records.  Returns MOE_ERR_INVALID_ARG if buf is too small.
  */
 int moe_profile_enable(int on);
 int moe_profile_report(char* buf, size_t buf_len);

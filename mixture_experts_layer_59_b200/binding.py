@@ -365,14 +365,15 @@ def moe_profile_enable(on: bool = True):
 
 
 def moe_profile_report() -> dict:
-    """{kernel name: (launches, total_ms)} of the launches recorded since the
-    last report (waits for their events)."""
+    """{kernel name: (launches, total_ms, median_ms)} of the launches recorded
+    since the last report (waits for their events); median_ms is the median
+    time of one launch."""
     buf = ctypes.create_string_buffer(1 << 16)
     _check(lib().moe_profile_report(buf, len(buf)))
     out = {}
     for line in buf.value.decode().splitlines():
-        name, n, ms = line.split()
-        out[name] = (int(n), float(ms))
+        name, n, ms, med = line.split()
+        out[name] = (int(n), float(ms), float(med))
     return out
 
 

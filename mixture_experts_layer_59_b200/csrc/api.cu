@@ -1,4 +1,5 @@
 // extern "C" entry points: argument checks, workspace layout, kernel order.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -771,24 +772,28 @@ int moe_profile_enable(int on) {
 int moe_profile_report(char* buf, size_t buf_len) {
   if (buf == nullptr || buf_len == 0) return fail(MOE_ERR_INVALID_ARG, "buf must not be NULL");
   std::lock_guard<std::mutex> lk(g_prof_mu);
-  std::map<std::string, std::pair<int, double>> agg;
+  std::map<std::string, std::vector<float>> agg;   // launch times per kernel name
   int rc = MOE_OK;
   for (auto& r : g_recs) {
     float ms = 0.f;
     cudaError_t e = cudaEventSynchronize(r.b);
     if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.a, r.b);
     if (e != cudaSuccess) rc = cuda_fail(e, "profile event");
-    auto& v = agg[r.name];
-    v.first += 1;
-    v.second += ms;
+    agg[r.name].push_back(ms);
     g_pool.push_back(r.a);
     g_pool.push_back(r.b);
   }
   g_recs.clear();
   std::string out;
-  char line[160];
+  char line[192];
   for (auto& kv : agg) {
-    snprintf(line, sizeof(line), "%s %d %.6f\n", kv.first.c_str(), kv.second.first, kv.second.second);
+    std::vector<float>& v = kv.second;
+    double total = 0.0;
+    for (float ms : v) total += ms;
+    std::sort(v.begin(), v.end());
+    const size_t n = v.size();
+    const double median = n % 2 ? v[n / 2] : 0.5 * ((double)v[n / 2 - 1] + v[n / 2]);
+    snprintf(line, sizeof(line), "%s %d %.6f %.6f\n", kv.first.c_str(), (int)n, total, median);
     out += line;
   }
   if (out.size() + 1 > buf_len) return fail(MOE_ERR_INVALID_ARG, "report buffer too small");
