@@ -473,7 +473,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
-    n_prof = min(args.steps, 20)
+    n_prof = args.steps       # the profiled pass repeats the timed steps' length too
     t0 = time.time()
     for i in range(args.steps):
         flush.zero_()
@@ -488,9 +488,9 @@ def run_ours(args, cfg, rank, world, local_rank):
     # Per-kernel live times come from a separate profiled pass: the library's
     # profiling events around every kernel would otherwise sit inside the timed
     # steps (they serialise the dependent launches and lengthened the step by
-    # ~4 %).  The pass repeats the timed steps' history (0.3 s idle, then the
-    # steps), because the GPU's clock under its power cap depends on how long
-    # it has been busy: a pass run straight after the timed steps measured
+    # ~4 %).  The pass repeats the timed steps' history (0.3 s idle, then as
+    # many steps), because the GPU's clock under its power cap depends on how
+    # long it has been busy: a pass run straight after the timed steps measured
     # every kernel 7-14 % slower than the timed steps implied.  Each kernel's
     # rate is set by its median launch time, so that a one-off stall (seen
     # once as a 50 % longer mean for one kernel) does not set it.
