@@ -55,7 +55,7 @@ Readings taken where the pages are silent:
 
 parity pins: tests/test_oracle_pins.py (brute force, dense masked evaluation,
 closed-form 2-expert example, central finite differences, the 145 -> 128
-rounding example, invariants; MXFP8 against torch's float8_e4m3fn conversion,
+rounding example, invariants, hand-derived values at every bf16 staging point; MXFP8 against torch's float8_e4m3fn conversion,
 the 256-code table, closed-form scales and saturation).  No function here is
 unpinned.
 """

@@ -261,6 +261,52 @@ def test_forward_matches_per_expert_masked_loop():
     np.testing.assert_allclose(fwd["out"], out, rtol=1e-12, atol=1e-12)
 
 
+SILU1 = 0.7310585786300049      # silu(1) = 1 / (1 + e^-1)
+DSILU1 = 0.9276705118714869     # silu'(1) = sigmoid(1) * (1 + (1 - sigmoid(1)))
+
+
+def test_bf16_staging_points_on_hand_derived_scalars():
+    """Each bf16 staging point of one expert's rows -- H, A and Y forward; A
+    (recomputed), dH, s*A and dX_perm backward -- on 1 x 1 operands whose
+    staged values were worked out by hand: bf16 keeps 8 significant bits, so
+    values in [2^(e-1), 2^e) lie on a grid of 2^(e-8), ties to even.  Each
+    case is chosen so that dropping or moving one rounding changes a result
+    (the alternative is given beside each value)."""
+    one = np.ones((1, 1))
+    # H: h1 = 1 + 2^-9 is below 1 + 2^-8 (half the grid step at 1), so it is
+    # stored as 1 and A = bf16(silu(1)) = bf16(187.15 / 256) = 187/256; from
+    # the unrounded h1, silu(1 + 2^-9) = 187.62 / 256 would give 188/256.
+    h1, h3, a, y = O.expert_rows_forward(one, one * (1 + 2.0 ** -9), one, one, staged=True)
+    assert (h1[0, 0], h3[0, 0], a[0, 0], y[0, 0]) == (1.0, 1.0, 187 / 256, 187 / 256)
+    # A and Y: with W2 = 9/16, A W2 = 187/256 * 9/16 = 210.375 * 2^-9, stored as
+    # Y = 210/512; from an unrounded A, silu(1) * 9/16 = 210.55 * 2^-9 -> 211/512.
+    _, _, a, y = O.expert_rows_forward(one, one, one, one * 9 / 16, staged=True)
+    assert (a[0, 0], y[0, 0]) == (187 / 256, 210 / 512)
+    _, _, a, y = O.expert_rows_forward(one, one, one, one * 9 / 16, staged=False)
+    assert abs(a[0, 0] - SILU1) < 1e-15 and abs(y[0, 0] - SILU1 * 9 / 16) < 1e-15
+    # Backward with x = 1, W1 = 1, W3 = 5/4, W2 = 1/4, dO = 5/4, gate g = 3/8:
+    # h1 = 1, h3 = 5/4, A = bf16(silu(1) * 5/4 = 233.94 / 256) = 234/256.
+    w3, w2, dout, g = one * 5 / 4, one / 4, one * 5 / 4, np.array([3 / 8])
+    ds, da1, da3, ga, dxp = O.expert_rows_backward(dout, g, one, w3, one, w3, w2, staged=True)
+    # dS = <dA', A> with dA' = dO W2^T = 5/16: 5/16 * 234/256 = 585/2048
+    # (0.285567 from an unrounded A)
+    assert ds[0] == 585 / 2048
+    # dA = g dA' = 15/128; dH3 = bf16(dA silu(1) = 175.45 * 2^-11) = 175/2048
+    assert da3[0, 0] == 175 / 2048
+    # dH1 = bf16(dA h3 silu'(1) = 139.15 * 2^-10) = 139/1024
+    assert da1[0, 0] == 139 / 1024
+    # s*A = bf16(3/8 * 234/256 = 175.5 * 2^-9): a tie, to even -> 176/512
+    # (175/512 from an unrounded A, 175.45 * 2^-9)
+    assert ga[0, 0] == 176 / 512
+    # dX_perm = bf16(dH1 W1 + dH3 W3 = 139/1024 + 175/2048 * 5/4 = 248.375 * 2^-10)
+    # = 248/1024 (from unrounded dH1, dH3: 248.81 * 2^-10 -> 249/1024)
+    assert dxp[0, 0] == 248 / 1024
+    ds, da1, da3, ga, dxp = O.expert_rows_backward(dout, g, one, w3, one, w3, w2, staged=False)
+    assert abs(ds[0] - 5 / 16 * SILU1 * 5 / 4) < 1e-15
+    assert abs(da1[0, 0] - 15 / 128 * 5 / 4 * DSILU1) < 1e-15
+    assert abs(dxp[0, 0] - (15 / 128 * 5 / 4 * DSILU1 + 15 / 128 * SILU1 * 5 / 4)) < 1e-15
+
+
 def test_staged_forward_close_to_ideal():
     rng = np.random.default_rng(10)
     x, wg, w1, w3, w2, _ = _rand_layer(rng, 50, 32, 16, 4, scale=0.2)
