@@ -625,7 +625,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     if rank != 0:
         return 0
 
-    # ---- roofline of the dominant kernel (measured live over the timed region)
+    # ---- roofline of the dominant kernel (live CUDA-event times of the profiled pass)
     peaks, peak_src = load_peaks()
     gemm = {n: v for n, v in prof.items() if gemm_flops(n, cfg.T, cfg.d, cfg.f, cfg.k)}
     # avg_us: the median launch time over the profiled pass
