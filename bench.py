@@ -572,7 +572,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                            chunks(objs[b].out) + chunks(objs[b].grads["dx"]))) for b in range(2)]
 
     def pipeline(n):
-        done, down = [None] * n, [None] * n
+        # The first nch copies of a step move x (up) or out (down), the next
+        # nch dO (up) or dx (down): the forward waits only for x, the
+        # backward for dO, out is read back as soon as the forward is done.
+        done, fwd_done, down = [None] * n, [None] * n, [None] * n
         start = torch.cuda.Event(enable_timing=True)
         start.record(up_s[0])
         for s_ in up_s[1:]:
@@ -589,19 +592,26 @@ def run_ours(args, cfg, rank, world, local_rank):
                     ev.record(s_)
                     ups.append(ev)
             with torch.cuda.stream(comp_s):
-                for ev in ups:
+                for ev in ups[:nch]:                    # x
                     comp_s.wait_event(ev)
                 if i >= 2:
-                    for ev in down[i - 2]:              # step i-2's results are read back
+                    for ev in down[i - 2][:nch]:        # step i-2's out is read back
                         comp_s.wait_event(ev)
                 objs[b].forward(x_d[b], wg, w1, w3, w2, lo, lb, logit_noise=noise)
+                fwd_done[i] = torch.cuda.Event()
+                fwd_done[i].record(comp_s)
+                for ev in ups[nch:]:                    # dO
+                    comp_s.wait_event(ev)
+                if i >= 2:
+                    for ev in down[i - 2][nch:]:        # step i-2's dx is read back
+                        comp_s.wait_event(ev)
                 objs[b].backward(d_d[b])
                 done[i] = torch.cuda.Event()
                 done[i].record(comp_s)
             down[i] = []
-            for s_, (dst, src) in zip(down_s, down_pairs[b]):
+            for j, (s_, (dst, src)) in enumerate(zip(down_s, down_pairs[b])):
                 with torch.cuda.stream(s_):
-                    s_.wait_event(done[i])
+                    s_.wait_event(fwd_done[i] if j < nch else done[i])
                     dst.copy_(src, non_blocking=True)
                     ev = torch.cuda.Event(enable_timing=True)
                     ev.record(s_)
