@@ -555,16 +555,17 @@ def run_ours(args, cfg, rank, world, local_rank):
     dx_h = [torch.empty_like(step.grads["dx"], device="cpu").pin_memory() for _ in range(2)]
     x_d = [torch.empty_like(x) for _ in range(2)]
     d_d = [torch.empty_like(dout) for _ in range(2)]
-    # the copies are split into row chunks, one copy stream per chunk and
-    # direction (x and dO up, out and dx down), so that they spread over the
-    # copy engines
+    # the copies are split into row chunks, one copy stream per chunk index
+    # and direction: up, each stream copies its chunk of x and then its chunk
+    # of dO (so x, which the forward needs first, arrives first); down, its
+    # chunk of out and then of dx
     nch = max(1, args.e2e_chunks)
 
     def chunks(t):
         return list(t.chunk(nch, dim=0))
 
-    up_s = [torch.cuda.Stream() for _ in range(2 * nch)]
-    down_s = [torch.cuda.Stream() for _ in range(2 * nch)]
+    up_s = [torch.cuda.Stream() for _ in range(nch)] * 2      # x chunks, then dO chunks
+    down_s = [torch.cuda.Stream() for _ in range(nch)] * 2    # out chunks, then dx chunks
     comp_s = torch.cuda.Stream()
     up_pairs = [list(zip(chunks(x_d[b]) + chunks(d_d[b]), chunks(x_h) + chunks(d_h)))
                 for b in range(2)]
@@ -729,7 +730,9 @@ def run_ours(args, cfg, rank, world, local_rank):
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_total / len(e2e_ms) if e2e_ms else None,
                 "pipelined": "upload of step i+1 and read-back of step i-1 overlap step i's kernels; "
-                             f"{nch} row chunk(s) per tensor, one copy stream per chunk and direction"},
+                             f"{nch} row chunk(s) per tensor, one copy stream per chunk index and "
+                             "direction (x before dO up, out before dx down); the forward waits "
+                             "for x only, out is read back once the forward is done"},
         "clocks": clocks,
         "sustained": sustained,
         "gpu_launches": launches,
