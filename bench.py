@@ -625,9 +625,18 @@ def run_ours(args, cfg, rank, world, local_rank):
         return start.elapsed_time(end)
 
     e2e_ms = []
+    e2e_match = None
     if args.e2e_steps > 0:
+        # every step sees the same inputs and the kernels are deterministic,
+        # so the results read back must equal the device-resident step's
+        out_ref, dx_ref = step.out.clone(), step.grads["dx"].clone()
         pipeline(3)                                     # warm-up
         e2e_ms = [pipeline(args.e2e_steps) / args.e2e_steps] * args.e2e_steps
+        e2e_match = all(torch.equal(out_h[b].to(dev), out_ref) and torch.equal(dx_h[b].to(dev), dx_ref)
+                        for b in range(2))
+        if not e2e_match:
+            print("warning: end-to-end pipeline results read back differ from the device step's",
+                  file=sys.stderr, flush=True)
     e2e_total = max_over_ranks(sum(e2e_ms), world, dev)
     e2e_value = job_tokens_per_s(world, cfg.T, len(e2e_ms), e2e_total) if e2e_ms else None
     h2d = x.numel() * x.element_size() + dout.numel() * dout.element_size()
@@ -729,6 +738,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_total / len(e2e_ms) if e2e_ms else None,
+                "results_match_device": e2e_match,
                 "pipelined": "upload of step i+1 and read-back of step i-1 overlap step i's kernels; "
                              f"{nch} row chunk(s) per tensor, one copy stream per chunk index and "
                              "direction (x before dO up, out before dx down); the forward waits "
